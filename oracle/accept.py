@@ -1,0 +1,146 @@
+"""Lossless acceptance of k drafted tokens, the correction draw and the bonus draw, float64.
+
+Test infrastructure (CPU oracle): never imported by the product path.
+
+The rule (the pages cite Leviathan et al., "Fast Inference from Transformers via
+Speculative Decoding", for it -- Google blog translation, section "how speculative
+decoding works"; Gemma 4 MTP serving guide, section 1 -- and state its property: rejected
+tokens are replaced by a token the target generates itself, so the output is
+distributionally identical to decoding without a drafter -- "Gemma 4 MTP: drafter drafts,
+target verifies", section "basic structure of speculative decoding"):
+
+  target logits z [B, k+1, V], draft logits y [B, k, V], drafts d [B, k].
+  p_i = softmax(z[i-1] / T), q_i = softmax(y[i-1] / T) for i = 1..k; p_{k+1} from z[k].
+  For i = 1..k: accept d_i iff u_i < p_i(d_i) / q_i(d_i), u_i uniform in [0, 1); stop at
+  the first rejection (serving guide, section 4: from the first rejected token on the
+  rest of the draft is discarded and the target generates the token itself).
+  Rejected at i: emit x ~ norm(max(0, p_i - q_i)) (p_i itself when that is all zero).
+  All k accepted: emit the bonus token x ~ p_{k+1} (GeekNews summary, section "how MTP
+  works": when the target agrees with the drafts it accepts them and adds one token).
+  Outputs: a = accepted count, tokens [d_1 .. d_a, x, -1 ...] of length k+1.
+
+  T = 0 (greedy): accept d_i iff d_i == argmax z[i-1]; emit argmax z[a]; the lowest id
+  wins ties.
+
+Readings of points the pages leave open:
+  * q(d) = 0 accepts iff p(d) > 0 (the ratio is +inf).
+  * Categorical draws are exponential races: x = argmin_v E_v / w_v over w_v > 0 with
+    E_v = -ln(1 - V_v), V_v the per-token Philox uniform of the draw's row and purpose;
+    lowest v wins ties.  This is an exact categorical draw needing no normalisation.
+    Implemented as argmax of ln w_v - ln E_v.
+  * Margins (decisions a float32 implementation may take differently): an acceptance
+    with |u - p/q| < MARGIN, a draw whose winner leads some other token by less than
+    MARGIN plus both tokens' error bounds on the ln-key scale, a greedy argmax whose top
+    two logits differ by less than MARGIN * max(1, |top|).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .philox import accept_uniform, token_uniform_rows
+
+MARGIN = 1e-4          # spec margin on |u - p/q|; reused for draws and argmaxes
+REL_P = 1e-5           # assumed float32 relative error bound on a probability p_v or q_v
+ABS_KEY = 1e-6         # assumed float32 absolute error bound on ln E_v and z_v / T
+
+PURPOSE_ACCEPT = 0
+PURPOSE_TARGET = 1
+PURPOSE_DRAFTER = 2
+
+
+def softmax(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, np.float64)
+    m = x.max(axis=-1, keepdims=True)
+    e = np.exp(x - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def race(w: np.ndarray, V: np.ndarray):
+    """Exponential race per row: returns (winner ids, ln-keys g)."""
+    E = -np.log1p(-V)
+    with np.errstate(divide="ignore"):
+        g = np.log(w) - np.log(E)
+    g = np.where(w > 0, g, -np.inf)
+    return np.argmax(g, axis=-1), g
+
+
+def _race_margin(g: np.ndarray, err: np.ndarray, x: np.ndarray) -> np.ndarray:
+    R = g.shape[0]
+    gx = g[np.arange(R), x]
+    ex = err[np.arange(R), x]
+    with np.errstate(invalid="ignore"):
+        upper = np.where(np.isfinite(g), g + err, g)
+    upper[np.arange(R), x] = -np.inf
+    return upper.max(axis=-1) > gx - ex - MARGIN
+
+
+def greedy_gap(z: np.ndarray) -> np.ndarray:
+    """(top1 - top2) / max(1, |top1|) over the last axis."""
+    part = np.partition(z, -2, axis=-1)
+    t1, t2 = part[..., -1], part[..., -2]
+    return (t1 - t2) / np.maximum(1.0, np.abs(t1))
+
+
+def accept(z, y, drafts, temperature: float, seed: int, step: int,
+           purpose: int = PURPOSE_TARGET):
+    """Apply the rule to a batch.  z [B, k+1, V], y [B, k, V] (unused when k = 0 or T = 0),
+    drafts [B, k].  Returns dict(n_accepted [B], out_tokens [B, k+1], margin [B] bool)."""
+    z = np.asarray(z, np.float64)
+    B, n_q, V = z.shape
+    k = n_q - 1
+    drafts = np.asarray(drafts, np.int64).reshape(B, k)
+    n_acc = np.zeros(B, np.int64)
+    margin = np.zeros(B, bool)
+    bidx = np.arange(B)
+
+    if temperature == 0.0:
+        am = np.argmax(z, axis=-1)
+        gap = greedy_gap(z)
+        active = np.ones(B, bool)
+        for i in range(1, k + 1):
+            margin |= active & (gap[:, i - 1] < MARGIN)
+            ok = active & (drafts[:, i - 1] == am[:, i - 1])
+            n_acc += ok
+            active = ok
+        margin |= gap[bidx, n_acc] < MARGIN
+        x = am[bidx, n_acc]
+    else:
+        T = float(temperature)
+        p = softmax(z / T)
+        q = softmax(np.asarray(y, np.float64) / T) if k > 0 else None
+        rows = bidx * n_q
+        active = np.ones(B, bool)
+        for i in range(1, k + 1):
+            d = drafts[:, i - 1]
+            pd = p[bidx, i - 1, d]
+            qd = q[bidx, i - 1, d]
+            with np.errstate(divide="ignore", invalid="ignore"):
+                ratio = np.where(qd > 0, pd / qd, np.where(pd > 0, np.inf, 0.0))
+            u = accept_uniform(seed, step, rows + i - 1)
+            margin |= active & (np.abs(u - ratio) < MARGIN)
+            active = active & (u < ratio)
+            n_acc += active
+        pa = p[bidx, n_acc]
+        if k > 0:
+            qa = q[bidx, np.minimum(n_acc, k - 1)]
+            resid = np.maximum(0.0, pa - qa)
+            bonus = n_acc == k
+            empty = resid.sum(axis=-1) == 0.0
+            use_p = (bonus | empty)[:, None]
+            w = np.where(use_p, pa, resid)
+            with np.errstate(divide="ignore", invalid="ignore"):
+                err = np.where(use_p, ABS_KEY * (1.0 + np.abs(z[bidx, n_acc] / T)),
+                               REL_P * (pa + qa) / w + ABS_KEY)
+        else:
+            w = pa
+            err = ABS_KEY * (1.0 + np.abs(z[:, 0] / T))
+        Vu = token_uniform_rows(seed, step, rows + n_acc, purpose, V)
+        x, g = race(w, Vu)
+        margin |= _race_margin(g, np.nan_to_num(err, nan=np.inf, posinf=np.inf), x)
+
+    out = np.full((B, n_q), -1, np.int64)
+    for b in range(B):
+        a = int(n_acc[b])
+        out[b, :a] = drafts[b, :a]
+        out[b, a] = x[b]
+    return dict(n_accepted=n_acc, out_tokens=out, margin=margin)
