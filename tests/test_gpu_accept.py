@@ -1,0 +1,172 @@
+"""GPU parity of sd_accept against the float64 oracle on identical float32 inputs.
+
+Integer outputs must match bit for bit, except sequences the oracle flags as within the
+spec margin (|u - p/q| < 1e-4, or a draw / argmax whose best keys are that close);
+those are counted and checked for validity only.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy import stats
+
+import synthetic as S
+import verify_step_b200 as sd
+from oracle import accept as OACC
+from tests.gpu_util import DEV, status_ok, to_dev, workspace
+
+pytestmark = pytest.mark.gpu
+
+NOISE = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "draft_noise.json")))
+
+
+def gpu_accept(z, y, drafts, T, seed, step, purpose=1):
+    B, n_q, V = z.shape
+    k = n_q - 1
+    desc = sd.AcceptDesc(batch=B, k=k, vocab=V, temperature=float(T), seed=seed, step=step,
+                         purpose=purpose)
+    n_acc = torch.full((B,), -9, dtype=torch.int32, device=DEV)
+    out = torch.full((B, n_q), -9, dtype=torch.int32, device=DEV)
+    flags = torch.full((B,), -9, dtype=torch.int32, device=DEV)
+    ws = workspace(sd.sd_accept_workspace_size(desc))
+    sd.sd_accept(desc, to_dev(z), to_dev(y) if (y is not None and k > 0) else None,
+                 to_dev(drafts) if k > 0 else None, n_acc, out, flags, ws)
+    torch.cuda.synchronize()
+    return n_acc.cpu().numpy(), out.cpu().numpy(), flags.cpu().numpy()
+
+
+def draw_drafts(y, T, seed, step):
+    """Drafts drawn from q = softmax(y / T) by the oracle's own draw (drafter purpose)."""
+    B, k, V = y.shape
+    d = np.zeros((B, k), np.int64)
+    for i in range(k):
+        if T == 0:
+            d[:, i] = np.argmax(y[:, i].numpy(), axis=-1)
+        else:
+            r = OACC.accept(y[:, i:i + 1].numpy(), None, np.zeros((B, 0)), T, seed=seed,
+                            step=step * 64 + i, purpose=OACC.PURPOSE_DRAFTER)
+            d[:, i] = r["out_tokens"][:, 0]
+    return torch.from_numpy(d.astype(np.int32))
+
+
+def compare(z, y, drafts, T, seed, step, purpose=1, max_flag_frac=0.05):
+    n_acc, out, gflags = gpu_accept(z, y, drafts, T, seed, step, purpose)
+    ref = OACC.accept(z.double().numpy(), None if y is None else y.double().numpy(),
+                      drafts.numpy(), T, seed=seed, step=step, purpose=purpose)
+    ok = ~ref["margin"]
+    assert np.array_equal(n_acc[ok], ref["n_accepted"][ok])
+    assert np.array_equal(out[ok], ref["out_tokens"][ok])
+    # flagged sequences: outputs still well formed
+    B, n_q = out.shape
+    for b in np.nonzero(~ok)[0]:
+        a = n_acc[b]
+        assert 0 <= a < n_q and np.all(out[b, :a] == drafts[b, :a].numpy())
+        assert 0 <= out[b, a] < z.shape[-1] and np.all(out[b, a + 1:] == -1)
+    assert (~ok).mean() <= max_flag_frac
+    assert np.all((gflags == 0) | (gflags == 1))
+    assert status_ok()
+    return n_acc, out, ref
+
+
+def tuned_inputs(seed, B, k, V=262144):
+    z = S.make_logits(seed, B * (k + 1), V).reshape(B, k + 1, V)
+    sig = [NOISE["sigma_pos0"]] + [NOISE["sigma_later"]] * (k - 1)
+    y = torch.stack([S.perturb(seed * 100 + i, z[:, i], sig[i]) for i in range(k)], dim=1)
+    return z, y
+
+
+@pytest.mark.parametrize("k", [1, 2, 4, 6])
+def test_full_vocab_sampling(k):
+    """B8, V262144, T=1, draft logits tuned to the serving guide's acceptance."""
+    z, y = tuned_inputs(100 + k, 8, k)
+    drafts = draw_drafts(y, 1.0, seed=5, step=k)
+    compare(z, y, drafts, 1.0, seed=11, step=k)
+
+
+def test_full_vocab_temperature_and_batch64():
+    z, y = tuned_inputs(7, 64, 2)
+    drafts = draw_drafts(y, 0.7, seed=6, step=1)
+    compare(z, y, drafts, 0.7, seed=12, step=3)
+
+
+def test_full_vocab_greedy():
+    z, y = tuned_inputs(8, 16, 3)
+    drafts = draw_drafts(y, 0, seed=0, step=0)
+    drafts[::2, 0] = torch.from_numpy(np.argmax(z[::2, 0].numpy(), axis=-1).astype(np.int32))
+    n_acc, _, _ = compare(z, None, drafts, 0.0, seed=0, step=0)
+
+
+def test_drafter_draw_with_masked_logits():
+    """k = 0 (the drafter sampling its own token, purpose 2) on clustered-style logits that
+    are -inf outside a subset of tokens."""
+    B, V = 8, 262144
+    z = S.make_logits(9, B, V)
+    mask = torch.from_numpy(np.random.default_rng(1).random((B, V)) < 0.03)
+    z = torch.where(mask, z, torch.full_like(z, float("-inf"))).reshape(B, 1, V)
+    n_acc, out, _ = compare(z, None, torch.zeros(B, 0, dtype=torch.int32), 1.0, seed=3, step=2,
+                            purpose=2)
+    assert np.all(mask.numpy()[np.arange(B), out[:, 0]])
+
+
+def test_small_vocab_exact_many_sequences():
+    """V=8, k=3, 100000 sequences: every unflagged output equals the oracle."""
+    B, k, V = 100_000, 3, 8
+    z = S.make_logits(21, B * (k + 1), V, std=1.5).reshape(B, k + 1, V)
+    y = torch.stack([S.perturb(22 + i, z[:, i], 1.0) for i in range(k)], dim=1)
+    drafts = draw_drafts(y, 1.0, seed=1, step=0)
+    compare(z, y, drafts, 1.0, seed=99, step=4, max_flag_frac=0.01)
+
+
+def _tables(seed, V, k):
+    rng = np.random.default_rng(seed)
+    P, Q = {}, {}
+    for i in range(1, k + 2):
+        for pre in itertools.product(range(V), repeat=i - 1):
+            zp = rng.standard_normal(V)
+            P[pre] = np.exp(zp) / np.exp(zp).sum()
+            if i <= k:
+                zq = zp + rng.standard_normal(V) * 1.2
+                Q[pre] = np.exp(zq) / np.exp(zq).sum()
+    return P, Q
+
+
+def test_gpu_reproduces_target_distribution():
+    """The pages' guarantee on the GPU: with 10^6 sequences the first emitted token follows
+    p_1 and the first two follow p_1 * p_2 (chi-square, p > 0.01)."""
+    V, k, n = 8, 2, 1_000_000
+    P, Q = _tables(5, V, k)
+    rng = np.random.default_rng(2)
+    d = np.zeros((n, k), np.int64)
+    d[:, 0] = rng.choice(V, n, p=Q[()])
+    for v in range(V):
+        s = d[:, 0] == v
+        d[s, 1] = rng.choice(V, int(s.sum()), p=Q[(v,)])
+    z = np.zeros((n, k + 1, V), np.float32)
+    y = np.zeros((n, k, V), np.float32)
+    z[:, 0] = np.log(P[()])
+    y[:, 0] = np.log(Q[()])
+    for v in range(V):
+        s = d[:, 0] == v
+        z[s, 1] = np.log(P[(v,)])
+        y[s, 1] = np.log(Q[(v,)])
+        for u in range(V):
+            s2 = s & (d[:, 1] == u)
+            z[s2, 2] = np.log(P[(v, u)])
+    n_acc, out, _ = gpu_accept(torch.from_numpy(z), torch.from_numpy(y),
+                               torch.from_numpy(d.astype(np.int32)), 1.0, seed=17, step=0)
+    first = np.bincount(out[:, 0], minlength=V)
+    assert stats.chisquare(first, P[()] * n).pvalue > 0.01
+    # two-token joint over the sequences that emitted >= 2 tokens, compared with the
+    # probability of that event per pair: P(e1, e2, a >= 1)
+    two = np.zeros((V, V))
+    sel = n_acc >= 1
+    np.add.at(two, (out[sel, 0], out[sel, 1]), 1)
+    exp = np.zeros((V, V))
+    for v in range(V):
+        alpha = min(1.0, P[()][v] / Q[()][v])
+        exp[v] = Q[()][v] * alpha * P[(v,)]  # d1 = v accepted; next token ~ p_2(.|v) exactly
+    exp = exp / exp.sum() * two.sum()
+    assert stats.chisquare(two.ravel(), exp.ravel()).pvalue > 0.01

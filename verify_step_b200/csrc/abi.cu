@@ -1,0 +1,109 @@
+// Library-wide host helpers and the status entry points of the C ABI.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "host.cuh"
+
+namespace sdv {
+
+// Per-device status word: kernels record the first device-side error here.
+__device__ int g_status_word;
+
+int *device_status_word() {
+  static std::mutex mu;
+  static int *addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    addr[dev] = reinterpret_cast<int *>(p);
+  }
+  return addr[dev];
+}
+
+int sm_count() {
+  static int cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace sdv
+
+extern "C" {
+
+const char *sd_status_string(sd_status s) {
+  switch (s) {
+    case SD_OK: return "ok";
+    case SD_ERR_INVALID_ARG: return "invalid argument";
+    case SD_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SD_ERR_WORKSPACE: return "workspace too small";
+    case SD_ERR_CUDA: return "CUDA error";
+    case SD_ERR_TIMEOUT: return "device wait timed out";
+    case SD_ERR_DEVICE: return "out-of-range index on the device";
+  }
+  return "unknown status";
+}
+
+sd_status sd_device_status_read(int *out, sd_stream stream) {
+  if (!out) return SD_ERR_INVALID_ARG;
+  int *w = sdv::device_status_word();
+  if (!w) return SD_ERR_CUDA;
+  if (cudaMemcpyAsync(out, w, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream) !=
+      cudaSuccess)
+    return SD_ERR_CUDA;
+  return sdv::cuda_status(cudaStreamSynchronize((cudaStream_t)stream));
+}
+
+sd_status sd_device_status_clear(sd_stream stream) {
+  int *w = sdv::device_status_word();
+  if (!w) return SD_ERR_CUDA;
+  return sdv::cuda_status(cudaMemsetAsync(w, 0, sizeof(int), (cudaStream_t)stream));
+}
+
+int sd_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,409 @@
+// Lossless acceptance of k drafts, correction / bonus draw, greedy rule (sm_100a).
+//
+// The rule (pages cite Leviathan et al. for it: Google blog translation, section "how
+// speculative decoding works"; property stated in "Gemma 4 MTP: drafter drafts, target
+// verifies", section "basic structure of speculative decoding"): accept d_i iff
+// u_i < p_i(d_i) / q_i(d_i); at the first rejection emit x ~ norm(max(0, p_i - q_i)); if all
+// are accepted emit the bonus x ~ p_{k+1}.  T = 0: accept iff d_i == argmax, emit argmax.
+//
+// Two kernels, both bandwidth-bound scans of float32 logits (vectorised 16-byte loads):
+//  1. accept_stats: one CTA per (row, 8192-token chunk): online max / sum of exp(x / T)
+//     (T > 0) or the top two values and the argmax (T = 0) of the chunk.
+//  2. accept_draw: one CTA per (sequence, chunk).  Every CTA merges the row statistics in
+//     chunk order, takes the acceptance decisions (a handful of single-element reads and
+//     Philox uniforms), then runs the exponential race of the draw row over its chunk:
+//     key_v = ln w_v - ln(-ln(1 - V_v)), V_v the token's Philox uniform, for both the
+//     residual weights max(0, p - q) and for p (the fallback when the residual is empty).
+//     The last CTA of a sequence (atomic ticket; no waiting) merges the chunk winners in chunk
+//     order, lowest token id first on ties, and writes the outputs.
+#include <cfloat>
+
+#include "common.cuh"
+#include "host.cuh"
+#include "philox.cuh"
+
+namespace sdv {
+namespace acc {
+
+constexpr int kChunk = 8192;
+constexpr int kThreads = 256;
+constexpr float kMargin = 1e-4f;
+
+struct Params {
+  int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, rows_t, rows_total;
+  float T;
+  unsigned long long seed;
+  uint32_t step;
+  const float *z;
+  const float *y;
+  const int32_t *drafts;
+  int32_t *n_acc;
+  int32_t *out;
+  int32_t *margin;
+  float4 *stats;   // [rows_total][nchunks]
+  float4 *cand;    // [B][nchunks][2]
+  unsigned int *counters;  // [B]
+  int *status;
+};
+
+struct Cand {  // best and runner-up key of a race, best token id
+  float g1, g2;
+  int v1;
+};
+
+__device__ __forceinline__ void cand_push(Cand &c, float g, int v) {
+  // tokens arrive in increasing v per thread; strict > keeps the lowest id on ties
+  if (g > c.g1) {
+    c.g2 = c.g1;
+    c.g1 = g;
+    c.v1 = v;
+  } else if (g > c.g2) {
+    c.g2 = g;
+  }
+}
+
+__device__ __forceinline__ Cand cand_merge(const Cand &a, const Cand &b) {
+  // a holds lower token ids than b when ids tie in key
+  Cand r;
+  if (b.g1 > a.g1 || (b.g1 == a.g1 && b.v1 < a.v1 && b.v1 >= 0)) {
+    r.g1 = b.g1;
+    r.v1 = b.v1;
+    r.g2 = fmaxf(b.g2, a.g1);
+  } else {
+    r.g1 = a.g1;
+    r.v1 = a.v1;
+    r.g2 = fmaxf(a.g2, b.g1);
+  }
+  return r;
+}
+
+__device__ __forceinline__ Cand cand_shfl(const Cand &c, int off) {
+  Cand o;
+  o.g1 = __shfl_xor_sync(0xffffffffu, c.g1, off);
+  o.g2 = __shfl_xor_sync(0xffffffffu, c.g2, off);
+  o.v1 = __shfl_xor_sync(0xffffffffu, c.v1, off);
+  return o;
+}
+
+// (max, sum exp(x - max)) pairs
+__device__ __forceinline__ void ms_merge(float &m, float &s, float m2, float s2) {
+  const float mm = fmaxf(m, m2);
+  if (mm == -INFINITY) return;
+  s = s * expf(m - mm) + s2 * expf(m2 - mm);
+  m = mm;
+}
+
+__device__ __forceinline__ const float *row_ptr(const Params &p, int r) {
+  return r < p.rows_t ? p.z + (size_t)r * p.ld_t : p.y + (size_t)(r - p.rows_t) * p.ld_d;
+}
+
+__global__ void __launch_bounds__(kThreads) accept_stats_kernel(const Params p) {
+  const int r = blockIdx.x, c = blockIdx.y;
+  if (c == 0 && r == 0)
+    for (int b = threadIdx.x; b < p.B; b += blockDim.x) p.counters[b] = 0u;
+  const float *row = row_ptr(p, r);
+  const int v0 = c * kChunk;
+  const int v1 = min(p.V, v0 + kChunk);
+  const float4 *row4 = reinterpret_cast<const float4 *>(row + v0);
+  const int n4 = (v1 - v0) >> 2;
+  __shared__ float4 red[kThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (p.T > 0.f) {
+    float m = -INFINITY, s = 0.f;
+    for (int i = threadIdx.x; i < n4; i += kThreads) {
+      const float4 x4 = __ldg(row4 + i);
+      const float a = x4.x / p.T, b = x4.y / p.T, cc = x4.z / p.T, d = x4.w / p.T;
+      const float mx = fmaxf(fmaxf(a, b), fmaxf(cc, d));
+      if (mx > m) {
+        s = s * expf(m - mx);
+        m = mx;
+      }
+      if (m != -INFINITY) s += expf(a - m) + expf(b - m) + expf(cc - m) + expf(d - m);
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+      const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+      ms_merge(m, s, m2, s2);
+    }
+    if (lane == 0) red[warp] = make_float4(m, s, 0.f, 0.f);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float M = red[0].x, S = red[0].y;
+      for (int w = 1; w < kThreads / 32; ++w) ms_merge(M, S, red[w].x, red[w].y);
+      p.stats[(size_t)r * p.nchunks + c] = make_float4(M, S, 0.f, 0.f);
+    }
+  } else {
+    Cand cd{-INFINITY, -INFINITY, -1};
+    for (int i = threadIdx.x; i < n4; i += kThreads) {
+      const float4 x4 = __ldg(row4 + i);
+      const int v = v0 + 4 * i;
+      cand_push(cd, x4.x, v);
+      cand_push(cd, x4.y, v + 1);
+      cand_push(cd, x4.z, v + 2);
+      cand_push(cd, x4.w, v + 3);
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+      const Cand o = cand_shfl(cd, off);
+      // lane order is not token order inside a warp: break ties by id explicitly
+      cd = (lane & off) ? cand_merge(o, cd) : cand_merge(cd, o);
+    }
+    if (lane == 0) red[warp] = make_float4(cd.g1, __int_as_float(cd.v1), cd.g2, 0.f);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      Cand t{red[0].x, red[0].z, __float_as_int(red[0].y)};
+      for (int w = 1; w < kThreads / 32; ++w) {
+        Cand o{red[w].x, red[w].z, __float_as_int(red[w].y)};
+        t = cand_merge(t, o);
+      }
+      p.stats[(size_t)r * p.nchunks + c] = make_float4(t.g1, __int_as_float(t.v1), t.g2, 0.f);
+    }
+  }
+}
+
+// Merged statistics of one row: (max, sum) for T > 0; (top1, argmax, top2) for T = 0.
+__device__ __forceinline__ float4 row_stats(const Params &p, int r) {
+  const float4 *st = p.stats + (size_t)r * p.nchunks;
+  if (p.T > 0.f) {
+    float M = st[0].x, S = st[0].y;
+    for (int c = 1; c < p.nchunks; ++c) ms_merge(M, S, st[c].x, st[c].y);
+    return make_float4(M, S, 0.f, 0.f);
+  }
+  Cand t{st[0].x, st[0].z, __float_as_int(st[0].y)};
+  for (int c = 1; c < p.nchunks; ++c) {
+    Cand o{st[c].x, st[c].z, __float_as_int(st[c].y)};
+    t = cand_merge(t, o);
+  }
+  return make_float4(t.g1, __int_as_float(t.v1), t.g2, 0.f);
+}
+
+__global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
+  const int b = blockIdx.x, c = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int s_a, s_flag;
+  __shared__ float s_mz, s_isz, s_my, s_isy;
+  __shared__ float4 red[2][kThreads / 32];
+  __shared__ int s_last;
+
+  if (threadIdx.x == 0) {
+    int a = 0, flag = 0;
+    for (int i = 1; i <= p.k; ++i) {
+      const int d = p.drafts[(size_t)b * p.k + i - 1];
+      const int rt = b * p.n_q + i - 1;
+      bool acc = false;
+      if (d < 0 || d >= p.V) {
+        record_status(p.status, SD_ERR_DEVICE);
+      } else if (p.T > 0.f) {
+        const float4 sz = row_stats(p, rt);
+        const float4 sy = row_stats(p, p.rows_t + b * p.k + i - 1);
+        const float pd = expf(p.z[(size_t)rt * p.ld_t + d] / p.T - sz.x) / sz.y;
+        const float qd =
+            expf(p.y[((size_t)b * p.k + i - 1) * p.ld_d + d] / p.T - sy.x) / sy.y;
+        const float ratio = qd > 0.f ? pd / qd : (pd > 0.f ? INFINITY : 0.f);
+        const float u = accept_uniform(p.seed, p.step, (uint32_t)rt);
+        if (fabsf(u - ratio) < kMargin) flag = 1;
+        acc = u < ratio;
+      } else {
+        const float4 sz = row_stats(p, rt);
+        if ((sz.x - sz.z) / fmaxf(1.f, fabsf(sz.x)) < kMargin) flag = 1;
+        acc = d == __float_as_int(sz.y);
+      }
+      if (!acc) break;
+      ++a;
+    }
+    s_a = a;
+    s_flag = flag;
+    if (p.T > 0.f) {
+      const float4 sz = row_stats(p, b * p.n_q + a);
+      s_mz = sz.x;
+      s_isz = 1.f / sz.y;
+      if (a < p.k) {
+        const float4 sy = row_stats(p, p.rows_t + b * p.k + a);
+        s_my = sy.x;
+        s_isy = 1.f / sy.y;
+      }
+    }
+  }
+  __syncthreads();
+  const int a = s_a;
+
+  if (p.T == 0.f) {  // greedy: one CTA per sequence, no race
+    if (threadIdx.x == 0) {
+      const float4 sz = row_stats(p, b * p.n_q + a);
+      int flag = s_flag;
+      if ((sz.x - sz.z) / fmaxf(1.f, fabsf(sz.x)) < kMargin) flag = 1;
+      int32_t *o = p.out + (size_t)b * p.ld_o;
+      for (int j = 0; j < p.n_q; ++j)
+        o[j] = j < a ? p.drafts[(size_t)b * p.k + j] : (j == a ? __float_as_int(sz.y) : -1);
+      p.n_acc[b] = a;
+      if (p.margin) p.margin[b] = flag;
+    }
+    return;
+  }
+
+  // ---- exponential race over this CTA's chunk of the draw row
+  const bool resid = a < p.k;
+  const int rt = b * p.n_q + a;
+  const float *zr = p.z + (size_t)rt * p.ld_t;
+  const float *yr = resid ? p.y + ((size_t)b * p.k + a) * p.ld_d : nullptr;
+  const float mz = s_mz, isz = s_isz, my = resid ? s_my : 0.f, isy = resid ? s_isy : 0.f;
+  const int v0 = c * kChunk;
+  const int v1 = min(p.V, v0 + kChunk);
+  const int n4 = (v1 - v0) >> 2;
+  Cand cr{-INFINITY, -INFINITY, -1}, cp{-INFINITY, -INFINITY, -1};
+  for (int i = threadIdx.x; i < n4; i += kThreads) {
+    const int v = v0 + 4 * i;
+    const float4 z4 = __ldg(reinterpret_cast<const float4 *>(zr + v));
+    float4 y4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (resid) y4 = __ldg(reinterpret_cast<const float4 *>(yr + v));
+    float U[4];
+    token_uniform_pair(p.seed, p.step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1), U[0],
+                       U[1]);
+    token_uniform_pair(p.seed, p.step, (uint32_t)rt, (uint32_t)p.purpose,
+                       (uint32_t)(v >> 1) + 1u, U[2], U[3]);
+    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
+    const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float E = -log1pf(-U[e]);
+      const float lnE = logf(E);  // E == 0 gives -inf: that token wins if its weight > 0
+      const float zt = zz[e] / p.T;
+      const float gp = zt == -INFINITY ? -INFINITY : zt - lnE;
+      cand_push(cp, gp, v + e);
+      if (resid) {
+        const float pv = expf(zt - mz) * isz;
+        const float qv = expf(yy[e] / p.T - my) * isy;
+        const float w = pv - qv;
+        cand_push(cr, w > 0.f ? logf(w) - lnE : -INFINITY, v + e);
+      }
+    }
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    const Cand o1 = cand_shfl(cp, off), o2 = cand_shfl(cr, off);
+    cp = (lane & off) ? cand_merge(o1, cp) : cand_merge(cp, o1);
+    cr = (lane & off) ? cand_merge(o2, cr) : cand_merge(cr, o2);
+  }
+  if (lane == 0) {
+    red[0][warp] = make_float4(cp.g1, __int_as_float(cp.v1), cp.g2, 0.f);
+    red[1][warp] = make_float4(cr.g1, __int_as_float(cr.v1), cr.g2, 0.f);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Cand tp{red[0][0].x, red[0][0].z, __float_as_int(red[0][0].y)};
+    Cand tr{red[1][0].x, red[1][0].z, __float_as_int(red[1][0].y)};
+    for (int w = 1; w < kThreads / 32; ++w) {
+      tp = cand_merge(tp, Cand{red[0][w].x, red[0][w].z, __float_as_int(red[0][w].y)});
+      tr = cand_merge(tr, Cand{red[1][w].x, red[1][w].z, __float_as_int(red[1][w].y)});
+    }
+    float4 *slot = p.cand + ((size_t)b * p.nchunks + c) * 2;
+    slot[0] = make_float4(tp.g1, __int_as_float(tp.v1), tp.g2, 0.f);
+    slot[1] = make_float4(tr.g1, __int_as_float(tr.v1), tr.g2, 0.f);
+    __threadfence();
+    const unsigned int ticket = atomicAdd(&p.counters[b], 1u);
+    s_last = ticket == (unsigned int)(p.nchunks - 1);
+  }
+  __syncthreads();
+  if (!s_last || threadIdx.x != 0) return;
+  __threadfence();
+  // ---- last CTA of the sequence: merge chunk winners in chunk (token) order
+  const volatile float4 *cv = reinterpret_cast<const volatile float4 *>(p.cand) +
+                              (size_t)b * p.nchunks * 2;
+  Cand tp{-INFINITY, -INFINITY, -1}, tr{-INFINITY, -INFINITY, -1};
+  for (int cc = 0; cc < p.nchunks; ++cc) {
+    const float4 a0 = make_float4(cv[2 * cc].x, cv[2 * cc].y, cv[2 * cc].z, 0.f);
+    const float4 a1 = make_float4(cv[2 * cc + 1].x, cv[2 * cc + 1].y, cv[2 * cc + 1].z, 0.f);
+    tp = cand_merge(tp, Cand{a0.x, a0.z, __float_as_int(a0.y)});
+    tr = cand_merge(tr, Cand{a1.x, a1.z, __float_as_int(a1.y)});
+  }
+  const Cand &w = (resid && tr.v1 >= 0 && tr.g1 > -INFINITY) ? tr : tp;
+  int flag = s_flag;
+  if (w.g1 - w.g2 < kMargin) flag = 1;
+  int32_t *o = p.out + (size_t)b * p.ld_o;
+  for (int j = 0; j < p.n_q; ++j)
+    o[j] = j < a ? p.drafts[(size_t)b * p.k + j] : (j == a ? w.v1 : -1);
+  p.n_acc[b] = a;
+  if (p.margin) p.margin[b] = flag;
+  p.counters[b] = 0u;
+}
+
+static sd_status validate(const sd_accept_desc *d) {
+  if (!d) return SD_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->k < 0 || d->k > 15 || d->vocab < 1) return SD_ERR_INVALID_ARG;
+  if (!(d->temperature >= 0.f) || d->temperature > 1e30f) return SD_ERR_INVALID_ARG;
+  if (d->purpose < 1) return SD_ERR_INVALID_ARG;
+  const int ldt = d->ld_target ? d->ld_target : d->vocab;
+  const int ldd = d->ld_draft ? d->ld_draft : d->vocab;
+  const int ldo = d->ld_out ? d->ld_out : d->k + 1;
+  if (ldt < d->vocab || ldd < d->vocab || ldo < d->k + 1) return SD_ERR_INVALID_ARG;
+  if (d->vocab % 4 || ldt % 4 || ldd % 4) return SD_ERR_UNSUPPORTED;
+  return SD_OK;
+}
+
+static int nchunks_of(int V) { return (V + kChunk - 1) / kChunk; }
+
+static size_t ws_size(const sd_accept_desc *d) {
+  if (validate(d) != SD_OK) return 0;
+  const size_t nc = nchunks_of(d->vocab);
+  const size_t rows = (size_t)d->batch * (d->k + 1) + (size_t)d->batch * d->k;
+  return round_up(rows * nc * 16, 256) + round_up((size_t)d->batch * nc * 32, 256) +
+         round_up((size_t)d->batch * 4, 256);
+}
+
+}  // namespace acc
+}  // namespace sdv
+
+extern "C" {
+
+size_t sd_accept_workspace_size(const sd_accept_desc *desc) { return sdv::acc::ws_size(desc); }
+
+sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
+                    const float *draft_logits, const int32_t *draft_tokens,
+                    int32_t *n_accepted, int32_t *out_tokens, int32_t *margin_flags,
+                    void *ws, size_t ws_bytes, sd_stream stream) {
+  using namespace sdv;
+  using namespace sdv::acc;
+  sd_status s = validate(desc);
+  if (s != SD_OK) return s;
+  const bool sampling = desc->temperature > 0.f;
+  if (!target_logits || !n_accepted || !out_tokens) return SD_ERR_INVALID_ARG;
+  if (desc->k > 0 && !draft_tokens) return SD_ERR_INVALID_ARG;
+  if (sampling && desc->k > 0 && !draft_logits) return SD_ERR_INVALID_ARG;
+  if (!aligned16(target_logits) || (sampling && desc->k > 0 && !aligned16(draft_logits)))
+    return SD_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < ws_size(desc)) return SD_ERR_WORKSPACE;
+  Params p{};
+  p.B = desc->batch;
+  p.k = desc->k;
+  p.V = desc->vocab;
+  p.n_q = desc->k + 1;
+  p.ld_t = desc->ld_target ? desc->ld_target : desc->vocab;
+  p.ld_d = desc->ld_draft ? desc->ld_draft : desc->vocab;
+  p.ld_o = desc->ld_out ? desc->ld_out : desc->k + 1;
+  p.purpose = desc->purpose;
+  p.nchunks = nchunks_of(desc->vocab);
+  p.rows_t = p.B * p.n_q;
+  p.rows_total = p.rows_t + (sampling ? p.B * p.k : 0);
+  p.T = desc->temperature;
+  p.seed = desc->seed;
+  p.step = (uint32_t)desc->step;
+  p.z = target_logits;
+  p.y = draft_logits;
+  p.drafts = draft_tokens;
+  p.n_acc = n_accepted;
+  p.out = out_tokens;
+  p.margin = margin_flags;
+  const size_t rows = (size_t)p.B * (p.k + 1) + (size_t)p.B * p.k;
+  uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+  p.stats = reinterpret_cast<float4 *>(w8);
+  w8 += round_up(rows * p.nchunks * 16, 256);
+  p.cand = reinterpret_cast<float4 *>(w8);
+  w8 += round_up((size_t)p.B * p.nchunks * 32, 256);
+  p.counters = reinterpret_cast<unsigned int *>(w8);
+  p.status = device_status_word();
+  cudaStream_t st = (cudaStream_t)stream;
+  accept_stats_kernel<<<dim3(p.rows_total, p.nchunks), kThreads, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+  accept_draw_kernel<<<dim3(p.B, sampling ? p.nchunks : 1), kThreads, 0, st>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,848 @@
+// Verify attention and drafter cross-attention over a paged KV cache (sm_100a).
+//
+// What is computed: "Gemma 4 MTP: drafter drafts, target verifies", section "drafter internal
+// architecture" (k+1 positions verified in one pass; each drafter layer attends directly into
+// the target's KV cache).  Query j of sequence b sits at t = L_b + j (verify) or q_pos[b]
+// (drafter) and attends to keys p in [lo, hi]: lo = max(0, t - window + 1) on a sliding layer,
+// 0 on a global one; hi = t (verify) or min(t, L_b - 1) (drafter).  Query head h reads kv head
+// h / G.
+//
+// bf16 design (decode attention is bandwidth-bound: GeekNews summary of the Google blog,
+// section "why speculative decoding"):
+//  * Persistent CTAs split the flattened list of (sequence, kv head, 16-key tile) work evenly
+//    (stream-K): every CTA streams the same number of KV bytes however ragged the contexts.
+//  * A producer warp moves each 16-key K and V tile of one kv head (contiguous in the
+//    [num_blocks, h_kv, block_size, D] layout) into shared memory once, by TMA
+//    (cp.async.bulk.tensor, 128-byte swizzle, no multicast), through an mbarrier ring.
+//  * The tile is reused by every query row of the item: the G query heads of the kv head times
+//    the n_q verify positions (M = G * n_q rows, padded to 16-row MMA tiles).
+//  * Compute warps own (16-row tile, D slice of 128 columns).  Q K^T partials over the slices
+//    are summed through shared memory (fixed order, so every warp of a row tile gets the same
+//    scores); the online softmax and P V run in registers on bf16 mma.sync tensor cores with
+//    float32 accumulation.
+//  * Items split across CTAs leave (m, l, o) partials in the workspace; a combine kernel merges
+//    them in CTA order (deterministic).  Items one CTA finishes are written directly.
+//
+// float32 path: one warp per query row, plain FMA (the tiny float32 configuration).
+#include <cfloat>
+
+#include "common.cuh"
+#include "host.cuh"
+
+namespace sdv {
+namespace attn {
+
+constexpr int kTile = 16;
+
+struct Params {
+  int B, n_q, Hq, Hkv, G, D, bs, mbps, num_blocks, window, M, Mpad;
+  int is_draft;
+  float scale_log2;  // scale * log2(e)
+  float scale;
+  const void *q;
+  const int32_t *table;
+  const int32_t *ctx_len;
+  const int32_t *q_pos;
+  void *out;
+  float *ws_o;   // [slots][Mpad][D]
+  float *ws_ml;  // [slots][Mpad][2]
+  int P;         // CTAs of the persistent grid
+  int *status;
+};
+
+// Keys an item (sequence b, any kv head) reads: tiles [tf, tf + n) of 16 positions, with
+// lo_min / hi_max the union of the rows' key ranges.
+struct SeqRange {
+  int L, tf, n, lo_min, hi_max;
+};
+
+__device__ __forceinline__ SeqRange seq_range(const Params &p, int b, bool report) {
+  SeqRange r;
+  r.L = p.ctx_len[b];
+  r.tf = 0;
+  r.n = 0;
+  r.lo_min = 0;
+  r.hi_max = -1;
+  int lo, hi;
+  if (!p.is_draft) {
+    if (r.L < 0) {
+      if (report) record_status(p.status, SD_ERR_DEVICE);
+      return r;
+    }
+    hi = r.L + p.n_q - 1;
+    lo = p.window > 0 ? max(0, r.L - p.window + 1) : 0;
+  } else {
+    const int qp = p.q_pos[b];
+    if (r.L < 0 || qp < 0) {
+      if (report) record_status(p.status, SD_ERR_DEVICE);
+      return r;
+    }
+    hi = min(qp, r.L - 1);
+    lo = p.window > 0 ? max(0, qp - p.window + 1) : 0;
+  }
+  if (hi < lo) return r;
+  if (hi >= p.mbps * p.bs) {  // positions beyond the block table
+    if (report) record_status(p.status, SD_ERR_DEVICE);
+    return r;
+  }
+  r.tf = lo / kTile;
+  r.n = hi / kTile - r.tf + 1;
+  r.lo_min = lo;
+  r.hi_max = hi;
+  return r;
+}
+
+// Key range of query row `row` (row = j * G + hh) of sequence b.
+__device__ __forceinline__ void row_range(const Params &p, const SeqRange &s, int b, int row,
+                                          int &lo, int &hi) {
+  if (row >= p.M || s.n == 0) {
+    lo = 1;
+    hi = 0;
+    return;
+  }
+  if (!p.is_draft) {
+    const int t = s.L + row / p.G;
+    hi = t;
+    lo = p.window > 0 ? max(0, t - p.window + 1) : 0;
+  } else {
+    const int t = p.q_pos[b];
+    hi = min(t, s.L - 1);
+    lo = p.window > 0 ? max(0, t - p.window + 1) : 0;
+  }
+}
+
+__device__ __forceinline__ long long total_tiles(const Params &p) {
+  long long T = 0;
+  for (int b = 0; b < p.B; ++b) T += (long long)p.Hkv * seq_range(p, b, false).n;
+  return T;
+}
+
+// Cursor over the flattened (b, g, tile) list of one CTA.
+struct Cursor {
+  int b, g, tau;         // current item and tile index inside it
+  SeqRange s;            // range of sequence b
+  long long left;        // tiles still to process by this CTA
+  long long item_first;  // flattened index of tile 0 of the current item
+};
+
+__device__ __forceinline__ void cursor_begin(const Params &p, long long start, long long count,
+                                             Cursor &c) {
+  c.left = count;
+  long long pre = 0;
+  c.b = 0;
+  c.g = 0;
+  c.tau = 0;
+  c.s = seq_range(p, 0, false);
+  if (count <= 0) return;
+  for (int b = 0; b < p.B; ++b) {
+    SeqRange s = seq_range(p, b, false);
+    const long long len = (long long)p.Hkv * s.n;
+    if (start < pre + len) {
+      c.b = b;
+      c.s = s;
+      const long long off = start - pre;
+      c.g = (int)(off / s.n);
+      c.tau = (int)(off % s.n);
+      c.item_first = pre + (long long)c.g * s.n;
+      return;
+    }
+    pre += len;
+  }
+  c.left = 0;
+}
+
+// Advances to the next item after the current one finished (tau == n).
+__device__ __forceinline__ void cursor_next_item(const Params &p, Cursor &c) {
+  c.item_first += c.s.n;
+  c.tau = 0;
+  if (++c.g < p.Hkv) return;
+  c.g = 0;
+  for (int b = c.b + 1; b < p.B; ++b) {
+    SeqRange s = seq_range(p, b, false);
+    if (s.n > 0) {
+      c.b = b;
+      c.s = s;
+      return;
+    }
+  }
+  c.left = 0;
+}
+
+// Byte offset of element (row, col) inside a [16 rows x D] bf16 tile stored as D/64 chunks of
+// [16 rows x 128 B] with the 128-byte swizzle (16-byte unit u of row r stored at u ^ (r & 7)).
+__device__ __forceinline__ uint32_t swz(int row, int col) {
+  const int chunk = col >> 6;
+  const int unit = (col >> 3) & 7;
+  return (uint32_t)(chunk * (kTile * 128) + row * 128 + ((unit ^ (row & 7)) << 4) +
+                    ((col & 7) << 1));
+}
+
+template <int D, int MT, int STAGES>
+struct Cfg {
+  static constexpr int DS = D >= 128 ? 128 : 64;
+  static constexpr int NDG = D / DS;
+  static constexpr int NCW = MT * NDG;
+  static constexpr int THREADS = 32 * (NCW + 1);
+  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + RED_FLOATS * 4 +
+                                 16 * STAGES + 16 + 4 * (1 + STAGES) + 64;
+};
+
+template <int D, int MT, int STAGES>
+__global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap, const Params p) {
+  using C = Cfg<D, MT, STAGES>;
+  constexpr int DS = C::DS, NDG = C::NDG, NCW = C::NCW;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *stages = smem;
+  float *red = reinterpret_cast<float *>(smem + (size_t)STAGES * C::STAGE_BYTES);
+  uint64_t *full = reinterpret_cast<uint64_t *>(red + C::RED_FLOATS);
+  uint64_t *empty = full + STAGES;
+  uint64_t *red_bar = empty + STAGES;  // [2]: partial scores of a tile are in red[buf]
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(red_bar + 2);
+  volatile int *bad = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW * 32);
+      bad[s] = 0;
+    }
+    mbar_init(&red_bar[0], NCW * 32);
+    mbar_init(&red_bar[1], NCW * 32);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const long long T = total_tiles(p);
+  const long long start = T * blockIdx.x / p.P;
+  const long long end = T * (blockIdx.x + 1) / p.P;
+
+  if (warp == NCW) {
+    // ------------------------------------------------------------------- producer warp
+    if (lane != 0) return;
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+    Cursor c;
+    cursor_begin(p, start, end - start, c);
+    uint32_t it = 0;
+    while (c.left > 0) {
+      const int stage = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) {
+        record_status(p.status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      const int p0 = (c.s.tf + c.tau) * kTile;
+      const int bidx = p0 / p.bs;
+      int blk = -1;
+      if (bidx < p.mbps) blk = p.table[(size_t)c.b * p.mbps + bidx];
+      if (blk < 0 || blk >= p.num_blocks) {
+        record_status(p.status, SD_ERR_DEVICE);
+        bad[stage] = 1;
+        mbar_arrive(&full[stage]);
+      } else {
+        bad[stage] = 0;
+        const int row = (blk * p.Hkv + c.g) * p.bs + (p0 % p.bs);
+        uint8_t *kd = stages + (size_t)stage * C::STAGE_BYTES;
+        uint8_t *vd = kd + C::TILE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+#pragma unroll
+        for (int ch = 0; ch < D / 64; ++ch) {
+          tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
+          tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+        }
+      }
+      ++it;
+      --c.left;
+      if (++c.tau == c.s.n && c.left > 0) cursor_next_item(p, c);
+    }
+    if (*abort_flag) {
+      // wait (bounded) for the copies this CTA issued before leaving
+      for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+        mbar_wait_timed(&full[j % STAGES], (j / STAGES) & 1);
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------------- compute warps
+  const int mg = warp / NDG, dg = warp % NDG;
+  const int r0 = mg * 16 + (lane >> 2);  // rows r0 and r0 + 8 of the item
+  const int kq = 2 * (lane & 3);         // column pair inside an 8-wide n tile
+  const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(p.q);
+
+  Cursor c;
+  cursor_begin(p, start, end - start, c);
+  uint32_t it = 0;
+  int buf = 0;
+  bool ok = true;
+  while (c.left > 0 && ok) {
+    // ---- segment setup: item (c.b, c.g), tiles [c.tau, seg_end)
+    const int b = c.b, g = c.g;
+    const int t_begin = c.tau;
+    const long long rest = (long long)(c.s.n - c.tau);
+    const int seg_n = (int)(c.left < rest ? c.left : rest);
+    const bool whole = (t_begin == 0 && seg_n == c.s.n);
+    const SeqRange s = c.s;
+
+    uint32_t qa[DS / 16][4];
+#pragma unroll
+    for (int ks = 0; ks < DS / 16; ++ks) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = r0 + ((e & 1) ? 8 : 0);
+        const int col = dg * DS + ks * 16 + kq + ((e & 2) ? 8 : 0);
+        uint32_t v = 0;
+        if (row < p.M) {
+          const int j = row / p.G, hh = row % p.G;
+          const size_t off = (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D + col;
+          v = *reinterpret_cast<const uint32_t *>(qg + off);
+        }
+        qa[ks][e] = v;
+      }
+    }
+    int lo0, hi0, lo1, hi1;
+    row_range(p, s, b, r0, lo0, hi0);
+    row_range(p, s, b, r0 + 8, lo1, hi1);
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float o[DS / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < DS / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+
+    for (int t = 0; t < seg_n; ++t) {
+      const int stage = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      if (!mbar_wait(&full[stage], ph, abort_flag)) {
+        record_status(p.status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+        ok = false;
+        break;
+      }
+      const int is_bad = bad[stage];
+      const uint32_t kbase = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
+      const uint32_t vbase = kbase + C::TILE_BYTES;
+      const int p0 = (s.tf + t_begin + t) * kTile;
+
+      // ---- partial S = Q K^T over this warp's D slice
+      float sp[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sp[nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < DS / 16; ++ks) {
+        const int d0 = dg * DS + ks * 16;
+        uint32_t kb[4];
+        const int key = ((lane >> 4) << 3) + (lane & 7);
+        const int col = d0 + ((lane >> 3) & 1) * 8;
+        ldsm_x4(kb, kbase + swz(key, col));
+        mma_bf16_16816(sp[0], qa[ks], kb[0], kb[1]);
+        mma_bf16_16816(sp[1], qa[ks], kb[2], kb[3]);
+      }
+      float *myred = red + ((size_t)(buf * NCW + warp) * 32 + lane) * 8;
+      reinterpret_cast<float4 *>(myred)[0] = make_float4(sp[0][0], sp[0][1], sp[0][2], sp[0][3]);
+      reinterpret_cast<float4 *>(myred)[1] = make_float4(sp[1][0], sp[1][1], sp[1][2], sp[1][3]);
+      mbar_arrive(&red_bar[buf]);
+      if (!mbar_wait(&red_bar[buf], (it >> 1) & 1, abort_flag)) {
+        record_status(p.status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+        ok = false;
+        break;
+      }
+      float sc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+#pragma unroll
+      for (int dd = 0; dd < NDG; ++dd) {
+        const float *src = red + ((size_t)(buf * NCW + mg * NDG + dd) * 32 + lane) * 8;
+        const float4 a = reinterpret_cast<const float4 *>(src)[0];
+        const float4 bq = reinterpret_cast<const float4 *>(src)[1];
+        sc[0][0] += a.x;
+        sc[0][1] += a.y;
+        sc[0][2] += a.z;
+        sc[0][3] += a.w;
+        sc[1][0] += bq.x;
+        sc[1][1] += bq.y;
+        sc[1][2] += bq.z;
+        sc[1][3] += bq.w;
+      }
+      buf ^= 1;
+
+      // ---- mask, online softmax (base-2 exponent with the scale folded in)
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pos = p0 + nt * 8 + kq + (e & 1);
+          const int lo = (e & 2) ? lo1 : lo0, hi = (e & 2) ? hi1 : hi0;
+          const bool valid = !is_bad && pos >= lo && pos <= hi;
+          const float x = valid ? sc[nt][e] * p.scale_log2 : -INFINITY;
+          sc[nt][e] = x;
+          mx[e >> 1] = fmaxf(mx[e >> 1], x);
+        }
+      float alpha[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+        const float m_new = fmaxf(m_run[h], mx[h]);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha[h] = exp2f(m_run[h] - m_use);
+        m_run[h] = m_new;
+        l_run[h] *= alpha[h];
+        mx[h] = m_use;
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+          sc[nt][e] = pv;
+          l_run[e >> 1] += pv;
+        }
+#pragma unroll
+      for (int nt = 0; nt < DS / 8; ++nt) {
+        o[nt][0] *= alpha[0];
+        o[nt][1] *= alpha[0];
+        o[nt][2] *= alpha[1];
+        o[nt][3] *= alpha[1];
+      }
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
+      pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
+      pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
+      pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+
+      // ---- V rows no query of the item may read can hold anything (rolled-back or never
+      // written slots, NaN included); zero this warp's slice of them so 0 * V stays 0.
+      {
+        int zlo = max(0, min(kTile, s.lo_min - p0));
+        int zhi = max(0, min(kTile, s.hi_max - p0 + 1));
+        if (is_bad) {
+          zlo = kTile;
+          zhi = kTile;
+        }
+        if (zlo > 0 || zhi < kTile) {
+          uint8_t *vt = stages + (size_t)stage * C::STAGE_BYTES + C::TILE_BYTES;
+          // rows [0, zlo) and [zhi, 16); slice columns [dg*DS, dg*DS+DS) = DS/64 chunks
+          for (int u = lane; u < kTile * (DS / 64) * 8; u += 32) {
+            const int row = u / ((DS / 64) * 8);
+            const int rem = u % ((DS / 64) * 8);
+            const int chunk = dg * (DS / 64) + rem / 8;
+            const int unit = rem % 8;
+            if (row < zlo || row >= zhi)
+              *reinterpret_cast<uint4 *>(vt + chunk * (kTile * 128) + row * 128 + unit * 16) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();  // before the stage is handed back to TMA
+          __syncwarp();
+        }
+      }
+
+      // ---- O += P V over this warp's D slice
+#pragma unroll
+      for (int np = 0; np < DS / 16; ++np) {
+        const int d0 = dg * DS + np * 16;
+        uint32_t vb[4];
+        const int key = ((lane >> 3) & 1) * 8 + (lane & 7);
+        const int col = d0 + (lane >> 4) * 8;
+        ldsm_x4_trans(vb, vbase + swz(key, col));
+        mma_bf16_16816(o[2 * np], pa, vb[0], vb[1]);
+        mma_bf16_16816(o[2 * np + 1], pa, vb[2], vb[3]);
+      }
+      mbar_arrive(&empty[stage]);
+      ++it;
+    }
+    if (!ok) break;
+
+    // ---- segment end: final rows or a partial for the combine kernel
+    float l_tot[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float l = l_run[h];
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      l_tot[h] = l;
+    }
+    if (whole) {
+      __nv_bfloat16 *outg = reinterpret_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = r0 + 8 * h;
+        if (row >= p.M) continue;
+        const int j = row / p.G, hh = row % p.G;
+        const float inv = l_tot[h] > 0.f ? 1.f / l_tot[h] : 0.f;
+        __nv_bfloat16 *dst =
+            outg + (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D + dg * DS + kq;
+#pragma unroll
+        for (int nt = 0; nt < DS / 8; ++nt)
+          *reinterpret_cast<uint32_t *>(dst + nt * 8) =
+              pack_bf16x2(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
+      }
+    } else {
+      const size_t slot = (size_t)b * p.Hkv + g + blockIdx.x;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = r0 + 8 * h;
+        if (row >= p.M) continue;
+        float *dst = p.ws_o + (slot * p.Mpad + row) * D + dg * DS + kq;
+#pragma unroll
+        for (int nt = 0; nt < DS / 8; ++nt)
+          *reinterpret_cast<float2 *>(dst + nt * 8) = make_float2(o[nt][2 * h], o[nt][2 * h + 1]);
+        if (dg == 0 && (lane & 3) == 0) {
+          p.ws_ml[(slot * p.Mpad + row) * 2 + 0] = m_run[h];
+          p.ws_ml[(slot * p.Mpad + row) * 2 + 1] = l_tot[h];
+        }
+      }
+    }
+    c.tau += seg_n;
+    c.left -= seg_n;
+    if (c.left > 0) cursor_next_item(p, c);
+  }
+}
+
+// Merges the partials of items that several CTAs shared, in CTA order; writes zero rows for
+// drafter items with an empty key range.
+template <typename T>
+__global__ void attn_combine_kernel(const Params p) {
+  const int item = blockIdx.x;
+  const int b = item / p.Hkv, g = item % p.Hkv;
+  long long pre = 0, T_all = 0;
+  SeqRange sb;
+  for (int bb = 0; bb < p.B; ++bb) {
+    SeqRange s = seq_range(p, bb, threadIdx.x == 0 && bb == b && item % p.Hkv == 0);
+    if (bb == b) sb = s;
+    if (bb < b) pre += (long long)p.Hkv * s.n;
+    T_all += (long long)p.Hkv * s.n;
+  }
+  T *outg = reinterpret_cast<T *>(p.out);
+  if (sb.n == 0) {
+    for (int idx = threadIdx.x; idx < p.M * p.D; idx += blockDim.x) {
+      const int row = idx / p.D, d = idx % p.D;
+      const int j = row / p.G, hh = row % p.G;
+      outg[(((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * p.D + d] = T(0.f);
+    }
+    return;
+  }
+  const long long F = pre + (long long)g * sb.n;
+  const long long Fl = F + sb.n - 1;
+  const int c_first = (int)(((F + 1) * p.P - 1) / T_all);
+  const int c_last = (int)(((Fl + 1) * p.P - 1) / T_all);
+  if (c_first == c_last) return;  // written directly by its only CTA
+  const size_t slot0 = (size_t)b * p.Hkv + g;
+  for (int idx = threadIdx.x; idx < p.M * p.D; idx += blockDim.x) {
+    const int row = idx / p.D, d = idx % p.D;
+    float mmax = -INFINITY;
+    for (int c = c_first; c <= c_last; ++c)
+      mmax = fmaxf(mmax, p.ws_ml[((slot0 + c) * p.Mpad + row) * 2]);
+    float num = 0.f, den = 0.f;
+    if (mmax != -INFINITY) {
+      for (int c = c_first; c <= c_last; ++c) {
+        const size_t sl = (slot0 + c) * p.Mpad + row;
+        const float w = exp2f(p.ws_ml[sl * 2] - mmax);
+        num += w * p.ws_o[sl * p.D + d];
+        den += w * p.ws_ml[sl * 2 + 1];
+      }
+    }
+    const int j = row / p.G, hh = row % p.G;
+    outg[(((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * p.D + d] =
+        T(den > 0.f ? num / den : 0.f);
+  }
+}
+
+// Writes the n_q new K/V rows of every sequence into the cache (verify only).
+template <typename T>
+__global__ void append_kv_kernel(const Params p, const T *k_new, const T *v_new, T *k_cache,
+                                 T *v_cache) {
+  const int b = blockIdx.x / p.n_q, j = blockIdx.x % p.n_q;
+  const int L = p.ctx_len[b];
+  if (L < 0) return;  // reported by the attention kernel
+  const int pos = L + j;
+  const int bidx = pos / p.bs;
+  if (bidx >= p.mbps) {
+    if (threadIdx.x == 0) record_status(p.status, SD_ERR_DEVICE);
+    return;
+  }
+  const int blk = p.table[(size_t)b * p.mbps + bidx];
+  if (blk < 0 || blk >= p.num_blocks) {
+    if (threadIdx.x == 0) record_status(p.status, SD_ERR_DEVICE);
+    return;
+  }
+  const int n = p.Hkv * p.D;
+  for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
+    const int g = idx / p.D, d = idx % p.D;
+    const size_t src = (((size_t)b * p.n_q + j) * p.Hkv + g) * p.D + d;
+    const size_t dst = (((size_t)blk * p.Hkv + g) * p.bs + pos % p.bs) * p.D + d;
+    k_cache[dst] = k_new[src];
+    v_cache[dst] = v_new[src];
+  }
+}
+
+// float32 path: one warp per (sequence, query position, head).
+__global__ void attn_f32_kernel(const Params p, const float *k_cache, const float *v_cache) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int total = p.B * p.n_q * p.Hq;
+  if (wid >= total) return;
+  const int h = wid % p.Hq;
+  const int j = (wid / p.Hq) % p.n_q;
+  const int b = wid / (p.Hq * p.n_q);
+  const int g = h / p.G;
+  const SeqRange s = seq_range(p, b, lane == 0);
+  int lo, hi;
+  row_range(p, s, b, j * p.G + (h % p.G), lo, hi);
+  constexpr int MAXE = 16;  // D <= 512
+  const int per = p.D / 32;
+  const float *qv = reinterpret_cast<const float *>(p.q) + (((size_t)b * p.n_q + j) * p.Hq + h) * p.D;
+  float qr[MAXE], acc[MAXE];
+  for (int e = 0; e < MAXE; ++e) {
+    qr[e] = e < per ? qv[lane + 32 * e] : 0.f;
+    acc[e] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int pos = lo; pos <= hi; ++pos) {
+    const int blk = p.table[(size_t)b * p.mbps + pos / p.bs];
+    if (blk < 0 || blk >= p.num_blocks) {
+      if (lane == 0) record_status(p.status, SD_ERR_DEVICE);
+      continue;
+    }
+    const size_t row = (((size_t)blk * p.Hkv + g) * p.bs + pos % p.bs) * p.D;
+    float dot = 0.f;
+    for (int e = 0; e < per; ++e) dot = fmaf(qr[e], k_cache[row + lane + 32 * e], dot);
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    const float x = dot * p.scale;
+    const float m_new = fmaxf(m, x);
+    const float alpha = expf(m - m_new);
+    const float w = expf(x - m_new);
+    l = l * alpha + w;
+    for (int e = 0; e < per; ++e) acc[e] = acc[e] * alpha + w * v_cache[row + lane + 32 * e];
+    m = m_new;
+  }
+  float *ov = reinterpret_cast<float *>(p.out) + (((size_t)b * p.n_q + j) * p.Hq + h) * p.D;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  for (int e = 0; e < per; ++e) ov[lane + 32 * e] = acc[e] * inv;
+}
+
+// ------------------------------------------------------------------------------- host side
+
+template <int D, int MT, int STAGES>
+struct Launcher {
+  using C = Cfg<D, MT, STAGES>;
+  static int ctas_per_sm() {
+    static int dev_cache[64];
+    static int occ_cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && dev_cache[dev] == dev + 1) return occ_cache[dev];
+    cudaFuncSetAttribute(attn_bf16_kernel<D, MT, STAGES>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_bf16_kernel<D, MT, STAGES>,
+                                                      C::THREADS, C::SMEM) != cudaSuccess)
+      occ = 0;
+    if (dev < 64) {
+      occ_cache[dev] = occ;
+      dev_cache[dev] = dev + 1;
+    }
+    return occ;
+  }
+  static sd_status launch(const CUtensorMap &km, const CUtensorMap &vm, const Params &p,
+                          cudaStream_t st) {
+    attn_bf16_kernel<D, MT, STAGES><<<p.P, C::THREADS, C::SMEM, st>>>(km, vm, p);
+    return cuda_status(cudaGetLastError());
+  }
+};
+
+template <int D, int MT>
+struct Pick;
+#define SDV_STAGES(D) ((D) == 512 ? 3 : (D) == 256 ? 4 : (D) == 128 ? 6 : 8)
+
+// Persistent CTAs for a (head_dim, row tiles) pair on the current device.
+static int persistent_ctas(int D, int MT) {
+  int occ = 0;
+#define SDV_CASE(DD, MM)                                      \
+  if (D == DD && MT == MM) occ = Launcher<DD, MM, SDV_STAGES(DD)>::ctas_per_sm();
+  SDV_CASE(64, 1) SDV_CASE(64, 2) SDV_CASE(64, 3) SDV_CASE(64, 4)
+  SDV_CASE(128, 1) SDV_CASE(128, 2) SDV_CASE(128, 3) SDV_CASE(128, 4)
+  SDV_CASE(256, 1) SDV_CASE(256, 2) SDV_CASE(256, 3) SDV_CASE(256, 4)
+  SDV_CASE(512, 1) SDV_CASE(512, 2) SDV_CASE(512, 3) SDV_CASE(512, 4)
+#undef SDV_CASE
+  const int sms = sm_count();
+  if (occ <= 0 || sms <= 0) return 0;
+  return occ * sms;
+}
+
+static sd_status launch_bf16(int D, int MT, const CUtensorMap &km, const CUtensorMap &vm,
+                             const Params &p, cudaStream_t st) {
+#define SDV_CASE(DD, MM) \
+  if (D == DD && MT == MM) return Launcher<DD, MM, SDV_STAGES(DD)>::launch(km, vm, p, st);
+  SDV_CASE(64, 1) SDV_CASE(64, 2) SDV_CASE(64, 3) SDV_CASE(64, 4)
+  SDV_CASE(128, 1) SDV_CASE(128, 2) SDV_CASE(128, 3) SDV_CASE(128, 4)
+  SDV_CASE(256, 1) SDV_CASE(256, 2) SDV_CASE(256, 3) SDV_CASE(256, 4)
+  SDV_CASE(512, 1) SDV_CASE(512, 2) SDV_CASE(512, 3) SDV_CASE(512, 4)
+#undef SDV_CASE
+  return SD_ERR_UNSUPPORTED;
+}
+
+static sd_status validate(const sd_attn_desc *d, bool draft) {
+  if (!d) return SD_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_q < 1 || d->h_q < 1 || d->h_kv < 1 || d->h_q % d->h_kv)
+    return SD_ERR_INVALID_ARG;
+  if (draft && d->n_q != 1) return SD_ERR_INVALID_ARG;
+  if (d->block_size < 1 || d->max_blocks_per_seq < 1 || d->num_blocks < 1)
+    return SD_ERR_INVALID_ARG;
+  if (!(d->scale > 0.f) || d->scale != d->scale) return SD_ERR_INVALID_ARG;
+  if ((long long)d->num_blocks * d->h_kv * d->block_size >= (1ll << 31))
+    return SD_ERR_UNSUPPORTED;
+  const int G = d->h_q / d->h_kv;
+  if ((long long)G * d->n_q > 64) return SD_ERR_UNSUPPORTED;
+  if (d->dtype == SD_BF16) {
+    if (!(d->head_dim == 64 || d->head_dim == 128 || d->head_dim == 256 || d->head_dim == 512))
+      return SD_ERR_UNSUPPORTED;
+    if (d->block_size % 16) return SD_ERR_UNSUPPORTED;
+  } else if (d->dtype == SD_F32) {
+    if (d->head_dim < 32 || d->head_dim > 512 || d->head_dim % 32) return SD_ERR_UNSUPPORTED;
+  } else {
+    return SD_ERR_INVALID_ARG;
+  }
+  return SD_OK;
+}
+
+static int grid_ctas(const sd_attn_desc *d) {
+  if (d->dtype != SD_BF16) return 0;
+  const int G = d->h_q / d->h_kv;
+  const int MT = (G * d->n_q + 15) / 16;
+  return persistent_ctas(d->head_dim, MT);
+}
+
+static size_t ws_size(const sd_attn_desc *d) {
+  if (validate(d, false) != SD_OK && validate(d, true) != SD_OK) return 0;
+  if (d->dtype != SD_BF16) return 0;
+  const int G = d->h_q / d->h_kv;
+  const int Mpad = (G * d->n_q + 15) / 16 * 16;
+  const size_t slots = (size_t)d->batch * d->h_kv + (size_t)grid_ctas(d);
+  return round_up(slots * Mpad * d->head_dim * 4, 256) + round_up(slots * Mpad * 2 * 4, 256);
+}
+
+static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const void *k_new,
+                     const void *v_new, void *k_cache, void *v_cache, const int32_t *table,
+                     const int32_t *ctx_len, const int32_t *q_pos, void *out, void *ws,
+                     size_t ws_bytes, cudaStream_t st) {
+  sd_status s = validate(d, draft);
+  if (s != SD_OK) return s;
+  if (!q || !k_cache || !v_cache || !table || !ctx_len || !out) return SD_ERR_INVALID_ARG;
+  if (draft && !q_pos) return SD_ERR_INVALID_ARG;
+  if (!draft && (!k_new || !v_new)) return SD_ERR_INVALID_ARG;
+  Params p{};
+  p.B = d->batch;
+  p.n_q = d->n_q;
+  p.Hq = d->h_q;
+  p.Hkv = d->h_kv;
+  p.G = d->h_q / d->h_kv;
+  p.D = d->head_dim;
+  p.bs = d->block_size;
+  p.mbps = d->max_blocks_per_seq;
+  p.num_blocks = d->num_blocks;
+  p.window = d->window > 0 ? d->window : 0;
+  p.M = p.G * p.n_q;
+  p.Mpad = (p.M + 15) / 16 * 16;
+  p.is_draft = draft ? 1 : 0;
+  p.scale = d->scale;
+  p.scale_log2 = d->scale * 1.4426950408889634f;
+  p.q = q;
+  p.table = table;
+  p.ctx_len = ctx_len;
+  p.q_pos = q_pos;
+  p.out = out;
+  p.status = device_status_word();
+
+  if (d->dtype == SD_F32) {
+    if (!draft) {
+      append_kv_kernel<float><<<p.B * p.n_q, 256, 0, st>>>(
+          p, (const float *)k_new, (const float *)v_new, (float *)k_cache, (float *)v_cache);
+      if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+    }
+    const int warps = p.B * p.n_q * p.Hq;
+    attn_f32_kernel<<<(warps + 3) / 4, 128, 0, st>>>(p, (const float *)k_cache,
+                                                      (const float *)v_cache);
+    return cuda_status(cudaGetLastError());
+  }
+
+  // bf16
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (!draft && (!aligned16(k_new) || !aligned16(v_new))))
+    return SD_ERR_INVALID_ARG;
+  const int MT = p.Mpad / 16;
+  p.P = persistent_ctas(p.D, MT);
+  if (p.P <= 0) return SD_ERR_CUDA;
+  const size_t need = ws_size(d);
+  if (!ws || ws_bytes < need) return SD_ERR_WORKSPACE;
+  const size_t slots = (size_t)p.B * p.Hkv + p.P;
+  p.ws_o = reinterpret_cast<float *>(ws);
+  p.ws_ml = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ws) +
+                                      round_up(slots * p.Mpad * p.D * 4, 256));
+  CUtensorMap km, vm;
+  const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
+  if (!encode_tmap_2d_bf16(&km, k_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile) ||
+      !encode_tmap_2d_bf16(&vm, v_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile))
+    return SD_ERR_CUDA;
+  if (!draft) {
+    append_kv_kernel<__nv_bfloat16><<<p.B * p.n_q, 256, 0, st>>>(
+        p, (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new,
+        (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache);
+    if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+  }
+  s = launch_bf16(p.D, MT, km, vm, p, st);
+  if (s != SD_OK) return s;
+  attn_combine_kernel<__nv_bfloat16><<<p.B * p.Hkv, 256, 0, st>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace attn
+}  // namespace sdv
+
+extern "C" {
+
+size_t sd_verify_attn_workspace_size(const sd_attn_desc *desc) {
+  if (sdv::attn::validate(desc, false) != SD_OK) return 0;
+  return sdv::attn::ws_size(desc);
+}
+
+sd_status sd_verify_attn(const sd_attn_desc *desc, const void *q, const void *k_new,
+                         const void *v_new, void *k_cache, void *v_cache,
+                         const int32_t *block_table, const int32_t *ctx_len, void *out,
+                         void *ws, size_t ws_bytes, sd_stream stream) {
+  return sdv::attn::run(desc, false, q, k_new, v_new, k_cache, v_cache, block_table, ctx_len,
+                        nullptr, out, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+size_t sd_draft_xattn_workspace_size(const sd_attn_desc *desc) {
+  if (sdv::attn::validate(desc, true) != SD_OK) return 0;
+  return sdv::attn::ws_size(desc);
+}
+
+sd_status sd_draft_xattn(const sd_attn_desc *desc, const void *q, const void *k_cache,
+                         const void *v_cache, const int32_t *block_table,
+                         const int32_t *ctx_len, const int32_t *q_pos, void *out, void *ws,
+                         size_t ws_bytes, sd_stream stream) {
+  return sdv::attn::run(desc, true, q, nullptr, nullptr, const_cast<void *>(k_cache),
+                        const_cast<void *>(v_cache), block_table, ctx_len, q_pos, out, ws,
+                        ws_bytes, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,30 @@
+// Host-side helpers shared by the entry points (defined in abi.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sd_verify.h"
+
+namespace sdv {
+
+// Device address of the current device's status word (nullptr if it cannot be obtained).
+int *device_status_word();
+
+// Streaming multiprocessors of the current device (0 on failure).
+int sm_count();
+
+// 2D bf16 tensor map over a row-major matrix [outer, inner] with the given row stride in
+// bytes, box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
+bool encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+inline sd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_CUDA; }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace sdv

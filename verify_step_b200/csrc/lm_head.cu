@@ -1,0 +1,446 @@
+// LM head over the vocabulary, dense and clustered (sm_100a).
+//
+// Dense: logits[i, v] = h[i] . W[v] for a 262144-token vocabulary (Gemma 4 MTP serving guide,
+// section 1; GeekNews summary of the Google blog, section "MTP drafter internal optimisations":
+// the final logit projection is a major cost).  With m = B * (k+1) rows of h (24 at B = 8,
+// k = 2) the product is a weight stream: W is read once, 2.8 GB at d = 5376.
+//
+// bf16 design (tcgen05): swap A and B so the streamed operand is the MMA's M side.
+//   A = a 128-row vocab tile of W [128 x 64] per pipeline stage (K-major, 128-byte swizzle),
+//   B = h [N x 64] (N = m rounded up to the instruction's N, zero rows past m),
+//   D = logits^T tile [128 x N] float32 in tensor memory (two buffers, so the epilogue of
+//   one tile overlaps the MMAs of the next).
+//   Warp 0 issues TMA loads (cp.async.bulk.tensor, no multicast; W evict-first, h
+//   evict-last in L2), warp 1 allocates tensor memory and issues tcgen05.mma from one thread,
+//   warps 2-5 read the accumulator with tcgen05.ld (thread = vocab row) and store
+//   logits[i, v] coalesced along v.  Persistent: one CTA per SM walks vocab tiles.
+//
+// Clustered (drafter side; the pages give no algorithm, this is one flat level): centroid
+// scores with the same kernel, per-row top-c selection, -inf fill, exact logits of the kept
+// clusters' tokens gathered from cluster-major weights.
+//
+// float32 dense path: one warp per vocab row, plain FMA.
+#include <cfloat>
+
+#include "common.cuh"
+#include "host.cuh"
+
+namespace sdv {
+namespace head {
+
+constexpr int BM = 128;  // vocab rows per tile (UMMA M)
+constexpr int BK = 64;   // K elements per stage (128-byte rows)
+
+struct Params {
+  int M, d, V, ld;
+  int num_tiles, kblocks;
+  float *logits;
+  int *status;
+};
+
+template <int N>
+struct UCfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = N * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < 8 ? (200 * 1024 / STAGE_BYTES) : 8;
+  static constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64
+                                      : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 8 * (2 * STAGES + 4) + 64;
+  static constexpr int THREADS = 192;
+};
+
+template <int N>
+__global__ void __launch_bounds__(192, 1)
+    lm_head_umma_kernel(const __grid_constant__ CUtensorMap wmap,
+                        const __grid_constant__ CUtensorMap hmap, const Params p) {
+  using C = UCfg<N>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)STAGES * C::STAGE_BYTES);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;   // [2] accumulator ready
+  uint64_t *tempty = tfull + 2;       // [2] accumulator drained
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ----------------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&wmap);
+      tma_prefetch_desc(&hmap);
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_h = l2_policy_evict_last();
+      uint32_t g = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < p.kblocks; ++kb, ++g) {
+          const int stage = g % STAGES;
+          const uint32_t ph = (g / STAGES) & 1;
+          if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) {
+            record_status(p.status, SD_ERR_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t *a = smem + (size_t)stage * C::STAGE_BYTES;
+          uint8_t *b = a + C::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d_hint(a, &wmap, &full[stage], kb * BK, tile * BM, pol_w);
+          tma_load_2d_hint(b, &hmap, &full[stage], kb * BK, 0, pol_h);
+        }
+      }
+      if (!ok) {
+        for (uint32_t j = (g > (uint32_t)STAGES ? g - STAGES : 0); j < g; ++j)
+          mbar_wait_timed(&full[j % STAGES], (j / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, N);
+      uint32_t g = 0, i = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++i) {
+        const uint32_t buf = i & 1, tph = (i >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], tph ^ 1, abort_flag)) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * N;
+        for (int kb = 0; kb < p.kblocks; ++kb, ++g) {
+          const int stage = g % STAGES;
+          const uint32_t ph = (g / STAGES) & 1;
+          if (!mbar_wait(&full[stage], ph, abort_flag)) {
+            record_status(p.status, SD_ERR_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + (size_t)stage * C::STAGE_BYTES);
+          const uint32_t b = a + C::A_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks)
+            umma_bf16(d_tmem, umma_desc_sw128(a + ks * 32), umma_desc_sw128(b + ks * 32), idesc,
+                      (kb | ks) != 0);
+          umma_commit(&empty[stage]);
+        }
+        if (ok) umma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------------------- epilogue
+    const int quad = warp & 3;  // tensor-memory lanes 32*quad .. 32*quad+31
+    uint32_t i = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
+      const uint32_t buf = i & 1, tph = (i >> 1) & 1;
+      if (!mbar_wait(&tfull[buf], tph, abort_flag)) {
+        record_status(p.status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int v = tile * BM + quad * 32 + lane;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * N;
+#pragma unroll
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + c0, r);
+        tmem_ld_wait();
+        if (v < p.V) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int m = c0 + e;
+            if (m < p.M) p.logits[(size_t)m * p.ld + v] = __uint_as_float(r[e]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    if (*abort_flag) {
+      // let MMAs already issued drain before the tensor memory is released
+      const unsigned long long t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 1000000ull) {
+      }
+    }
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// float32: one warp per (vocab row); all m rows.
+__global__ void lm_head_f32_kernel(const float *h, const float *w, const Params p) {
+  const int v = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (v >= p.V) return;
+  const float *wr = w + (size_t)v * p.d;
+  for (int m = 0; m < p.M; ++m) {
+    const float *hr = h + (size_t)m * p.d;
+    float acc = 0.f;
+    for (int c = lane; c < p.d; c += 32) acc = fmaf(hr[c], wr[c], acc);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) p.logits[(size_t)m * p.ld + v] = acc;
+  }
+}
+
+// Per row: the top_c clusters by score (ties -> lower id), written in ascending id order.
+// Bitonic sort of (descending score, ascending id) keys in shared memory.
+__global__ void topc_kernel(const float *scores, int C, int top_c, int32_t *sel) {
+  extern __shared__ unsigned long long keys[];
+  const int m = blockIdx.x;
+  int n = 1;
+  while (n < C) n <<= 1;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    unsigned long long key = ~0ull;
+    if (i < C) {
+      uint32_t u = __float_as_uint(scores[(size_t)m * C + i]);
+      u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending order of floats
+      key = ((unsigned long long)(~u) << 32) | (uint32_t)i;  // descending score, then id
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const unsigned long long a = keys[i], b = keys[j];
+          if ((a > b) == up) {
+            keys[i] = b;
+            keys[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // the first top_c keys are the kept clusters; order their ids ascending (top_c <= 64)
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int t = lane; t < top_c; t += 32) {
+      const int id = (int)(keys[t] & 0xFFFFFFFFu);
+      int rank = 0;
+      for (int u = 0; u < top_c; ++u) rank += (int)(keys[u] & 0xFFFFFFFFu) < id;
+      sel[(size_t)m * top_c + rank] = id;
+    }
+  }
+}
+
+__global__ void fill_neg_inf_kernel(float *logits, int M, int V, int ld) {
+  const size_t total = (size_t)M * V;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t m = i / V, v = i % V;
+    logits[m * ld + v] = -INFINITY;
+  }
+}
+
+// One CTA per (row m, kept cluster slot): exact logits of the cluster's tokens.
+__global__ void cluster_logits_kernel(const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm,
+                                      const int32_t *cluster_tokens, const int32_t *sel,
+                                      int top_c, int cs, int d, int C, int V, int ld,
+                                      float *logits, int *status) {
+  extern __shared__ float hs[];
+  const int m = blockIdx.x / top_c, slot = blockIdx.x % top_c;
+  const int c = sel[(size_t)m * top_c + slot];
+  for (int i = threadIdx.x; i < d; i += blockDim.x)
+    hs[i] = __bfloat162float(h[(size_t)m * d + i]);
+  __syncthreads();
+  if (c < 0 || c >= C) {
+    if (threadIdx.x == 0) record_status(status, SD_ERR_DEVICE);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int t = warp; t < cs; t += nw) {
+    const __nv_bfloat16 *wr = w_cm + ((size_t)c * cs + t) * d;
+    float acc = 0.f;
+    for (int k0 = lane * 8; k0 < d; k0 += 256) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(wr + k0);
+      const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc = fmaf(__bfloat162float(e[q]), hs[k0 + q], acc);
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const int tok = cluster_tokens[(size_t)c * cs + t];
+      if (tok < 0 || tok >= V)
+        record_status(status, SD_ERR_DEVICE);
+      else
+        logits[(size_t)m * ld + tok] = acc;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------- host side
+
+template <int N>
+static sd_status launch_umma(const void *h, const void *w, int M, int d, int V, float *logits,
+                             int ld, cudaStream_t st) {
+  using C = UCfg<N>;
+  static bool attr_set[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(lm_head_umma_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C::SMEM) != cudaSuccess)
+      return SD_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  CUtensorMap wm, hm;
+  if (!encode_tmap_2d_bf16(&wm, w, d, V, (uint64_t)d * 2, BK, BM) ||
+      !encode_tmap_2d_bf16(&hm, h, d, M, (uint64_t)d * 2, BK, N))
+    return SD_ERR_CUDA;
+  Params p{};
+  p.M = M;
+  p.d = d;
+  p.V = V;
+  p.ld = ld;
+  p.num_tiles = (V + BM - 1) / BM;
+  p.kblocks = d / BK;
+  p.logits = logits;
+  p.status = device_status_word();
+  const int sms = sm_count();
+  if (sms <= 0) return SD_ERR_CUDA;
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  lm_head_umma_kernel<N><<<grid, C::THREADS, C::SMEM, st>>>(wm, hm, p);
+  return cuda_status(cudaGetLastError());
+}
+
+// Dense bf16 projection of up to 256 rows.
+static sd_status dense_bf16(const void *h, const void *w, int M, int d, int V, float *logits,
+                            int ld, cudaStream_t st) {
+  if (M <= 16) return launch_umma<16>(h, w, M, d, V, logits, ld, st);
+  if (M <= 32) return launch_umma<32>(h, w, M, d, V, logits, ld, st);
+  if (M <= 48) return launch_umma<48>(h, w, M, d, V, logits, ld, st);
+  if (M <= 64) return launch_umma<64>(h, w, M, d, V, logits, ld, st);
+  if (M <= 96) return launch_umma<96>(h, w, M, d, V, logits, ld, st);
+  if (M <= 128) return launch_umma<128>(h, w, M, d, V, logits, ld, st);
+  if (M <= 192) return launch_umma<192>(h, w, M, d, V, logits, ld, st);
+  return launch_umma<256>(h, w, M, d, V, logits, ld, st);
+}
+
+static sd_status validate(const sd_head_desc *d) {
+  if (!d) return SD_ERR_INVALID_ARG;
+  if (d->m < 1 || d->d < 1 || d->vocab < 1) return SD_ERR_INVALID_ARG;
+  const int ld = d->ld_logits ? d->ld_logits : d->vocab;
+  if (ld < d->vocab) return SD_ERR_INVALID_ARG;
+  if (d->dtype != SD_BF16 && d->dtype != SD_F32) return SD_ERR_INVALID_ARG;
+  if (d->top_c < 0) return SD_ERR_INVALID_ARG;
+  if (d->top_c > 0) {
+    if (d->dtype != SD_BF16) return SD_ERR_UNSUPPORTED;
+    if (d->n_clusters < 1 || d->cluster_size < 1 ||
+        (long long)d->n_clusters * d->cluster_size != d->vocab || d->top_c > d->n_clusters)
+      return SD_ERR_INVALID_ARG;
+    if (d->top_c > 64 || d->n_clusters > 8192) return SD_ERR_UNSUPPORTED;
+  }
+  if (d->dtype == SD_BF16 && d->d % 64) return SD_ERR_UNSUPPORTED;
+  if (d->dtype == SD_BF16 && (long long)d->vocab >= (1ll << 31)) return SD_ERR_UNSUPPORTED;
+  return SD_OK;
+}
+
+static size_t ws_size(const sd_head_desc *d) {
+  if (validate(d) != SD_OK) return 0;
+  if (d->top_c == 0) return 0;
+  return round_up((size_t)d->m * d->n_clusters * 4, 256);
+}
+
+}  // namespace head
+}  // namespace sdv
+
+extern "C" {
+
+size_t sd_lm_head_workspace_size(const sd_head_desc *desc) { return sdv::head::ws_size(desc); }
+
+sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
+                     const void *centroids, const int32_t *cluster_tokens, float *logits,
+                     int32_t *sel_clusters, void *ws, size_t ws_bytes, sd_stream stream) {
+  using namespace sdv;
+  using namespace sdv::head;
+  sd_status s = validate(desc);
+  if (s != SD_OK) return s;
+  if (!h || !w || !logits) return SD_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int ld = desc->ld_logits ? desc->ld_logits : desc->vocab;
+  if (desc->dtype == SD_F32) {
+    Params p{};
+    p.M = desc->m;
+    p.d = desc->d;
+    p.V = desc->vocab;
+    p.ld = ld;
+    p.logits = logits;
+    lm_head_f32_kernel<<<(desc->vocab + 7) / 8, 256, 0, st>>>((const float *)h, (const float *)w,
+                                                              p);
+    return cuda_status(cudaGetLastError());
+  }
+  if (!aligned16(h) || !aligned16(w)) return SD_ERR_INVALID_ARG;
+  const size_t hrow = (size_t)desc->d * 2;
+  if (desc->top_c == 0) {
+    for (int m0 = 0; m0 < desc->m; m0 += 256) {
+      const int mm = desc->m - m0 < 256 ? desc->m - m0 : 256;
+      s = dense_bf16((const uint8_t *)h + m0 * hrow, w, mm, desc->d, desc->vocab,
+                     logits + (size_t)m0 * ld, ld, st);
+      if (s != SD_OK) return s;
+    }
+    return SD_OK;
+  }
+  // clustered
+  if (!centroids || !cluster_tokens || !sel_clusters || !aligned16(centroids))
+    return SD_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < ws_size(desc)) return SD_ERR_WORKSPACE;
+  float *scores = reinterpret_cast<float *>(ws);
+  const int C = desc->n_clusters;
+  for (int m0 = 0; m0 < desc->m; m0 += 256) {
+    const int mm = desc->m - m0 < 256 ? desc->m - m0 : 256;
+    s = dense_bf16((const uint8_t *)h + m0 * hrow, centroids, mm, desc->d, C,
+                   scores + (size_t)m0 * C, C, st);
+    if (s != SD_OK) return s;
+  }
+  int n = 1;
+  while (n < C) n <<= 1;
+  topc_kernel<<<desc->m, 512, (size_t)n * 8, st>>>(scores, C, desc->top_c, sel_clusters);
+  if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+  const int sms = sm_count();
+  fill_neg_inf_kernel<<<sms > 0 ? 4 * sms : 512, 256, 0, st>>>(logits, desc->m, desc->vocab, ld);
+  if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+  cluster_logits_kernel<<<desc->m * desc->top_c, 256, (size_t)desc->d * 4, st>>>(
+      (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
+      desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
+      device_status_word());
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"
