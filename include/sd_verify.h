@@ -76,6 +76,8 @@ typedef struct {
                              p in [t - window + 1, t] (window keys including its own) */
   float scale;            /* logit scale, e.g. 1 / sqrt(head_dim) */
   sd_dtype dtype;         /* element type of q, k_new, v_new, caches and out */
+  int q_offset;           /* sd_draft_xattn with q_pos == NULL: the query of sequence b sits
+                             at ctx_len[b] + q_offset (step j of a drafter chain: j) */
 } sd_attn_desc;
 
 /*
@@ -108,7 +110,8 @@ sd_status sd_verify_attn(const sd_attn_desc *desc, const void *q, const void *k_
  * The query of sequence b sits at position q_pos[b] and attends to the committed keys
  * p in [lo, min(q_pos[b], L_b - 1)], lo relative to q_pos[b] as above; an empty range gives a
  * zero output row.
- *   q, out [B, 1, h_q, head_dim]      q_pos int32 [B] (>= 0)
+ *   q, out [B, 1, h_q, head_dim]      q_pos int32 [B] (>= 0), or NULL for
+ *   q_pos[b] = ctx_len[b] + desc->q_offset
  */
 size_t sd_draft_xattn_workspace_size(const sd_attn_desc *desc);
 sd_status sd_draft_xattn(const sd_attn_desc *desc, const void *q, const void *k_cache,

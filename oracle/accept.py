@@ -29,9 +29,10 @@ Readings of points the pages leave open:
     lowest v wins ties.  This is an exact categorical draw needing no normalisation.
     Implemented as argmax of ln w_v - ln E_v.
   * Margins (decisions a float32 implementation may take differently): an acceptance
-    with |u - p/q| < MARGIN, a draw whose winner leads some other token by less than
-    MARGIN plus both tokens' error bounds on the ln-key scale, a greedy argmax whose top
-    two logits differ by less than MARGIN * max(1, |top|).
+    with |u - p/q| < MARGIN; a draw whose winner's lowest possible key does not beat every
+    other token's highest possible key by MARGIN, the key bounds taking each weight as
+    w +- REL_P * (p + q) (the float32 error of p - q) and ln E, z / T to within ABS_KEY;
+    a greedy argmax whose top two logits differ by less than MARGIN * max(1, |top|).
 """
 from __future__ import annotations
 
@@ -64,14 +65,13 @@ def race(w: np.ndarray, V: np.ndarray):
     return np.argmax(g, axis=-1), g
 
 
-def _race_margin(g: np.ndarray, err: np.ndarray, x: np.ndarray) -> np.ndarray:
-    R = g.shape[0]
-    gx = g[np.arange(R), x]
-    ex = err[np.arange(R), x]
-    with np.errstate(invalid="ignore"):
-        upper = np.where(np.isfinite(g), g + err, g)
-    upper[np.arange(R), x] = -np.inf
-    return upper.max(axis=-1) > gx - ex - MARGIN
+def _race_margin(g_lo: np.ndarray, g_hi: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """True where the winner x might lose: its lowest possible key is not MARGIN above the
+    highest possible key of every other token."""
+    R = g_lo.shape[0]
+    hi = g_hi.copy()
+    hi[np.arange(R), x] = -np.inf
+    return hi.max(axis=-1) > g_lo[np.arange(R), x] - MARGIN
 
 
 def greedy_gap(z: np.ndarray) -> np.ndarray:
@@ -121,6 +121,7 @@ def accept(z, y, drafts, temperature: float, seed: int, step: int,
             active = active & (u < ratio)
             n_acc += active
         pa = p[bidx, n_acc]
+        za = z[bidx, n_acc] / T
         if k > 0:
             qa = q[bidx, np.minimum(n_acc, k - 1)]
             resid = np.maximum(0.0, pa - qa)
@@ -128,15 +129,20 @@ def accept(z, y, drafts, temperature: float, seed: int, step: int,
             empty = resid.sum(axis=-1) == 0.0
             use_p = (bonus | empty)[:, None]
             w = np.where(use_p, pa, resid)
-            with np.errstate(divide="ignore", invalid="ignore"):
-                err = np.where(use_p, ABS_KEY * (1.0 + np.abs(z[bidx, n_acc] / T)),
-                               REL_P * (pa + qa) / w + ABS_KEY)
+            slack = REL_P * (pa + qa)
+            w_hi = np.where(use_p, pa, resid + slack)
+            w_lo = np.where(use_p, pa, np.maximum(resid - slack, 0.0))
+            key_err = np.where(use_p, ABS_KEY * (1.0 + np.abs(za)), ABS_KEY)
         else:
-            w = pa
-            err = ABS_KEY * (1.0 + np.abs(z[:, 0] / T))
+            w = w_hi = w_lo = pa
+            key_err = ABS_KEY * (1.0 + np.abs(za))
         Vu = token_uniform_rows(seed, step, rows + n_acc, purpose, V)
         x, g = race(w, Vu)
-        margin |= _race_margin(g, np.nan_to_num(err, nan=np.inf, posinf=np.inf), x)
+        lnE = np.log(-np.log1p(-Vu))
+        with np.errstate(divide="ignore"):
+            g_hi = np.log(w_hi) - lnE + key_err
+            g_lo = np.log(w_lo) - lnE - key_err
+        margin |= _race_margin(g_lo, g_hi, x)
 
     out = np.full((B, n_q), -1, np.int64)
     for b in range(B):

@@ -47,7 +47,9 @@ def attn_desc(B, n_q, hq, hkv, D, bs, mbps, nblocks, window, dtype=sd.SD_BF16, s
 
 
 def workspace(nbytes: int) -> torch.Tensor:
-    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=DEV)
+    """Scratch buffer filled with 0xFF bytes (NaN as float32), so a kernel that reads a
+    workspace slot it never wrote produces NaN instead of a stale but plausible value."""
+    return torch.full((max(int(nbytes), 16),), 255, dtype=torch.uint8, device=DEV)
 
 
 def to_dev(t: torch.Tensor) -> torch.Tensor:

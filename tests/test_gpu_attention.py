@@ -241,3 +241,28 @@ def test_drafter_config_full_size():
                                          qp.numpy(), lay.window, desc.scale, w.block_size)
             assert rel_err(out[b, 0, h].cpu().float().numpy()[None], ref[None]) <= BF16_TOL
     assert status_ok()
+
+
+def test_draft_xattn_position_from_context_length():
+    """q_pos == NULL: the query sits at ctx_len + q_offset (a drafter chain step)."""
+    seed, L, hq, hkv, D, bs, window = 24, [300, 40, 77], 16, 4, 256, 16, 64
+    B = len(L)
+    c = small_paged(seed, L, 1, hkv, D, bs)
+    q, _, _ = qkv(seed, B, 1, hq, hkv, D)
+    kc_d, vc_d, tab, Ld = to_dev(c["kc"]), to_dev(c["vc"]), to_dev(c["table"]), to_dev(c["L"])
+    for j in (0, 1, 3):
+        desc = attn_desc(B, 1, hq, hkv, D, bs, c["mbps"], c["nb"], window)
+        desc.q_offset = j
+        ws = workspace(sd.sd_draft_xattn_workspace_size(desc))
+        out_a = torch.empty(q.shape, dtype=q.dtype, device=DEV)
+        out_b = torch.empty(q.shape, dtype=q.dtype, device=DEV)
+        sd.sd_draft_xattn(desc, to_dev(q), kc_d, vc_d, tab, Ld, None, out_a, ws)
+        qp = to_dev(c["L"] + j)
+        sd.sd_draft_xattn(desc, to_dev(q), kc_d, vc_d, tab, Ld, qp, out_b, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out_a, out_b)
+        f = lambda t: t.to(torch.float64).numpy()
+        ref = OA.draft_attention(f(q), f(c["kc"]), f(c["vc"]), c["table"].numpy(),
+                                 c["L"].numpy(), (c["L"] + j).numpy(), window, desc.scale, bs)
+        assert rel_err(out_a.cpu().float().numpy(), ref) <= BF16_TOL
+    assert status_ok()

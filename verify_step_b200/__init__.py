@@ -36,7 +36,8 @@ class AttnDesc(ctypes.Structure):
                 ("h_kv", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("max_blocks_per_seq", ctypes.c_int),
                 ("num_blocks", ctypes.c_int), ("window", ctypes.c_int),
-                ("scale", ctypes.c_float), ("dtype", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int),
+                ("q_offset", ctypes.c_int)]
 
 
 class HeadDesc(ctypes.Structure):

@@ -37,6 +37,7 @@ constexpr int kTile = 16;
 struct Params {
   int B, n_q, Hq, Hkv, G, D, bs, mbps, num_blocks, window, M, Mpad;
   int is_draft;
+  int q_offset;      // query position ctx_len[b] + q_offset when q_pos is null
   float scale_log2;  // scale * log2(e)
   float scale;
   const void *q;
@@ -56,6 +57,10 @@ struct SeqRange {
   int L, tf, n, lo_min, hi_max;
 };
 
+__device__ __forceinline__ int draft_qpos(const Params &p, int b) {
+  return p.q_pos != nullptr ? p.q_pos[b] : p.ctx_len[b] + p.q_offset;
+}
+
 __device__ __forceinline__ SeqRange seq_range(const Params &p, int b, bool report) {
   SeqRange r;
   r.L = p.ctx_len[b];
@@ -72,7 +77,7 @@ __device__ __forceinline__ SeqRange seq_range(const Params &p, int b, bool repor
     hi = r.L + p.n_q - 1;
     lo = p.window > 0 ? max(0, r.L - p.window + 1) : 0;
   } else {
-    const int qp = p.q_pos[b];
+    const int qp = draft_qpos(p, b);
     if (r.L < 0 || qp < 0) {
       if (report) record_status(p.status, SD_ERR_DEVICE);
       return r;
@@ -105,7 +110,7 @@ __device__ __forceinline__ void row_range(const Params &p, const SeqRange &s, in
     hi = t;
     lo = p.window > 0 ? max(0, t - p.window + 1) : 0;
   } else {
-    const int t = p.q_pos[b];
+    const int t = draft_qpos(p, b);
     hi = min(t, s.L - 1);
     lo = p.window > 0 ? max(0, t - p.window + 1) : 0;
   }
@@ -545,14 +550,21 @@ __global__ void attn_combine_kernel(const Params p) {
   const int c_last = (int)(((Fl + 1) * p.P - 1) / T_all);
   if (c_first == c_last) return;  // written directly by its only CTA
   const size_t slot0 = (size_t)b * p.Hkv + g;
+  // CTA c holds tiles [T*c/P, T*(c+1)/P); with fewer tiles than CTAs some hold none and
+  // wrote no partial for this item.
+  auto holds = [&](int c) {
+    const long long s_c = T_all * c / p.P, e_c = T_all * (c + 1) / p.P;
+    return e_c > F && s_c <= Fl && e_c > s_c;
+  };
   for (int idx = threadIdx.x; idx < p.M * p.D; idx += blockDim.x) {
     const int row = idx / p.D, d = idx % p.D;
     float mmax = -INFINITY;
     for (int c = c_first; c <= c_last; ++c)
-      mmax = fmaxf(mmax, p.ws_ml[((slot0 + c) * p.Mpad + row) * 2]);
+      if (holds(c)) mmax = fmaxf(mmax, p.ws_ml[((slot0 + c) * p.Mpad + row) * 2]);
     float num = 0.f, den = 0.f;
     if (mmax != -INFINITY) {
       for (int c = c_first; c <= c_last; ++c) {
+        if (!holds(c)) continue;
         const size_t sl = (slot0 + c) * p.Mpad + row;
         const float w = exp2f(p.ws_ml[sl * 2] - mmax);
         num += w * p.ws_o[sl * p.D + d];
@@ -746,7 +758,6 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   sd_status s = validate(d, draft);
   if (s != SD_OK) return s;
   if (!q || !k_cache || !v_cache || !table || !ctx_len || !out) return SD_ERR_INVALID_ARG;
-  if (draft && !q_pos) return SD_ERR_INVALID_ARG;
   if (!draft && (!k_new || !v_new)) return SD_ERR_INVALID_ARG;
   Params p{};
   p.B = d->batch;
@@ -762,6 +773,7 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   p.M = p.G * p.n_q;
   p.Mpad = (p.M + 15) / 16 * 16;
   p.is_draft = draft ? 1 : 0;
+  p.q_offset = d->q_offset;
   p.scale = d->scale;
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.q = q;
