@@ -142,15 +142,21 @@ class SpecStep:
         self.hdesc_cl = sd.HeadDesc(m=B, d=self.dh, vocab=self.V, ld_logits=k * self.V,
                                     n_clusters=self.C, cluster_size=self.cs, top_c=self.top_c,
                                     dtype=sd.SD_BF16)
+        # step counter on the device: the acceptance draws of step s use counter value s (the
+        # drafter's chain step j adds (j+1) << 28 to keep its uniforms apart); sd_commit
+        # advances it, so a step captured once in a CUDA graph draws fresh numbers each replay
+        self.step_dev = torch.zeros(1, dtype=torch.int64, device=dev)
+        sp = self.step_dev.data_ptr()
         self.adesc_draft = [sd.AcceptDesc(batch=B, k=0, vocab=self.V, temperature=1.0, seed=7,
-                                          step=0, purpose=2, ld_target=k * self.V, ld_out=k)
-                            for _ in range(k)]
+                                          step=(j + 1) << 28, purpose=2, ld_target=k * self.V,
+                                          ld_out=k, step_ptr=sp)
+                            for j in range(k)]
         self.adesc = sd.AcceptDesc(batch=B, k=k, vocab=self.V, temperature=1.0, seed=7, step=0,
-                                   purpose=1)
+                                   purpose=1, step_ptr=sp)
         self.cdesc = sd.CommitDesc(batch=B, k=k, block_size=self.bs,
                                    max_blocks_per_seq=self.cache[0]["mb"],
                                    num_blocks=self.cache[0]["nb"], d=self.d,
-                                   hidden_dtype=sd.SD_BF16)
+                                   hidden_dtype=sd.SD_BF16, step_ptr=sp)
         wsz = max([sd.sd_verify_attn_workspace_size(x) for x in self.vdesc] +
                   [sd.sd_draft_xattn_workspace_size(x) for row in self.xdesc for x in row] +
                   [sd.sd_lm_head_workspace_size(self.hdesc_cl),
@@ -175,19 +181,20 @@ class SpecStep:
         return (self.k * (4 * L["xattn"] + L["head_clustered"] + L["accept"]) +
                 2 * L["verify"] + L["head_dense"] + L["accept"] + L["commit"])
 
-    def run(self, s, ev=None):
-        """Issue one step on the current stream; ev maps a kernel group to a list that receives
-        (start, end) CUDA events around each call of that group."""
-        sd, torch, I = self.sd, self.torch, self.inputs
+    def run(self, ev=None):
+        """Issue one step on the current stream.  ev (used while capturing a CUDA graph) maps a
+        kernel group to a list that receives (start, end) events recorded as graph nodes
+        around each call of that group."""
+        sd, I = self.sd, self.inputs
 
         def timed(name, fn):
             if ev is None or name not in ev:
                 fn()
                 return
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
+            a, b = new_event(), new_event()
+            record_external(a)
             fn()
-            b.record()
+            record_external(b)
             ev[name].append((a, b))
 
         c0, c1 = self.cache
@@ -202,7 +209,6 @@ class SpecStep:
                 self.xout[0], self.ws))
             timed("head_clustered", lambda: self._clustered(j))
             ad = self.adesc_draft[j]
-            ad.step = s * 16 + j
             timed("accept_draft", lambda: sd.sd_accept(
                 ad, self._row_ptr(self.draft_logits, j), None, None, self.n_acc,
                 self._col_ptr(self.drafts, j), None, self.ws))
@@ -214,7 +220,6 @@ class SpecStep:
             self.attn_out[1], self.ws))
         timed("head_dense", lambda: sd.sd_lm_head(self.hdesc_dense, I["hidden"], self.W,
                                                   self.target_logits))
-        self.adesc.step = s
         timed("accept", lambda: sd.sd_accept(self.adesc, self.target_logits, self.draft_logits,
                                              self.drafts, self.n_acc, self.out_tokens,
                                              self.margin, self.ws))
@@ -270,6 +275,34 @@ class SpecStep:
     def reset(self):
         self.ctx.copy_(self.ctx0)
 
+    def capture(self, ev=None):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run(ev)
+        return g
+
+
+def new_event():
+    """A timing event whose CUDA handle exists (torch creates it lazily on first record)."""
+    import torch
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()
+    return e
+
+
+def record_external(ev):
+    """Record ``ev`` on the current stream as an event node of the graph being captured
+    (cudaEventRecordExternal), so every replay re-records it."""
+    import torch
+    from cuda.bindings import runtime as cudart
+    err, = cudart.cudaEventRecordWithFlags(
+        cudart.cudaEvent_t(ev.cuda_event),
+        cudart.cudaStream_t(torch.cuda.current_stream().cuda_stream),
+        cudart.cudaEventRecordExternal)
+    if err != cudart.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaEventRecordWithFlags: {err}")
+
 
 # --------------------------------------------------------------------------------- clocks
 
@@ -280,7 +313,7 @@ class ClockSampler:
 
     def __init__(self, dev_index):
         self.proc = None
-        self.t0 = None
+        self.err = None
         try:
             import torch
             props = torch.cuda.get_device_properties(dev_index)
@@ -288,22 +321,22 @@ class ClockSampler:
             dom = getattr(props, "pci_domain_id", 0)
             dvc = getattr(props, "pci_device_id", 0)
             sel = ["-i", "%08X:%02X:%02X.0" % (dom, bus, dvc)] if bus is not None else []
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", *sel, "--query-gpu=timestamp," + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+            self.cmd = ["nvidia-smi", *sel, "--query-gpu=timestamp," + self.FIELDS,
+                        "--format=csv,noheader,nounits", "-lms", "20"]
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.PIPE, text=True)
+        except Exception as e:  # no nvidia-smi: report why
+            self.err = repr(e)
 
     def stop(self):
         if self.proc is None:
-            return None
+            return {"error": self.err}
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=10)
+            out, errout = self.proc.communicate(timeout=10)
         except Exception:
             self.proc.kill()
-            return None
+            return {"error": "nvidia-smi did not stop"}
         rows = []
         for line in out.strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
@@ -317,7 +350,8 @@ class ClockSampler:
             except ValueError:
                 continue
         if not rows:
-            return None
+            return {"error": "no samples", "cmd": " ".join(self.cmd),
+                    "stdout": out.strip().splitlines()[:3], "stderr": errout.strip()[:300]}
         load = [r for r in rows if r["power"] > 300] or rows
         reasons = set()
         for r in load:
@@ -327,7 +361,9 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r["sm"] for r in load),
                 "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
-                "samples": len(load), "power_w_max": max(r["power"] for r in rows)}
+                "samples": len(load), "power_w_max": max(r["power"] for r in rows),
+                "window": "warm-up, timed, per-kernel and end-to-end passes (samples above "
+                          "300 W taken as under load)"}
 
 
 # --------------------------------------------------------------------------------- oracle
@@ -381,8 +417,8 @@ def oracle_sample(step_obj, seqs, s):
         lg, _, _ = OH.clustered_lm_head(f(hi[f"dh{j}"])[seqs], f(cl["centroids"]),
                                         F64(cl["w_cm"]), cl["cluster_tokens"].numpy(), st.top_c)
         draft_logits[:, j] = lg
-        r = OACC.accept(lg[:, None, :], None, np.zeros((m, 0)), 1.0, seed=7, step=s * 16 + j,
-                        purpose=OACC.PURPOSE_DRAFTER)
+        r = OACC.accept(lg[:, None, :], None, np.zeros((m, 0)), 1.0, seed=7,
+                        step=((j + 1) << 28) + s, purpose=OACC.PURPOSE_DRAFTER)
         drafts[:, j] = r["out_tokens"][:, 0]
     for layer, cache, D, W in ((0, c0, 512, 0), (1, c1, 256, 512)):
         q, kn, vn = f(hi[f"q{layer}"]), f(hi[f"kn{layer}"]), f(hi[f"vn{layer}"])
@@ -440,33 +476,34 @@ def main():
     import verify_step_b200 as sd
     sd.lib()
 
-    reserve = 3 * (a.warmup + a.steps + 2) * (a.k + 1) + 64
+    # every pass below runs a.steps steps (warm-up, timed, per-kernel, e2e): reserve the blocks
+    reserve = (a.warmup + 4 * a.steps + 8) * (a.k + 1) + 64
     st = SpecStep(k=a.k, B=a.batch, L=a.ctx, reserve=reserve, rank=rank)
     L_start = st.L0.copy()
-    for s in range(a.warmup):
-        st.run(s)
+    clock = ClockSampler(local)
+    for _ in range(a.warmup):
+        st.run()
     torch.cuda.synchronize()
     sd.sd_device_status_clear()
+    graph = st.capture()
+    graph.replay()
+    torch.cuda.synchronize()
+    ctx_a = st.ctx.cpu().numpy()
 
-    groups = list(st.calls_per_step())
-    ev = {g: [] for g in groups}
-    clock = ClockSampler(local)
-    # whole-step timing (no per-kernel events inside)
+    # ---- timed region: exactly K steps, one graph replay each
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
-    for s in range(a.warmup, a.warmup + a.steps):
-        st.run(s)
+    for _ in range(a.steps):
+        graph.replay()
     t1.record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clocks = clock.stop()
     ms = t0.elapsed_time(t1)
-    ctx_end = st.ctx.cpu().numpy()
-    status = sd.sd_device_status_read()
+    ctx_b = st.ctx.cpu().numpy()
     if world > 1:
         tms = torch.tensor([ms], device="cuda")
         dist.all_reduce(tms, op=dist.ReduceOp.MAX)
@@ -474,57 +511,58 @@ def main():
     ms_step = ms / a.steps
     value = world * st.B * st.n_q * a.steps / (ms / 1e3)
 
-    # per-kernel timing: a second pass of the same K steps with events around each call
-    st.reset()
-    for s in range(2):
-        st.run(s)
-    torch.cuda.synchronize()
-    for s in range(a.steps):
-        st.run(a.warmup + s, ev)
-    torch.cuda.synchronize()
-    kern_ms = {g: (sum(x.elapsed_time(y) for x, y in ev[g]) / len(ev[g])) if ev[g] else 0.0
-               for g in groups}
-    L_mid = (L_start + ctx_end) / 2.0
-    nbytes = st.bytes_per_call(L_mid)
+    # ---- per-kernel device times: the same step captured with event nodes around each call,
+    # replayed K times (synchronised per replay to read the events)
+    groups = list(st.calls_per_step())
+    ev = {g: [] for g in groups}
+    graph_ev = st.capture(ev)
+    sums = {g: 0.0 for g in groups}
+    ctx_c = st.ctx.cpu().numpy()
+    for _ in range(a.steps):
+        graph_ev.replay()
+        torch.cuda.synchronize()
+        for g in groups:
+            sums[g] += sum(x.elapsed_time(y) for x, y in ev[g])
+    ctx_d = st.ctx.cpu().numpy()
+    kern_ms = {g: sums[g] / (a.steps * len(ev[g])) if ev[g] else 0.0 for g in groups}
+    nbytes = st.bytes_per_call((ctx_c + ctx_d) / 2.0)
     hbm, tfl, src = peaks()
-    per_kernel = {g: {"ms": round(kern_ms[g], 4), "calls_per_step": st.calls_per_step()[g],
+    cps = st.calls_per_step()
+    per_kernel = {g: {"ms": round(kern_ms[g], 4), "calls_per_step": cps[g],
+                      "bytes_per_call": nbytes[g],
                       "GBps": round(nbytes[g] / (kern_ms[g] * 1e6), 1) if kern_ms[g] else None,
                       "frac_hbm": round(nbytes[g] / (kern_ms[g] * 1e6) / hbm, 3)
                       if kern_ms[g] else None}
                   for g in groups}
-    dom = max(groups, key=lambda g: kern_ms[g] * st.calls_per_step()[g])
-    ach = nbytes[dom] / (kern_ms[dom] * 1e6)
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
-                "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": None,
-                "peak_source": src, "bytes_per_launch": nbytes[dom],
-                "ms_per_launch": round(kern_ms[dom], 4)}
-    att = "verify_global"
-    ach_a = nbytes[att] / (kern_ms[att] * 1e6)
-    roof_attn = {"kernel": att, "bound": "hbm", "achieved": round(ach_a, 1), "peak": hbm,
-                 "unit": "GB/s", "frac": round(ach_a / hbm, 4), "traffic": None,
-                 "bytes_per_launch": nbytes[att], "ms_per_launch": round(kern_ms[att], 4)}
-    # telemetry of the acceptance rule on these (random) weights
-    n_acc_total = float(((ctx_end - L_start) - a.steps).sum()) / max(1, a.steps * st.B)
+    busy_ms = sum(kern_ms[g] * cps[g] for g in groups)
+    dom = max(groups, key=lambda g: kern_ms[g] * cps[g])
 
-    # end-to-end leg: inputs copied from pinned host memory each step, result read back
+    def roof(g):
+        ach = nbytes[g] / (kern_ms[g] * 1e6)
+        return {"kernel": g, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": None,
+                "peak_source": src, "bytes_per_launch": nbytes[g],
+                "ms_per_launch": round(kern_ms[g], 4)}
+    # telemetry of the acceptance rule on these (random) weights
+    mean_acc = float(((ctx_b - ctx_a) - a.steps).sum()) / max(1, a.steps * st.B)
+
+    # ---- end-to-end: every step copies its inputs from pinned host memory, replays the step
+    # and reads the accepted counts and tokens back to the host
     e2e = None
     if not a.no_e2e:
-        st.reset()
         pinned = {kk: v.pin_memory() for kk, v in st.host_inputs.items()}
         res_h = torch.empty(st.B * (st.n_q + 1), dtype=torch.int32).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in pinned.values())
         d2h = res_h.numel() * 4
-        for s in range(2):
-            st.run(s)
-        torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
+        torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for s in range(a.steps):
+        for _ in range(a.steps):
             for kk, v in pinned.items():
                 st.inputs[kk].copy_(v, non_blocking=True)
-            st.run(a.warmup + s)
+            graph.replay()
             res_h[:st.B].copy_(st.n_acc, non_blocking=True)
             res_h[st.B:].copy_(st.out_tokens.view(-1), non_blocking=True)
             torch.cuda.current_stream().synchronize()
@@ -537,7 +575,13 @@ def main():
             ems = float(tms.item())
         e2e = {"value": round(world * st.B * st.n_q * a.steps / (ems / 1e3), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(ems / a.steps, 4)}
+               "ms_per_step": round(ems / a.steps, 4),
+               "path": "public C ABI calls captured once in a CUDA graph; per step: H2D of "
+                       "the step inputs from pinned memory, replay, D2H of n_accepted and "
+                       "out_tokens, stream synchronise"}
+    clocks = clock.stop()
+    status = sd.sd_device_status_read()
+    del graph, graph_ev
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -568,13 +612,15 @@ def main():
                    "l2": "inputs larger than L2 (~6 GB read per step)",
                    "ctx_growth": "contexts advance by the accepted length each step"},
         "gpu_launches": st.launches_per_step() * a.steps,
-        "roofline": roofline,
-        "roofline_attention": roof_attn,
+        "roofline": roof(dom),
+        "roofline_attention": roof("verify_global"),
+        "roofline_lm_head": roof("head_dense"),
         "kernels": per_kernel,
+        "kernel_busy_ms_per_step": round(busy_ms, 4),
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "mean_accepted": round(n_acc_total, 4),
+        "mean_accepted": round(mean_acc, 4),
         "device_status": status,
     }
     print(json.dumps(line))

@@ -188,6 +188,9 @@ typedef struct {
   int ld_target;       /* floats between target rows r = b*(k+1)+i; 0 means vocab */
   int ld_draft;        /* floats between draft rows b*k+i; 0 means vocab */
   int ld_out;          /* int32 between sequences of out_tokens; 0 means k+1 */
+  const uint64_t *step_ptr; /* nullable DEVICE word: when set, the step entering the counter
+                               is *step_ptr + step, read when the kernels run (a decode loop
+                               replayed from a CUDA graph advances it with sd_commit) */
 } sd_accept_desc;
 
 /*
@@ -216,6 +219,7 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
  *                                 both may be NULL to skip)
  *   poison (n_poison > 0): the rows of the rolled-back positions L+a+1 .. L+k are set to NaN
  *   in every listed cache (debugging aid; the next verify step overwrites them).
+ *   step_ptr (nullable): *step_ptr += 1 once the commit is done.
  */
 typedef struct {
   void *cache;          /* [num_blocks, h_kv, block_size, head_dim] sharing block_table */
@@ -234,6 +238,7 @@ typedef struct {
   sd_dtype hidden_dtype;
   int n_poison;         /* entries in poison (0: no poisoning) */
   const sd_poison_cache *poison;  /* HOST array of n_poison entries */
+  uint64_t *step_ptr;   /* nullable DEVICE word: incremented by one after the commit */
 } sd_commit_desc;
 
 sd_status sd_commit(const sd_commit_desc *desc, const int32_t *block_table, int32_t *ctx_len,

@@ -170,3 +170,23 @@ def test_gpu_reproduces_target_distribution():
         exp[v] = Q[()][v] * alpha * P[(v,)]  # d1 = v accepted; next token ~ p_2(.|v) exactly
     exp = exp / exp.sum() * two.sum()
     assert stats.chisquare(two.ravel(), exp.ravel()).pvalue > 0.01
+
+
+def test_step_read_from_device_word():
+    """step_ptr set: the counter uses *step_ptr + step (what a graph-replayed loop relies on)."""
+    z, y = tuned_inputs(41, 8, 2)
+    drafts = draw_drafts(y, 1.0, seed=2, step=9)
+    B, n_q, V = z.shape
+    counter = torch.tensor([123456], dtype=torch.int64, device=DEV)
+    desc = sd.AcceptDesc(batch=B, k=2, vocab=V, temperature=1.0, seed=77, step=1000,
+                         purpose=1, step_ptr=counter.data_ptr())
+    n_acc = torch.empty(B, dtype=torch.int32, device=DEV)
+    out = torch.empty((B, n_q), dtype=torch.int32, device=DEV)
+    ws = workspace(sd.sd_accept_workspace_size(desc))
+    sd.sd_accept(desc, to_dev(z), to_dev(y), to_dev(drafts), n_acc, out, None, ws)
+    torch.cuda.synchronize()
+    ref = OACC.accept(z.double().numpy(), y.double().numpy(), drafts.numpy(), 1.0, seed=77,
+                      step=123456 + 1000)
+    ok = ~ref["margin"]
+    assert np.array_equal(n_acc.cpu().numpy()[ok], ref["n_accepted"][ok])
+    assert np.array_equal(out.cpu().numpy()[ok], ref["out_tokens"][ok])

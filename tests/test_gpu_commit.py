@@ -60,3 +60,20 @@ def test_commit_flags_out_of_range_accept_count():
     assert sd.sd_device_status_read() == sd.SD_ERR_DEVICE
     sd.sd_device_status_clear()
     assert status_ok()
+
+
+def test_commit_advances_step_counter():
+    B, k, bs = 4, 2, 16
+    L = np.array([5, 17, 0, 40], np.int32)
+    table, nb = S.block_table(0, L, k + 1, bs, shuffle=False)
+    counter = torch.tensor([41], dtype=torch.int64, device=DEV)
+    ctx = to_dev(torch.from_numpy(L))
+    a = torch.tensor([0, 2, 1, 2], dtype=torch.int32, device=DEV)
+    slots = torch.empty((B, k + 1), dtype=torch.int32, device=DEV)
+    desc = sd.CommitDesc(batch=B, k=k, block_size=bs, max_blocks_per_seq=table.shape[1],
+                         num_blocks=nb, step_ptr=counter.data_ptr())
+    for _ in range(3):
+        sd.sd_commit(desc, to_dev(torch.from_numpy(table)), ctx, a, slots)
+    torch.cuda.synchronize()
+    assert counter.item() == 44
+    assert ctx.cpu().tolist() == [5 + 3, 17 + 9, 0 + 6, 40 + 9]

@@ -52,7 +52,7 @@ class AcceptDesc(ctypes.Structure):
                 ("temperature", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("step", ctypes.c_uint64), ("purpose", ctypes.c_int),
                 ("ld_target", ctypes.c_int), ("ld_draft", ctypes.c_int),
-                ("ld_out", ctypes.c_int)]
+                ("ld_out", ctypes.c_int), ("step_ptr", ctypes.c_void_p)]
 
 
 class PoisonCache(ctypes.Structure):
@@ -64,7 +64,8 @@ class CommitDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("k", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("max_blocks_per_seq", ctypes.c_int), ("num_blocks", ctypes.c_int),
                 ("d", ctypes.c_int), ("hidden_dtype", ctypes.c_int),
-                ("n_poison", ctypes.c_int), ("poison", ctypes.POINTER(PoisonCache))]
+                ("n_poison", ctypes.c_int), ("poison", ctypes.POINTER(PoisonCache)),
+                ("step_ptr", ctypes.c_void_p)]
 
 
 _lib = None

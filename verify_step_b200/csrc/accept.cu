@@ -33,7 +33,8 @@ struct Params {
   int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, rows_t, rows_total;
   float T;
   unsigned long long seed;
-  uint32_t step;
+  unsigned long long step;
+  const unsigned long long *step_ptr;  // nullable: step = *step_ptr + step
   const float *z;
   const float *y;
   const int32_t *drafts;
@@ -183,8 +184,10 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   __shared__ float s_mz, s_isz, s_my, s_isy;
   __shared__ float4 red[2][kThreads / 32];
   __shared__ int s_last;
+  __shared__ uint32_t s_step;
 
   if (threadIdx.x == 0) {
+    s_step = (uint32_t)(p.step + (p.step_ptr != nullptr ? *p.step_ptr : 0ull));
     int a = 0, flag = 0;
     for (int i = 1; i <= p.k; ++i) {
       const int d = p.drafts[(size_t)b * p.k + i - 1];
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
         const float qd =
             expf(p.y[((size_t)b * p.k + i - 1) * p.ld_d + d] / p.T - sy.x) / sy.y;
         const float ratio = qd > 0.f ? pd / qd : (pd > 0.f ? INFINITY : 0.f);
-        const float u = accept_uniform(p.seed, p.step, (uint32_t)rt);
+        const float u = accept_uniform(p.seed, s_step, (uint32_t)rt);
         if (fabsf(u - ratio) < kMargin) flag = 1;
         acc = u < ratio;
       } else {
@@ -225,6 +228,7 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   }
   __syncthreads();
   const int a = s_a;
+  const uint32_t step = s_step;
 
   if (p.T == 0.f) {  // greedy: one CTA per sequence, no race
     if (threadIdx.x == 0) {
@@ -256,10 +260,10 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
     float4 y4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (resid) y4 = __ldg(reinterpret_cast<const float4 *>(yr + v));
     float U[4];
-    token_uniform_pair(p.seed, p.step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1), U[0],
+    token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1), U[0],
                        U[1]);
-    token_uniform_pair(p.seed, p.step, (uint32_t)rt, (uint32_t)p.purpose,
-                       (uint32_t)(v >> 1) + 1u, U[2], U[3]);
+    token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1) + 1u,
+                       U[2], U[3]);
     const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
     const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
 #pragma unroll
@@ -384,7 +388,8 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.rows_total = p.rows_t + (sampling ? p.B * p.k : 0);
   p.T = desc->temperature;
   p.seed = desc->seed;
-  p.step = (uint32_t)desc->step;
+  p.step = desc->step;
+  p.step_ptr = reinterpret_cast<const unsigned long long *>(desc->step_ptr);
   p.z = target_logits;
   p.y = draft_logits;
   p.drafts = draft_tokens;

@@ -31,6 +31,7 @@ struct Params {
   const uint8_t *hidden;
   uint8_t *next_hidden;
   PoisonList poison;
+  unsigned long long *step_ptr;
   int *status;
 };
 
@@ -49,6 +50,7 @@ __global__ void commit_kernel(const Params p) {
   }
   __syncthreads();
   const int a = s_a, L = s_L;
+  if (b == 0 && threadIdx.x == 0 && p.step_ptr != nullptr) *p.step_ptr += 1ull;
   if (a < 0) return;
   for (int j = threadIdx.x; j < p.n_q; j += blockDim.x) {
     int slot = -1;
@@ -137,6 +139,7 @@ extern "C" sd_status sd_commit(const sd_commit_desc *desc, const int32_t *block_
     p.poison.head_dim[i] = c.head_dim;
     p.poison.is_bf16[i] = c.dtype == SD_BF16;
   }
+  p.step_ptr = reinterpret_cast<unsigned long long *>(desc->step_ptr);
   p.status = device_status_word();
   commit_kernel<<<p.B, 128, 0, (cudaStream_t)stream>>>(p);
   return cuda_status(cudaGetLastError());
