@@ -65,7 +65,7 @@ def test_commit_flags_out_of_range_accept_count():
 def test_commit_advances_step_counter():
     B, k, bs = 4, 2, 16
     L = np.array([5, 17, 0, 40], np.int32)
-    table, nb = S.block_table(0, L, k + 1, bs, shuffle=False)
+    table, nb = S.block_table(0, L, 4 * (k + 1), bs, shuffle=False)
     counter = torch.tensor([41], dtype=torch.int64, device=DEV)
     ctx = to_dev(torch.from_numpy(L))
     a = torch.tensor([0, 2, 1, 2], dtype=torch.int32, device=DEV)
@@ -77,3 +77,4 @@ def test_commit_advances_step_counter():
     torch.cuda.synchronize()
     assert counter.item() == 44
     assert ctx.cpu().tolist() == [5 + 3, 17 + 9, 0 + 6, 40 + 9]
+    assert status_ok()
