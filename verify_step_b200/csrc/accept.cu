@@ -25,12 +25,13 @@
 namespace sdv {
 namespace acc {
 
-constexpr int kChunk = 8192;
+constexpr int kChunk = 8192;      // tokens per CTA of the statistics pass
+constexpr int kDrawChunk = 2048;  // tokens per CTA of the race
 constexpr int kThreads = 256;
 constexpr float kMargin = 1e-4f;
 
 struct Params {
-  int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, rows_t, rows_total;
+  int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, ndraw, rows_t, rows_total;
   float T;
   unsigned long long seed;
   unsigned long long step;
@@ -42,7 +43,7 @@ struct Params {
   int32_t *out;
   int32_t *margin;
   float4 *stats;   // [rows_total][nchunks]
-  float4 *cand;    // [B][nchunks][2]
+  float4 *cand;    // [B][ndraw][2]
   unsigned int *counters;  // [B]
   int *status;
 };
@@ -110,16 +111,25 @@ __global__ void __launch_bounds__(kThreads) accept_stats_kernel(const Params p) 
   __shared__ float4 red[kThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (p.T > 0.f) {
+    // all of this thread's values first (independent loads), then max, then the sum
+    constexpr int PER = kChunk / 4 / kThreads;
+    float4 x[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int i = threadIdx.x + u * kThreads;
+      x[u] = i < n4 ? __ldg(row4 + i)
+                    : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
     float m = -INFINITY, s = 0.f;
-    for (int i = threadIdx.x; i < n4; i += kThreads) {
-      const float4 x4 = __ldg(row4 + i);
-      const float a = x4.x / p.T, b = x4.y / p.T, cc = x4.z / p.T, d = x4.w / p.T;
-      const float mx = fmaxf(fmaxf(a, b), fmaxf(cc, d));
-      if (mx > m) {
-        s = s * expf(m - mx);
-        m = mx;
-      }
-      if (m != -INFINITY) s += expf(a - m) + expf(b - m) + expf(cc - m) + expf(d - m);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      x[u] = make_float4(x[u].x / p.T, x[u].y / p.T, x[u].z / p.T, x[u].w / p.T);
+      m = fmaxf(m, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
+    }
+    if (m != -INFINITY) {
+#pragma unroll
+      for (int u = 0; u < PER; ++u)
+        s += (expf(x[u].x - m) + expf(x[u].y - m)) + (expf(x[u].z - m) + expf(x[u].w - m));
     }
     for (int off = 16; off > 0; off >>= 1) {
       const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
@@ -250,8 +260,8 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   const float *zr = p.z + (size_t)rt * p.ld_t;
   const float *yr = resid ? p.y + ((size_t)b * p.k + a) * p.ld_d : nullptr;
   const float mz = s_mz, isz = s_isz, my = resid ? s_my : 0.f, isy = resid ? s_isy : 0.f;
-  const int v0 = c * kChunk;
-  const int v1 = min(p.V, v0 + kChunk);
+  const int v0 = c * kDrawChunk;
+  const int v1 = min(p.V, v0 + kDrawChunk);
   const int n4 = (v1 - v0) >> 2;
   Cand cr{-INFINITY, -INFINITY, -1}, cp{-INFINITY, -INFINITY, -1};
   for (int i = threadIdx.x; i < n4; i += kThreads) {
@@ -298,21 +308,21 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
       tp = cand_merge(tp, Cand{red[0][w].x, red[0][w].z, __float_as_int(red[0][w].y)});
       tr = cand_merge(tr, Cand{red[1][w].x, red[1][w].z, __float_as_int(red[1][w].y)});
     }
-    float4 *slot = p.cand + ((size_t)b * p.nchunks + c) * 2;
+    float4 *slot = p.cand + ((size_t)b * p.ndraw + c) * 2;
     slot[0] = make_float4(tp.g1, __int_as_float(tp.v1), tp.g2, 0.f);
     slot[1] = make_float4(tr.g1, __int_as_float(tr.v1), tr.g2, 0.f);
     __threadfence();
     const unsigned int ticket = atomicAdd(&p.counters[b], 1u);
-    s_last = ticket == (unsigned int)(p.nchunks - 1);
+    s_last = ticket == (unsigned int)(p.ndraw - 1);
   }
   __syncthreads();
   if (!s_last || threadIdx.x != 0) return;
   __threadfence();
   // ---- last CTA of the sequence: merge chunk winners in chunk (token) order
   const volatile float4 *cv = reinterpret_cast<const volatile float4 *>(p.cand) +
-                              (size_t)b * p.nchunks * 2;
+                              (size_t)b * p.ndraw * 2;
   Cand tp{-INFINITY, -INFINITY, -1}, tr{-INFINITY, -INFINITY, -1};
-  for (int cc = 0; cc < p.nchunks; ++cc) {
+  for (int cc = 0; cc < p.ndraw; ++cc) {
     const float4 a0 = make_float4(cv[2 * cc].x, cv[2 * cc].y, cv[2 * cc].z, 0.f);
     const float4 a1 = make_float4(cv[2 * cc + 1].x, cv[2 * cc + 1].y, cv[2 * cc + 1].z, 0.f);
     tp = cand_merge(tp, Cand{a0.x, a0.z, __float_as_int(a0.y)});
@@ -343,12 +353,14 @@ static sd_status validate(const sd_accept_desc *d) {
 }
 
 static int nchunks_of(int V) { return (V + kChunk - 1) / kChunk; }
+static int ndraw_of(int V) { return (V + kDrawChunk - 1) / kDrawChunk; }
 
 static size_t ws_size(const sd_accept_desc *d) {
   if (validate(d) != SD_OK) return 0;
   const size_t nc = nchunks_of(d->vocab);
   const size_t rows = (size_t)d->batch * (d->k + 1) + (size_t)d->batch * d->k;
-  return round_up(rows * nc * 16, 256) + round_up((size_t)d->batch * nc * 32, 256) +
+  return round_up(rows * nc * 16, 256) +
+         round_up((size_t)d->batch * ndraw_of(d->vocab) * 32, 256) +
          round_up((size_t)d->batch * 4, 256);
 }
 
@@ -384,6 +396,7 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.ld_o = desc->ld_out ? desc->ld_out : desc->k + 1;
   p.purpose = desc->purpose;
   p.nchunks = nchunks_of(desc->vocab);
+  p.ndraw = ndraw_of(desc->vocab);
   p.rows_t = p.B * p.n_q;
   p.rows_total = p.rows_t + (sampling ? p.B * p.k : 0);
   p.T = desc->temperature;
@@ -401,13 +414,13 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.stats = reinterpret_cast<float4 *>(w8);
   w8 += round_up(rows * p.nchunks * 16, 256);
   p.cand = reinterpret_cast<float4 *>(w8);
-  w8 += round_up((size_t)p.B * p.nchunks * 32, 256);
+  w8 += round_up((size_t)p.B * p.ndraw * 32, 256);
   p.counters = reinterpret_cast<unsigned int *>(w8);
   p.status = device_status_word();
   cudaStream_t st = (cudaStream_t)stream;
   accept_stats_kernel<<<dim3(p.rows_total, p.nchunks), kThreads, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
-  accept_draw_kernel<<<dim3(p.B, sampling ? p.nchunks : 1), kThreads, 0, st>>>(p);
+  accept_draw_kernel<<<dim3(p.B, sampling ? p.ndraw : 1), kThreads, 0, st>>>(p);
   return cuda_status(cudaGetLastError());
 }
 

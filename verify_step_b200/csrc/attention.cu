@@ -193,10 +193,13 @@ struct Cfg {
   static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + RED_FLOATS * 4 +
                                  16 * STAGES + 16 + 4 * (1 + STAGES) + 64;
+  // two independent tile pipelines per SM where registers allow (one CTA's per-tile chain
+  // of waits, MMAs and the cross-warp score exchange is latency-bound on its own)
+  static constexpr int MIN_CTAS = NCW <= 4 ? 2 : 1;
 };
 
 template <int D, int MT, int STAGES>
-__global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS)
+__global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES>::MIN_CTAS)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const Params p) {
   using C = Cfg<D, MT, STAGES>;
@@ -522,30 +525,39 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS)
 }
 
 // Merges the partials of items that several CTAs shared, in CTA order; writes zero rows for
-// drafter items with an empty key range.
+// drafter items with an empty key range.  One CTA per (item, query row).
 template <typename T>
-__global__ void attn_combine_kernel(const Params p) {
-  const int item = blockIdx.x;
+__global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
+  constexpr int kChunk = 512;
+  __shared__ long long s_F, s_Fl, s_T;
+  __shared__ int s_n;
+  __shared__ float s_w[kChunk];
+  __shared__ float s_red[4];
+  const int item = blockIdx.x, row = blockIdx.y;
   const int b = item / p.Hkv, g = item % p.Hkv;
-  long long pre = 0, T_all = 0;
-  SeqRange sb;
-  for (int bb = 0; bb < p.B; ++bb) {
-    SeqRange s = seq_range(p, bb, threadIdx.x == 0 && bb == b && item % p.Hkv == 0);
-    if (bb == b) sb = s;
-    if (bb < b) pre += (long long)p.Hkv * s.n;
-    T_all += (long long)p.Hkv * s.n;
-  }
-  T *outg = reinterpret_cast<T *>(p.out);
-  if (sb.n == 0) {
-    for (int idx = threadIdx.x; idx < p.M * p.D; idx += blockDim.x) {
-      const int row = idx / p.D, d = idx % p.D;
-      const int j = row / p.G, hh = row % p.G;
-      outg[(((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * p.D + d] = T(0.f);
+  if (threadIdx.x == 0) {
+    long long pre = 0, T_all = 0;
+    int n = 0;
+    for (int bb = 0; bb < p.B; ++bb) {
+      SeqRange sr = seq_range(p, bb, bb == b && g == 0 && row == 0);
+      if (bb == b) n = sr.n;
+      if (bb < b) pre += (long long)p.Hkv * sr.n;
+      T_all += (long long)p.Hkv * sr.n;
     }
+    s_n = n;
+    s_F = pre + (long long)g * n;
+    s_Fl = s_F + n - 1;
+    s_T = T_all;
+  }
+  __syncthreads();
+  const int j = row / p.G, hh = row % p.G;
+  T *dst = reinterpret_cast<T *>(p.out) +
+           (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * p.D;
+  if (s_n == 0) {
+    for (int d = threadIdx.x; d < p.D; d += blockDim.x) dst[d] = T(0.f);
     return;
   }
-  const long long F = pre + (long long)g * sb.n;
-  const long long Fl = F + sb.n - 1;
+  const long long F = s_F, Fl = s_Fl, T_all = s_T;
   const int c_first = (int)(((F + 1) * p.P - 1) / T_all);
   const int c_last = (int)(((Fl + 1) * p.P - 1) / T_all);
   if (c_first == c_last) return;  // written directly by its only CTA
@@ -556,28 +568,65 @@ __global__ void attn_combine_kernel(const Params p) {
     const long long s_c = T_all * c / p.P, e_c = T_all * (c + 1) / p.P;
     return e_c > F && s_c <= Fl && e_c > s_c;
   };
-  for (int idx = threadIdx.x; idx < p.M * p.D; idx += blockDim.x) {
-    const int row = idx / p.D, d = idx % p.D;
-    float mmax = -INFINITY;
-    for (int c = c_first; c <= c_last; ++c)
-      if (holds(c)) mmax = fmaxf(mmax, p.ws_ml[((slot0 + c) * p.Mpad + row) * 2]);
-    float num = 0.f, den = 0.f;
-    if (mmax != -INFINITY) {
-      for (int c = c_first; c <= c_last; ++c) {
-        if (!holds(c)) continue;
-        const size_t sl = (slot0 + c) * p.Mpad + row;
-        const float w = exp2f(p.ws_ml[sl * 2] - mmax);
-        num += w * p.ws_o[sl * p.D + d];
-        den += w * p.ws_ml[sl * 2 + 1];
+  auto block_reduce = [&](float v, bool is_max) {
+    for (int o = 16; o > 0; o >>= 1) {
+      const float u = __shfl_xor_sync(0xffffffffu, v, o);
+      v = is_max ? fmaxf(v, u) : v + u;
+    }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = s_red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = is_max ? fmaxf(r, s_red[w]) : r + s_red[w];
+    return r;
+  };
+  const int S = c_last - c_first + 1;
+  float mloc = -INFINITY;
+  for (int t = threadIdx.x; t < S; t += blockDim.x)
+    if (holds(c_first + t))
+      mloc = fmaxf(mloc, p.ws_ml[((slot0 + c_first + t) * p.Mpad + row) * 2]);
+  const float mmax = block_reduce(mloc, true);
+  float den_loc = 0.f;
+  if (mmax != -INFINITY)
+    for (int t = threadIdx.x; t < S; t += blockDim.x)
+      if (holds(c_first + t)) {
+        const size_t sl = (slot0 + c_first + t) * p.Mpad + row;
+        den_loc += exp2f(p.ws_ml[sl * 2] - mmax) * p.ws_ml[sl * 2 + 1];
+      }
+  const float den = block_reduce(den_loc, false);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  // weighted sum of the partial rows, slots in CTA order, kChunk slots at a time
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // D <= 512 with 128 threads
+  for (int t0 = 0; t0 < S; t0 += kChunk) {
+    const int n = min(kChunk, S - t0);
+    __syncthreads();
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+      const int c = c_first + t0 + t;
+      s_w[t] = (mmax != -INFINITY && holds(c))
+                   ? exp2f(p.ws_ml[((slot0 + c) * p.Mpad + row) * 2] - mmax)
+                   : 0.f;
+    }
+    __syncthreads();
+    for (int t = 0; t < n; ++t) {
+      const float w = s_w[t];
+      if (w == 0.f) continue;
+      const float *o = p.ws_o + ((slot0 + c_first + t0 + t) * p.Mpad + row) * p.D;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int d = threadIdx.x + e * 128;
+        if (d < p.D) acc[e] = fmaf(w, o[d], acc[e]);
       }
     }
-    const int j = row / p.G, hh = row % p.G;
-    outg[(((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * p.D + d] =
-        T(den > 0.f ? num / den : 0.f);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int d = threadIdx.x + e * 128;
+    if (d < p.D) dst[d] = T(acc[e] * inv);
   }
 }
 
-// Writes the n_q new K/V rows of every sequence into the cache (verify only).
+// Writes the n_q new K/V rows of every sequence into the cache (verify only).  The h_kv rows
+// of one position are h_kv * D contiguous elements both in k_new and in the cache block.
 template <typename T>
 __global__ void append_kv_kernel(const Params p, const T *k_new, const T *v_new, T *k_cache,
                                  T *v_cache) {
@@ -595,13 +644,15 @@ __global__ void append_kv_kernel(const Params p, const T *k_new, const T *v_new,
     if (threadIdx.x == 0) record_status(p.status, SD_ERR_DEVICE);
     return;
   }
-  const int n = p.Hkv * p.D;
+  constexpr int E = 16 / sizeof(T);  // elements per 16-byte vector (D is a multiple of E)
+  const int per_head = p.D / E;
+  const int n = p.Hkv * per_head;
   for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
-    const int g = idx / p.D, d = idx % p.D;
-    const size_t src = (((size_t)b * p.n_q + j) * p.Hkv + g) * p.D + d;
-    const size_t dst = (((size_t)blk * p.Hkv + g) * p.bs + pos % p.bs) * p.D + d;
-    k_cache[dst] = k_new[src];
-    v_cache[dst] = v_new[src];
+    const int g = idx / per_head, e = idx % per_head;
+    const size_t src = (((size_t)b * p.n_q + j) * p.Hkv + g) * per_head + e;
+    const size_t dst = (((size_t)blk * p.Hkv + g) * p.bs + pos % p.bs) * per_head + e;
+    reinterpret_cast<uint4 *>(k_cache)[dst] = reinterpret_cast<const uint4 *>(k_new)[src];
+    reinterpret_cast<uint4 *>(v_cache)[dst] = reinterpret_cast<const uint4 *>(v_new)[src];
   }
 }
 
@@ -663,6 +714,9 @@ struct Launcher {
     if (dev < 64 && dev_cache[dev] == dev + 1) return occ_cache[dev];
     cudaFuncSetAttribute(attn_bf16_kernel<D, MT, STAGES>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    cudaFuncSetAttribute(attn_bf16_kernel<D, MT, STAGES>,
+                         cudaFuncAttributePreferredSharedMemoryCarveout,
+                         (int)cudaSharedmemCarveoutMaxShared);
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_bf16_kernel<D, MT, STAGES>,
                                                       C::THREADS, C::SMEM) != cudaSuccess)
@@ -821,7 +875,7 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   }
   s = launch_bf16(p.D, MT, km, vm, p, st);
   if (s != SD_OK) return s;
-  attn_combine_kernel<__nv_bfloat16><<<p.B * p.Hkv, 256, 0, st>>>(p);
+  attn_combine_kernel<__nv_bfloat16><<<dim3(p.B * p.Hkv, p.M), 128, 0, st>>>(p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -260,12 +260,16 @@ __global__ void topc_kernel(const float *scores, int C, int top_c, int32_t *sel)
   }
 }
 
-__global__ void fill_neg_inf_kernel(float *logits, int M, int V, int ld) {
-  const size_t total = (size_t)M * V;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const size_t m = i / V, v = i % V;
-    logits[m * ld + v] = -INFINITY;
+// -inf into rows [m, 0 .. V) of the logits; blockIdx.y = row.
+__global__ void fill_neg_inf_kernel(float *logits, int V, int ld, int vec4) {
+  float *row = logits + (size_t)blockIdx.y * ld;
+  const int stride = gridDim.x * blockDim.x;
+  if (vec4) {
+    float4 *r4 = reinterpret_cast<float4 *>(row);
+    const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < V / 4; i += stride) r4[i] = ninf;
+  } else {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < V; i += stride) row[i] = -INFINITY;
   }
 }
 
@@ -285,22 +289,39 @@ __global__ void cluster_logits_kernel(const __nv_bfloat16 *h, const __nv_bfloat1
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int t = warp; t < cs; t += nw) {
-    const __nv_bfloat16 *wr = w_cm + ((size_t)c * cs + t) * d;
-    float acc = 0.f;
-    for (int k0 = lane * 8; k0 < d; k0 += 256) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(wr + k0);
-      const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+  // four tokens per warp iteration: their weight loads are independent and overlap
+  constexpr int TK = 4;
+  for (int t0 = warp * TK; t0 < cs; t0 += nw * TK) {
+    float acc[TK];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc = fmaf(__bfloat162float(e[q]), hs[k0 + q], acc);
+    for (int u = 0; u < TK; ++u) acc[u] = 0.f;
+    for (int k0 = lane * 8; k0 < d; k0 += 256) {
+      uint4 raw[TK];
+#pragma unroll
+      for (int u = 0; u < TK; ++u)
+        raw[u] = t0 + u < cs ? __ldg(reinterpret_cast<const uint4 *>(
+                                   w_cm + ((size_t)c * cs + t0 + u) * d + k0))
+                             : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < TK; ++u) {
+        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[u]);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[u] = fmaf(__bfloat162float(e[q]), hs[k0 + q], acc[u]);
+      }
     }
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      const int tok = cluster_tokens[(size_t)c * cs + t];
+#pragma unroll
+    for (int u = 0; u < TK; ++u)
+      for (int o = 16; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+    if (lane < TK && t0 + lane < cs) {
+      float mine = acc[0];
+#pragma unroll
+      for (int u = 1; u < TK; ++u)
+        if (lane == u) mine = acc[u];
+      const int tok = cluster_tokens[(size_t)c * cs + t0 + lane];
       if (tok < 0 || tok >= V)
         record_status(status, SD_ERR_DEVICE);
       else
-        logits[(size_t)m * ld + tok] = acc;
+        logits[(size_t)m * ld + tok] = mine;
     }
   }
 }
@@ -433,8 +454,10 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   while (n < C) n <<= 1;
   topc_kernel<<<desc->m, 512, (size_t)n * 8, st>>>(scores, C, desc->top_c, sel_clusters);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
-  const int sms = sm_count();
-  fill_neg_inf_kernel<<<sms > 0 ? 4 * sms : 512, 256, 0, st>>>(logits, desc->m, desc->vocab, ld);
+  const int vec4 = aligned16(logits) && desc->vocab % 4 == 0 && ld % 4 == 0;
+  const int per_row = (desc->vocab / (vec4 ? 4 : 1) + 255) / 256;
+  fill_neg_inf_kernel<<<dim3(per_row < 64 ? per_row : 64, desc->m), 256, 0, st>>>(
+      logits, desc->vocab, ld, vec4);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
   cluster_logits_kernel<<<desc->m * desc->top_c, 256, (size_t)desc->d * 4, st>>>(
       (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
