@@ -121,15 +121,20 @@ __global__ void __launch_bounds__(kThreads) accept_stats_kernel(const Params p) 
                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
     }
     float m = -INFINITY, s = 0.f;
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      x[u] = make_float4(x[u].x / p.T, x[u].y / p.T, x[u].z / p.T, x[u].w / p.T);
-      m = fmaxf(m, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
-    }
-    if (m != -INFINITY) {
+    if (p.T != 1.f) {
 #pragma unroll
       for (int u = 0; u < PER; ++u)
-        s += (expf(x[u].x - m) + expf(x[u].y - m)) + (expf(x[u].z - m) + expf(x[u].w - m));
+        x[u] = make_float4(x[u].x / p.T, x[u].y / p.T, x[u].z / p.T, x[u].w / p.T);
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u)
+      m = fmaxf(m, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
+    if (m != -INFINITY) {
+      constexpr float L2E = 1.4426950408889634f;
+#pragma unroll
+      for (int u = 0; u < PER; ++u)
+        s += (exp2f((x[u].x - m) * L2E) + exp2f((x[u].y - m) * L2E)) +
+             (exp2f((x[u].z - m) * L2E) + exp2f((x[u].w - m) * L2E));
     }
     for (int off = 16; off > 0; off >>= 1) {
       const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
@@ -171,19 +176,26 @@ __global__ void __launch_bounds__(kThreads) accept_stats_kernel(const Params p) 
   }
 }
 
-// Merged statistics of one row: (max, sum) for T > 0; (top1, argmax, top2) for T = 0.
-__device__ __forceinline__ float4 row_stats(const Params &p, int r) {
+// Merged statistics of one row, computed by a full warp (every lane gets the result):
+// (max, sum) for T > 0; (top1, argmax, top2) for T = 0.  The argmax merge breaks ties by the
+// lower token id, so it does not depend on the merge order.
+__device__ __forceinline__ float4 row_stats_warp(const Params &p, int r) {
+  const int lane = threadIdx.x & 31;
   const float4 *st = p.stats + (size_t)r * p.nchunks;
   if (p.T > 0.f) {
-    float M = st[0].x, S = st[0].y;
-    for (int c = 1; c < p.nchunks; ++c) ms_merge(M, S, st[c].x, st[c].y);
+    float M = -INFINITY, S = 0.f;
+    for (int c = lane; c < p.nchunks; c += 32) ms_merge(M, S, st[c].x, st[c].y);
+    for (int off = 16; off > 0; off >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, M, off);
+      const float s2 = __shfl_xor_sync(0xffffffffu, S, off);
+      ms_merge(M, S, m2, s2);
+    }
     return make_float4(M, S, 0.f, 0.f);
   }
-  Cand t{st[0].x, st[0].z, __float_as_int(st[0].y)};
-  for (int c = 1; c < p.nchunks; ++c) {
-    Cand o{st[c].x, st[c].z, __float_as_int(st[c].y)};
-    t = cand_merge(t, o);
-  }
+  Cand t{-INFINITY, -INFINITY, -1};
+  for (int c = lane; c < p.nchunks; c += 32)
+    t = cand_merge(t, Cand{st[c].x, st[c].z, __float_as_int(st[c].y)});
+  for (int off = 16; off > 0; off >>= 1) t = cand_merge(t, cand_shfl(t, off));
   return make_float4(t.g1, __int_as_float(t.v1), t.g2, 0.f);
 }
 
@@ -195,19 +207,23 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   __shared__ float4 red[2][kThreads / 32];
   __shared__ int s_last;
   __shared__ uint32_t s_step;
+  __shared__ float s_top1, s_top2;
+  __shared__ int s_arg;
 
-  if (threadIdx.x == 0) {
-    s_step = (uint32_t)(p.step + (p.step_ptr != nullptr ? *p.step_ptr : 0ull));
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    if (lane == 0) s_step = (uint32_t)(p.step + (p.step_ptr != nullptr ? *p.step_ptr : 0ull));
+    __syncwarp();
     int a = 0, flag = 0;
     for (int i = 1; i <= p.k; ++i) {
       const int d = p.drafts[(size_t)b * p.k + i - 1];
       const int rt = b * p.n_q + i - 1;
+      const float4 sz = row_stats_warp(p, rt);
       bool acc = false;
       if (d < 0 || d >= p.V) {
-        record_status(p.status, SD_ERR_DEVICE);
+        if (lane == 0) record_status(p.status, SD_ERR_DEVICE);
       } else if (p.T > 0.f) {
-        const float4 sz = row_stats(p, rt);
-        const float4 sy = row_stats(p, p.rows_t + b * p.k + i - 1);
+        const float4 sy = row_stats_warp(p, p.rows_t + b * p.k + i - 1);
         const float pd = expf(p.z[(size_t)rt * p.ld_t + d] / p.T - sz.x) / sz.y;
         const float qd =
             expf(p.y[((size_t)b * p.k + i - 1) * p.ld_d + d] / p.T - sy.x) / sy.y;
@@ -216,24 +232,25 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
         if (fabsf(u - ratio) < kMargin) flag = 1;
         acc = u < ratio;
       } else {
-        const float4 sz = row_stats(p, rt);
         if ((sz.x - sz.z) / fmaxf(1.f, fabsf(sz.x)) < kMargin) flag = 1;
         acc = d == __float_as_int(sz.y);
       }
       if (!acc) break;
       ++a;
     }
-    s_a = a;
-    s_flag = flag;
-    if (p.T > 0.f) {
-      const float4 sz = row_stats(p, b * p.n_q + a);
+    const float4 sz = row_stats_warp(p, b * p.n_q + a);
+    float4 sy = make_float4(0.f, 1.f, 0.f, 0.f);
+    if (p.T > 0.f && a < p.k) sy = row_stats_warp(p, p.rows_t + b * p.k + a);
+    if (lane == 0) {
+      s_a = a;
+      s_flag = flag;
       s_mz = sz.x;
       s_isz = 1.f / sz.y;
-      if (a < p.k) {
-        const float4 sy = row_stats(p, p.rows_t + b * p.k + a);
-        s_my = sy.x;
-        s_isy = 1.f / sy.y;
-      }
+      s_my = sy.x;
+      s_isy = 1.f / sy.y;
+      s_top1 = sz.x;
+      s_arg = __float_as_int(sz.y);
+      s_top2 = sz.z;
     }
   }
   __syncthreads();
@@ -242,12 +259,11 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
 
   if (p.T == 0.f) {  // greedy: one CTA per sequence, no race
     if (threadIdx.x == 0) {
-      const float4 sz = row_stats(p, b * p.n_q + a);
       int flag = s_flag;
-      if ((sz.x - sz.z) / fmaxf(1.f, fabsf(sz.x)) < kMargin) flag = 1;
+      if ((s_top1 - s_top2) / fmaxf(1.f, fabsf(s_top1)) < kMargin) flag = 1;
       int32_t *o = p.out + (size_t)b * p.ld_o;
       for (int j = 0; j < p.n_q; ++j)
-        o[j] = j < a ? p.drafts[(size_t)b * p.k + j] : (j == a ? __float_as_int(sz.y) : -1);
+        o[j] = j < a ? p.drafts[(size_t)b * p.k + j] : (j == a ? s_arg : -1);
       p.n_acc[b] = a;
       if (p.margin) p.margin[b] = flag;
     }
@@ -316,18 +332,25 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
     s_last = ticket == (unsigned int)(p.ndraw - 1);
   }
   __syncthreads();
-  if (!s_last || threadIdx.x != 0) return;
+  if (!s_last) return;
   __threadfence();
-  // ---- last CTA of the sequence: merge chunk winners in chunk (token) order
+  // ---- last CTA of the sequence: merge the chunk winners (order-independent: ties go to the
+  // lower token id), one warp
+  if (threadIdx.x >= 32) return;
   const volatile float4 *cv = reinterpret_cast<const volatile float4 *>(p.cand) +
                               (size_t)b * p.ndraw * 2;
   Cand tp{-INFINITY, -INFINITY, -1}, tr{-INFINITY, -INFINITY, -1};
-  for (int cc = 0; cc < p.ndraw; ++cc) {
-    const float4 a0 = make_float4(cv[2 * cc].x, cv[2 * cc].y, cv[2 * cc].z, 0.f);
-    const float4 a1 = make_float4(cv[2 * cc + 1].x, cv[2 * cc + 1].y, cv[2 * cc + 1].z, 0.f);
-    tp = cand_merge(tp, Cand{a0.x, a0.z, __float_as_int(a0.y)});
-    tr = cand_merge(tr, Cand{a1.x, a1.z, __float_as_int(a1.y)});
+  for (int cc = lane; cc < p.ndraw; cc += 32) {
+    const float a0x = cv[2 * cc].x, a0y = cv[2 * cc].y, a0z = cv[2 * cc].z;
+    const float a1x = cv[2 * cc + 1].x, a1y = cv[2 * cc + 1].y, a1z = cv[2 * cc + 1].z;
+    tp = cand_merge(tp, Cand{a0x, a0z, __float_as_int(a0y)});
+    tr = cand_merge(tr, Cand{a1x, a1z, __float_as_int(a1y)});
   }
+  for (int off = 16; off > 0; off >>= 1) {
+    tp = cand_merge(tp, cand_shfl(tp, off));
+    tr = cand_merge(tr, cand_shfl(tr, off));
+  }
+  if (lane != 0) return;
   const Cand &w = (resid && tr.v1 >= 0 && tr.g1 > -INFINITY) ? tr : tp;
   int flag = s_flag;
   if (w.g1 - w.g2 < kMargin) flag = 1;

@@ -116,7 +116,50 @@ __device__ __forceinline__ void row_range(const Params &p, const SeqRange &s, in
   }
 }
 
-__device__ __forceinline__ long long total_tiles(const Params &p) {
+// Per-sequence ranges cached in shared memory for batches up to kTabB (built once per CTA by
+// one warp); larger batches recompute them from global memory.
+constexpr int kTabB = 64;
+
+struct SeqTab {
+  SeqRange r[kTabB];
+  long long pre[kTabB + 1];  // pre[b] = tiles of sequences before b (times h_kv)
+  int ok;
+};
+
+__device__ __forceinline__ void build_tab(const Params &p, SeqTab *t) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  if (p.B > kTabB) {
+    if (lane == 0) t->ok = 0;
+    return;
+  }
+  long long carry = 0;
+  for (int base = 0; base < p.B; base += 32) {
+    const int b = base + lane;
+    long long v = 0;
+    if (b < p.B) {
+      t->r[b] = seq_range(p, b, false);
+      v = (long long)p.Hkv * t->r[b].n;
+    }
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    if (b < p.B) t->pre[b + 1] = carry + v;
+    carry += __shfl_sync(0xffffffffu, v, 31);
+  }
+  if (lane == 0) {
+    t->pre[0] = 0;
+    t->ok = 1;
+  }
+}
+
+__device__ __forceinline__ SeqRange tab_range(const Params &p, const SeqTab *t, int b) {
+  return t->ok ? t->r[b] : seq_range(p, b, false);
+}
+
+__device__ __forceinline__ long long total_tiles(const Params &p, const SeqTab *t) {
+  if (t->ok) return t->pre[p.B];
   long long T = 0;
   for (int b = 0; b < p.B; ++b) T += (long long)p.Hkv * seq_range(p, b, false).n;
   return T;
@@ -127,20 +170,19 @@ struct Cursor {
   int b, g, tau;         // current item and tile index inside it
   SeqRange s;            // range of sequence b
   long long left;        // tiles still to process by this CTA
-  long long item_first;  // flattened index of tile 0 of the current item
 };
 
-__device__ __forceinline__ void cursor_begin(const Params &p, long long start, long long count,
-                                             Cursor &c) {
+__device__ __forceinline__ void cursor_begin(const Params &p, const SeqTab *t, long long start,
+                                             long long count, Cursor &c) {
   c.left = count;
   long long pre = 0;
   c.b = 0;
   c.g = 0;
   c.tau = 0;
-  c.s = seq_range(p, 0, false);
+  c.s = tab_range(p, t, 0);
   if (count <= 0) return;
   for (int b = 0; b < p.B; ++b) {
-    SeqRange s = seq_range(p, b, false);
+    SeqRange s = tab_range(p, t, b);
     const long long len = (long long)p.Hkv * s.n;
     if (start < pre + len) {
       c.b = b;
@@ -148,7 +190,6 @@ __device__ __forceinline__ void cursor_begin(const Params &p, long long start, l
       const long long off = start - pre;
       c.g = (int)(off / s.n);
       c.tau = (int)(off % s.n);
-      c.item_first = pre + (long long)c.g * s.n;
       return;
     }
     pre += len;
@@ -157,13 +198,12 @@ __device__ __forceinline__ void cursor_begin(const Params &p, long long start, l
 }
 
 // Advances to the next item after the current one finished (tau == n).
-__device__ __forceinline__ void cursor_next_item(const Params &p, Cursor &c) {
-  c.item_first += c.s.n;
+__device__ __forceinline__ void cursor_next_item(const Params &p, const SeqTab *t, Cursor &c) {
   c.tau = 0;
   if (++c.g < p.Hkv) return;
   c.g = 0;
   for (int b = c.b + 1; b < p.B; ++b) {
-    SeqRange s = seq_range(p, b, false);
+    SeqRange s = tab_range(p, t, b);
     if (s.n > 0) {
       c.b = b;
       c.s = s;
@@ -192,7 +232,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + RED_FLOATS * 4 +
-                                 16 * STAGES + 16 + 4 * (1 + STAGES) + 64;
+                                 16 * STAGES + 16 + 4 * (1 + STAGES) + 64 + sizeof(SeqTab) + 16;
   // two independent tile pipelines per SM where registers allow (one CTA's per-tile chain
   // of waits, MMAs and the cross-warp score exchange is latency-bound on its own)
   static constexpr int MIN_CTAS = NCW <= 4 ? 2 : 1;
@@ -214,6 +254,8 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   uint64_t *red_bar = empty + STAGES;  // [2]: partial scores of a tile are in red[buf]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(red_bar + 2);
   volatile int *bad = abort_flag + 1;
+  SeqTab *tab = reinterpret_cast<SeqTab *>(
+      (reinterpret_cast<uintptr_t>(bad + STAGES) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -227,9 +269,10 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     *abort_flag = 0;
     fence_mbar_init();
   }
+  build_tab(p, tab);
   __syncthreads();
 
-  const long long T = total_tiles(p);
+  const long long T = total_tiles(p, tab);
   const long long start = T * blockIdx.x / p.P;
   const long long end = T * (blockIdx.x + 1) / p.P;
 
@@ -239,7 +282,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
     Cursor c;
-    cursor_begin(p, start, end - start, c);
+    cursor_begin(p, tab, start, end - start, c);
     uint32_t it = 0;
     while (c.left > 0) {
       const int stage = it % STAGES;
@@ -271,7 +314,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
       }
       ++it;
       --c.left;
-      if (++c.tau == c.s.n && c.left > 0) cursor_next_item(p, c);
+      if (++c.tau == c.s.n && c.left > 0) cursor_next_item(p, tab, c);
     }
     if (*abort_flag) {
       // wait (bounded) for the copies this CTA issued before leaving
@@ -288,7 +331,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(p.q);
 
   Cursor c;
-  cursor_begin(p, start, end - start, c);
+  cursor_begin(p, tab, start, end - start, c);
   uint32_t it = 0;
   int buf = 0;
   bool ok = true;
@@ -520,7 +563,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     }
     c.tau += seg_n;
     c.left -= seg_n;
-    if (c.left > 0) cursor_next_item(p, c);
+    if (c.left > 0) cursor_next_item(p, tab, c);
   }
 }
 
@@ -535,19 +578,26 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
   __shared__ float s_red[4];
   const int item = blockIdx.x, row = blockIdx.y;
   const int b = item / p.Hkv, g = item % p.Hkv;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {  // tile counts of all sequences, one warp
     long long pre = 0, T_all = 0;
     int n = 0;
-    for (int bb = 0; bb < p.B; ++bb) {
+    for (int bb = threadIdx.x; bb < p.B; bb += 32) {
       SeqRange sr = seq_range(p, bb, bb == b && g == 0 && row == 0);
       if (bb == b) n = sr.n;
       if (bb < b) pre += (long long)p.Hkv * sr.n;
       T_all += (long long)p.Hkv * sr.n;
     }
-    s_n = n;
-    s_F = pre + (long long)g * n;
-    s_Fl = s_F + n - 1;
-    s_T = T_all;
+    for (int o = 16; o > 0; o >>= 1) {
+      pre += __shfl_xor_sync(0xffffffffu, pre, o);
+      T_all += __shfl_xor_sync(0xffffffffu, T_all, o);
+      n += __shfl_xor_sync(0xffffffffu, n, o);
+    }
+    if (threadIdx.x == 0) {
+      s_n = n;
+      s_F = pre + (long long)g * n;
+      s_Fl = s_F + n - 1;
+      s_T = T_all;
+    }
   }
   __syncthreads();
   const int j = row / p.G, hh = row % p.G;
