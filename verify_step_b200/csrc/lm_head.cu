@@ -217,6 +217,43 @@ __global__ void lm_head_f32_kernel(const float *h, const float *w, const Params 
 
 // Per row: the top_c clusters by score (ties -> lower id), written in ascending id order.
 // Bitonic sort of (descending score, ascending id) keys in shared memory.
+__device__ __forceinline__ unsigned long long topc_key(float score, int id) {
+  uint32_t u = __float_as_uint(score);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);         // ascending order of floats
+  return ((unsigned long long)(~u) << 32) | (uint32_t)id;  // descending score, then id
+}
+
+// Same selection for n_pow2 <= 1024 clusters: one key per thread, bitonic sort with warp
+// shuffles for strides below 32 and shared memory above.
+__global__ void topc_small_kernel(const float *scores, int C, int top_c, int32_t *sel) {
+  __shared__ unsigned long long sk[1024];
+  const int m = blockIdx.x, i = threadIdx.x, n = blockDim.x;
+  unsigned long long key = i < C ? topc_key(scores[(size_t)m * C + i], i) : ~0ull;
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      unsigned long long other;
+      if (stride >= 32) {
+        sk[i] = key;
+        __syncthreads();
+        other = sk[i ^ stride];
+        __syncthreads();
+      } else {
+        other = __shfl_xor_sync(0xffffffffu, key, stride);
+      }
+      const bool up = (i & size) == 0, lower = (i & stride) == 0;
+      key = (lower == up) ? (key < other ? key : other) : (key < other ? other : key);
+    }
+  }
+  sk[i] = key;
+  __syncthreads();
+  if (i < top_c) {
+    const int id = (int)(key & 0xFFFFFFFFu);
+    int rank = 0;
+    for (int u = 0; u < top_c; ++u) rank += (int)(sk[u] & 0xFFFFFFFFu) < id;
+    sel[(size_t)m * top_c + rank] = id;
+  }
+}
+
 __global__ void topc_kernel(const float *scores, int C, int top_c, int32_t *sel) {
   extern __shared__ unsigned long long keys[];
   const int m = blockIdx.x;
@@ -273,13 +310,18 @@ __global__ void fill_neg_inf_kernel(float *logits, int V, int ld, int vec4) {
   }
 }
 
-// One CTA per (row m, kept cluster slot): exact logits of the cluster's tokens.
-__global__ void cluster_logits_kernel(const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm,
-                                      const int32_t *cluster_tokens, const int32_t *sel,
-                                      int top_c, int cs, int d, int C, int V, int ld,
-                                      float *logits, int *status) {
+// Exact logits of the kept clusters' tokens: CTA (m, slot, part) takes tokens
+// [part * tpc, (part+1) * tpc) of cluster sel[m, slot]; each warp takes TK tokens at a time
+// with all their weight loads in flight (d <= 256 * KMAX) before the dot products.
+template <int KMAX>
+__global__ void __launch_bounds__(256) cluster_logits_kernel(
+    const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm, const int32_t *cluster_tokens,
+    const int32_t *sel, int top_c, int cs, int d, int C, int V, int ld, int parts, float *logits,
+    int *status) {
   extern __shared__ float hs[];
-  const int m = blockIdx.x / top_c, slot = blockIdx.x % top_c;
+  const int part = blockIdx.x % parts;
+  const int ms = blockIdx.x / parts;
+  const int m = ms / top_c, slot = ms % top_c;
   const int c = sel[(size_t)m * top_c + slot];
   for (int i = threadIdx.x; i < d; i += blockDim.x)
     hs[i] = __bfloat162float(h[(size_t)m * d + i]);
@@ -288,31 +330,41 @@ __global__ void cluster_logits_kernel(const __nv_bfloat16 *h, const __nv_bfloat1
     if (threadIdx.x == 0) record_status(status, SD_ERR_DEVICE);
     return;
   }
+  const int tpc = (cs + parts - 1) / parts;
+  const int t_begin = part * tpc, t_end = min(cs, t_begin + tpc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  // four tokens per warp iteration: their weight loads are independent and overlap
   constexpr int TK = 4;
-  for (int t0 = warp * TK; t0 < cs; t0 += nw * TK) {
+  const int nk = (d + 255) / 256;  // 256 elements per warp-wide 16-byte load
+  for (int t0 = t_begin + warp * TK; t0 < t_end; t0 += nw * TK) {
+    uint4 raw[TK][KMAX];
+#pragma unroll
+    for (int u = 0; u < TK; ++u)
+#pragma unroll
+      for (int q = 0; q < KMAX; ++q) {
+        const int k0 = lane * 8 + q * 256;
+        raw[u][q] = (q < nk && k0 < d && t0 + u < t_end)
+                        ? __ldg(reinterpret_cast<const uint4 *>(
+                              w_cm + ((size_t)c * cs + t0 + u) * d + k0))
+                        : make_uint4(0, 0, 0, 0);
+      }
     float acc[TK];
 #pragma unroll
-    for (int u = 0; u < TK; ++u) acc[u] = 0.f;
-    for (int k0 = lane * 8; k0 < d; k0 += 256) {
-      uint4 raw[TK];
+    for (int u = 0; u < TK; ++u) {
+      acc[u] = 0.f;
 #pragma unroll
-      for (int u = 0; u < TK; ++u)
-        raw[u] = t0 + u < cs ? __ldg(reinterpret_cast<const uint4 *>(
-                                   w_cm + ((size_t)c * cs + t0 + u) * d + k0))
-                             : make_uint4(0, 0, 0, 0);
+      for (int q = 0; q < KMAX; ++q) {
+        const int k0 = lane * 8 + q * 256;
+        if (q < nk && k0 < d) {
+          const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][q]);
 #pragma unroll
-      for (int u = 0; u < TK; ++u) {
-        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[u]);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[u] = fmaf(__bfloat162float(e[q]), hs[k0 + q], acc[u]);
+          for (int r = 0; r < 8; ++r) acc[u] = fmaf(__bfloat162float(e[r]), hs[k0 + r], acc[u]);
+        }
       }
     }
 #pragma unroll
     for (int u = 0; u < TK; ++u)
       for (int o = 16; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
-    if (lane < TK && t0 + lane < cs) {
+    if (lane < TK && t0 + lane < t_end) {
       float mine = acc[0];
 #pragma unroll
       for (int u = 1; u < TK; ++u)
@@ -386,7 +438,7 @@ static sd_status validate(const sd_head_desc *d) {
     if (d->n_clusters < 1 || d->cluster_size < 1 ||
         (long long)d->n_clusters * d->cluster_size != d->vocab || d->top_c > d->n_clusters)
       return SD_ERR_INVALID_ARG;
-    if (d->top_c > 64 || d->n_clusters > 8192) return SD_ERR_UNSUPPORTED;
+    if (d->top_c > 64 || d->n_clusters > 8192 || d->d > 4096) return SD_ERR_UNSUPPORTED;
   }
   if (d->dtype == SD_BF16 && d->d % 64) return SD_ERR_UNSUPPORTED;
   if (d->dtype == SD_BF16 && (long long)d->vocab >= (1ll << 31)) return SD_ERR_UNSUPPORTED;
@@ -452,17 +504,35 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   }
   int n = 1;
   while (n < C) n <<= 1;
-  topc_kernel<<<desc->m, 512, (size_t)n * 8, st>>>(scores, C, desc->top_c, sel_clusters);
+  if (n < 32) n = 32;
+  if (n <= 1024)
+    topc_small_kernel<<<desc->m, n, 0, st>>>(scores, C, desc->top_c, sel_clusters);
+  else
+    topc_kernel<<<desc->m, 512, (size_t)n * 8, st>>>(scores, C, desc->top_c, sel_clusters);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
   const int vec4 = aligned16(logits) && desc->vocab % 4 == 0 && ld % 4 == 0;
   const int per_row = (desc->vocab / (vec4 ? 4 : 1) + 255) / 256;
   fill_neg_inf_kernel<<<dim3(per_row < 64 ? per_row : 64, desc->m), 256, 0, st>>>(
       logits, desc->vocab, ld, vec4);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
-  cluster_logits_kernel<<<desc->m * desc->top_c, 256, (size_t)desc->d * 4, st>>>(
-      (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
-      desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
-      device_status_word());
+  // enough CTAs to keep every SM streaming: split a cluster's tokens over `parts` CTAs
+  const int sms = sm_count();
+  int parts = 1;
+  while (parts < 8 && (long long)desc->m * desc->top_c * parts < 4ll * (sms > 0 ? sms : 148) &&
+         desc->cluster_size / (parts * 2) >= 32)
+    parts *= 2;
+  const dim3 grid(desc->m * desc->top_c * parts);
+  const size_t shm = (size_t)desc->d * 4;
+  if (desc->d <= 1024)
+    cluster_logits_kernel<4><<<grid, 256, shm, st>>>(
+        (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
+        desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, parts, logits,
+        device_status_word());
+  else
+    cluster_logits_kernel<16><<<grid, 256, shm, st>>>(
+        (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
+        desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, parts, logits,
+        device_status_word());
   return cuda_status(cudaGetLastError());
 }
 
