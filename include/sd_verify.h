@@ -19,7 +19,9 @@
  *   - Every data pointer is a caller-owned DEVICE buffer, densely packed in the layout
  *     stated for it (row-major, last index fastest).  Descriptors are HOST structs read
  *     during the call only.  The library allocates no device memory; scratch space is the
- *     caller's workspace (ws, ws_bytes), sized by the matching *_workspace_size call.
+ *     caller's workspace (ws, ws_bytes), sized by the matching *_workspace_size call.  A
+ *     workspace needs no initialisation and carries nothing from one call to the next, so
+ *     calls that share one must not overlap on the GPU.
  *   - Calls are stream-ordered and return after enqueueing; results are valid once the
  *     stream has reached them.  The library keeps no state between calls except a
  *     per-device status word (sd_device_status_read).
