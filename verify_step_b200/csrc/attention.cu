@@ -601,7 +601,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     }
     if (!ok) break;
 
-    // ---- segment end: final rows or a partial for the combine kernel
+    // ---- segment end: final rows, or a partial merged by the last CTA of the item
     float l_tot[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
