@@ -20,10 +20,8 @@
 //    are summed through shared memory (fixed order, so every warp of a row tile gets the same
 //    scores); the online softmax and P V run in registers on bf16 mma.sync tensor cores with
 //    float32 accumulation.
-//  * Items split across CTAs leave (m, l, o) partials in the workspace and arrive on a per-item
-//    counter; the CTA whose arrival completes the item merges the partials (slots summed in CTA
-//    order, so the result does not depend on arrival order).  No CTA ever waits for another.
-//    Items one CTA finishes are written directly.
+//  * Items split across CTAs leave (m, l, o) partials in the workspace; a combine kernel merges
+//    them in CTA order (deterministic).  Items one CTA finishes are written directly.
 //
 // float32 path: one warp per query row, plain FMA (the tiny float32 configuration).
 #include <cfloat>
@@ -49,7 +47,6 @@ struct Params {
   void *out;
   float *ws_o;   // [slots][Mpad][D]
   float *ws_ml;  // [slots][Mpad][2]
-  int *counters; // [B * Hkv] partials arrived per item (zero between launches)
   int P;         // CTAs of the persistent grid
   int *status;
 };
@@ -173,7 +170,6 @@ struct Cursor {
   int b, g, tau;         // current item and tile index inside it
   SeqRange s;            // range of sequence b
   long long left;        // tiles still to process by this CTA
-  long long item_first;  // flattened index of tile 0 of the current item
 };
 
 __device__ __forceinline__ void cursor_begin(const Params &p, const SeqTab *t, long long start,
@@ -194,7 +190,6 @@ __device__ __forceinline__ void cursor_begin(const Params &p, const SeqTab *t, l
       const long long off = start - pre;
       c.g = (int)(off / s.n);
       c.tau = (int)(off % s.n);
-      c.item_first = pre + (long long)c.g * s.n;
       return;
     }
     pre += len;
@@ -204,7 +199,6 @@ __device__ __forceinline__ void cursor_begin(const Params &p, const SeqTab *t, l
 
 // Advances to the next item after the current one finished (tau == n).
 __device__ __forceinline__ void cursor_next_item(const Params &p, const SeqTab *t, Cursor &c) {
-  c.item_first += c.s.n;
   c.tau = 0;
   if (++c.g < p.Hkv) return;
   c.g = 0;
@@ -217,63 +211,6 @@ __device__ __forceinline__ void cursor_next_item(const Params &p, const SeqTab *
     }
   }
   c.left = 0;
-}
-
-// CTA c of the persistent grid holds tiles [T*c/P, T*(c+1)/P) of the flattened list.  The CTAs
-// that hold tiles of an item whose tiles are [F, Fl] form the range [c_first, c_last]; with
-// fewer tiles than CTAs some CTAs inside that range hold none.
-__device__ __forceinline__ bool cta_holds(long long T, int P, int c, long long F, long long Fl) {
-  const long long s_c = T * c / P, e_c = T * (c + 1) / P;
-  return e_c > F && s_c <= Fl && e_c > s_c;
-}
-
-// Merges the partials of item (b, g) left by the CTAs that held its tiles, in any order of
-// arrival (the sums run over the slots in CTA order).  Called by the last CTA to arrive; the
-// rows are spread over the compute warps.
-template <int D, int NCW>
-__device__ __forceinline__ void merge_item(const Params &p, int b, int g, long long T,
-                                           long long F, long long Fl, int warp, int lane) {
-  const int c_first = (int)(((F + 1) * p.P - 1) / T);
-  const int c_last = (int)(((Fl + 1) * p.P - 1) / T);
-  const int S = c_last - c_first + 1;
-  const size_t slot0 = (size_t)b * p.Hkv + g;
-  for (int row = warp; row < p.M; row += NCW) {
-    float mmax = -INFINITY;
-    for (int t0 = 0; t0 < S; t0 += 32) {
-      const int c = c_first + t0 + lane;
-      if (t0 + lane < S && cta_holds(T, p.P, c, F, Fl))
-        mmax = fmaxf(mmax, __ldcg(p.ws_ml + ((slot0 + c) * p.Mpad + row) * 2));
-    }
-    for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
-    float den = 0.f;
-    float acc[D / 32];
-#pragma unroll
-    for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
-    for (int t0 = 0; t0 < S; t0 += 32) {
-      const int c = c_first + t0 + lane;
-      float w = 0.f;
-      if (mmax != -INFINITY && t0 + lane < S && cta_holds(T, p.P, c, F, Fl)) {
-        const size_t sl = (slot0 + c) * p.Mpad + row;
-        w = exp2f(__ldcg(p.ws_ml + sl * 2) - mmax);
-        den += w * __ldcg(p.ws_ml + sl * 2 + 1);
-      }
-      const int n = min(32, S - t0);
-      for (int u = 0; u < n; ++u) {
-        const float wu = __shfl_sync(0xffffffffu, w, u);
-        if (wu == 0.f) continue;
-        const float *o = p.ws_o + ((slot0 + c_first + t0 + u) * p.Mpad + row) * D;
-#pragma unroll
-        for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(wu, __ldcg(o + lane + 32 * e), acc[e]);
-      }
-    }
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    const int j = row / p.G, hh = row % p.G;
-    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) +
-                         (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D;
-#pragma unroll
-    for (int e = 0; e < D / 32; ++e) dst[lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
-  }
 }
 
 // Byte offset of element (row, col) inside a [16 rows x D] bf16 tile stored as D/64 chunks of
@@ -295,7 +232,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + RED_FLOATS * 4 +
-                                 16 * STAGES + 24 + 4 * (2 + STAGES) + 64 + sizeof(SeqTab) + 16;
+                                 16 * STAGES + 16 + 4 * (1 + STAGES) + 64 + sizeof(SeqTab) + 16;
   // two independent tile pipelines per SM where registers allow (one CTA's per-tile chain
   // of waits, MMAs and the cross-warp score exchange is latency-bound on its own)
   static constexpr int MIN_CTAS = NCW <= 4 ? 2 : 1;
@@ -315,12 +252,10 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   uint64_t *full = reinterpret_cast<uint64_t *>(red + C::RED_FLOATS);
   uint64_t *empty = full + STAGES;
   uint64_t *red_bar = empty + STAGES;  // [2]: partial scores of a tile are in red[buf]
-  uint64_t *seg_bar = red_bar + 2;     // compute warps at a segment end
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(seg_bar + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(red_bar + 2);
   volatile int *bad = abort_flag + 1;
-  volatile int *merge_flag = bad + STAGES;
   SeqTab *tab = reinterpret_cast<SeqTab *>(
-      (reinterpret_cast<uintptr_t>(merge_flag + 1) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(bad + STAGES) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -331,7 +266,6 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     }
     mbar_init(&red_bar[0], NCW * 32);
     mbar_init(&red_bar[1], NCW * 32);
-    mbar_init(seg_bar, NCW * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -339,19 +273,6 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   __syncthreads();
 
   const long long T = total_tiles(p, tab);
-  if (p.is_draft && blockIdx.x == 0 && warp == 0) {
-    // drafter items whose key range is empty get zero rows (no CTA visits them)
-    for (int b = 0; b < p.B; ++b) {
-      if (tab_range(p, tab, b).n != 0) continue;
-      for (int idx = lane; idx < p.Hkv * p.M * D; idx += 32) {
-        const int g = idx / (p.M * D), row = (idx / D) % p.M, d = idx % D;
-        const int j = row / p.G, hh = row % p.G;
-        reinterpret_cast<__nv_bfloat16 *>(p.out)[(((size_t)b * p.n_q + j) * p.Hq +
-                                                   (size_t)g * p.G + hh) * D + d] =
-            __float2bfloat16_rn(0.f);
-      }
-    }
-  }
   const long long start = T * blockIdx.x / p.P;
   const long long end = T * (blockIdx.x + 1) / p.P;
 
@@ -413,7 +334,6 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   cursor_begin(p, tab, start, end - start, c);
   uint32_t it = 0;
   int buf = 0;
-  uint32_t seg_phase = 0;
   bool ok = true;
   while (c.left > 0 && ok) {
     // ---- segment setup: item (c.b, c.g), tiles [c.tau, seg_end)
@@ -601,7 +521,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     }
     if (!ok) break;
 
-    // ---- segment end: final rows, or a partial merged by the last CTA of the item
+    // ---- segment end: final rows or a partial for the combine kernel
     float l_tot[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -640,38 +560,128 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
           p.ws_ml[(slot * p.Mpad + row) * 2 + 1] = l_tot[h];
         }
       }
-      // publish this CTA's partial, then one arrival on the item's counter; the CTA that
-      // brings the count to the number of contributors merges the item (no waiting)
-      __threadfence();
-      mbar_arrive(seg_bar);
-      bool ok2 = mbar_wait(seg_bar, seg_phase & 1, abort_flag);
-      ++seg_phase;
-      const long long F = c.item_first, Fl = F + c.s.n - 1;
-      if (ok2 && warp == 0 && lane == 0) {
-        const int c_first = (int)(((F + 1) * p.P - 1) / T);
-        const int c_last = (int)(((Fl + 1) * p.P - 1) / T);
-        int contributors = 0;
-        for (int cc = c_first; cc <= c_last; ++cc) contributors += cta_holds(T, p.P, cc, F, Fl);
-        const int ticket = atomicAdd(&p.counters[(size_t)b * p.Hkv + g], 1);
-        *merge_flag = ticket == contributors - 1;
-      }
-      mbar_arrive(seg_bar);
-      ok2 = ok2 && mbar_wait(seg_bar, seg_phase & 1, abort_flag);
-      ++seg_phase;
-      if (!ok2) {
-        record_status(p.status, SD_ERR_TIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
-      if (*merge_flag) {
-        __threadfence();
-        merge_item<D, NCW>(p, b, g, T, F, Fl, warp, lane);
-        if (warp == 0 && lane == 0) p.counters[(size_t)b * p.Hkv + g] = 0;
-      }
     }
     c.tau += seg_n;
     c.left -= seg_n;
     if (c.left > 0) cursor_next_item(p, tab, c);
+  }
+}
+
+// Merges the partials of items that several CTAs shared, in CTA order; writes zero rows for
+// drafter items with an empty key range.  One CTA per (item, query row).
+template <typename T>
+__global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
+  constexpr int kChunk = 512;
+  __shared__ long long s_F, s_Fl, s_T;
+  __shared__ int s_n;
+  __shared__ float s_w[kChunk];
+  __shared__ float s_red[4];
+  const int item = blockIdx.x, row = blockIdx.y;
+  const int b = item / p.Hkv, g = item % p.Hkv;
+  if (threadIdx.x < 32) {  // tile counts of all sequences, one warp
+    long long pre = 0, T_all = 0;
+    int n = 0;
+    for (int bb = threadIdx.x; bb < p.B; bb += 32) {
+      SeqRange sr = seq_range(p, bb, bb == b && g == 0 && row == 0);
+      if (bb == b) n = sr.n;
+      if (bb < b) pre += (long long)p.Hkv * sr.n;
+      T_all += (long long)p.Hkv * sr.n;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      pre += __shfl_xor_sync(0xffffffffu, pre, o);
+      T_all += __shfl_xor_sync(0xffffffffu, T_all, o);
+      n += __shfl_xor_sync(0xffffffffu, n, o);
+    }
+    if (threadIdx.x == 0) {
+      s_n = n;
+      s_F = pre + (long long)g * n;
+      s_Fl = s_F + n - 1;
+      s_T = T_all;
+    }
+  }
+  __syncthreads();
+  const int j = row / p.G, hh = row % p.G;
+  T *dst = reinterpret_cast<T *>(p.out) +
+           (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * p.D;
+  if (s_n == 0) {
+    for (int d = threadIdx.x; d < p.D; d += blockDim.x) dst[d] = T(0.f);
+    return;
+  }
+  const long long F = s_F, Fl = s_Fl, T_all = s_T;
+  const int c_first = (int)(((F + 1) * p.P - 1) / T_all);
+  const int c_last = (int)(((Fl + 1) * p.P - 1) / T_all);
+  if (c_first == c_last) return;  // written directly by its only CTA
+  const size_t slot0 = (size_t)b * p.Hkv + g;
+  // CTA c holds tiles [T*c/P, T*(c+1)/P); with fewer tiles than CTAs some hold none and
+  // wrote no partial for this item.
+  auto holds = [&](int c) {
+    const long long s_c = T_all * c / p.P, e_c = T_all * (c + 1) / p.P;
+    return e_c > F && s_c <= Fl && e_c > s_c;
+  };
+  auto block_reduce = [&](float v, bool is_max) {
+    for (int o = 16; o > 0; o >>= 1) {
+      const float u = __shfl_xor_sync(0xffffffffu, v, o);
+      v = is_max ? fmaxf(v, u) : v + u;
+    }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = s_red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = is_max ? fmaxf(r, s_red[w]) : r + s_red[w];
+    return r;
+  };
+  const int S = c_last - c_first + 1;
+  float mloc = -INFINITY;
+  for (int t = threadIdx.x; t < S; t += blockDim.x)
+    if (holds(c_first + t))
+      mloc = fmaxf(mloc, p.ws_ml[((slot0 + c_first + t) * p.Mpad + row) * 2]);
+  const float mmax = block_reduce(mloc, true);
+  float den_loc = 0.f;
+  if (mmax != -INFINITY)
+    for (int t = threadIdx.x; t < S; t += blockDim.x)
+      if (holds(c_first + t)) {
+        const size_t sl = (slot0 + c_first + t) * p.Mpad + row;
+        den_loc += exp2f(p.ws_ml[sl * 2] - mmax) * p.ws_ml[sl * 2 + 1];
+      }
+  const float den = block_reduce(den_loc, false);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  // weighted sum of the partial rows, slots in CTA order, kChunk slots at a time; the loads
+  // of 8 slots are issued before their multiply-adds (they are independent L2 reads)
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // D <= 512 with 128 threads
+  for (int t0 = 0; t0 < S; t0 += kChunk) {
+    const int n = min(kChunk, S - t0);
+    __syncthreads();
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+      const int c = c_first + t0 + t;
+      s_w[t] = (mmax != -INFINITY && holds(c))
+                   ? exp2f(p.ws_ml[((slot0 + c) * p.Mpad + row) * 2] - mmax)
+                   : 0.f;
+    }
+    __syncthreads();
+    for (int u0 = 0; u0 < n; u0 += 8) {
+      float v[8][4];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = u0 + u < n ? s_w[u0 + u] : 0.f;
+        const float *o = p.ws_o + ((slot0 + c_first + t0 + u0 + u) * p.Mpad + row) * p.D;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int d = threadIdx.x + e * 128;
+          v[u][e] = (w != 0.f && d < p.D) ? __ldcg(o + d) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = u0 + u < n ? s_w[u0 + u] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int d = threadIdx.x + e * 128;
+    if (d < p.D) dst[d] = T(acc[e] * inv);
   }
 }
 
@@ -852,8 +862,7 @@ static size_t ws_size(const sd_attn_desc *d) {
   const int G = d->h_q / d->h_kv;
   const int Mpad = (G * d->n_q + 15) / 16 * 16;
   const size_t slots = (size_t)d->batch * d->h_kv + (size_t)grid_ctas(d);
-  return round_up(slots * Mpad * d->head_dim * 4, 256) + round_up(slots * Mpad * 2 * 4, 256) +
-         round_up((size_t)d->batch * d->h_kv * 4, 256);
+  return round_up(slots * Mpad * d->head_dim * 4, 256) + round_up(slots * Mpad * 2 * 4, 256);
 }
 
 static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const void *k_new,
@@ -913,10 +922,6 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   p.ws_o = reinterpret_cast<float *>(ws);
   p.ws_ml = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ws) +
                                       round_up(slots * p.Mpad * p.D * 4, 256));
-  p.counters = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(p.ws_ml) +
-                                       round_up(slots * p.Mpad * 2 * 4, 256));
-  if (cudaMemsetAsync(p.counters, 0, (size_t)p.B * p.Hkv * sizeof(int), st) != cudaSuccess)
-    return SD_ERR_CUDA;
   CUtensorMap km, vm;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
   if (!encode_tmap_2d_bf16(&km, k_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile) ||
@@ -928,7 +933,10 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
         (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache);
     if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
   }
-  return launch_bf16(p.D, MT, km, vm, p, st);
+  s = launch_bf16(p.D, MT, km, vm, p, st);
+  if (s != SD_OK) return s;
+  attn_combine_kernel<__nv_bfloat16><<<dim3(p.B * p.Hkv, p.M), 128, 0, st>>>(p);
+  return cuda_status(cudaGetLastError());
 }
 
 }  // namespace attn
