@@ -209,41 +209,53 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   __shared__ uint32_t s_step;
   __shared__ float s_top1, s_top2;
   __shared__ int s_arg;
+  __shared__ float4 s_rows[32];  // merged statistics: target rows 0..k, then draft rows 0..k-1
 
+  // ---- statistics of every row this sequence may need, one warp per row (in parallel)
+  const int n_rows = p.n_q + (p.T > 0.f ? p.k : 0);
+  for (int ri = warp; ri < n_rows; ri += kThreads / 32) {
+    const int r = ri < p.n_q ? b * p.n_q + ri : p.rows_t + b * p.k + (ri - p.n_q);
+    const float4 st = row_stats_warp(p, r);
+    if (lane == 0) s_rows[ri] = st;
+  }
+  if (threadIdx.x == 0) s_step = (uint32_t)(p.step + (p.step_ptr != nullptr ? *p.step_ptr : 0ull));
+  __syncthreads();
+
+  // ---- acceptance tests of the k drafts in parallel (lane i-1 tests draft i), first rejection
   if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    if (lane == 0) s_step = (uint32_t)(p.step + (p.step_ptr != nullptr ? *p.step_ptr : 0ull));
-    __syncwarp();
-    int a = 0, flag = 0;
-    for (int i = 1; i <= p.k; ++i) {
+    bool acc = true;
+    int flag = 0;
+    if (lane < p.k) {
+      const int i = lane + 1;
       const int d = p.drafts[(size_t)b * p.k + i - 1];
       const int rt = b * p.n_q + i - 1;
-      const float4 sz = row_stats_warp(p, rt);
-      bool acc = false;
+      const float4 sz = s_rows[i - 1];
       if (d < 0 || d >= p.V) {
-        if (lane == 0) record_status(p.status, SD_ERR_DEVICE);
+        record_status(p.status, SD_ERR_DEVICE);
+        acc = false;
       } else if (p.T > 0.f) {
-        const float4 sy = row_stats_warp(p, p.rows_t + b * p.k + i - 1);
+        const float4 sy = s_rows[p.n_q + i - 1];
         const float pd = expf(p.z[(size_t)rt * p.ld_t + d] / p.T - sz.x) / sz.y;
         const float qd =
             expf(p.y[((size_t)b * p.k + i - 1) * p.ld_d + d] / p.T - sy.x) / sy.y;
         const float ratio = qd > 0.f ? pd / qd : (pd > 0.f ? INFINITY : 0.f);
         const float u = accept_uniform(p.seed, s_step, (uint32_t)rt);
-        if (fabsf(u - ratio) < kMargin) flag = 1;
+        flag = fabsf(u - ratio) < kMargin;
         acc = u < ratio;
       } else {
-        if ((sz.x - sz.z) / fmaxf(1.f, fabsf(sz.x)) < kMargin) flag = 1;
+        flag = (sz.x - sz.z) / fmaxf(1.f, fabsf(sz.x)) < kMargin;
         acc = d == __float_as_int(sz.y);
       }
-      if (!acc) break;
-      ++a;
     }
-    const float4 sz = row_stats_warp(p, b * p.n_q + a);
-    float4 sy = make_float4(0.f, 1.f, 0.f, 0.f);
-    if (p.T > 0.f && a < p.k) sy = row_stats_warp(p, p.rows_t + b * p.k + a);
+    const unsigned rej = __ballot_sync(0xffffffffu, !acc && lane < p.k);
+    const int a = rej ? __ffs(rej) - 1 : p.k;
+    // margins count for the decisions actually taken: drafts 1 .. a+1
+    const unsigned flags = __ballot_sync(0xffffffffu, flag && lane <= a);
     if (lane == 0) {
+      const float4 sz = s_rows[a];
+      const float4 sy = (p.T > 0.f && a < p.k) ? s_rows[p.n_q + a] : make_float4(0.f, 1.f, 0.f, 0.f);
       s_a = a;
-      s_flag = flag;
+      s_flag = flags != 0;
       s_mz = sz.x;
       s_isz = 1.f / sz.y;
       s_my = sy.x;
@@ -280,6 +292,12 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   const int v1 = min(p.V, v0 + kDrawChunk);
   const int n4 = (v1 - v0) >> 2;
   Cand cr{-INFINITY, -INFINITY, -1}, cp{-INFINITY, -INFINITY, -1};
+  // Keys in float32 with fast exp2 / log where the error (<~1e-6 absolute on a key, <~1e-6
+  // relative on p and q) is far inside the 1e-4 margin below which a draw is flagged; the
+  // log1p of the uniform stays accurate because small uniforms decide the winners.
+  constexpr float L2E = 1.4426950408889634f;
+  const bool unit_t = p.T == 1.f;
+  const float mzl = mz * L2E, myl = my * L2E;
   for (int i = threadIdx.x; i < n4; i += kThreads) {
     const int v = v0 + 4 * i;
     const float4 z4 = __ldg(reinterpret_cast<const float4 *>(zr + v));
@@ -295,15 +313,16 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float E = -log1pf(-U[e]);
-      const float lnE = logf(E);  // E == 0 gives -inf: that token wins if its weight > 0
-      const float zt = zz[e] / p.T;
+      const float lnE = __logf(E);  // E == 0 gives -inf: that token wins if its weight > 0
+      const float zt = unit_t ? zz[e] : zz[e] / p.T;
       const float gp = zt == -INFINITY ? -INFINITY : zt - lnE;
       cand_push(cp, gp, v + e);
       if (resid) {
-        const float pv = expf(zt - mz) * isz;
-        const float qv = expf(yy[e] / p.T - my) * isy;
+        const float yt = unit_t ? yy[e] : yy[e] / p.T;
+        const float pv = exp2f(fmaf(zt, L2E, -mzl)) * isz;
+        const float qv = exp2f(fmaf(yt, L2E, -myl)) * isy;
         const float w = pv - qv;
-        cand_push(cr, w > 0.f ? logf(w) - lnE : -INFINITY, v + e);
+        cand_push(cr, w > 0.f ? __logf(w) - lnE : -INFINITY, v + e);
       }
     }
   }

@@ -48,8 +48,9 @@ __device__ __forceinline__ float accept_uniform(uint64_t seed, uint32_t step, ui
 __device__ __forceinline__ float float_uniform64(uint64_t w) {
   if (w == 0) return 0.0f;
   const int n = __clzll((long long)w);
-  const uint32_t m = (uint32_t)((w << n) >> 40);
-  return ldexpf((float)m, -24 - n);
+  const uint32_t m = (uint32_t)((w << n) >> 40);  // in [2^23, 2^24): the leading bit is set
+  // m * 2^(-24-n) = (m / 2^23) * 2^(-1-n): a normal float with biased exponent 126 - n
+  return __uint_as_float(((uint32_t)(126 - n) << 23) | (m & 0x7FFFFFu));
 }
 
 // Token uniforms of tokens 2*c and 2*c+1 of a row (one Philox call).
