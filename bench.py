@@ -56,6 +56,37 @@ def parse():
     return ap.parse_args()
 
 
+# kernel group -> the CUDA source whose ncu counters a committed profile summary holds
+GROUP_SOURCE = {"head_dense": "lm_head.cu", "head_clustered": "lm_head.cu",
+                "verify_global": "attention.cu", "verify_sliding": "attention.cu",
+                "xattn_global": "attention.cu", "xattn_sliding": "attention.cu",
+                "accept": "accept.cu", "accept_draft": "accept.cu", "commit": "commit.cu"}
+
+
+def source_hash(name):
+    import hashlib
+    h = hashlib.sha256()
+    for f in (name, "common.cuh", "philox.cuh"):
+        path = os.path.join(ROOT, "verify_step_b200", "csrc", f)
+        if os.path.exists(path):
+            h.update(open(path, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(group):
+    """DRAM bytes per launch of a kernel group from the committed ncu summary, or None when
+    the summary is missing or the kernel source changed since its counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic_%s.json" % WORKLOAD)
+    try:
+        d = json.load(open(path))
+        e = d["groups"][group]
+        if e["source_sha"] != source_hash(GROUP_SOURCE[group]):
+            return None
+        return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -540,7 +571,7 @@ def main():
     def roof(g):
         ach = nbytes[g] / (kern_ms[g] * 1e6)
         return {"kernel": g, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
-                "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": None,
+                "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": dram_traffic(g),
                 "peak_source": src, "bytes_per_launch": nbytes[g],
                 "ms_per_launch": round(kern_ms[g], 4)}
     # telemetry of the acceptance rule on these (random) weights
