@@ -208,6 +208,28 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
                     int32_t *n_accepted, int32_t *out_tokens, int32_t *margin_flags,
                     void *ws, size_t ws_bytes, sd_stream stream);
 
+/*
+ * sd_accept_noalloc -- the same computation as sd_accept, for callers that cannot allocate
+ * device memory (for example code that must not call cudaMalloc inside a latency-critical
+ * serving loop, or a host framework that only lends out its own input and output buffers).
+ * There is no counterpart on the pages; it exists only for such callers.
+ *
+ * The caller still passes every input and output; the scratch space is a fixed array of
+ * SD_ACCEPT_NOALLOC_MAX_SCRATCH bytes compiled into the library, which every GPU that loads the
+ * library holds until the process exits.  A request whose sd_accept_workspace_size exceeds that
+ * limit is rejected with SD_ERR_WORKSPACE before anything is launched (at V = 262144 the limit
+ * covers up to 389 sequences at k = 6, 629 at k = 2).  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * All calls share the one array: calls that may overlap on the GPU (other streams, other host
+ * threads) race and must be ordered by the caller.  Nothing in the array needs clearing by the
+ * caller: the state that must start at zero is reset by every call.  Allocates nothing.
+ */
+#define SD_ACCEPT_NOALLOC_MAX_SCRATCH (4u << 20)
+sd_status sd_accept_noalloc(const sd_accept_desc *desc, const float *target_logits,
+                            const float *draft_logits, const int32_t *draft_tokens,
+                            int32_t *n_accepted, int32_t *out_tokens, int32_t *margin_flags,
+                            sd_stream stream);
+
 /* ---------------------------------------------------------------------------------------
  * Commit ("Gemma 4 MTP: drafter drafts, target verifies", section "basic structure of
  * speculative decoding": only the prefix up to the rejected position is kept; Gemma 4 MTP

@@ -84,6 +84,8 @@ _SIGS = {
     "sd_accept_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(AcceptDesc)]),
     "sd_accept": (ctypes.c_int, [ctypes.POINTER(AcceptDesc), _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.c_size_t, _P]),
+    "sd_accept_noalloc": (ctypes.c_int, [ctypes.POINTER(AcceptDesc), _P, _P, _P, _P, _P, _P,
+                                         _P]),
     "sd_commit": (ctypes.c_int, [ctypes.POINTER(CommitDesc), _P, _P, _P, _P, _P, _P, _P]),
     "sd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sd_device_status_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), _P]),
@@ -186,6 +188,15 @@ def sd_accept(desc, target_logits, draft_logits, draft_tokens, n_accepted, out_t
         ctypes.byref(desc), _ptr(target_logits), _ptr(draft_logits), _ptr(draft_tokens),
         _ptr(n_accepted), _ptr(out_tokens), _ptr(margin_flags), _ptr(ws), _nbytes(ws),
         _stream(stream)))
+
+
+def sd_accept_noalloc(desc, target_logits, draft_logits, draft_tokens, n_accepted, out_tokens,
+                      margin_flags, stream=None):
+    """sd_accept without a caller workspace: the library's fixed scratch array is used (see
+    include/sd_verify.h for its size limit and the rule that overlapping calls race)."""
+    _check("sd_accept_noalloc", lib().sd_accept_noalloc(
+        ctypes.byref(desc), _ptr(target_logits), _ptr(draft_logits), _ptr(draft_tokens),
+        _ptr(n_accepted), _ptr(out_tokens), _ptr(margin_flags), _stream(stream)))
 
 
 def sd_commit(desc, block_table, ctx_len, n_accepted, committed_slots, hidden=None,

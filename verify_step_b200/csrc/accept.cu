@@ -17,6 +17,7 @@
 //     The last CTA of a sequence (atomic ticket; no waiting) merges the chunk winners in chunk
 //     order, lowest token id first on ties, and writes the outputs.
 #include <cfloat>
+#include <mutex>
 
 #include "common.cuh"
 #include "host.cuh"
@@ -467,3 +468,50 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------- no-allocation
+// sd_accept_noalloc: the same acceptance step for callers that cannot allocate device memory
+// themselves -- for example code running where a device allocation would synchronise or is
+// forbidden (inside a real-time serving loop with a fixed memory budget, or a host framework
+// that hands out only its own buffers).  The scratch lives in a fixed array compiled into this
+// library; every GPU that loads the library keeps it until the process exits.
+
+namespace sdv {
+namespace acc {
+
+static __device__ __align__(256) unsigned char g_accept_noalloc_scratch[SD_ACCEPT_NOALLOC_MAX_SCRATCH];
+
+// Device address of the scratch array on the current device, looked up once per device.  A
+// symbol's host-side name is not a device address, so it is never passed to a kernel directly.
+static void *noalloc_scratch() {
+  static std::mutex mu;
+  static void *addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_accept_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace acc
+}  // namespace sdv
+
+extern "C" sd_status sd_accept_noalloc(const sd_accept_desc *desc, const float *target_logits,
+                                       const float *draft_logits, const int32_t *draft_tokens,
+                                       int32_t *n_accepted, int32_t *out_tokens,
+                                       int32_t *margin_flags, sd_stream stream) {
+  const sd_status v = sdv::acc::validate(desc);
+  if (v != SD_OK) return v;
+  if (sd_accept_workspace_size(desc) > (size_t)SD_ACCEPT_NOALLOC_MAX_SCRATCH)
+    return SD_ERR_WORKSPACE;
+  void *scratch = sdv::acc::noalloc_scratch();
+  if (scratch == nullptr) return SD_ERR_CUDA;
+  // The per-sequence counters in the scratch are cleared by the statistics kernel at the start
+  // of every call, so the array's leftover contents from an earlier call do not matter.
+  return sd_accept(desc, target_logits, draft_logits, draft_tokens, n_accepted, out_tokens,
+                   margin_flags, scratch, (size_t)SD_ACCEPT_NOALLOC_MAX_SCRATCH, stream);
+}
