@@ -42,7 +42,7 @@ from .philox import accept_uniform, token_uniform_rows
 
 MARGIN = 1e-4          # spec margin on |u - p/q|; reused for draws and argmaxes
 REL_P = 1e-5           # assumed float32 relative error bound on a probability p_v or q_v
-ABS_KEY = 1e-6         # assumed float32 absolute error bound on ln E_v and z_v / T
+ABS_KEY = 1e-5         # assumed float32 absolute error bound on ln E_v and z_v / T
 
 PURPOSE_ACCEPT = 0
 PURPOSE_TARGET = 1

@@ -49,6 +49,24 @@ struct Params {
   int *status;
 };
 
+// E = -ln(1 - V) for V in [0, 1): the series V + V^2/2 + ... + V^8/8 below 1/16 (truncation
+// below 3e-11 relative), else -ln(1 - V) with 1 - V formed exactly or within 2^-25 and the fast
+// logarithm (absolute error below 4e-7, i.e. below 6e-6 relative to E >= 0.0645).
+__device__ __forceinline__ float neg_log1m(float V) {
+  if (V < 0.0625f) {
+    float t = 0.125f;
+    t = fmaf(V, t, 0.14285714f);
+    t = fmaf(V, t, 0.16666667f);
+    t = fmaf(V, t, 0.2f);
+    t = fmaf(V, t, 0.25f);
+    t = fmaf(V, t, 0.33333333f);
+    t = fmaf(V, t, 0.5f);
+    t = fmaf(V, t, 1.f);
+    return V * t;
+  }
+  return -__logf(1.f - V);
+}
+
 struct Cand {  // best and runner-up key of a race, best token id
   float g1, g2;
   int v1;
@@ -304,27 +322,33 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
     const float4 z4 = __ldg(reinterpret_cast<const float4 *>(zr + v));
     float4 y4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (resid) y4 = __ldg(reinterpret_cast<const float4 *>(yr + v));
+    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
+    const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
+    float zt[4], w[4];
+    bool any = false;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      zt[e] = unit_t ? zz[e] : zz[e] / p.T;
+      w[e] = 0.f;
+      if (resid) {
+        const float yt = unit_t ? yy[e] : yy[e] / p.T;
+        const float pv = exp2f(fmaf(zt[e], L2E, -mzl)) * isz;
+        const float qv = exp2f(fmaf(yt, L2E, -myl)) * isy;
+        w[e] = pv - qv;
+      }
+      any |= zt[e] != -INFINITY || w[e] > 0.f;
+    }
+    if (!any) continue;  // no token of the group can win either race: no uniforms needed
     float U[4];
     token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1), U[0],
                        U[1]);
     token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1) + 1u,
                        U[2], U[3]);
-    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
-    const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float E = -log1pf(-U[e]);
-      const float lnE = __logf(E);  // E == 0 gives -inf: that token wins if its weight > 0
-      const float zt = unit_t ? zz[e] : zz[e] / p.T;
-      const float gp = zt == -INFINITY ? -INFINITY : zt - lnE;
-      cand_push(cp, gp, v + e);
-      if (resid) {
-        const float yt = unit_t ? yy[e] : yy[e] / p.T;
-        const float pv = exp2f(fmaf(zt, L2E, -mzl)) * isz;
-        const float qv = exp2f(fmaf(yt, L2E, -myl)) * isy;
-        const float w = pv - qv;
-        cand_push(cr, w > 0.f ? __logf(w) - lnE : -INFINITY, v + e);
-      }
+      const float lnE = __logf(neg_log1m(U[e]));  // E == 0 gives -inf: that token wins
+      cand_push(cp, zt[e] == -INFINITY ? -INFINITY : zt[e] - lnE, v + e);
+      if (resid) cand_push(cr, w[e] > 0.f ? __logf(w[e]) - lnE : -INFINITY, v + e);
     }
   }
   for (int off = 16; off > 0; off >>= 1) {

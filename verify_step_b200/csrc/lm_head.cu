@@ -311,30 +311,37 @@ __global__ void fill_neg_inf_kernel(float *logits, int V, int ld, int vec4) {
 }
 
 // Exact logits of the kept clusters' tokens: CTA (m, slot, part) takes tokens
-// [part * tpc, (part+1) * tpc) of cluster sel[m, slot]; each warp takes TK tokens at a time
-// with all their weight loads in flight (d <= 256 * KMAX) before the dot products.
+// [part * tpc, (part+1) * tpc) of cluster sel[m, slot].  Lane l multiplies elements
+// l*8 + q*256 + [0, 8) of every weight row, so it keeps those hidden values in registers;
+// each warp takes TK tokens at a time with all their weight loads in flight (d <= 256 * KMAX).
 template <int KMAX>
 __global__ void __launch_bounds__(256) cluster_logits_kernel(
     const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm, const int32_t *cluster_tokens,
     const int32_t *sel, int top_c, int cs, int d, int C, int V, int ld, int parts, float *logits,
     int *status) {
-  extern __shared__ float hs[];
   const int part = blockIdx.x % parts;
   const int ms = blockIdx.x / parts;
   const int m = ms / top_c, slot = ms % top_c;
   const int c = sel[(size_t)m * top_c + slot];
-  for (int i = threadIdx.x; i < d; i += blockDim.x)
-    hs[i] = __bfloat162float(h[(size_t)m * d + i]);
-  __syncthreads();
   if (c < 0 || c >= C) {
     if (threadIdx.x == 0) record_status(status, SD_ERR_DEVICE);
     return;
   }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int nk = (d + 255) / 256;  // 256 elements per warp-wide 16-byte load
+  float hr[KMAX][8];
+#pragma unroll
+  for (int q = 0; q < KMAX; ++q) {
+    const int k0 = lane * 8 + q * 256;
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (q < nk && k0 < d) raw = __ldg(reinterpret_cast<const uint4 *>(h + (size_t)m * d + k0));
+    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) hr[q][r] = __bfloat162float(e[r]);
+  }
   const int tpc = (cs + parts - 1) / parts;
   const int t_begin = part * tpc, t_end = min(cs, t_begin + tpc);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  constexpr int TK = 4;
-  const int nk = (d + 255) / 256;  // 256 elements per warp-wide 16-byte load
+  constexpr int TK = 2;
   for (int t0 = t_begin + warp * TK; t0 < t_end; t0 += nw * TK) {
     uint4 raw[TK][KMAX];
 #pragma unroll
@@ -353,27 +360,68 @@ __global__ void __launch_bounds__(256) cluster_logits_kernel(
       acc[u] = 0.f;
 #pragma unroll
       for (int q = 0; q < KMAX; ++q) {
-        const int k0 = lane * 8 + q * 256;
-        if (q < nk && k0 < d) {
-          const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][q]);
+        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][q]);
 #pragma unroll
-          for (int r = 0; r < 8; ++r) acc[u] = fmaf(__bfloat162float(e[r]), hs[k0 + r], acc[u]);
-        }
+        for (int r = 0; r < 8; ++r) acc[u] = fmaf(__bfloat162float(e[r]), hr[q][r], acc[u]);
       }
     }
 #pragma unroll
     for (int u = 0; u < TK; ++u)
       for (int o = 16; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
     if (lane < TK && t0 + lane < t_end) {
-      float mine = acc[0];
-#pragma unroll
-      for (int u = 1; u < TK; ++u)
-        if (lane == u) mine = acc[u];
+      const float mine = lane == 0 ? acc[0] : acc[1];
       const int tok = cluster_tokens[(size_t)c * cs + t0 + lane];
       if (tok < 0 || tok >= V)
         record_status(status, SD_ERR_DEVICE);
       else
         logits[(size_t)m * ld + tok] = mine;
+    }
+  }
+}
+
+// Centroid scores of the clustered head, score[i, c] = h[i] . centroid[c], for up to 16 rows:
+// one warp per centroid (its row read once, 16-byte loads), the rows of h in shared memory.
+// A GEMV this small (2 MB of centroids) needs many CTAs in flight rather than tensor cores.
+__global__ void __launch_bounds__(256) centroid_scores_kernel(const __nv_bfloat16 *h,
+                                                              const __nv_bfloat16 *cent, int M,
+                                                              int d, int C, float *scores) {
+  extern __shared__ float hs[];  // [M][d]
+  for (int i = threadIdx.x; i < M * d; i += blockDim.x) hs[i] = __bfloat162float(h[i]);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (c >= C) return;
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  for (int k0 = lane * 8; k0 < d; k0 += 256) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(cent + (size_t)c * d + k0));
+    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+    float w[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) w[r] = __bfloat162float(e[r]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i < M) {
+        const float4 a = *reinterpret_cast<const float4 *>(hs + i * d + k0);
+        const float4 b = *reinterpret_cast<const float4 *>(hs + i * d + k0 + 4);
+        acc[i] = fmaf(w[0], a.x, acc[i]);
+        acc[i] = fmaf(w[1], a.y, acc[i]);
+        acc[i] = fmaf(w[2], a.z, acc[i]);
+        acc[i] = fmaf(w[3], a.w, acc[i]);
+        acc[i] = fmaf(w[4], b.x, acc[i]);
+        acc[i] = fmaf(w[5], b.y, acc[i]);
+        acc[i] = fmaf(w[6], b.z, acc[i]);
+        acc[i] = fmaf(w[7], b.w, acc[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i < M) {
+      float v = acc[i];
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) scores[(size_t)i * C + c] = v;
     }
   }
 }
@@ -496,11 +544,17 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   if (!ws || ws_bytes < ws_size(desc)) return SD_ERR_WORKSPACE;
   float *scores = reinterpret_cast<float *>(ws);
   const int C = desc->n_clusters;
-  for (int m0 = 0; m0 < desc->m; m0 += 256) {
-    const int mm = desc->m - m0 < 256 ? desc->m - m0 : 256;
-    s = dense_bf16((const uint8_t *)h + m0 * hrow, centroids, mm, desc->d, C,
-                   scores + (size_t)m0 * C, C, st);
-    if (s != SD_OK) return s;
+  if (desc->m <= 16 && (size_t)desc->m * desc->d * 4 <= 48 * 1024) {
+    centroid_scores_kernel<<<(C + 7) / 8, 256, (size_t)desc->m * desc->d * 4, st>>>(
+        (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)centroids, desc->m, desc->d, C, scores);
+    if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+  } else {
+    for (int m0 = 0; m0 < desc->m; m0 += 256) {
+      const int mm = desc->m - m0 < 256 ? desc->m - m0 : 256;
+      s = dense_bf16((const uint8_t *)h + m0 * hrow, centroids, mm, desc->d, C,
+                     scores + (size_t)m0 * C, C, st);
+      if (s != SD_OK) return s;
+    }
   }
   int n = 1;
   while (n < C) n <<= 1;
@@ -522,7 +576,7 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
          desc->cluster_size / (parts * 2) >= 32)
     parts *= 2;
   const dim3 grid(desc->m * desc->top_c * parts);
-  const size_t shm = (size_t)desc->d * 4;
+  const size_t shm = 0;
   if (desc->d <= 1024)
     cluster_logits_kernel<4><<<grid, 256, shm, st>>>(
         (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
