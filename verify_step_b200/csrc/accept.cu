@@ -27,12 +27,12 @@ namespace sdv {
 namespace acc {
 
 constexpr int kChunk = 8192;      // tokens per CTA of the statistics pass
-constexpr int kDrawChunk = 2048;  // tokens per CTA of the race
+constexpr int kDrawSlots = 592;  // draw CTAs aimed at: one wave at 4 CTAs on each of 148 SMs
 constexpr int kThreads = 256;
 constexpr float kMargin = 1e-4f;
 
 struct Params {
-  int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, ndraw, rows_t, rows_total;
+  int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, ndraw, draw_chunk, rows_t, rows_total;
   float T;
   unsigned long long seed;
   unsigned long long step;
@@ -307,8 +307,8 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   const float *zr = p.z + (size_t)rt * p.ld_t;
   const float *yr = resid ? p.y + ((size_t)b * p.k + a) * p.ld_d : nullptr;
   const float mz = s_mz, isz = s_isz, my = resid ? s_my : 0.f, isy = resid ? s_isy : 0.f;
-  const int v0 = c * kDrawChunk;
-  const int v1 = min(p.V, v0 + kDrawChunk);
+  const int v0 = c * p.draw_chunk;
+  const int v1 = min(p.V, v0 + p.draw_chunk);
   const int n4 = (v1 - v0) >> 2;
   Cand cr{-INFINITY, -INFINITY, -1}, cp{-INFINITY, -INFINITY, -1};
   // Keys in float32 with fast exp2 / log where the error (<~1e-6 absolute on a key, <~1e-6
@@ -420,14 +420,27 @@ static sd_status validate(const sd_accept_desc *d) {
 }
 
 static int nchunks_of(int V) { return (V + kChunk - 1) / kChunk; }
-static int ndraw_of(int V) { return (V + kDrawChunk - 1) / kDrawChunk; }
+// Tokens per draw CTA: the race of one sequence is split so that all B sequences together give
+// about one wave of CTAs (the per-CTA chain of dependent memory round trips, not the token work,
+// dominates at small B); multiples of 1024 tokens.
+static int draw_chunk_of(int B, int V) {
+  int per_seq = kDrawSlots / (B > 0 ? B : 1);
+  if (per_seq < 1) per_seq = 1;
+  int chunk = (V + per_seq - 1) / per_seq;
+  chunk = (chunk + 1023) / 1024 * 1024;
+  return chunk;
+}
+static int ndraw_of(int B, int V) {
+  const int c = draw_chunk_of(B, V);
+  return (V + c - 1) / c;
+}
 
 static size_t ws_size(const sd_accept_desc *d) {
   if (validate(d) != SD_OK) return 0;
   const size_t nc = nchunks_of(d->vocab);
   const size_t rows = (size_t)d->batch * (d->k + 1) + (size_t)d->batch * d->k;
   return round_up(rows * nc * 16, 256) +
-         round_up((size_t)d->batch * ndraw_of(d->vocab) * 32, 256) +
+         round_up((size_t)d->batch * ndraw_of(d->batch, d->vocab) * 32, 256) +
          round_up((size_t)d->batch * 4, 256);
 }
 
@@ -463,7 +476,8 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.ld_o = desc->ld_out ? desc->ld_out : desc->k + 1;
   p.purpose = desc->purpose;
   p.nchunks = nchunks_of(desc->vocab);
-  p.ndraw = ndraw_of(desc->vocab);
+  p.draw_chunk = draw_chunk_of(desc->batch, desc->vocab);
+  p.ndraw = ndraw_of(desc->batch, desc->vocab);
   p.rows_t = p.B * p.n_q;
   p.rows_total = p.rows_t + (sampling ? p.B * p.k : 0);
   p.T = desc->temperature;

@@ -310,65 +310,73 @@ __global__ void fill_neg_inf_kernel(float *logits, int V, int ld, int vec4) {
   }
 }
 
-// Exact logits of the kept clusters' tokens: CTA (m, slot, part) takes tokens
-// [part * tpc, (part+1) * tpc) of cluster sel[m, slot].  Lane l multiplies elements
-// l*8 + q*256 + [0, 8) of every weight row, so it keeps those hidden values in registers;
-// each warp takes TK tokens at a time with all their weight loads in flight (d <= 256 * KMAX).
+// Exact logits of the kept clusters' tokens.  The work is M * top_c * ceil(cs / TK) units of TK
+// tokens; a persistent grid of warps takes contiguous ranges of units, so consecutive units of
+// a warp almost always share the row m.  Lane l multiplies elements l*8 + q*256 + [0, 8) of a
+// weight row and keeps those hidden values in registers (reloaded only when m changes); the
+// weight loads of a unit's TK tokens are all in flight before the dot products (d <= 256 * KMAX).
 template <int KMAX>
 __global__ void __launch_bounds__(256) cluster_logits_kernel(
     const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm, const int32_t *cluster_tokens,
-    const int32_t *sel, int top_c, int cs, int d, int C, int V, int ld, int parts, float *logits,
+    const int32_t *sel, int M, int top_c, int cs, int d, int C, int V, int ld, float *logits,
     int *status) {
-  const int part = blockIdx.x % parts;
-  const int ms = blockIdx.x / parts;
-  const int m = ms / top_c, slot = ms % top_c;
-  const int c = sel[(size_t)m * top_c + slot];
-  if (c < 0 || c >= C) {
-    if (threadIdx.x == 0) record_status(status, SD_ERR_DEVICE);
-    return;
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int nk = (d + 255) / 256;  // 256 elements per warp-wide 16-byte load
-  float hr[KMAX][8];
-#pragma unroll
-  for (int q = 0; q < KMAX; ++q) {
-    const int k0 = lane * 8 + q * 256;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (q < nk && k0 < d) raw = __ldg(reinterpret_cast<const uint4 *>(h + (size_t)m * d + k0));
-    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) hr[q][r] = __bfloat162float(e[r]);
-  }
-  const int tpc = (cs + parts - 1) / parts;
-  const int t_begin = part * tpc, t_end = min(cs, t_begin + tpc);
   constexpr int TK = 2;
-  for (int t0 = t_begin + warp * TK; t0 < t_end; t0 += nw * TK) {
+  const int lane = threadIdx.x & 31;
+  const long long n_warps = (long long)gridDim.x * (blockDim.x >> 5);
+  const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int upc = (cs + TK - 1) / TK;  // units per (row, cluster)
+  const long long U = (long long)M * top_c * upc;
+  const long long u_begin = U * wid / n_warps, u_end = U * (wid + 1) / n_warps;
+  const int nk = (d + 255) / 256;
+  float hr[KMAX][8];
+  int m_loaded = -1;
+  for (long long u = u_begin; u < u_end; ++u) {
+    const int ms = (int)(u / upc);
+    const int t0 = (int)(u % upc) * TK;
+    const int m = ms / top_c, slot = ms % top_c;
+    const int c = sel[(size_t)m * top_c + slot];
+    if (c < 0 || c >= C) {
+      if (lane == 0) record_status(status, SD_ERR_DEVICE);
+      continue;
+    }
     uint4 raw[TK][KMAX];
 #pragma unroll
-    for (int u = 0; u < TK; ++u)
+    for (int t = 0; t < TK; ++t)
 #pragma unroll
       for (int q = 0; q < KMAX; ++q) {
         const int k0 = lane * 8 + q * 256;
-        raw[u][q] = (q < nk && k0 < d && t0 + u < t_end)
+        raw[t][q] = (q < nk && k0 < d && t0 + t < cs)
                         ? __ldg(reinterpret_cast<const uint4 *>(
-                              w_cm + ((size_t)c * cs + t0 + u) * d + k0))
+                              w_cm + ((size_t)c * cs + t0 + t) * d + k0))
                         : make_uint4(0, 0, 0, 0);
       }
-    float acc[TK];
-#pragma unroll
-    for (int u = 0; u < TK; ++u) {
-      acc[u] = 0.f;
+    if (m != m_loaded) {
 #pragma unroll
       for (int q = 0; q < KMAX; ++q) {
-        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[u][q]);
+        const int k0 = lane * 8 + q * 256;
+        uint4 hv = make_uint4(0, 0, 0, 0);
+        if (q < nk && k0 < d) hv = __ldg(reinterpret_cast<const uint4 *>(h + (size_t)m * d + k0));
+        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&hv);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) acc[u] = fmaf(__bfloat162float(e[r]), hr[q][r], acc[u]);
+        for (int r = 0; r < 8; ++r) hr[q][r] = __bfloat162float(e[r]);
+      }
+      m_loaded = m;
+    }
+    float acc[TK];
+#pragma unroll
+    for (int t = 0; t < TK; ++t) {
+      acc[t] = 0.f;
+#pragma unroll
+      for (int q = 0; q < KMAX; ++q) {
+        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[t][q]);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[t] = fmaf(__bfloat162float(e[r]), hr[q][r], acc[t]);
       }
     }
 #pragma unroll
-    for (int u = 0; u < TK; ++u)
-      for (int o = 16; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
-    if (lane < TK && t0 + lane < t_end) {
+    for (int t = 0; t < TK; ++t)
+      for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+    if (lane < TK && t0 + lane < cs) {
       const float mine = lane == 0 ? acc[0] : acc[1];
       const int tok = cluster_tokens[(size_t)c * cs + t0 + lane];
       if (tok < 0 || tok >= V)
@@ -386,17 +394,32 @@ __global__ void __launch_bounds__(256) centroid_scores_kernel(const __nv_bfloat1
                                                               const __nv_bfloat16 *cent, int M,
                                                               int d, int C, float *scores) {
   extern __shared__ float hs[];  // [M][d]
-  for (int i = threadIdx.x; i < M * d; i += blockDim.x) hs[i] = __bfloat162float(h[i]);
-  __syncthreads();
+  for (int i = threadIdx.x; i < M * d / 8; i += blockDim.x) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(h) + i);
+    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) hs[i * 8 + r] = __bfloat162float(e[r]);
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x * (blockDim.x >> 5) + warp;
+  // this lane's part of the centroid row, loaded before the rows of h are needed (d <= 1024)
+  uint4 raw[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int k0 = lane * 8 + q * 256;
+    raw[q] = (c < C && k0 < d) ? __ldg(reinterpret_cast<const uint4 *>(cent + (size_t)c * d + k0))
+                               : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();
   if (c >= C) return;
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int k0 = lane * 8; k0 < d; k0 += 256) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(cent + (size_t)c * d + k0));
-    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int k0 = lane * 8 + q * 256;
+    if (k0 >= d) break;
+    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw[q]);
     float w[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) w[r] = __bfloat162float(e[r]);
@@ -544,7 +567,7 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   if (!ws || ws_bytes < ws_size(desc)) return SD_ERR_WORKSPACE;
   float *scores = reinterpret_cast<float *>(ws);
   const int C = desc->n_clusters;
-  if (desc->m <= 16 && (size_t)desc->m * desc->d * 4 <= 48 * 1024) {
+  if (desc->m <= 16 && desc->d <= 1024 && (size_t)desc->m * desc->d * 4 <= 48 * 1024) {
     centroid_scores_kernel<<<(C + 7) / 8, 256, (size_t)desc->m * desc->d * 4, st>>>(
         (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)centroids, desc->m, desc->d, C, scores);
     if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
@@ -569,23 +592,23 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   fill_neg_inf_kernel<<<dim3(per_row < 64 ? per_row : 64, desc->m), 256, 0, st>>>(
       logits, desc->vocab, ld, vec4);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
-  // enough CTAs to keep every SM streaming: split a cluster's tokens over `parts` CTAs
+  // persistent warps: as many 8-warp CTAs as fit on the device at once
   const int sms = sm_count();
-  int parts = 1;
-  while (parts < 8 && (long long)desc->m * desc->top_c * parts < 4ll * (sms > 0 ? sms : 148) &&
-         desc->cluster_size / (parts * 2) >= 32)
-    parts *= 2;
-  const dim3 grid(desc->m * desc->top_c * parts);
-  const size_t shm = 0;
+  int occ = 0;
   if (desc->d <= 1024)
-    cluster_logits_kernel<4><<<grid, 256, shm, st>>>(
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<4>, 256, 0);
+  else
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<16>, 256, 0);
+  const dim3 grid((occ > 0 ? occ : 1) * (sms > 0 ? sms : 148));
+  if (desc->d <= 1024)
+    cluster_logits_kernel<4><<<grid, 256, 0, st>>>(
         (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
-        desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, parts, logits,
+        desc->m, desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
         device_status_word());
   else
-    cluster_logits_kernel<16><<<grid, 256, shm, st>>>(
+    cluster_logits_kernel<16><<<grid, 256, 0, st>>>(
         (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
-        desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, parts, logits,
+        desc->m, desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
         device_status_word());
   return cuda_status(cudaGetLastError());
 }
