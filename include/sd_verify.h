@@ -218,7 +218,7 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
  * SD_ACCEPT_NOALLOC_MAX_SCRATCH bytes compiled into the library, which every GPU that loads the
  * library holds until the process exits.  A request whose sd_accept_workspace_size exceeds that
  * limit is rejected with SD_ERR_WORKSPACE before anything is launched (at V = 262144 the limit
- * covers up to 389 sequences at k = 6, 629 at k = 2).  The first call on a device looks up the array's
+ * covers up to 626 sequences at k = 6, 1615 at k = 2).  The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress), so make that first call before any stream capture.
  * All calls share the one array: calls that may overlap on the GPU (other streams, other host
  * threads) race and must be ordered by the caller.  Nothing in the array needs clearing by the

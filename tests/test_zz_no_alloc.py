@@ -58,7 +58,7 @@ def test_noalloc_matches_workspace_version_twice():
 
 def test_noalloc_refuses_requests_beyond_its_scratch():
     V, k = 262144, 6
-    desc = sd.AcceptDesc(batch=390, k=k, vocab=V, temperature=1.0, seed=0, step=0, purpose=1)
+    desc = sd.AcceptDesc(batch=627, k=k, vocab=V, temperature=1.0, seed=0, step=0, purpose=1)
     assert sd.sd_accept_workspace_size(desc) > (4 << 20)
     # nothing is dereferenced or launched: null data pointers are fine for the size check
     st = sd.lib().sd_accept_noalloc(ctypes.byref(desc), None, None, None, None, None, None,
