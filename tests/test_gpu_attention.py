@@ -123,6 +123,75 @@ def test_verify_ignores_nan_in_unread_slots():
     assert rel_err(out.float().numpy(), ref) <= BF16_TOL
 
 
+# Sliding windows of at most 2048 keys run on the cluster kernel (one cluster of CTAs per
+# (sequence, kv head), partials merged in distributed shared memory); longer windows on the
+# persistent split-KV kernel.  Cases cover two 16-row tiles, head dims 64..512, a single
+# sequence (largest clusters), a batch too large for clusters (one CTA per item), tile rings
+# that wrap (more tiles per CTA than stages) and a window past the cluster limit.
+WINDOW_CASES = [
+    # (seed, L list, n_q, hq, hkv, D, bs, window)
+    (31, [700, 20, 513], 7, 16, 4, 256, 16, 100),   # 28 rows
+    (32, [1000], 3, 8, 2, 64, 16, 300),             # B1: clusters of 8
+    (33, [2500, 2200, 3000], 1, 16, 4, 512, 32, 2048),  # 129 tiles per item: the ring wraps
+    (34, [600] * 40, 3, 8, 2, 128, 16, 512),        # 80 items: one CTA each, ring wraps
+    (35, [5000, 4100], 3, 16, 4, 256, 16, 3000),    # past the cluster limit: split-KV kernel
+    (36, [8, 1, 40], 2, 8, 2, 256, 16, 512),        # window longer than every context
+]
+
+
+@pytest.mark.parametrize("case", WINDOW_CASES, ids=[str(c[0]) for c in WINDOW_CASES])
+def test_verify_window(case):
+    seed, L, n_q, hq, hkv, D, bs, window = case
+    B = len(L)
+    c = small_paged(seed, L, n_q, hkv, D, bs, window=window)
+    q, kn, vn = qkv(seed, B, n_q, hq, hkv, D)
+    desc = attn_desc(B, n_q, hq, hkv, D, bs, c["mbps"], c["nb"], window)
+    out, kco, vco = run_verify(desc, q, kn, vn, c["kc"], c["vc"], c["table"], c["L"])
+    ref = oracle_verify(q, kn, vn, c["kc"], c["vc"], c["table"], c["L"], window, desc.scale, bs)
+    assert rel_err(out.float().numpy(), ref) <= BF16_TOL
+    check_append(kco, vco, kn, vn, c["table"], c["L"], bs)
+    assert status_ok()
+
+
+def test_window_ignores_nan_outside_the_window():
+    """Slots older than the window and slots past the new rows may hold NaN."""
+    seed, L, n_q, hq, hkv, D, bs, window = 37, [300, 90], 3, 16, 4, 256, 16, 64
+    c = small_paged(seed, L, n_q, hkv, D, bs, reserve=30)
+    kc, vc = c["kc"].clone(), c["vc"].clone()
+    for b in range(2):
+        old = range(0, max(0, L[b] + 1 - window))
+        new = range(L[b] + n_q, L[b] + 30)
+        for p in list(old) + list(new):
+            blk = int(c["table"][b, p // bs])
+            kc[blk, :, p % bs] = float("nan")
+            vc[blk, :, p % bs] = float("nan")
+    q, kn, vn = qkv(seed, 2, n_q, hq, hkv, D)
+    desc = attn_desc(2, n_q, hq, hkv, D, bs, c["mbps"], c["nb"], window)
+    out, _, _ = run_verify(desc, q, kn, vn, kc, vc, c["table"], c["L"])
+    assert torch.isfinite(out.float()).all()
+    ref = oracle_verify(q, kn, vn, c["kc"], c["vc"], c["table"], c["L"], window, desc.scale, bs)
+    assert rel_err(out.float().numpy(), ref) <= BF16_TOL
+    assert status_ok()
+
+
+@pytest.mark.parametrize("window", [0, 64])
+def test_out_of_range_block_is_flagged(window):
+    """A block-table entry outside [0, num_blocks) inside the key range: the tile is skipped
+    (never copied) and the device status reports SD_ERR_DEVICE."""
+    seed, L, n_q, hq, hkv, D, bs = 38, [100, 50], 3, 8, 2, 256, 16
+    c = small_paged(seed, L, n_q, hkv, D, bs)
+    table = c["table"].clone()
+    table[0, 5] = c["nb"] + 7  # positions 80..95 of sequence 0: inside both key ranges
+    q, kn, vn = qkv(seed, 2, n_q, hq, hkv, D)
+    desc = attn_desc(2, n_q, hq, hkv, D, bs, c["mbps"], c["nb"], window)
+    out, _, _ = run_verify(desc, q, kn, vn, c["kc"], c["vc"], table, c["L"])
+    assert sd.sd_device_status_read() == sd.SD_ERR_DEVICE
+    sd.sd_device_status_clear()
+    # the other sequence is untouched by the bad entry
+    ref = oracle_verify(q, kn, vn, c["kc"], c["vc"], c["table"], c["L"], window, desc.scale, bs)
+    assert rel_err(out[1].float().numpy(), ref[1]) <= BF16_TOL
+
+
 DRAFT_CASES = [
     (21, [37, 100, 5], [40, 99, 0], 8, 2, 256, 16, 24),
     (22, [300, 17], [299, 500], 16, 4, 512, 16, 0),

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "host.cuh"
@@ -24,6 +26,14 @@ int *device_status_word() {
     addr[dev] = reinterpret_cast<int *>(p);
   }
   return addr[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char *e = getenv("SDV_PDL");
+    return e && strcmp(e, "1") == 0;
+  }();
+  return on;
 }
 
 int sm_count() {

@@ -119,6 +119,7 @@ __device__ __forceinline__ const float *row_ptr(const Params &p, int r) {
 }
 
 __global__ void __launch_bounds__(kThreads) accept_stats_kernel(const Params p) {
+  pdl_wait();  // many waves: no early trigger, so the next kernel does not take their slots
   const int r = blockIdx.x, c = blockIdx.y;
   if (c == 0 && r == 0)
     for (int b = threadIdx.x; b < p.B; b += blockDim.x) p.counters[b] = 0u;
@@ -219,6 +220,8 @@ __device__ __forceinline__ float4 row_stats_warp(const Params &p, int r) {
 }
 
 __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x, c = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   __shared__ int s_a, s_flag;
@@ -499,10 +502,11 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.counters = reinterpret_cast<unsigned int *>(w8);
   p.status = device_status_word();
   cudaStream_t st = (cudaStream_t)stream;
-  accept_stats_kernel<<<dim3(p.rows_total, p.nchunks), kThreads, 0, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
-  accept_draw_kernel<<<dim3(p.B, sampling ? p.ndraw : 1), kThreads, 0, st>>>(p);
-  return cuda_status(cudaGetLastError());
+  if (launch(accept_stats_kernel, dim3(p.rows_total, p.nchunks), dim3(kThreads), 0, st, p) !=
+      cudaSuccess)
+    return SD_ERR_CUDA;
+  return cuda_status(
+      launch(accept_draw_kernel, dim3(p.B, sampling ? p.ndraw : 1), dim3(kThreads), 0, st, p));
 }
 
 }  // extern "C"

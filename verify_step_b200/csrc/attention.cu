@@ -269,6 +269,8 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     *abort_flag = 0;
     fence_mbar_init();
   }
+  pdl_trigger();
+  pdl_wait();  // everything below reads memory earlier kernels may have written
   build_tab(p, tab);
   __syncthreads();
 
@@ -567,6 +569,395 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   }
 }
 
+// ------------------------------------------------------------ short key ranges (clusters)
+// Sliding-window layers read at most window + n_q - 1 keys per item, too few to amortise a
+// separate merge kernel.  A cluster of CS CTAs takes one item (sequence b, kv head g); CTA
+// rank r streams tiles [n r / CS, n (r+1) / CS) of it, all of them in flight at once where the
+// shared-memory ring holds them.  Inside a CTA, KG key groups of warps take the CTA's tiles
+// round robin, each with its own online softmax.  The CS * KG partials (m, l, o) are merged
+// through distributed shared memory in (rank, key group) order: CTA r writes output columns
+// [D r / CS, D (r+1) / CS).  No workspace, one launch per call.
+
+template <int D, int MT>
+struct WCfg {
+  static constexpr int DS = D >= 128 ? 128 : 64;
+  static constexpr int NDG = D / DS;
+  static constexpr int WPG = MT * NDG;                  // warps of one key group
+  static constexpr int KG = 8 / WPG > 0 ? 8 / WPG : 1;  // key groups per CTA
+  static constexpr int NCW = KG * WPG;
+  static constexpr int THREADS = 32 * (NCW + 1);
+  static constexpr int MP = 16 * MT;  // padded rows of an item
+  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  // A multiple of KG: tiles t and t + STAGES share a stage and belong to the same key group,
+  // which consumes them in order (so a parity wait never sees the stage's previous phase).
+  static constexpr int RING = (192 * 1024) / STAGE_BYTES > 16 ? 16 : (192 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = RING / KG * KG;
+  static_assert(STAGES >= KG, "at least one stage per key group");
+  static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
+  static constexpr int ML_FLOATS = KG * MP * 2;
+  static constexpr size_t PART_BYTES = (size_t)KG * MP * D * 4;
+  static_assert(PART_BYTES <= (size_t)STAGES * STAGE_BYTES, "partials reuse the tile ring");
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + RED_FLOATS * 4 +
+                                 ML_FLOATS * 4 + 8 * (2 * STAGES + 2 * KG + 1) + 4 * (1 + STAGES) +
+                                 16;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+template <int D, int MT>
+__global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
+    attn_window_kernel(const __grid_constant__ CUtensorMap kmap,
+                       const __grid_constant__ CUtensorMap vmap, const Params p, int CS) {
+  using C = WCfg<D, MT>;
+  constexpr int DS = C::DS, NDG = C::NDG, WPG = C::WPG, KG = C::KG, NCW = C::NCW;
+  constexpr int STAGES = C::STAGES, MP = C::MP;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *stages = smem;
+  float *red = reinterpret_cast<float *>(smem + (size_t)STAGES * C::STAGE_BYTES);
+  float *ml = red + C::RED_FLOATS;  // [KG][MP][2] partial (m, l) per row
+  uint64_t *full = reinterpret_cast<uint64_t *>(ml + C::ML_FLOATS);
+  uint64_t *empty = full + STAGES;
+  uint64_t *red_bar = empty + STAGES;  // [KG][2]
+  uint64_t *done_bar = red_bar + 2 * KG;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(done_bar + 1);
+  volatile int *bad = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int item = blockIdx.x / CS;
+  const int b = item / p.Hkv, g = item % p.Hkv;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], WPG * 32);
+      bad[s] = 0;
+    }
+    for (int k = 0; k < 2 * KG; ++k) mbar_init(&red_bar[k], WPG * 32);
+    mbar_init(done_bar, NCW * 32);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  pdl_trigger();
+  pdl_wait();
+  __syncthreads();
+  const SeqRange s = seq_range(p, b, threadIdx.x == 0 && g == 0 && rank == 0);
+  const int t_lo = (int)((long long)s.n * rank / CS);
+  const int nl = (int)((long long)s.n * (rank + 1) / CS) - t_lo;
+
+  if (warp == NCW) {
+    // ------------------------------------------------------------------- producer warp
+    // The whole warp walks the tiles; its lanes fetch the block-table entries of the next
+    // 32 tiles at once, lane 0 issues the copies.
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+    }
+    int base = -32, blk_l = -1, t = 0;
+    for (; t < nl; ++t) {
+      if (t - base >= 32) {
+        base = t;
+        blk_l = -1;
+        if (t + lane < nl) {
+          const int bidx = (s.tf + t_lo + t + lane) * kTile / p.bs;
+          if (bidx < p.mbps) blk_l = p.table[(size_t)b * p.mbps + bidx];
+        }
+      }
+      const int blk = __shfl_sync(0xffffffffu, blk_l, t - base);
+      int go = 1;
+      if (lane == 0) {
+        const int stage = t % STAGES;
+        if (!mbar_wait(&empty[stage], ((t / STAGES) & 1) ^ 1, abort_flag)) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          go = 0;
+        } else if (blk < 0 || blk >= p.num_blocks) {
+          record_status(p.status, SD_ERR_DEVICE);
+          bad[stage] = 1;
+          mbar_arrive(&full[stage]);
+        } else {
+          bad[stage] = 0;
+          const int p0 = (s.tf + t_lo + t) * kTile;
+          const int row = (blk * p.Hkv + g) * p.bs + (p0 % p.bs);
+          uint8_t *kd = stages + (size_t)stage * C::STAGE_BYTES;
+          uint8_t *vd = kd + C::TILE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+            tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
+            tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+          }
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+    }
+    if (lane == 0 && *abort_flag) {
+      // wait (bounded) for the copies this CTA issued before its shared memory is reused
+      for (int j = (t > STAGES ? t - STAGES : 0); j < t; ++j)
+        mbar_wait_timed(&full[j % STAGES], (j / STAGES) & 1);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------------------------- compute warps
+    const int kg = warp / WPG, wi = warp % WPG, mg = wi / NDG, dg = wi % NDG;
+    const int r0 = mg * 16 + (lane >> 2);
+    const int kq = 2 * (lane & 3);
+    const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(p.q);
+    uint32_t qa[DS / 16][4];
+#pragma unroll
+    for (int ks = 0; ks < DS / 16; ++ks) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = r0 + ((e & 1) ? 8 : 0);
+        const int col = dg * DS + ks * 16 + kq + ((e & 2) ? 8 : 0);
+        uint32_t v = 0;
+        if (row < p.M && nl > 0) {
+          const int j = row / p.G, hh = row % p.G;
+          const size_t off = (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D + col;
+          v = *reinterpret_cast<const uint32_t *>(qg + off);
+        }
+        qa[ks][e] = v;
+      }
+    }
+    int lo0, hi0, lo1, hi1;
+    row_range(p, s, b, r0, lo0, hi0);
+    row_range(p, s, b, r0 + 8, lo1, hi1);
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float o[DS / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < DS / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+
+    int j = 0;
+    for (int t = kg; t < nl; t += KG, ++j) {
+      const int stage = t % STAGES;
+      // warp-uniform decisions: a lane that gave up must not leave the others in a shuffle
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], (t / STAGES) & 1, abort_flag))) {
+        record_status(p.status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      const int buf = j & 1;
+      const int is_bad = bad[stage];
+      const uint32_t kbase = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
+      const uint32_t vbase = kbase + C::TILE_BYTES;
+      const int p0 = (s.tf + t_lo + t) * kTile;
+
+      // ---- partial S = Q K^T over this warp's D slice, summed over the key group's slices
+      float sp[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sp[nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < DS / 16; ++ks) {
+        const int d0 = dg * DS + ks * 16;
+        uint32_t kb[4];
+        const int key = ((lane >> 4) << 3) + (lane & 7);
+        const int col = d0 + ((lane >> 3) & 1) * 8;
+        ldsm_x4(kb, kbase + swz(key, col));
+        mma_bf16_16816(sp[0], qa[ks], kb[0], kb[1]);
+        mma_bf16_16816(sp[1], qa[ks], kb[2], kb[3]);
+      }
+      float sc[2][4];
+      if (NDG == 1) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nt][e] = sp[nt][e];
+      } else {
+        float *myred = red + ((size_t)((kg * 2 + buf) * WPG + wi) * 32 + lane) * 8;
+        reinterpret_cast<float4 *>(myred)[0] =
+            make_float4(sp[0][0], sp[0][1], sp[0][2], sp[0][3]);
+        reinterpret_cast<float4 *>(myred)[1] =
+            make_float4(sp[1][0], sp[1][1], sp[1][2], sp[1][3]);
+        mbar_arrive(&red_bar[kg * 2 + buf]);
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&red_bar[kg * 2 + buf], (j >> 1) & 1, abort_flag))) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+#pragma unroll
+        for (int dd = 0; dd < NDG; ++dd) {
+          const float *src =
+              red + ((size_t)((kg * 2 + buf) * WPG + mg * NDG + dd) * 32 + lane) * 8;
+          const float4 a = reinterpret_cast<const float4 *>(src)[0];
+          const float4 bq = reinterpret_cast<const float4 *>(src)[1];
+          sc[0][0] += a.x;
+          sc[0][1] += a.y;
+          sc[0][2] += a.z;
+          sc[0][3] += a.w;
+          sc[1][0] += bq.x;
+          sc[1][1] += bq.y;
+          sc[1][2] += bq.z;
+          sc[1][3] += bq.w;
+        }
+      }
+
+      // ---- mask, online softmax (base-2 exponent with the scale folded in)
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pos = p0 + nt * 8 + kq + (e & 1);
+          const int lo = (e & 2) ? lo1 : lo0, hi = (e & 2) ? hi1 : hi0;
+          const bool valid = !is_bad && pos >= lo && pos <= hi;
+          const float x = valid ? sc[nt][e] * p.scale_log2 : -INFINITY;
+          sc[nt][e] = x;
+          mx[e >> 1] = fmaxf(mx[e >> 1], x);
+        }
+      float alpha[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+        const float m_new = fmaxf(m_run[h], mx[h]);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha[h] = exp2f(m_run[h] - m_use);
+        m_run[h] = m_new;
+        l_run[h] *= alpha[h];
+        mx[h] = m_use;
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+          sc[nt][e] = pv;
+          l_run[e >> 1] += pv;
+        }
+#pragma unroll
+      for (int nt = 0; nt < DS / 8; ++nt) {
+        o[nt][0] *= alpha[0];
+        o[nt][1] *= alpha[0];
+        o[nt][2] *= alpha[1];
+        o[nt][3] *= alpha[1];
+      }
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
+      pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
+      pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
+      pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+
+      // ---- V rows no query of the item may read can hold anything (rolled-back or never
+      // written slots, NaN included); zero this warp's slice of them so 0 * V stays 0.
+      {
+        int zlo = max(0, min(kTile, s.lo_min - p0));
+        int zhi = max(0, min(kTile, s.hi_max - p0 + 1));
+        if (is_bad) {
+          zlo = kTile;
+          zhi = kTile;
+        }
+        if (zlo > 0 || zhi < kTile) {
+          uint8_t *vt = stages + (size_t)stage * C::STAGE_BYTES + C::TILE_BYTES;
+          for (int u = lane; u < kTile * (DS / 64) * 8; u += 32) {
+            const int row = u / ((DS / 64) * 8);
+            const int rem = u % ((DS / 64) * 8);
+            const int chunk = dg * (DS / 64) + rem / 8;
+            const int unit = rem % 8;
+            if (row < zlo || row >= zhi)
+              *reinterpret_cast<uint4 *>(vt + chunk * (kTile * 128) + row * 128 + unit * 16) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+      }
+
+      // ---- O += P V over this warp's D slice
+#pragma unroll
+      for (int np = 0; np < DS / 16; ++np) {
+        const int d0 = dg * DS + np * 16;
+        uint32_t vb[4];
+        const int key = ((lane >> 3) & 1) * 8 + (lane & 7);
+        const int col = d0 + (lane >> 4) * 8;
+        ldsm_x4_trans(vb, vbase + swz(key, col));
+        mma_bf16_16816(o[2 * np], pa, vb[0], vb[1]);
+        mma_bf16_16816(o[2 * np + 1], pa, vb[2], vb[3]);
+      }
+      mbar_arrive(&empty[stage]);
+    }
+    float l_tot[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float l = l_run[h];
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      l_tot[h] = l;
+    }
+    // every compute warp is done with the tile ring before it holds the partials
+    mbar_arrive(done_bar);
+    if (!mbar_wait(done_bar, 0, abort_flag)) {
+      record_status(p.status, SD_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    float *po = reinterpret_cast<float *>(stages);  // [KG][MP][D]
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = r0 + 8 * h;
+      float *dst = po + ((size_t)kg * MP + row) * D + dg * DS + kq;
+#pragma unroll
+      for (int nt = 0; nt < DS / 8; ++nt)
+        *reinterpret_cast<float2 *>(dst + nt * 8) = make_float2(o[nt][2 * h], o[nt][2 * h + 1]);
+      if (dg == 0 && (lane & 3) == 0)
+        *reinterpret_cast<float2 *>(ml + ((size_t)kg * MP + row) * 2) =
+            make_float2(m_run[h], l_tot[h]);
+    }
+  }
+
+  // ---- merge the cluster's partials: this CTA writes columns [D r / CS, D (r+1) / CS)
+  cluster_sync();
+  {
+    const int cols = D / CS, c4 = cols / 4;
+    const uint32_t po_base = smem_u32(stages), ml_base = smem_u32(ml);
+    __nv_bfloat16 *outg = reinterpret_cast<__nv_bfloat16 *>(p.out);
+    for (int u = threadIdx.x; u < p.M * c4; u += C::THREADS) {
+      const int row = u / c4, col = (int)rank * cols + (u % c4) * 4;
+      float m_acc = -INFINITY, l_acc = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < CS; ++q) {
+        float2 mlv[KG];
+        float4 ov[KG];
+#pragma unroll
+        for (int k = 0; k < KG; ++k) {
+          mlv[k] = ld_dsmem_f2(dsmem_addr(ml_base + (uint32_t)((k * MP + row) * 2 * 4), q));
+          ov[k] = ld_dsmem_f4(
+              dsmem_addr(po_base + (uint32_t)(((size_t)(k * MP + row) * D + col) * 4), q));
+        }
+#pragma unroll
+        for (int k = 0; k < KG; ++k) {
+          if (mlv[k].x == -INFINITY) continue;
+          const float m_new = fmaxf(m_acc, mlv[k].x);
+          const float a = exp2f(m_acc - m_new), w = exp2f(mlv[k].x - m_new);
+          l_acc = l_acc * a + mlv[k].y * w;
+          acc.x = acc.x * a + ov[k].x * w;
+          acc.y = acc.y * a + ov[k].y * w;
+          acc.z = acc.z * a + ov[k].z * w;
+          acc.w = acc.w * a + ov[k].w * w;
+          m_acc = m_new;
+        }
+      }
+      const float inv = l_acc > 0.f ? 1.f / l_acc : 0.f;
+      const int jq = row / p.G, hh = row % p.G;
+      __nv_bfloat16 *dst =
+          outg + (((size_t)b * p.n_q + jq) * p.Hq + (size_t)g * p.G + hh) * D + col;
+      *reinterpret_cast<uint2 *>(dst) =
+          make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    }
+  }
+  cluster_sync();  // no CTA leaves while another may still read its shared memory
+}
+
 // Merges the partials of items that several CTAs shared, in CTA order; writes zero rows for
 // drafter items with an empty key range.  One CTA per (item, query row).
 template <typename T>
@@ -576,6 +967,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
   __shared__ int s_n;
   __shared__ float s_w[kChunk];
   __shared__ float s_red[4];
+  pdl_trigger();
+  pdl_wait();
   const int item = blockIdx.x, row = blockIdx.y;
   const int b = item / p.Hkv, g = item % p.Hkv;
   if (threadIdx.x < 32) {  // tile counts of all sequences, one warp
@@ -690,6 +1083,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
 template <typename T>
 __global__ void append_kv_kernel(const Params p, const T *k_new, const T *v_new, T *k_cache,
                                  T *v_cache) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x / p.n_q, j = blockIdx.x % p.n_q;
   const int L = p.ctx_len[b];
   if (L < 0) return;  // reported by the attention kernel
@@ -718,6 +1113,7 @@ __global__ void append_kv_kernel(const Params p, const T *k_new, const T *v_new,
 
 // float32 path: one warp per (sequence, query position, head).
 __global__ void attn_f32_kernel(const Params p, const float *k_cache, const float *v_cache) {
+  pdl_wait();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int total = p.B * p.n_q * p.Hq;
@@ -789,8 +1185,9 @@ struct Launcher {
   }
   static sd_status launch(const CUtensorMap &km, const CUtensorMap &vm, const Params &p,
                           cudaStream_t st) {
-    attn_bf16_kernel<D, MT, STAGES><<<p.P, C::THREADS, C::SMEM, st>>>(km, vm, p);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(
+        sdv::launch(attn_bf16_kernel<D, MT, STAGES>, dim3(p.P), dim3(C::THREADS), C::SMEM, st,
+                    km, vm, p));
   }
 };
 
@@ -821,6 +1218,85 @@ static sd_status launch_bf16(int D, int MT, const CUtensorMap &km, const CUtenso
   SDV_CASE(128, 1) SDV_CASE(128, 2) SDV_CASE(128, 3) SDV_CASE(128, 4)
   SDV_CASE(256, 1) SDV_CASE(256, 2) SDV_CASE(256, 3) SDV_CASE(256, 4)
   SDV_CASE(512, 1) SDV_CASE(512, 2) SDV_CASE(512, 3) SDV_CASE(512, 4)
+#undef SDV_CASE
+  return SD_ERR_UNSUPPORTED;
+}
+
+// Sliding windows up to this many keys take the cluster path (one launch, no workspace).
+constexpr int kWinMax = 2048;
+
+template <int D, int MT>
+struct WLauncher {
+  using C = WCfg<D, MT>;
+  // Clusters of 1, 2, 4 and 8 CTAs resident at once on the current device.
+  static const int *max_clusters() {
+    static int cache[64][4];
+    static int dev_ok[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && dev_ok[dev] == dev + 1) return cache[dev];
+    static int scratch[4];
+    int *out = dev < 64 ? cache[dev] : scratch;
+    cudaFuncSetAttribute(attn_window_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)C::SMEM);
+    for (int i = 0; i < 4; ++i) {
+      const int cs = 1 << i;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs);
+      cfg.blockDim = dim3(C::THREADS);
+      cfg.dynamicSmemBytes = C::SMEM;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = cs;
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      cfg.attrs = a;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, attn_window_kernel<D, MT>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      out[i] = n;
+    }
+    if (dev < 64) dev_ok[dev] = dev + 1;
+    return out;
+  }
+  static sd_status launch(const CUtensorMap &km, const CUtensorMap &vm, const Params &p,
+                          int tiles_max, cudaStream_t st) {
+    const int *mc = max_clusters();
+    if (mc[0] <= 0) return SD_ERR_CUDA;
+    const int items = p.B * p.Hkv;
+    int cs = 1;
+    for (int i = 3; i >= 1; --i)
+      if ((1 << i) <= tiles_max && items <= mc[i]) {
+        cs = 1 << i;
+        break;
+      }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(items * cs);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute a[2];
+    a[0].id = cudaLaunchAttributeClusterDimension;
+    a[0].val.clusterDim.x = cs;
+    a[0].val.clusterDim.y = 1;
+    a[0].val.clusterDim.z = 1;
+    a[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, attn_window_kernel<D, MT>, km, vm, p, cs));
+  }
+};
+
+static sd_status launch_window(int D, int MT, const CUtensorMap &km, const CUtensorMap &vm,
+                               const Params &p, int tiles_max, cudaStream_t st) {
+#define SDV_CASE(DD, MM) \
+  if (D == DD && MT == MM) return WLauncher<DD, MM>::launch(km, vm, p, tiles_max, st);
+  SDV_CASE(64, 1) SDV_CASE(64, 2) SDV_CASE(128, 1) SDV_CASE(128, 2)
+  SDV_CASE(256, 1) SDV_CASE(256, 2) SDV_CASE(512, 1) SDV_CASE(512, 2)
 #undef SDV_CASE
   return SD_ERR_UNSUPPORTED;
 }
@@ -899,14 +1375,14 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
 
   if (d->dtype == SD_F32) {
     if (!draft) {
-      append_kv_kernel<float><<<p.B * p.n_q, 256, 0, st>>>(
-          p, (const float *)k_new, (const float *)v_new, (float *)k_cache, (float *)v_cache);
-      if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+      if (launch(append_kv_kernel<float>, dim3(p.B * p.n_q), dim3(256), 0, st, p,
+                 (const float *)k_new, (const float *)v_new, (float *)k_cache,
+                 (float *)v_cache) != cudaSuccess)
+        return SD_ERR_CUDA;
     }
     const int warps = p.B * p.n_q * p.Hq;
-    attn_f32_kernel<<<(warps + 3) / 4, 128, 0, st>>>(p, (const float *)k_cache,
-                                                      (const float *)v_cache);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch(attn_f32_kernel, dim3((warps + 3) / 4), dim3(128), 0, st, p,
+                              (const float *)k_cache, (const float *)v_cache));
   }
 
   // bf16
@@ -928,15 +1404,20 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
       !encode_tmap_2d_bf16(&vm, v_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile))
     return SD_ERR_CUDA;
   if (!draft) {
-    append_kv_kernel<__nv_bfloat16><<<p.B * p.n_q, 256, 0, st>>>(
-        p, (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new,
-        (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache);
-    if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+    if (launch(append_kv_kernel<__nv_bfloat16>, dim3(p.B * p.n_q), dim3(256), 0, st, p,
+               (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new,
+               (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache) != cudaSuccess)
+      return SD_ERR_CUDA;
+  }
+  if (p.window > 0 && p.window <= kWinMax && MT <= 2) {
+    // every item reads at most window + n_q - 1 keys, over at most this many 16-key tiles
+    const int tiles_max = (p.window + p.n_q - 1 + kTile - 1) / kTile + 1;
+    return launch_window(p.D, MT, km, vm, p, tiles_max, st);
   }
   s = launch_bf16(p.D, MT, km, vm, p, st);
   if (s != SD_OK) return s;
-  attn_combine_kernel<__nv_bfloat16><<<dim3(p.B * p.Hkv, p.M), 128, 0, st>>>(p);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(
+      launch(attn_combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hkv, p.M), dim3(128), 0, st, p));
 }
 
 }  // namespace attn

@@ -36,6 +36,8 @@ struct Params {
 };
 
 __global__ void commit_kernel(const Params p) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   __shared__ int s_a, s_L;
   if (threadIdx.x == 0) {
@@ -149,6 +151,5 @@ extern "C" sd_status sd_commit(const sd_commit_desc *desc, const int32_t *block_
   }
   p.step_ptr = reinterpret_cast<unsigned long long *>(desc->step_ptr);
   p.status = device_status_word();
-  commit_kernel<<<p.B, 256, 0, (cudaStream_t)stream>>>(p);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch(commit_kernel, dim3(p.B), dim3(256), 0, (cudaStream_t)stream, p));
 }

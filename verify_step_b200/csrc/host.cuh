@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/sd_verify.h"
 
 namespace sdv {
@@ -22,6 +24,29 @@ bool encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uin
                          uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 
 inline sd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_CUDA; }
+
+// Programmatic dependent launch: off unless the environment sets SDV_PDL=1 (read once per
+// process).  Every kernel calls pdl_wait() before its first global access, so either way is
+// correct; on the spec step the plain stream order measured faster.
+bool pdl_enabled();
+
+// Launches ``kernel`` with programmatic stream serialization (the kernel must call pdl_wait()
+// before touching global memory written by earlier work in the stream).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

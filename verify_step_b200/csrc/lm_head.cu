@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // h (and the logits buffer) may come from earlier kernels
 
   if (warp == 0) {
     // ----------------------------------------------------------------------- producer
@@ -202,6 +204,7 @@ __global__ void __launch_bounds__(192, 1)
 
 // float32: one warp per (vocab row); all m rows.
 __global__ void lm_head_f32_kernel(const float *h, const float *w, const Params p) {
+  pdl_wait();
   const int v = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (v >= p.V) return;
@@ -227,6 +230,8 @@ __device__ __forceinline__ unsigned long long topc_key(float score, int id) {
 // shuffles for strides below 32 and shared memory above.
 __global__ void topc_small_kernel(const float *scores, int C, int top_c, int32_t *sel) {
   __shared__ unsigned long long sk[1024];
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x, i = threadIdx.x, n = blockDim.x;
   unsigned long long key = i < C ? topc_key(scores[(size_t)m * C + i], i) : ~0ull;
   for (int size = 2; size <= n; size <<= 1) {
@@ -256,6 +261,7 @@ __global__ void topc_small_kernel(const float *scores, int C, int top_c, int32_t
 
 __global__ void topc_kernel(const float *scores, int C, int top_c, int32_t *sel) {
   extern __shared__ unsigned long long keys[];
+  pdl_wait();
   const int m = blockIdx.x;
   int n = 1;
   while (n < C) n <<= 1;
@@ -299,6 +305,7 @@ __global__ void topc_kernel(const float *scores, int C, int top_c, int32_t *sel)
 
 // -inf into rows [m, 0 .. V) of the logits; blockIdx.y = row.
 __global__ void fill_neg_inf_kernel(float *logits, int V, int ld, int vec4) {
+  pdl_wait();
   float *row = logits + (size_t)blockIdx.y * ld;
   const int stride = gridDim.x * blockDim.x;
   if (vec4) {
@@ -320,6 +327,8 @@ __global__ void __launch_bounds__(256) cluster_logits_kernel(
     const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm, const int32_t *cluster_tokens,
     const int32_t *sel, int M, int top_c, int cs, int d, int C, int V, int ld, float *logits,
     int *status) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int TK = 2;
   const int lane = threadIdx.x & 31;
   const long long n_warps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -394,6 +403,8 @@ __global__ void __launch_bounds__(256) centroid_scores_kernel(const __nv_bfloat1
                                                               const __nv_bfloat16 *cent, int M,
                                                               int d, int C, float *scores) {
   extern __shared__ float hs[];  // [M][d]
+  pdl_trigger();
+  pdl_wait();
   for (int i = threadIdx.x; i < M * d / 8; i += blockDim.x) {
     const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(h) + i);
     const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
@@ -480,8 +491,8 @@ static sd_status launch_umma(const void *h, const void *w, int M, int d, int V, 
   const int sms = sm_count();
   if (sms <= 0) return SD_ERR_CUDA;
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  lm_head_umma_kernel<N><<<grid, C::THREADS, C::SMEM, st>>>(wm, hm, p);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(
+      launch(lm_head_umma_kernel<N>, dim3(grid), dim3(C::THREADS), C::SMEM, st, wm, hm, p));
 }
 
 // Dense bf16 projection of up to 256 rows.
@@ -546,9 +557,8 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
     p.V = desc->vocab;
     p.ld = ld;
     p.logits = logits;
-    lm_head_f32_kernel<<<(desc->vocab + 7) / 8, 256, 0, st>>>((const float *)h, (const float *)w,
-                                                              p);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch(lm_head_f32_kernel, dim3((desc->vocab + 7) / 8), dim3(256), 0, st,
+                              (const float *)h, (const float *)w, p));
   }
   if (!aligned16(h) || !aligned16(w)) return SD_ERR_INVALID_ARG;
   const size_t hrow = (size_t)desc->d * 2;
@@ -568,9 +578,10 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   float *scores = reinterpret_cast<float *>(ws);
   const int C = desc->n_clusters;
   if (desc->m <= 16 && desc->d <= 1024 && (size_t)desc->m * desc->d * 4 <= 48 * 1024) {
-    centroid_scores_kernel<<<(C + 7) / 8, 256, (size_t)desc->m * desc->d * 4, st>>>(
-        (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)centroids, desc->m, desc->d, C, scores);
-    if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+    if (launch(centroid_scores_kernel, dim3((C + 7) / 8), dim3(256),
+               (size_t)desc->m * desc->d * 4, st, (const __nv_bfloat16 *)h,
+               (const __nv_bfloat16 *)centroids, desc->m, desc->d, C, scores) != cudaSuccess)
+      return SD_ERR_CUDA;
   } else {
     for (int m0 = 0; m0 < desc->m; m0 += 256) {
       const int mm = desc->m - m0 < 256 ? desc->m - m0 : 256;
@@ -583,15 +594,17 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   while (n < C) n <<= 1;
   if (n < 32) n = 32;
   if (n <= 1024)
-    topc_small_kernel<<<desc->m, n, 0, st>>>(scores, C, desc->top_c, sel_clusters);
+    s = cuda_status(launch(topc_small_kernel, dim3(desc->m), dim3(n), 0, st, (const float *)scores,
+                           C, desc->top_c, sel_clusters));
   else
-    topc_kernel<<<desc->m, 512, (size_t)n * 8, st>>>(scores, C, desc->top_c, sel_clusters);
-  if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+    s = cuda_status(launch(topc_kernel, dim3(desc->m), dim3(512), (size_t)n * 8, st,
+                           (const float *)scores, C, desc->top_c, sel_clusters));
+  if (s != SD_OK) return s;
   const int vec4 = aligned16(logits) && desc->vocab % 4 == 0 && ld % 4 == 0;
   const int per_row = (desc->vocab / (vec4 ? 4 : 1) + 255) / 256;
-  fill_neg_inf_kernel<<<dim3(per_row < 64 ? per_row : 64, desc->m), 256, 0, st>>>(
-      logits, desc->vocab, ld, vec4);
-  if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
+  if (launch(fill_neg_inf_kernel, dim3(per_row < 64 ? per_row : 64, desc->m), dim3(256), 0, st,
+             logits, desc->vocab, ld, vec4) != cudaSuccess)
+    return SD_ERR_CUDA;
   // persistent warps: as many 8-warp CTAs as fit on the device at once
   const int sms = sm_count();
   int occ = 0;
@@ -601,15 +614,18 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<16>, 256, 0);
   const dim3 grid((occ > 0 ? occ : 1) * (sms > 0 ? sms : 148));
   if (desc->d <= 1024)
-    cluster_logits_kernel<4><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
-        desc->m, desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
-        device_status_word());
+    s = cuda_status(launch(cluster_logits_kernel<4>, grid, dim3(256), 0, st,
+                           (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens,
+                           (const int32_t *)sel_clusters, desc->m, desc->top_c,
+                           desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
+                           device_status_word()));
   else
-    cluster_logits_kernel<16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens, sel_clusters,
-        desc->m, desc->top_c, desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
-        device_status_word());
+    s = cuda_status(launch(cluster_logits_kernel<16>, grid, dim3(256), 0, st,
+                           (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens,
+                           (const int32_t *)sel_clusters, desc->m, desc->top_c,
+                           desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
+                           device_status_word()));
+  return s;
   return cuda_status(cudaGetLastError());
 }
 
