@@ -280,45 +280,59 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
 
   if (warp == NCW) {
     // ------------------------------------------------------------------- producer warp
-    if (lane != 0) return;
-    tma_prefetch_desc(&kmap);
-    tma_prefetch_desc(&vmap);
+    // The whole warp walks the cursor; its lanes fetch the block-table entries of the next 32
+    // tiles of the current sequence at once (off the per-tile path), lane 0 issues the copies.
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+    }
     Cursor c;
     cursor_begin(p, tab, start, end - start, c);
     uint32_t it = 0;
+    int pf_b = -1, pf_base = 0, blk_l = -1;
     while (c.left > 0) {
-      const int stage = it % STAGES;
-      const uint32_t ph = (it / STAGES) & 1;
-      if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) {
-        record_status(p.status, SD_ERR_TIMEOUT);
-        *abort_flag = 1;
-        break;
+      const int ti = c.s.tf + c.tau;  // tile index inside sequence c.b
+      if (c.b != pf_b || ti < pf_base || ti >= pf_base + 32) {
+        pf_b = c.b;
+        pf_base = ti;
+        blk_l = -1;
+        const int bidx = (ti + lane) * kTile / p.bs;
+        if (ti + lane < c.s.tf + c.s.n && bidx < p.mbps)
+          blk_l = p.table[(size_t)c.b * p.mbps + bidx];
       }
-      const int p0 = (c.s.tf + c.tau) * kTile;
-      const int bidx = p0 / p.bs;
-      int blk = -1;
-      if (bidx < p.mbps) blk = p.table[(size_t)c.b * p.mbps + bidx];
-      if (blk < 0 || blk >= p.num_blocks) {
-        record_status(p.status, SD_ERR_DEVICE);
-        bad[stage] = 1;
-        mbar_arrive(&full[stage]);
-      } else {
-        bad[stage] = 0;
-        const int row = (blk * p.Hkv + c.g) * p.bs + (p0 % p.bs);
-        uint8_t *kd = stages + (size_t)stage * C::STAGE_BYTES;
-        uint8_t *vd = kd + C::TILE_BYTES;
-        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+      const int blk = __shfl_sync(0xffffffffu, blk_l, ti - pf_base);
+      int go = 1;
+      if (lane == 0) {
+        const int stage = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          go = 0;
+        } else if (blk < 0 || blk >= p.num_blocks) {
+          record_status(p.status, SD_ERR_DEVICE);
+          bad[stage] = 1;
+          mbar_arrive(&full[stage]);
+        } else {
+          bad[stage] = 0;
+          const int p0 = ti * kTile;
+          const int row = (blk * p.Hkv + c.g) * p.bs + (p0 % p.bs);
+          uint8_t *kd = stages + (size_t)stage * C::STAGE_BYTES;
+          uint8_t *vd = kd + C::TILE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
 #pragma unroll
-        for (int ch = 0; ch < D / 64; ++ch) {
-          tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
-          tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+          for (int ch = 0; ch < D / 64; ++ch) {
+            tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
+            tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+          }
         }
       }
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
       ++it;
       --c.left;
       if (++c.tau == c.s.n && c.left > 0) cursor_next_item(p, tab, c);
     }
-    if (*abort_flag) {
+    if (lane == 0 && *abort_flag) {
       // wait (bounded) for the copies this CTA issued before leaving
       for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
         mbar_wait_timed(&full[j % STAGES], (j / STAGES) & 1);
@@ -574,33 +588,43 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
 // separate merge kernel.  A cluster of CS CTAs takes one item (sequence b, kv head g); CTA
 // rank r streams tiles [n r / CS, n (r+1) / CS) of it, all of them in flight at once where the
 // shared-memory ring holds them.  Inside a CTA, KG key groups of warps take the CTA's tiles
-// round robin, each with its own online softmax.  The CS * KG partials (m, l, o) are merged
-// through distributed shared memory in (rank, key group) order: CTA r writes output columns
-// [D r / CS, D (r+1) / CS).  No workspace, one launch per call.
+// round robin, each with its own online softmax.  Each CTA merges its KG partials (m, l, o) in
+// key-group order and pushes the result, column slice by column slice, into the shared memory
+// of the CTA owning that slice (CTA r owns output columns [D r / CS, D (r+1) / CS)); after one
+// cluster barrier every CTA merges the CS partials of its slice in rank order and writes it.
+// No workspace, one launch per call.
 
 template <int D, int MT>
 struct WCfg {
   static constexpr int DS = D >= 128 ? 128 : 64;
   static constexpr int NDG = D / DS;
   static constexpr int WPG = MT * NDG;                  // warps of one key group
-  static constexpr int KG = 8 / WPG > 0 ? 8 / WPG : 1;  // key groups per CTA
+  // key groups per CTA: at most 7 warps with two 16x128 slices or more per warp group, so the
+  // register file of a sub-partition holds two warps of 255 registers (no spills)
+  static constexpr int KG = WPG == 1 ? 8 : (6 / WPG > 0 ? 6 / WPG : 1);
   static constexpr int NCW = KG * WPG;
   static constexpr int THREADS = 32 * (NCW + 1);
   static constexpr int MP = 16 * MT;  // padded rows of an item
+  static constexpr int MAX_CS = 8;    // CTAs per cluster at most
   static constexpr int TILE_BYTES = kTile * D * 2;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
+  static constexpr int ML_FLOATS = KG * MP * 2;       // key-group (m, l) partials
+  static constexpr int RECV_FLOATS = MP * D;          // [CS][MP][D / CS] pushed column slices
+  static constexpr int RECV_ML_FLOATS = MAX_CS * MP * 2;
+  static constexpr size_t PART_BYTES = (size_t)KG * MP * D * 4;
+  static constexpr size_t FIXED = 1024 + (size_t)(RED_FLOATS + ML_FLOATS + RECV_FLOATS +
+                                                  RECV_ML_FLOATS) * 4 + 8 * (2 * 16 + 2 * KG + 1) +
+                                  4 * (1 + 16) + 16;
   // A multiple of KG: tiles t and t + STAGES share a stage and belong to the same key group,
   // which consumes them in order (so a parity wait never sees the stage's previous phase).
-  static constexpr int RING = (192 * 1024) / STAGE_BYTES > 16 ? 16 : (192 * 1024) / STAGE_BYTES;
+  static constexpr int RING = (227 * 1024 - FIXED) / STAGE_BYTES > 16
+                                  ? 16
+                                  : (int)((227 * 1024 - FIXED) / STAGE_BYTES);
   static constexpr int STAGES = RING / KG * KG;
   static_assert(STAGES >= KG, "at least one stage per key group");
-  static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
-  static constexpr int ML_FLOATS = KG * MP * 2;
-  static constexpr size_t PART_BYTES = (size_t)KG * MP * D * 4;
   static_assert(PART_BYTES <= (size_t)STAGES * STAGE_BYTES, "partials reuse the tile ring");
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + RED_FLOATS * 4 +
-                                 ML_FLOATS * 4 + 8 * (2 * STAGES + 2 * KG + 1) + 4 * (1 + STAGES) +
-                                 16;
+  static constexpr size_t SMEM = FIXED + (size_t)STAGES * STAGE_BYTES;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -617,7 +641,9 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
   uint8_t *stages = smem;
   float *red = reinterpret_cast<float *>(smem + (size_t)STAGES * C::STAGE_BYTES);
   float *ml = red + C::RED_FLOATS;  // [KG][MP][2] partial (m, l) per row
-  uint64_t *full = reinterpret_cast<uint64_t *>(ml + C::ML_FLOATS);
+  float *recv = ml + C::ML_FLOATS;  // [CS][MP][D / CS] partials of this CTA's column slice
+  float *recv_ml = recv + C::RECV_FLOATS;  // [CS][MP][2]
+  uint64_t *full = reinterpret_cast<uint64_t *>(recv_ml + C::RECV_ML_FLOATS);
   uint64_t *empty = full + STAGES;
   uint64_t *red_bar = empty + STAGES;  // [KG][2]
   uint64_t *done_bar = red_bar + 2 * KG;
@@ -628,6 +654,10 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const int item = blockIdx.x / CS;
   const int b = item / p.Hkv, g = item % p.Hkv;
+  pdl_trigger();
+  pdl_wait();
+  // thread 0 sets up the barriers while the other threads' loads of the sequence's range and
+  // the tensor-map prefetch are in flight
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -639,10 +669,12 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  pdl_trigger();
-  pdl_wait();
-  __syncthreads();
+  if (warp == NCW && lane == 0) {
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+  }
   const SeqRange s = seq_range(p, b, threadIdx.x == 0 && g == 0 && rank == 0);
+  __syncthreads();
   const int t_lo = (int)((long long)s.n * rank / CS);
   const int nl = (int)((long long)s.n * (rank + 1) / CS) - t_lo;
 
@@ -650,10 +682,6 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
     // ------------------------------------------------------------------- producer warp
     // The whole warp walks the tiles; its lanes fetch the block-table entries of the next
     // 32 tiles at once, lane 0 issues the copies.
-    if (lane == 0) {
-      tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
-    }
     int base = -32, blk_l = -1, t = 0;
     for (; t < nl; ++t) {
       if (t - base >= 32) {
@@ -905,6 +933,7 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int row = r0 + 8 * h;
+      if (row >= p.M) continue;
       float *dst = po + ((size_t)kg * MP + row) * D + dg * DS + kq;
 #pragma unroll
       for (int nt = 0; nt < DS / 8; ++nt)
@@ -914,48 +943,69 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
             make_float2(m_run[h], l_tot[h]);
     }
   }
+  __syncthreads();
 
-  // ---- merge the cluster's partials: this CTA writes columns [D r / CS, D (r+1) / CS)
-  cluster_sync();
-  {
-    const int cols = D / CS, c4 = cols / 4;
-    const uint32_t po_base = smem_u32(stages), ml_base = smem_u32(ml);
-    __nv_bfloat16 *outg = reinterpret_cast<__nv_bfloat16 *>(p.out);
-    for (int u = threadIdx.x; u < p.M * c4; u += C::THREADS) {
-      const int row = u / c4, col = (int)rank * cols + (u % c4) * 4;
-      float m_acc = -INFINITY, l_acc = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q = 0; q < CS; ++q) {
-        float2 mlv[KG];
-        float4 ov[KG];
+  // ---- key-group merge of each (row, 4 columns), pushed to the CTA owning the columns
+  const int cols = D / CS;
+  for (int u = threadIdx.x; u < p.M * (D / 4); u += C::THREADS) {
+    const int row = u / (D / 4), col = (u % (D / 4)) * 4;
+    float2 mlv[KG];
+    float4 ov[KG];
 #pragma unroll
-        for (int k = 0; k < KG; ++k) {
-          mlv[k] = ld_dsmem_f2(dsmem_addr(ml_base + (uint32_t)((k * MP + row) * 2 * 4), q));
-          ov[k] = ld_dsmem_f4(
-              dsmem_addr(po_base + (uint32_t)(((size_t)(k * MP + row) * D + col) * 4), q));
-        }
-#pragma unroll
-        for (int k = 0; k < KG; ++k) {
-          if (mlv[k].x == -INFINITY) continue;
-          const float m_new = fmaxf(m_acc, mlv[k].x);
-          const float a = exp2f(m_acc - m_new), w = exp2f(mlv[k].x - m_new);
-          l_acc = l_acc * a + mlv[k].y * w;
-          acc.x = acc.x * a + ov[k].x * w;
-          acc.y = acc.y * a + ov[k].y * w;
-          acc.z = acc.z * a + ov[k].z * w;
-          acc.w = acc.w * a + ov[k].w * w;
-          m_acc = m_new;
-        }
-      }
-      const float inv = l_acc > 0.f ? 1.f / l_acc : 0.f;
-      const int jq = row / p.G, hh = row % p.G;
-      __nv_bfloat16 *dst =
-          outg + (((size_t)b * p.n_q + jq) * p.Hq + (size_t)g * p.G + hh) * D + col;
-      *reinterpret_cast<uint2 *>(dst) =
-          make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    for (int k = 0; k < KG; ++k) {
+      mlv[k] = *reinterpret_cast<const float2 *>(ml + ((size_t)k * MP + row) * 2);
+      ov[k] = *reinterpret_cast<const float4 *>(
+          reinterpret_cast<const float *>(stages) + ((size_t)k * MP + row) * D + col);
     }
+    float m_acc = -INFINITY, l_acc = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < KG; ++k) {
+      if (mlv[k].x == -INFINITY) continue;
+      const float m_new = fmaxf(m_acc, mlv[k].x);
+      const float a = exp2f(m_acc - m_new), w = exp2f(mlv[k].x - m_new);
+      l_acc = l_acc * a + mlv[k].y * w;
+      acc.x = acc.x * a + ov[k].x * w;
+      acc.y = acc.y * a + ov[k].y * w;
+      acc.z = acc.z * a + ov[k].z * w;
+      acc.w = acc.w * a + ov[k].w * w;
+      m_acc = m_new;
+    }
+    const int owner = col / cols, cc = col % cols;
+    st_dsmem_f4(dsmem_addr(smem_u32(recv + ((size_t)rank * MP + row) * cols + cc), owner), acc);
+    if (cc == 0)
+      st_dsmem_f2(dsmem_addr(smem_u32(recv_ml + ((size_t)rank * MP + row) * 2), owner),
+                  make_float2(m_acc, l_acc));
   }
-  cluster_sync();  // no CTA leaves while another may still read its shared memory
+  cluster_sync();  // every CTA's pushes have landed; nothing below touches another CTA
+
+  // ---- this CTA's column slice: the CS partials merged in rank order
+  __nv_bfloat16 *outg = reinterpret_cast<__nv_bfloat16 *>(p.out);
+  for (int u = threadIdx.x; u < p.M * (cols / 4); u += C::THREADS) {
+    const int row = u / (cols / 4), cc = (u % (cols / 4)) * 4;
+    float m_acc = -INFINITY, l_acc = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < CS; ++q) {
+      const float2 mlq = *reinterpret_cast<const float2 *>(recv_ml + ((size_t)q * MP + row) * 2);
+      if (mlq.x == -INFINITY) continue;
+      const float4 oq =
+          *reinterpret_cast<const float4 *>(recv + ((size_t)q * MP + row) * cols + cc);
+      const float m_new = fmaxf(m_acc, mlq.x);
+      const float a = exp2f(m_acc - m_new), w = exp2f(mlq.x - m_new);
+      l_acc = l_acc * a + mlq.y * w;
+      acc.x = acc.x * a + oq.x * w;
+      acc.y = acc.y * a + oq.y * w;
+      acc.z = acc.z * a + oq.z * w;
+      acc.w = acc.w * a + oq.w * w;
+      m_acc = m_new;
+    }
+    const float inv = l_acc > 0.f ? 1.f / l_acc : 0.f;
+    const int jq = row / p.G, hh = row % p.G;
+    __nv_bfloat16 *dst = outg + (((size_t)b * p.n_q + jq) * p.Hq + (size_t)g * p.G + hh) * D +
+                         (int)rank * cols + cc;
+    *reinterpret_cast<uint2 *>(dst) =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+  }
 }
 
 // Merges the partials of items that several CTAs shared, in CTA order; writes zero rows for
