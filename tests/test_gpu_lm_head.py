@@ -144,3 +144,36 @@ def test_drafter_clustered_config():
     h = S.make_hidden(w, w.batch, d=w.drafter_hidden)
     assert _check_clustered(h, cl, w.top_c) <= 2
     assert status_ok()
+
+
+@pytest.mark.parametrize("C,cs,top_c", [(300, 3, 17), (4096, 2, 64), (8192, 1, 5)])
+def test_clustered_cluster_counts(C, cs, top_c):
+    """Cluster counts that are not multiples of the selection block, up to the 8192 limit."""
+    w = S.Workload("c", 4, 0, 0, 4, 1, [], 64, C * cs, n_clusters=C, cluster_size=cs,
+                   drafter_hidden=64, seed=33)
+    cl = S.make_clustered_head(w)
+    h = S.bf16(S.normal(7, (6, 64)))
+    assert _check_clustered(h, cl, top_c) <= 1
+    assert status_ok()
+
+
+def test_clustered_exact_ties_go_to_lower_ids():
+    """Equal scores at the selection boundary: the lower cluster ids are kept.  Centroids are
+    +v for a scattered set of 100 clusters and -v elsewhere, so every row's scores take two
+    bit-identical values and the kept set is the 40 lowest ids of the +v set."""
+    C, cs, d, top_c = 512, 2, 64, 40
+    w = S.Workload("c", 4, 0, 0, 4, 1, [], d, C * cs, n_clusters=C, cluster_size=cs,
+                   drafter_hidden=d, seed=34)
+    cl = S.make_clustered_head(w)
+    rng = np.random.default_rng(34)
+    plus = np.sort(rng.choice(C, size=100, replace=False))
+    v = S.bf16(S.normal(8, (1, d)))[0]
+    cent = (-v).repeat(C, 1)
+    cent[torch.from_numpy(plus).long()] = v
+    cl["centroids"] = cent.contiguous()
+    h = v.float().repeat(3, 1)
+    h[1] *= 2.0
+    h = h.to(torch.bfloat16)
+    _, sel = _run_clustered(h, cl, top_c)
+    assert sel.tolist() == [plus[:top_c].tolist()] * 3
+    assert status_ok()

@@ -218,103 +218,133 @@ __global__ void lm_head_f32_kernel(const float *h, const float *w, const Params 
   }
 }
 
-// Per row: the top_c clusters by score (ties -> lower id), written in ascending id order.
-// Bitonic sort of (descending score, ascending id) keys in shared memory.
-__device__ __forceinline__ unsigned long long topc_key(float score, int id) {
-  uint32_t u = __float_as_uint(score);
-  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);         // ascending order of floats
-  return ((unsigned long long)(~u) << 32) | (uint32_t)id;  // descending score, then id
+// Per row m (blockIdx.y): block 0 selects the top_c clusters by score (ties -> lower id) and
+// writes them in ascending id order; blocks 1.. write -inf over the row's logits meanwhile
+// (the kept clusters' tokens are overwritten by the next kernel).
+//
+// Selection: an exact radix select over 32-bit keys ordered by descending score (smaller key =
+// higher score; -0.0 and +0.0 are one key), most significant byte first, finds the key T of
+// the top_c-th best cluster and how many clusters with key T are kept; the kept set is then
+// read out in id order with two block scans (ties at T go to the lowest ids).
+constexpr int kSelThreads = 256;
+
+__device__ __forceinline__ uint32_t desc_key(float score) {
+  uint32_t u = __float_as_uint(score == 0.f ? 0.f : score);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending order of floats
+  return ~u;
 }
 
-// Same selection for n_pow2 <= 1024 clusters: one key per thread, bitonic sort with warp
-// shuffles for strides below 32 and shared memory above.
-__global__ void topc_small_kernel(const float *scores, int C, int top_c, int32_t *sel) {
-  __shared__ unsigned long long sk[1024];
-  pdl_trigger();
+// Exclusive prefix sum of v over the block (kSelThreads threads); also returns the total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *s_warp, int &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  int base = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    const int t = s_warp[w];
+    base += w < warp ? t : 0;
+    total += t;
+  }
+  __syncthreads();
+  return base + x - v;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_fill_kernel(const float *scores, int C,
+                                                                  int top_c, int32_t *sel,
+                                                                  float *logits, int V, int ld,
+                                                                  int vec4) {
+  extern __shared__ uint32_t skey[];  // [C]
+  __shared__ int hist[256];
+  __shared__ int s_warp[kSelThreads / 32];
+  __shared__ int s_digit, s_before;
   pdl_wait();
-  const int m = blockIdx.x, i = threadIdx.x, n = blockDim.x;
-  unsigned long long key = i < C ? topc_key(scores[(size_t)m * C + i], i) : ~0ull;
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      unsigned long long other;
-      if (stride >= 32) {
-        sk[i] = key;
-        __syncthreads();
-        other = sk[i ^ stride];
-        __syncthreads();
-      } else {
-        other = __shfl_xor_sync(0xffffffffu, key, stride);
+  const int m = blockIdx.y;
+  if (blockIdx.x > 0) {
+    float *row = logits + (size_t)m * ld;
+    const int nb = gridDim.x - 1, bx = blockIdx.x - 1;
+    if (vec4) {
+      float4 *r4 = reinterpret_cast<float4 *>(row);
+      const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      for (int i = bx * kSelThreads + threadIdx.x; i < V / 4; i += nb * kSelThreads) r4[i] = ninf;
+    } else {
+      for (int i = bx * kSelThreads + threadIdx.x; i < V; i += nb * kSelThreads)
+        row[i] = -INFINITY;
+    }
+    return;
+  }
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i < C; i += kSelThreads) skey[i] = desc_key(scores[(size_t)m * C + i]);
+  uint32_t prefix = 0, mask = 0;
+  int need = top_c;  // clusters still to take among the keys matching prefix under mask
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    hist[tid] = 0;  // kSelThreads == 256 bins
+    __syncthreads();
+    for (int i = tid; i < C; i += kSelThreads) {
+      const uint32_t k = skey[i];
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane owns digits [8 lane, 8 lane + 8): find the digit where the count reaches need
+      int cnt[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[lane * 8 + j];
+        sum += cnt[j];
       }
-      const bool up = (i & size) == 0, lower = (i & stride) == 0;
-      key = (lower == up) ? (key < other ? key : other) : (key < other ? other : key);
-    }
-  }
-  sk[i] = key;
-  __syncthreads();
-  if (i < top_c) {
-    const int id = (int)(key & 0xFFFFFFFFu);
-    int rank = 0;
-    for (int u = 0; u < top_c; ++u) rank += (int)(sk[u] & 0xFFFFFFFFu) < id;
-    sel[(size_t)m * top_c + rank] = id;
-  }
-}
-
-__global__ void topc_kernel(const float *scores, int C, int top_c, int32_t *sel) {
-  extern __shared__ unsigned long long keys[];
-  pdl_wait();
-  const int m = blockIdx.x;
-  int n = 1;
-  while (n < C) n <<= 1;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    unsigned long long key = ~0ull;
-    if (i < C) {
-      uint32_t u = __float_as_uint(scores[(size_t)m * C + i]);
-      u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending order of floats
-      key = ((unsigned long long)(~u) << 32) | (uint32_t)i;  // descending score, then id
-    }
-    keys[i] = key;
-  }
-  __syncthreads();
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool up = (i & size) == 0;
-          const unsigned long long a = keys[i], b = keys[j];
-          if ((a > b) == up) {
-            keys[i] = b;
-            keys[j] = a;
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int run = incl - sum;  // keys with a smaller digit in lower lanes
+      const unsigned hit = __ballot_sync(0xffffffffu, run < need && need <= incl);
+      if (lane == __ffs(hit) - 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (run < need && need <= run + cnt[j]) {
+            s_digit = lane * 8 + j;
+            s_before = run;
           }
+          run += cnt[j];
         }
       }
-      __syncthreads();
     }
+    __syncthreads();
+    prefix |= (uint32_t)s_digit << shift;
+    mask |= 255u << shift;
+    need -= s_before;
+    __syncthreads();
   }
-  // the first top_c keys are the kept clusters; order their ids ascending (top_c <= 64)
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    for (int t = lane; t < top_c; t += 32) {
-      const int id = (int)(keys[t] & 0xFFFFFFFFu);
-      int rank = 0;
-      for (int u = 0; u < top_c; ++u) rank += (int)(keys[u] & 0xFFFFFFFFu) < id;
-      sel[(size_t)m * top_c + rank] = id;
-    }
+  // prefix is the key T of the top_c-th cluster; every key < T is kept, and the `need` keys
+  // equal to T with the lowest ids.  Thread tid reads ids [tid * per, tid * per + per).
+  const int per = (C + kSelThreads - 1) / kSelThreads;
+  const int i0 = tid * per, i1 = min(C, i0 + per);
+  int ties = 0;
+  for (int i = i0; i < i1; ++i) ties += skey[i] == prefix;
+  int total;
+  int tie_rank = block_exclusive_scan(ties, s_warp, total);
+  int takes = 0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t k = skey[i];
+    takes += k < prefix || (k == prefix && tie_rank++ < need);
   }
-}
-
-// -inf into rows [m, 0 .. V) of the logits; blockIdx.y = row.
-__global__ void fill_neg_inf_kernel(float *logits, int V, int ld, int vec4) {
-  pdl_wait();
-  float *row = logits + (size_t)blockIdx.y * ld;
-  const int stride = gridDim.x * blockDim.x;
-  if (vec4) {
-    float4 *r4 = reinterpret_cast<float4 *>(row);
-    const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < V / 4; i += stride) r4[i] = ninf;
-  } else {
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < V; i += stride) row[i] = -INFINITY;
+  int out = block_exclusive_scan(takes, s_warp, total);
+  tie_rank -= ties;  // back to this thread's first tie
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t k = skey[i];
+    if (k < prefix || (k == prefix && tie_rank++ < need)) sel[(size_t)m * top_c + out++] = i;
   }
+  (void)lane;
 }
 
 // Exact logits of the kept clusters' tokens.  The work is M * top_c * ceil(cs / TK) units of TK
@@ -590,23 +620,24 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
       if (s != SD_OK) return s;
     }
   }
-  int n = 1;
-  while (n < C) n <<= 1;
-  if (n < 32) n = 32;
-  if (n <= 1024)
-    s = cuda_status(launch(topc_small_kernel, dim3(desc->m), dim3(n), 0, st, (const float *)scores,
-                           C, desc->top_c, sel_clusters));
-  else
-    s = cuda_status(launch(topc_kernel, dim3(desc->m), dim3(512), (size_t)n * 8, st,
-                           (const float *)scores, C, desc->top_c, sel_clusters));
-  if (s != SD_OK) return s;
+  // selection (block 0 of each row) and the -inf fill of the row (the other blocks): about
+  // one wave of blocks over all rows
   const int vec4 = aligned16(logits) && desc->vocab % 4 == 0 && ld % 4 == 0;
-  const int per_row = (desc->vocab / (vec4 ? 4 : 1) + 255) / 256;
-  if (launch(fill_neg_inf_kernel, dim3(per_row < 64 ? per_row : 64, desc->m), dim3(256), 0, st,
-             logits, desc->vocab, ld, vec4) != cudaSuccess)
+  const int per_row = (desc->vocab / (vec4 ? 4 : 1) + kSelThreads - 1) / kSelThreads;
+  const int sms = sm_count();
+  int fill_blocks = ((sms > 0 ? sms : 148) + desc->m - 1) / desc->m;
+  if (fill_blocks > per_row) fill_blocks = per_row;
+  if (fill_blocks < 1) fill_blocks = 1;
+  const size_t sel_smem = (size_t)C * 4;
+  if (sel_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(select_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sel_smem) != cudaSuccess)
+    return SD_ERR_CUDA;
+  if (launch(select_fill_kernel, dim3(1 + fill_blocks, desc->m), dim3(kSelThreads), sel_smem, st,
+             (const float *)scores, C, desc->top_c, sel_clusters, logits, desc->vocab, ld,
+             vec4) != cudaSuccess)
     return SD_ERR_CUDA;
   // persistent warps: as many 8-warp CTAs as fit on the device at once
-  const int sms = sm_count();
   int occ = 0;
   if (desc->d <= 1024)
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<4>, 256, 0);
@@ -626,7 +657,6 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
                            desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
                            device_status_word()));
   return s;
-  return cuda_status(cudaGetLastError());
 }
 
 }  // extern "C"
