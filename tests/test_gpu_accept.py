@@ -190,3 +190,25 @@ def test_step_read_from_device_word():
     ok = ~ref["margin"]
     assert np.array_equal(n_acc.cpu().numpy()[ok], ref["n_accepted"][ok])
     assert np.array_equal(out.cpu().numpy()[ok], ref["out_tokens"][ok])
+
+
+def test_plain_draw_dense_rows_twice_on_one_workspace():
+    """k = 0 at T = 0.7 on dense rows (every token can win), B = 64: the draw takes no row
+    statistics; a second call on the same workspace reuses the per-sequence tickets."""
+    B, V = 64, 65536
+    z = S.make_logits(12, B, V).reshape(B, 1, V)
+    desc = sd.AcceptDesc(batch=B, k=0, vocab=V, temperature=0.7, seed=5, step=3, purpose=2)
+    ws = workspace(sd.sd_accept_workspace_size(desc))
+    for step in (3, 4):
+        desc.step = step
+        n_acc = torch.full((B,), -9, dtype=torch.int32, device=DEV)
+        out = torch.full((B, 1), -9, dtype=torch.int32, device=DEV)
+        sd.sd_accept(desc, to_dev(z), None, None, n_acc, out, None, ws)
+        torch.cuda.synchronize()
+        ref = OACC.accept(z.double().numpy(), None, np.zeros((B, 0), np.int64), 0.7, seed=5,
+                          step=step, purpose=2)
+        ok = ~ref["margin"]
+        assert (~ok).sum() <= 1
+        assert np.array_equal(n_acc.cpu().numpy(), np.zeros(B, np.int32))
+        assert np.array_equal(out.cpu().numpy()[ok], ref["out_tokens"][ok])
+    assert status_ok()

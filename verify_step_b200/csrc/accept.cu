@@ -32,7 +32,8 @@ constexpr int kThreads = 256;
 constexpr float kMargin = 1e-4f;
 
 struct Params {
-  int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, ndraw, draw_chunk, rows_t, rows_total;
+  int B, k, V, n_q, ld_t, ld_d, ld_o, purpose, nchunks, stats_chunk, ndraw, draw_chunk, rows_t,
+      rows_total;
   float T;
   unsigned long long seed;
   unsigned long long step;
@@ -124,37 +125,42 @@ __global__ void __launch_bounds__(kThreads) accept_stats_kernel(const Params p) 
   if (c == 0 && r == 0)
     for (int b = threadIdx.x; b < p.B; b += blockDim.x) p.counters[b] = 0u;
   const float *row = row_ptr(p, r);
-  const int v0 = c * kChunk;
-  const int v1 = min(p.V, v0 + kChunk);
+  const int v0 = c * p.stats_chunk;
+  const int v1 = min(p.V, v0 + p.stats_chunk);
   const float4 *row4 = reinterpret_cast<const float4 *>(row + v0);
   const int n4 = (v1 - v0) >> 2;
   __shared__ float4 red[kThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (p.T > 0.f) {
-    // all of this thread's values first (independent loads), then max, then the sum
+    // kChunk tokens at a time: all of this thread's values first (independent loads), then
+    // their max, then the sum, merged online across batches
     constexpr int PER = kChunk / 4 / kThreads;
-    float4 x[PER];
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int i = threadIdx.x + u * kThreads;
-      x[u] = i < n4 ? __ldg(row4 + i)
-                    : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-    }
     float m = -INFINITY, s = 0.f;
-    if (p.T != 1.f) {
+    for (int base = 0; base < n4; base += PER * kThreads) {
+      float4 x[PER];
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int i = base + threadIdx.x + u * kThreads;
+        x[u] = i < n4 ? __ldg(row4 + i)
+                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+      if (p.T != 1.f) {
+#pragma unroll
+        for (int u = 0; u < PER; ++u)
+          x[u] = make_float4(x[u].x / p.T, x[u].y / p.T, x[u].z / p.T, x[u].w / p.T);
+      }
+      float mb = -INFINITY, sb = 0.f;
 #pragma unroll
       for (int u = 0; u < PER; ++u)
-        x[u] = make_float4(x[u].x / p.T, x[u].y / p.T, x[u].z / p.T, x[u].w / p.T);
-    }
+        mb = fmaxf(mb, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
+      if (mb != -INFINITY) {
+        constexpr float L2E = 1.4426950408889634f;
 #pragma unroll
-    for (int u = 0; u < PER; ++u)
-      m = fmaxf(m, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
-    if (m != -INFINITY) {
-      constexpr float L2E = 1.4426950408889634f;
-#pragma unroll
-      for (int u = 0; u < PER; ++u)
-        s += (exp2f((x[u].x - m) * L2E) + exp2f((x[u].y - m) * L2E)) +
-             (exp2f((x[u].z - m) * L2E) + exp2f((x[u].w - m) * L2E));
+        for (int u = 0; u < PER; ++u)
+          sb += (exp2f((x[u].x - mb) * L2E) + exp2f((x[u].y - mb) * L2E)) +
+                (exp2f((x[u].z - mb) * L2E) + exp2f((x[u].w - mb) * L2E));
+      }
+      ms_merge(m, s, mb, sb);
     }
     for (int off = 16; off > 0; off >>= 1) {
       const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
@@ -233,8 +239,9 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   __shared__ int s_arg;
   __shared__ float4 s_rows[32];  // merged statistics: target rows 0..k, then draft rows 0..k-1
 
-  // ---- statistics of every row this sequence may need, one warp per row (in parallel)
-  const int n_rows = p.n_q + (p.T > 0.f ? p.k : 0);
+  // ---- statistics of every row this sequence may need, one warp per row (in parallel).  A
+  // plain draw (k = 0, T > 0) needs none: the race keys of p are unnormalised logits.
+  const int n_rows = (p.k == 0 && p.T > 0.f) ? 0 : p.n_q + (p.T > 0.f ? p.k : 0);
   for (int ri = warp; ri < n_rows; ri += kThreads / 32) {
     const int r = ri < p.n_q ? b * p.n_q + ri : p.rows_t + b * p.k + (ri - p.n_q);
     const float4 st = row_stats_warp(p, r);
@@ -274,8 +281,9 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
     // margins count for the decisions actually taken: drafts 1 .. a+1
     const unsigned flags = __ballot_sync(0xffffffffu, flag && lane <= a);
     if (lane == 0) {
-      const float4 sz = s_rows[a];
-      const float4 sy = (p.T > 0.f && a < p.k) ? s_rows[p.n_q + a] : make_float4(0.f, 1.f, 0.f, 0.f);
+      const float4 sz = n_rows > 0 ? s_rows[a] : make_float4(0.f, 1.f, 0.f, 0.f);
+      const float4 sy = (n_rows > 0 && p.T > 0.f && a < p.k) ? s_rows[p.n_q + a]
+                                                              : make_float4(0.f, 1.f, 0.f, 0.f);
       s_a = a;
       s_flag = flags != 0;
       s_mz = sz.x;
@@ -423,6 +431,31 @@ static sd_status validate(const sd_accept_desc *d) {
 }
 
 static int nchunks_of(int V) { return (V + kChunk - 1) / kChunk; }
+
+// Tokens per CTA of the statistics pass: kChunk, or more (multiples of 1024) when the rows
+// times kChunk-token chunks would not fit in one wave of CTAs.  Never more chunks per row than
+// nchunks_of(V), which sizes the workspace.
+static int stats_chunk_of(int rows, int V) {
+  static int occ_cache[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int occ = dev < 64 ? occ_cache[dev] : 0;
+  if (occ <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, accept_stats_kernel, kThreads, 0) !=
+            cudaSuccess ||
+        occ <= 0)
+      occ = 1;
+    if (dev < 64) occ_cache[dev] = occ;
+  }
+  const int sms = sm_count();
+  const long long slots = (long long)occ * (sms > 0 ? sms : 148);
+  long long n = slots / (rows > 0 ? rows : 1);
+  if (n < 1) n = 1;
+  if (n > nchunks_of(V)) n = nchunks_of(V);
+  int chunk = (int)((V + n - 1) / n);
+  chunk = (chunk + 1023) / 1024 * 1024;
+  return chunk < kChunk ? kChunk : chunk;
+}
 // Tokens per draw CTA: the race of one sequence is split so that all B sequences together give
 // about one wave of CTAs (the per-CTA chain of dependent memory round trips, not the token work,
 // dominates at small B); multiples of 1024 tokens.
@@ -478,11 +511,12 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.ld_d = desc->ld_draft ? desc->ld_draft : desc->vocab;
   p.ld_o = desc->ld_out ? desc->ld_out : desc->k + 1;
   p.purpose = desc->purpose;
-  p.nchunks = nchunks_of(desc->vocab);
   p.draw_chunk = draw_chunk_of(desc->batch, desc->vocab);
   p.ndraw = ndraw_of(desc->batch, desc->vocab);
   p.rows_t = p.B * p.n_q;
   p.rows_total = p.rows_t + (sampling ? p.B * p.k : 0);
+  p.stats_chunk = stats_chunk_of(p.rows_total, desc->vocab);
+  p.nchunks = (desc->vocab + p.stats_chunk - 1) / p.stats_chunk;
   p.T = desc->temperature;
   p.seed = desc->seed;
   p.step = desc->step;
@@ -502,9 +536,14 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.counters = reinterpret_cast<unsigned int *>(w8);
   p.status = device_status_word();
   cudaStream_t st = (cudaStream_t)stream;
-  if (launch(accept_stats_kernel, dim3(p.rows_total, p.nchunks), dim3(kThreads), 0, st, p) !=
-      cudaSuccess)
+  if (sampling && p.k == 0) {
+    // a plain draw reads no row statistics: only the per-sequence tickets need clearing
+    if (cudaMemsetAsync(p.counters, 0, (size_t)p.B * sizeof(unsigned int), st) != cudaSuccess)
+      return SD_ERR_CUDA;
+  } else if (launch(accept_stats_kernel, dim3(p.rows_total, p.nchunks), dim3(kThreads), 0, st,
+                    p) != cudaSuccess) {
     return SD_ERR_CUDA;
+  }
   return cuda_status(
       launch(accept_draw_kernel, dim3(p.B, sampling ? p.ndraw : 1), dim3(kThreads), 0, st, p));
 }
@@ -552,8 +591,9 @@ extern "C" sd_status sd_accept_noalloc(const sd_accept_desc *desc, const float *
     return SD_ERR_WORKSPACE;
   void *scratch = sdv::acc::noalloc_scratch();
   if (scratch == nullptr) return SD_ERR_CUDA;
-  // The per-sequence counters in the scratch are cleared by the statistics kernel at the start
-  // of every call, so the array's leftover contents from an earlier call do not matter.
+  // The per-sequence counters in the scratch are cleared at the start of every call (by the
+  // statistics kernel, or a memset for a plain draw), so the array's leftover contents from an
+  // earlier call do not matter.
   return sd_accept(desc, target_logits, draft_logits, draft_tokens, n_accepted, out_tokens,
                    margin_flags, scratch, (size_t)SD_ACCEPT_NOALLOC_MAX_SCRATCH, stream);
 }
