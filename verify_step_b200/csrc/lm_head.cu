@@ -352,14 +352,13 @@ __global__ void __launch_bounds__(kSelThreads) select_fill_kernel(const float *s
 // a warp almost always share the row m.  Lane l multiplies elements l*8 + q*256 + [0, 8) of a
 // weight row and keeps those hidden values in registers (reloaded only when m changes); the
 // weight loads of a unit's TK tokens are all in flight before the dot products (d <= 256 * KMAX).
-template <int KMAX>
+template <int KMAX, int TK>
 __global__ void __launch_bounds__(256) cluster_logits_kernel(
     const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm, const int32_t *cluster_tokens,
     const int32_t *sel, int M, int top_c, int cs, int d, int C, int V, int ld, float *logits,
     int *status) {
   pdl_trigger();
   pdl_wait();
-  constexpr int TK = 2;
   const int lane = threadIdx.x & 31;
   const long long n_warps = (long long)gridDim.x * (blockDim.x >> 5);
   const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -416,7 +415,10 @@ __global__ void __launch_bounds__(256) cluster_logits_kernel(
     for (int t = 0; t < TK; ++t)
       for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
     if (lane < TK && t0 + lane < cs) {
-      const float mine = lane == 0 ? acc[0] : acc[1];
+      float mine = acc[0];
+#pragma unroll
+      for (int t = 1; t < TK; ++t)
+        if (lane == t) mine = acc[t];
       const int tok = cluster_tokens[(size_t)c * cs + t0 + lane];
       if (tok < 0 || tok >= V)
         record_status(status, SD_ERR_DEVICE);
@@ -640,18 +642,18 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   // persistent warps: as many 8-warp CTAs as fit on the device at once
   int occ = 0;
   if (desc->d <= 1024)
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<4>, 256, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<4, 4>, 256, 0);
   else
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<16>, 256, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cluster_logits_kernel<16, 2>, 256, 0);
   const dim3 grid((occ > 0 ? occ : 1) * (sms > 0 ? sms : 148));
   if (desc->d <= 1024)
-    s = cuda_status(launch(cluster_logits_kernel<4>, grid, dim3(256), 0, st,
+    s = cuda_status(launch(cluster_logits_kernel<4, 4>, grid, dim3(256), 0, st,
                            (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens,
                            (const int32_t *)sel_clusters, desc->m, desc->top_c,
                            desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
                            device_status_word()));
   else
-    s = cuda_status(launch(cluster_logits_kernel<16>, grid, dim3(256), 0, st,
+    s = cuda_status(launch(cluster_logits_kernel<16, 2>, grid, dim3(256), 0, st,
                            (const __nv_bfloat16 *)h, (const __nv_bfloat16 *)w, cluster_tokens,
                            (const int32_t *)sel_clusters, desc->m, desc->top_c,
                            desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
