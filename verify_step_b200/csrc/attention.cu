@@ -47,6 +47,13 @@ struct Params {
   void *out;
   float *ws_o;   // [slots][Mpad][D]
   float *ws_ml;  // [slots][Mpad][2]
+  // Verify on the cluster (sliding-window) kernel with one 16-row query tile: the new rows
+  // come from k_new / v_new, and the kernel also writes them into the cache.  Null when a
+  // separate append kernel ran first (or for the drafter).
+  const void *k_new;
+  const void *v_new;
+  void *k_cache;
+  void *v_cache;
   int P;         // CTAs of the persistent grid
   int *status;
 };
@@ -220,6 +227,41 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
   const int unit = (col >> 3) & 7;
   return (uint32_t)(chunk * (kTile * 128) + row * 128 + ((unit ^ (row & 7)) << 4) +
                     ((col & 7) << 1));
+}
+
+// Verify with the fused append: the staged tile at positions [p0, p0 + 16) of sequence b may
+// hold some of the n_q new rows (positions L .. L + n_q - 1), which the cache does not have
+// yet.  The calling warp, sole owner of columns [col0, col0 + DS) of the tile, copies its slice
+// of those rows from k_new / v_new into the staged K and V tiles and into the cache.  Returns
+// whether it wrote shared memory (the stage then needs a proxy fence before TMA reuses it).
+template <int D, int DS>
+__device__ __forceinline__ bool patch_new_rows(const Params &p, int b, int g, int L, int p0,
+                                               int col0, uint8_t *ktile, uint8_t *vtile,
+                                               int lane) {
+  const int r_lo = max(L, p0) - p0, r_hi = min(L + p.n_q, p0 + kTile) - p0;
+  if (r_lo >= r_hi) return false;
+  constexpr int U = DS / 8;  // 16-byte units of one row's slice
+  const int n = (r_hi - r_lo) * 2 * U;
+  // all 16-byte pieces in flight at once (cp.async: no registers held), then from shared
+  // memory into the cache
+  for (int i = lane; i < n; i += 32) {
+    const int r = r_lo + i / (2 * U), kv = (i / U) & 1, u = i % U;
+    const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(kv == 0 ? p.k_new : p.v_new);
+    const __nv_bfloat16 *gp = src + (((size_t)b * p.n_q + (p0 + r - L)) * p.Hkv + g) * D + col0 + u * 8;
+    cp_async_16(smem_u32((kv == 0 ? ktile : vtile) + swz(r, col0 + u * 8)), gp);
+  }
+  cp_async_wait_all();
+  __syncwarp();
+  const int blk = p.table[(size_t)b * p.mbps + p0 / p.bs];  // the producer checked it
+  for (int i = lane; i < n; i += 32) {
+    const int r = r_lo + i / (2 * U), kv = (i / U) & 1, u = i % U;
+    const int col = col0 + u * 8, t = p0 + r;
+    const uint4 v = *reinterpret_cast<const uint4 *>((kv == 0 ? ktile : vtile) + swz(r, col));
+    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(kv == 0 ? p.k_cache : p.v_cache);
+    *reinterpret_cast<uint4 *>(dst + (((size_t)blk * p.Hkv + g) * p.bs + (t % p.bs)) * D + col) =
+        v;
+  }
+  return true;
 }
 
 template <int D, int MT, int STAGES>
@@ -656,18 +698,18 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
   const int b = item / p.Hkv, g = item % p.Hkv;
   pdl_trigger();
   pdl_wait();
-  // thread 0 sets up the barriers while the other threads' loads of the sequence's range and
-  // the tensor-map prefetch are in flight
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], WPG * 32);
-      bad[s] = 0;
+  // one barrier per thread (full[], empty[], red_bar[], done_bar are contiguous), while the
+  // loads of the sequence's range and the tensor-map prefetch are in flight
+  {
+    constexpr int NB = 2 * STAGES + 2 * KG + 1;
+    const int i = threadIdx.x;
+    if (i < NB) {
+      const uint32_t cnt = i < STAGES ? 1u : (i < NB - 1 ? (uint32_t)(WPG * 32) : NCW * 32u);
+      mbar_init(&full[i], cnt);
+      fence_mbar_init();
     }
-    for (int k = 0; k < 2 * KG; ++k) mbar_init(&red_bar[k], WPG * 32);
-    mbar_init(done_bar, NCW * 32);
-    *abort_flag = 0;
-    fence_mbar_init();
+    if (i < STAGES) bad[i] = 0;
+    if (i == 0) *abort_flag = 0;
   }
   if (warp == NCW && lane == 0) {
     tma_prefetch_desc(&kmap);
@@ -774,6 +816,11 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
       const uint32_t kbase = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
       const uint32_t vbase = kbase + C::TILE_BYTES;
       const int p0 = (s.tf + t_lo + t) * kTile;
+      bool patched = false;
+      if (MT == 1 && p.k_new != nullptr && !is_bad) {
+        uint8_t *kt = stages + (size_t)stage * C::STAGE_BYTES;
+        patched = patch_new_rows<D, DS>(p, b, g, s.L, p0, dg * DS, kt, kt + C::TILE_BYTES, lane);
+      }
 
       // ---- partial S = Q K^T over this warp's D slice, summed over the key group's slices
       float sp[2][4];
@@ -899,7 +946,9 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
           }
           fence_proxy_async_smem();
           __syncwarp();
+          patched = false;
         }
+        if (patched) fence_proxy_async_smem();
       }
 
       // ---- O += P V over this warp's D slice
@@ -1453,13 +1502,20 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   if (!encode_tmap_2d_bf16(&km, k_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile) ||
       !encode_tmap_2d_bf16(&vm, v_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile))
     return SD_ERR_CUDA;
-  if (!draft) {
+  const bool window = p.window > 0 && p.window <= kWinMax && MT <= 2;
+  if (!draft && window && MT == 1) {
+    // cluster kernel with one query tile: it appends the new rows itself
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+  } else if (!draft) {
     if (launch(append_kv_kernel<__nv_bfloat16>, dim3(p.B * p.n_q), dim3(256), 0, st, p,
                (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new,
                (__nv_bfloat16 *)k_cache, (__nv_bfloat16 *)v_cache) != cudaSuccess)
       return SD_ERR_CUDA;
   }
-  if (p.window > 0 && p.window <= kWinMax && MT <= 2) {
+  if (window) {
     // every item reads at most window + n_q - 1 keys, over at most this many 16-key tiles
     const int tiles_max = (p.window + p.n_q - 1 + kTile - 1) / kTile + 1;
     return launch_window(p.D, MT, km, vm, p, tiles_max, st);

@@ -261,6 +261,16 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// 16-byte global -> shared copy that holds no register until it lands (cp.async, L2 only).
+__device__ __forceinline__ void cp_async_16(uint32_t smem_addr, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gmem)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ thread-block clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
