@@ -220,12 +220,17 @@ class SpecStep:
                                 dtype=self.sd.SD_BF16, q_offset=q_offset)
 
     # kernels launched per call (bf16 paths)
-    LAUNCHES = dict(verify=3, xattn=2, head_dense=1, head_clustered=4, accept=2, commit=1)
+    # kernels per call of each group on this workload (the step graph's kernel nodes are
+    # counted directly where the CUDA runtime allows; this is the fallback)
+    LAUNCHES = dict(xattn_sliding=1, xattn_global=2, verify_sliding=1, verify_global=3,
+                    head_dense=1, head_clustered=3, accept_draft=1, accept=2, commit=1)
 
     def launches_per_step(self):
         L = self.LAUNCHES
-        return (self.k * (4 * L["xattn"] + L["head_clustered"] + L["accept"]) +
-                2 * L["verify"] + L["head_dense"] + L["accept"] + L["commit"])
+        return (self.k * (3 * L["xattn_sliding"] + L["xattn_global"] + L["head_clustered"] +
+                          L["accept_draft"]) +
+                L["verify_global"] + L["verify_sliding"] + L["head_dense"] + L["accept"] +
+                L["commit"])
 
     def run(self, ev=None):
         """Issue one step on the current stream.  ev (used while capturing a CUDA graph) maps a
@@ -335,6 +340,24 @@ def new_event():
     e = torch.cuda.Event(enable_timing=True)
     e.record()
     return e
+
+
+def graph_kernel_nodes(graph):
+    """Kernel nodes in a captured torch CUDA graph (None if the runtime cannot say)."""
+    try:
+        from cuda.bindings import runtime as cudart
+        g = cudart.cudaGraph_t(graph.raw_cuda_graph())
+        err, _, n = cudart.cudaGraphGetNodes(g, 0)
+        if err != cudart.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = cudart.cudaGraphGetNodes(g, n)
+        if err != cudart.cudaError_t.cudaSuccess:
+            return None
+        kinds = [cudart.cudaGraphNodeGetType(nd) for nd in nodes]
+        return sum(1 for e, t in kinds if e == cudart.cudaError_t.cudaSuccess and
+                   t == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
 
 
 def record_external(ev):
@@ -532,6 +555,9 @@ def main():
     torch.cuda.synchronize()
     sd.sd_device_status_clear()
     graph = st.capture()
+    kernels_per_step = graph_kernel_nodes(graph)
+    if kernels_per_step is None:
+        kernels_per_step = st.launches_per_step()
     graph.replay()
     torch.cuda.synchronize()
     ctx_a = st.ctx.cpu().numpy()
@@ -659,7 +685,7 @@ def main():
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "inputs larger than L2 (~6 GB read per step)",
                    "ctx_growth": "contexts advance by the accepted length each step"},
-        "gpu_launches": st.launches_per_step() * a.steps,
+        "gpu_launches": kernels_per_step * a.steps,
         "roofline": roof(dom),
         "roofline_attention": roof("verify_global"),
         "roofline_lm_head": roof("head_dense"),
