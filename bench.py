@@ -144,12 +144,19 @@ class SpecStep:
                                                         (n, B, 1, self.hq, D), 1 / math.sqrt(D)))
             inp[f"dh{j}"] = S.bf16(S.normal(seed * 37 + j, (B, self.dh)))
         self.host_inputs = inp
-        # all per-step inputs live in one device buffer (256-byte aligned views), so the
-        # end-to-end leg moves them with a single host-to-device copy
-        offs, total = {}, 0
-        for kk, v in inp.items():
-            offs[kk] = total
-            total += (v.numel() * v.element_size() + 255) // 256 * 256
+        # all per-step inputs live in one device buffer (256-byte aligned views) ordered by
+        # the phase that first reads them (drafter step 0, drafter step 1, ..., verify), so the
+        # end-to-end leg moves each phase's inputs with one host-to-device copy
+        phases = [[f"dq{j}_0", f"dq{j}_1", f"dh{j}"] for j in range(k)]
+        phases.append([kk for kk in inp if not kk.startswith("dq") and not kk.startswith("dh")])
+        offs, total, self.phase_ranges = {}, 0, []
+        for keys in phases:
+            start = total
+            for kk in keys:
+                v = inp[kk]
+                offs[kk] = total
+                total += (v.numel() * v.element_size() + 255) // 256 * 256
+            self.phase_ranges.append((start, total))
         self.input_buf = torch.empty(total, dtype=torch.uint8, device=dev)
         self.input_offs = offs
         self.inputs = {}
@@ -232,10 +239,11 @@ class SpecStep:
                 L["verify_global"] + L["verify_sliding"] + L["head_dense"] + L["accept"] +
                 L["commit"])
 
-    def run(self, ev=None):
+    def run(self, ev=None, before_phase=None):
         """Issue one step on the current stream.  ev (used while capturing a CUDA graph) maps a
         kernel group to a list that receives (start, end) events recorded as graph nodes
-        around each call of that group."""
+        around each call of that group.  before_phase(j) is called before drafter step j
+        (j < k) and before the verify (j = k)."""
         sd, I = self.sd, self.inputs
 
         def timed(name, fn):
@@ -250,6 +258,8 @@ class SpecStep:
 
         c0, c1 = self.cache
         for j in range(self.k):
+            if before_phase is not None:
+                before_phase(j)
             xd0, xd1 = self.xdesc[j]
             for r in range(3):
                 timed("xattn_sliding", lambda: sd.sd_draft_xattn(
@@ -263,6 +273,8 @@ class SpecStep:
             timed("accept_draft", lambda: sd.sd_accept(
                 ad, self._row_ptr(self.draft_logits, j), None, None, self.n_acc,
                 self._col_ptr(self.drafts, j), None, self.ws))
+        if before_phase is not None:
+            before_phase(self.k)
         timed("verify_global", lambda: sd.sd_verify_attn(
             self.vdesc[0], I["q0"], I["kn0"], I["vn0"], c0["k"], c0["v"], c0["table"], self.ctx,
             self.attn_out[0], self.ws))
@@ -331,6 +343,37 @@ class SpecStep:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             self.run(ev)
+        return g
+
+    def capture_e2e(self, pinned, res_h):
+        """The step with its host transfers as graph nodes: the first drafter step's inputs
+        are copied on the step's stream before it starts; the later phases' inputs are copied
+        on a second stream meanwhile, each phase waiting only for its own block; the results
+        are copied back to pinned host memory at the end."""
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        with torch.cuda.graph(g):
+            cur = torch.cuda.current_stream()
+            s0, e0 = self.phase_ranges[0]
+            self.input_buf[s0:e0].copy_(pinned[s0:e0], non_blocking=True)
+            fork = torch.cuda.Event()
+            fork.record(cur)
+            side.wait_event(fork)
+            ready = []
+            with torch.cuda.stream(side):
+                for s, e in self.phase_ranges[1:]:
+                    self.input_buf[s:e].copy_(pinned[s:e], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(side)
+                    ready.append(ev)
+
+            def before_phase(j):
+                if j >= 1:
+                    cur.wait_event(ready[j - 1])
+
+            self.run(before_phase=before_phase)
+            res_h.copy_(self.results, non_blocking=True)
         return g
 
 
@@ -621,6 +664,7 @@ def main():
     # ---- end-to-end: every step copies its inputs from pinned host memory, replays the step
     # and reads the accepted counts and tokens back to the host
     e2e = None
+    graph_e2e = None
     if not a.no_e2e:
         pinned = torch.empty(st.input_buf.numel(), dtype=torch.uint8).pin_memory()
         for kk, v in st.host_inputs.items():
@@ -632,13 +676,13 @@ def main():
         d2h = res_h.numel() * 4
         if world > 1:
             dist.barrier()
+        graph_e2e = st.capture_e2e(pinned, res_h)
+        graph_e2e.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(a.steps):
-            st.input_buf.copy_(pinned, non_blocking=True)
-            graph.replay()
-            res_h.copy_(st.results, non_blocking=True)
+            graph_e2e.replay()
             torch.cuda.current_stream().synchronize()
         e1.record()
         torch.cuda.synchronize()
@@ -650,12 +694,14 @@ def main():
         e2e = {"value": round(world * st.B * st.n_q * a.steps / (ems / 1e3), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(ems / a.steps, 4),
-               "path": "public C ABI calls captured once in a CUDA graph; per step: one H2D "
-                       "copy of the step inputs (one pinned block), replay, one D2H of "
-                       "n_accepted and out_tokens, stream synchronise"}
+               "path": "public C ABI calls and the step's host transfers captured once in a "
+                       "CUDA graph; per step: H2D of the step inputs from pinned memory in one "
+                       "block per phase (drafter step 0 first; drafter step 1 and the verify "
+                       "inputs on a second stream while the drafter runs), the kernels, one "
+                       "D2H of n_accepted and out_tokens, stream synchronise"}
     clocks = clock.stop()
     status = sd.sd_device_status_read()
-    del graph, graph_ev
+    del graph, graph_ev, graph_e2e
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
