@@ -50,6 +50,14 @@ struct Params {
   int *status;
 };
 
+// 2^x by the hardware approximation (relative error about 2^-22; arguments here are <= 0, and
+// results below 2^-126 flush to 0, far below any weight that could win a race).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // E = -ln(1 - V) for V in [0, 1): the series V + V^2/2 + ... + V^8/8 below 1/16 (truncation
 // below 3e-11 relative), else -ln(1 - V) with 1 - V formed exactly or within 2^-25 and the fast
 // logarithm (absolute error below 4e-7, i.e. below 6e-6 relative to E >= 0.0645).
@@ -343,8 +351,8 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
       w[e] = 0.f;
       if (resid) {
         const float yt = unit_t ? yy[e] : yy[e] / p.T;
-        const float pv = exp2f(fmaf(zt[e], L2E, -mzl)) * isz;
-        const float qv = exp2f(fmaf(yt, L2E, -myl)) * isy;
+        const float pv = ex2_approx(fmaf(zt[e], L2E, -mzl)) * isz;
+        const float qv = ex2_approx(fmaf(yt, L2E, -myl)) * isy;
         w[e] = pv - qv;
       }
       any |= zt[e] != -INFINITY || w[e] > 0.f;
@@ -415,6 +423,13 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   p.n_acc[b] = a;
   if (p.margin) p.margin[b] = flag;
   p.counters[b] = 0u;
+}
+
+// Zeroes the per-sequence tickets of the draw (plain draws, which skip the statistics pass
+// that otherwise clears them).
+__global__ void clear_tickets_kernel(unsigned int *counters, int B) {
+  pdl_wait();
+  for (int b = threadIdx.x; b < B; b += blockDim.x) counters[b] = 0u;
 }
 
 static sd_status validate(const sd_accept_desc *d) {
@@ -537,8 +552,10 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.status = device_status_word();
   cudaStream_t st = (cudaStream_t)stream;
   if (sampling && p.k == 0) {
-    // a plain draw reads no row statistics: only the per-sequence tickets need clearing
-    if (cudaMemsetAsync(p.counters, 0, (size_t)p.B * sizeof(unsigned int), st) != cudaSuccess)
+    // a plain draw reads no row statistics: only the per-sequence tickets need clearing (a
+    // one-block kernel: in a CUDA graph it costs less than a memset node)
+    if (launch(clear_tickets_kernel, dim3(1), dim3(kThreads), 0, st, p.counters, p.B) !=
+        cudaSuccess)
       return SD_ERR_CUDA;
   } else if (launch(accept_stats_kernel, dim3(p.rows_total, p.nchunks), dim3(kThreads), 0, st,
                     p) != cudaSuccess) {
@@ -592,8 +609,8 @@ extern "C" sd_status sd_accept_noalloc(const sd_accept_desc *desc, const float *
   void *scratch = sdv::acc::noalloc_scratch();
   if (scratch == nullptr) return SD_ERR_CUDA;
   // The per-sequence counters in the scratch are cleared at the start of every call (by the
-  // statistics kernel, or a memset for a plain draw), so the array's leftover contents from an
-  // earlier call do not matter.
+  // statistics kernel, or a one-block kernel for a plain draw), so the array's leftover
+  // contents from an earlier call do not matter.
   return sd_accept(desc, target_logits, draft_logits, draft_tokens, n_accepted, out_tokens,
                    margin_flags, scratch, (size_t)SD_ACCEPT_NOALLOC_MAX_SCRATCH, stream);
 }

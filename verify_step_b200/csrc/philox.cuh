@@ -44,13 +44,11 @@ __device__ __forceinline__ float accept_uniform(uint64_t seed, uint32_t step, ui
 }
 
 // 24 leading significant bits of a 64-bit word, scaled so the result lies in (0, 1); 0 -> 0.
-// The value m * 2^(-24-n) (m < 2^24, n <= 63) is exact in float32.
+// Converting the word to float32 rounding toward zero keeps exactly its 24 leading significant
+// bits, m * 2^(40-n) (n leading zeros); the power-of-two scale 2^-64 is exact (the result,
+// at least 2^-88, stays normal).
 __device__ __forceinline__ float float_uniform64(uint64_t w) {
-  if (w == 0) return 0.0f;
-  const int n = __clzll((long long)w);
-  const uint32_t m = (uint32_t)((w << n) >> 40);  // in [2^23, 2^24): the leading bit is set
-  // m * 2^(-24-n) = (m / 2^23) * 2^(-1-n): a normal float with biased exponent 126 - n
-  return __uint_as_float(((uint32_t)(126 - n) << 23) | (m & 0x7FFFFFu));
+  return __ull2float_rz(w) * 0x1.0p-64f;
 }
 
 // Token uniforms of tokens 2*c and 2*c+1 of a row (one Philox call).
