@@ -146,9 +146,10 @@ def test_drafter_clustered_config():
     assert status_ok()
 
 
-@pytest.mark.parametrize("C,cs,top_c", [(300, 3, 17), (4096, 2, 64), (8192, 1, 5)])
+@pytest.mark.parametrize("C,cs,top_c", [(300, 3, 17), (4096, 2, 64), (8192, 1, 5), (200, 32, 7)])
 def test_clustered_cluster_counts(C, cs, top_c):
-    """Cluster counts that are not multiples of the selection block, up to the 8192 limit."""
+    """Cluster counts that are not multiples of the selection block, up to the 8192 limit;
+    cluster sizes that take the per-warp gather (not a multiple of 16) and the staged one."""
     w = S.Workload("c", 4, 0, 0, 4, 1, [], 64, C * cs, n_clusters=C, cluster_size=cs,
                    drafter_hidden=64, seed=33)
     cl = S.make_clustered_head(w)

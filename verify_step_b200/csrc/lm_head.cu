@@ -428,6 +428,141 @@ __global__ void __launch_bounds__(256) cluster_logits_kernel(
   }
 }
 
+// Same logits with the weights staged by bulk copies (d <= 1024, cluster_size a multiple of
+// kClTok): the work is M * top_c * cs / kClTok units of kClTok tokens, each unit's weights one
+// contiguous block of the cluster-major matrix.  A persistent CTA per SM takes a contiguous
+// range of units; its producer warp streams them (weights and token ids, cp.async.bulk) through
+// a kClStages-deep mbarrier ring, and each of the kClWarps consumer warps takes two tokens of a
+// unit: lane l multiplies elements l*8 + q*256 + [0, 8) of the staged row with the hidden
+// values it keeps in registers (reloaded when the row m changes).
+constexpr int kClTok = 16;
+constexpr int kClStages = 6;
+constexpr int kClWarps = kClTok / 2;
+constexpr int kClUnitBytes = kClTok * 1024 * 2;  // largest unit (d = 1024)
+constexpr size_t kClSmem = 128 + (size_t)kClStages * kClUnitBytes + kClStages * kClTok * 4 +
+                           kClStages * 16 + kClStages * 16 + 16;
+
+__global__ void __launch_bounds__(32 * (kClWarps + 1), 1) cluster_logits_tma_kernel(
+    const __nv_bfloat16 *h, const __nv_bfloat16 *w_cm, const int32_t *cluster_tokens,
+    const int32_t *sel, int M, int top_c, int cs, int d, int C, int V, int ld, float *logits,
+    int *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t *stages = smem;  // [kClStages][kClTok * d * 2]
+  int32_t *tok = reinterpret_cast<int32_t *>(stages + (size_t)kClStages * kClUnitBytes);
+  int4 *rec = reinterpret_cast<int4 *>(tok + kClStages * kClTok);  // (m, c, t0, tokens)
+  uint64_t *full = reinterpret_cast<uint64_t *>(rec + kClStages);
+  uint64_t *empty = full + kClStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kClStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  if (threadIdx.x < 2 * kClStages) {
+    mbar_init(&full[threadIdx.x], threadIdx.x < kClStages ? 1u : (uint32_t)kClWarps);
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 0) *abort_flag = 0;
+  __syncthreads();
+  const int upc = cs / kClTok;  // units per (row, cluster)
+  const long long U = (long long)M * top_c * upc;
+  const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
+  const uint32_t wbytes = (uint32_t)kClTok * d * 2;
+
+  if (warp == kClWarps) {
+    // ------------------------------------------------------------------- producer warp
+    if (lane != 0) return;
+    long long u = u0;
+    for (; u < u1; ++u) {
+      const int it = (int)(u - u0), stg = it % kClStages;
+      if (!mbar_wait(&empty[stg], ((it / kClStages) & 1) ^ 1, abort_flag)) {
+        record_status(status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      const int ms = (int)(u / upc), t0 = (int)(u % upc) * kClTok;
+      const int m = ms / top_c, slot = ms % top_c;
+      const int c = sel[(size_t)m * top_c + slot];
+      if (c < 0 || c >= C) {
+        record_status(status, SD_ERR_DEVICE);
+        rec[stg] = make_int4(m, c, t0, 0);
+        mbar_arrive(&full[stg]);
+        continue;
+      }
+      rec[stg] = make_int4(m, c, t0, kClTok);
+      mbar_arrive_expect_tx(&full[stg], wbytes + kClTok * 4);
+      bulk_load(stages + (size_t)stg * kClUnitBytes, w_cm + ((size_t)c * cs + t0) * d, wbytes,
+                &full[stg]);
+      bulk_load(tok + stg * kClTok, cluster_tokens + (size_t)c * cs + t0, kClTok * 4,
+                &full[stg]);
+    }
+    if (*abort_flag) {
+      // wait (bounded) for the copies this CTA issued before leaving
+      const long long n = u - u0;
+      for (long long j = (n > kClStages ? n - kClStages : 0); j < n; ++j)
+        mbar_wait_timed(&full[j % kClStages], (uint32_t)((j / kClStages) & 1));
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------------- consumer warps
+  const int nk = d / 256 + (d % 256 != 0);
+  float hr[4][8];
+  int m_loaded = -1;
+  for (long long u = u0; u < u1; ++u) {
+    const int it = (int)(u - u0), stg = it % kClStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[stg], (it / kClStages) & 1, abort_flag))) {
+      record_status(status, SD_ERR_TIMEOUT);
+      *abort_flag = 1;
+      break;
+    }
+    const int4 r = rec[stg];
+    if (r.w > 0) {
+      if (r.x != m_loaded) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k0 = lane * 8 + q * 256;
+          uint4 hv = make_uint4(0, 0, 0, 0);
+          if (q < nk && k0 < d)
+            hv = __ldg(reinterpret_cast<const uint4 *>(h + (size_t)r.x * d + k0));
+          const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&hv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) hr[q][j] = __bfloat162float(e[j]);
+        }
+        m_loaded = r.x;
+      }
+      float acc[2];
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        const uint8_t *row = stages + (size_t)stg * kClUnitBytes + (size_t)(warp * 2 + tt) * d * 2;
+        acc[tt] = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k0 = lane * 8 + q * 256;
+          if (q < nk && k0 < d) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(row + (size_t)k0 * 2);
+            const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[tt] = fmaf(__bfloat162float(e[j]), hr[q][j], acc[tt]);
+          }
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt)
+        for (int o = 16; o > 0; o >>= 1) acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], o);
+      if (lane < 2) {
+        const int t = warp * 2 + lane;
+        const int id = tok[stg * kClTok + t];
+        if (id < 0 || id >= V)
+          record_status(status, SD_ERR_DEVICE);
+        else
+          logits[(size_t)r.x * ld + id] = lane == 0 ? acc[0] : acc[1];
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stg]);
+  }
+}
+
 // Centroid scores of the clustered head, score[i, c] = h[i] . centroid[c], for up to 16 rows:
 // one warp per centroid (its row read once, 16-byte loads), the rows of h in shared memory.
 // A GEMV this small (2 MB of centroids) needs many CTAs in flight rather than tensor cores.
@@ -639,6 +774,24 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
              (const float *)scores, C, desc->top_c, sel_clusters, logits, desc->vocab, ld,
              vec4) != cudaSuccess)
     return SD_ERR_CUDA;
+  if (desc->d <= 1024 && desc->cluster_size % kClTok == 0 && aligned16(cluster_tokens)) {
+    static bool attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+      if (cudaFuncSetAttribute(cluster_logits_tma_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kClSmem) != cudaSuccess)
+        return SD_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+    return cuda_status(launch(cluster_logits_tma_kernel, dim3(sms > 0 ? sms : 148),
+                              dim3(32 * (kClWarps + 1)), kClSmem, st, (const __nv_bfloat16 *)h,
+                              (const __nv_bfloat16 *)w, cluster_tokens,
+                              (const int32_t *)sel_clusters, desc->m, desc->top_c,
+                              desc->cluster_size, desc->d, C, desc->vocab, ld, logits,
+                              device_status_word()));
+  }
   // persistent warps: as many 8-warp CTAs as fit on the device at once
   int occ = 0;
   if (desc->d <= 1024)
