@@ -137,6 +137,14 @@ typedef struct {
   int top_c;        /* 0: dense mode; else clusters kept per row (1 <= top_c <= n_clusters,
                        top_c <= 64) */
   sd_dtype dtype;   /* element type of h, w and centroids (bf16; f32 in dense mode too) */
+  /* Optional softmax partials of the logit rows for sd_accept (dense bf16 mode, m <= 64):
+   * row_stats[2 * (i * ld_stats + s)] = M, [... + 1] = S with M the largest logit / T of the
+   * vocabulary entries of slot s and S = sum of exp(logit / T - M) over them (M = -inf, S = 0
+   * for an empty slot), for s < sd_lm_head_stats_slots(desc); T = stats_temperature > 0.
+   * NULL: none. */
+  float *row_stats;
+  int ld_stats;     /* pairs between consecutive rows; 0 means the slot count */
+  float stats_temperature;
 } sd_head_desc;
 
 /*
@@ -154,6 +162,9 @@ typedef struct {
  *   sel_clusters int32 [m, top_c].
  */
 size_t sd_lm_head_workspace_size(const sd_head_desc *desc);
+/* Slots per row of row_stats for this descriptor on the current device (0 if the descriptor
+ * cannot produce them). */
+int sd_lm_head_stats_slots(const sd_head_desc *desc);
 sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
                      const void *centroids, const int32_t *cluster_tokens, float *logits,
                      int32_t *sel_clusters, void *ws, size_t ws_bytes, sd_stream stream);
@@ -193,6 +204,21 @@ typedef struct {
   const uint64_t *step_ptr; /* nullable DEVICE word: when set, the step entering the counter
                                is *step_ptr + step, read when the kernels run (a decode loop
                                replayed from a CUDA graph advances it with sd_commit) */
+  /* Optional softmax partials of the rows from their producers (T > 0), in the row_stats form
+   * of sd_head_desc computed at this call's temperature: target row r = b*(k+1)+i at pairs
+   * target_stats[r * ld_target_stats + s], s < target_stats_slots; draft row b*k+i likewise.
+   * A row's statistics are the merge of its slots.  With both given the statistics pass over
+   * the logits is skipped.  NULL: computed from the logits. */
+  const float *target_stats;
+  int target_stats_slots;
+  int ld_target_stats;   /* pairs between rows; 0 means target_stats_slots */
+  const float *draft_stats;
+  int draft_stats_slots;
+  int ld_draft_stats;    /* pairs between rows; 0 means draft_stats_slots */
+  /* Plain draws (k == 0, T > 0) can also emit the drawn rows' partials in that form:
+   * stats_out pairs [b * ld_stats_out + s], s < sd_accept_stats_slots(desc).  NULL: none. */
+  float *stats_out;
+  int ld_stats_out;      /* pairs between sequences; 0 means the slot count */
 } sd_accept_desc;
 
 /*
@@ -203,6 +229,8 @@ typedef struct {
  *   (|u - p/q| < 1e-4, or a draw / argmax whose two best keys differ by < 1e-4).
  */
 size_t sd_accept_workspace_size(const sd_accept_desc *desc);
+/* Slots per row of stats_out for a plain draw with this descriptor (0 if not a plain draw). */
+int sd_accept_stats_slots(const sd_accept_desc *desc);
 sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
                     const float *draft_logits, const int32_t *draft_tokens,
                     int32_t *n_accepted, int32_t *out_tokens, int32_t *margin_flags,

@@ -44,7 +44,8 @@ class HeadDesc(ctypes.Structure):
     _fields_ = [("m", ctypes.c_int), ("d", ctypes.c_int), ("vocab", ctypes.c_int),
                 ("ld_logits", ctypes.c_int), ("n_clusters", ctypes.c_int),
                 ("cluster_size", ctypes.c_int), ("top_c", ctypes.c_int),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("row_stats", ctypes.c_void_p),
+                ("ld_stats", ctypes.c_int), ("stats_temperature", ctypes.c_float)]
 
 
 class AcceptDesc(ctypes.Structure):
@@ -52,7 +53,11 @@ class AcceptDesc(ctypes.Structure):
                 ("temperature", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("step", ctypes.c_uint64), ("purpose", ctypes.c_int),
                 ("ld_target", ctypes.c_int), ("ld_draft", ctypes.c_int),
-                ("ld_out", ctypes.c_int), ("step_ptr", ctypes.c_void_p)]
+                ("ld_out", ctypes.c_int), ("step_ptr", ctypes.c_void_p),
+                ("target_stats", ctypes.c_void_p), ("target_stats_slots", ctypes.c_int),
+                ("ld_target_stats", ctypes.c_int), ("draft_stats", ctypes.c_void_p),
+                ("draft_stats_slots", ctypes.c_int), ("ld_draft_stats", ctypes.c_int),
+                ("stats_out", ctypes.c_void_p), ("ld_stats_out", ctypes.c_int)]
 
 
 class PoisonCache(ctypes.Structure):
@@ -79,9 +84,11 @@ _SIGS = {
     "sd_draft_xattn": (ctypes.c_int, [ctypes.POINTER(AttnDesc), _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]),
     "sd_lm_head_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(HeadDesc)]),
+    "sd_lm_head_stats_slots": (ctypes.c_int, [ctypes.POINTER(HeadDesc)]),
     "sd_lm_head": (ctypes.c_int, [ctypes.POINTER(HeadDesc), _P, _P, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P]),
     "sd_accept_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(AcceptDesc)]),
+    "sd_accept_stats_slots": (ctypes.c_int, [ctypes.POINTER(AcceptDesc)]),
     "sd_accept": (ctypes.c_int, [ctypes.POINTER(AcceptDesc), _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.c_size_t, _P]),
     "sd_accept_noalloc": (ctypes.c_int, [ctypes.POINTER(AcceptDesc), _P, _P, _P, _P, _P, _P,
@@ -159,6 +166,14 @@ def sd_lm_head_workspace_size(desc: HeadDesc) -> int:
 
 def sd_accept_workspace_size(desc: AcceptDesc) -> int:
     return lib().sd_accept_workspace_size(ctypes.byref(desc))
+
+
+def sd_lm_head_stats_slots(desc: HeadDesc) -> int:
+    return lib().sd_lm_head_stats_slots(ctypes.byref(desc))
+
+
+def sd_accept_stats_slots(desc: AcceptDesc) -> int:
+    return lib().sd_accept_stats_slots(ctypes.byref(desc))
 
 
 def sd_verify_attn(desc, q, k_new, v_new, k_cache, v_cache, block_table, ctx_len, out, ws,

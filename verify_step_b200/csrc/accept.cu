@@ -45,6 +45,14 @@ struct Params {
   int32_t *out;
   int32_t *margin;
   float4 *stats;   // [rows_total][nchunks]
+  int stats_row0, stats_rows;  // rows the statistics pass computes
+  // optional producer partials (max, sum exp) per slot: target rows, draft rows
+  const float2 *tstats;
+  int tslots, tld;
+  const float2 *dstats;
+  int dslots, dld;
+  float2 *sout;  // plain draws: partials of the drawn row per draw chunk
+  int sld;
   float4 *cand;    // [B][ndraw][2]
   unsigned int *counters;  // [B]
   int *status;
@@ -129,8 +137,8 @@ __device__ __forceinline__ const float *row_ptr(const Params &p, int r) {
 
 __global__ void __launch_bounds__(kThreads) accept_stats_kernel(const Params p) {
   pdl_wait();  // many waves: no early trigger, so the next kernel does not take their slots
-  const int r = blockIdx.x, c = blockIdx.y;
-  if (c == 0 && r == 0)
+  const int r = p.stats_row0 + blockIdx.x, c = blockIdx.y;
+  if (c == 0 && blockIdx.x == 0)
     for (int b = threadIdx.x; b < p.B; b += blockDim.x) p.counters[b] = 0u;
   const float *row = row_ptr(p, r);
   const int v0 = c * p.stats_chunk;
@@ -218,7 +226,18 @@ __device__ __forceinline__ float4 row_stats_warp(const Params &p, int r) {
   const float4 *st = p.stats + (size_t)r * p.nchunks;
   if (p.T > 0.f) {
     float M = -INFINITY, S = 0.f;
-    for (int c = lane; c < p.nchunks; c += 32) ms_merge(M, S, st[c].x, st[c].y);
+    const bool target = r < p.rows_t;
+    const float2 *ext = target ? p.tstats : p.dstats;
+    if (ext != nullptr) {  // partials from the rows' producers
+      const int slots = target ? p.tslots : p.dslots;
+      const float2 *e = ext + (size_t)(target ? r : r - p.rows_t) * (target ? p.tld : p.dld);
+      for (int c = lane; c < slots; c += 32) {
+        const float2 v = e[c];
+        ms_merge(M, S, v.x, v.y);
+      }
+    } else {
+      for (int c = lane; c < p.nchunks; c += 32) ms_merge(M, S, st[c].x, st[c].y);
+    }
     for (int off = 16; off > 0; off >>= 1) {
       const float m2 = __shfl_xor_sync(0xffffffffu, M, off);
       const float s2 = __shfl_xor_sync(0xffffffffu, S, off);
@@ -241,6 +260,7 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   __shared__ int s_a, s_flag;
   __shared__ float s_mz, s_isz, s_my, s_isy;
   __shared__ float4 red[2][kThreads / 32];
+  __shared__ float2 s_part[kThreads / 32];  // plain draws: per-warp softmax partials
   __shared__ int s_last;
   __shared__ uint32_t s_step;
   __shared__ float s_top1, s_top2;
@@ -336,6 +356,8 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
   constexpr float L2E = 1.4426950408889634f;
   const bool unit_t = p.T == 1.f;
   const float mzl = mz * L2E, myl = my * L2E;
+  const bool want_part = p.sout != nullptr;
+  float pm = -INFINITY, ps = 0.f;
   for (int i = threadIdx.x; i < n4; i += kThreads) {
     const int v = v0 + 4 * i;
     const float4 z4 = __ldg(reinterpret_cast<const float4 *>(zr + v));
@@ -357,6 +379,18 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
       }
       any |= zt[e] != -INFINITY || w[e] > 0.f;
     }
+    if (want_part) {  // running (max, sum exp(x - max)) of the drawn row's logits / T
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (zt[e] == -INFINITY) continue;
+        if (zt[e] > pm) {
+          ps = ps * exp2f((pm - zt[e]) * L2E) + 1.f;
+          pm = zt[e];
+        } else {
+          ps += exp2f((zt[e] - pm) * L2E);
+        }
+      }
+    }
     if (!any) continue;  // no token of the group can win either race: no uniforms needed
     float U[4];
     token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1), U[0],
@@ -375,11 +409,24 @@ __global__ void __launch_bounds__(kThreads) accept_draw_kernel(const Params p) {
     cp = (lane & off) ? cand_merge(o1, cp) : cand_merge(cp, o1);
     cr = (lane & off) ? cand_merge(o2, cr) : cand_merge(cr, o2);
   }
+  if (want_part) {
+    for (int off = 16; off > 0; off >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, pm, off);
+      const float s2 = __shfl_xor_sync(0xffffffffu, ps, off);
+      ms_merge(pm, ps, m2, s2);
+    }
+  }
   if (lane == 0) {
     red[0][warp] = make_float4(cp.g1, __int_as_float(cp.v1), cp.g2, 0.f);
     red[1][warp] = make_float4(cr.g1, __int_as_float(cr.v1), cr.g2, 0.f);
+    s_part[warp] = make_float2(pm, ps);
   }
   __syncthreads();
+  if (want_part && threadIdx.x == 0) {
+    float M = s_part[0].x, S = s_part[0].y;
+    for (int w = 1; w < kThreads / 32; ++w) ms_merge(M, S, s_part[w].x, s_part[w].y);
+    p.sout[(size_t)b * p.sld + c] = make_float2(M, S);
+  }
   if (threadIdx.x == 0) {
     Cand tp{red[0][0].x, red[0][0].z, __float_as_int(red[0][0].y)};
     Cand tr{red[1][0].x, red[1][0].z, __float_as_int(red[1][0].y)};
@@ -432,6 +479,8 @@ __global__ void clear_tickets_kernel(unsigned int *counters, int B) {
   for (int b = threadIdx.x; b < B; b += blockDim.x) counters[b] = 0u;
 }
 
+static int ndraw_of(int B, int V);
+
 static sd_status validate(const sd_accept_desc *d) {
   if (!d) return SD_ERR_INVALID_ARG;
   if (d->batch < 1 || d->k < 0 || d->k > 15 || d->vocab < 1) return SD_ERR_INVALID_ARG;
@@ -442,6 +491,19 @@ static sd_status validate(const sd_accept_desc *d) {
   const int ldo = d->ld_out ? d->ld_out : d->k + 1;
   if (ldt < d->vocab || ldd < d->vocab || ldo < d->k + 1) return SD_ERR_INVALID_ARG;
   if (d->vocab % 4 || ldt % 4 || ldd % 4) return SD_ERR_UNSUPPORTED;
+  if (d->target_stats &&
+      (d->target_stats_slots < 1 ||
+       (d->ld_target_stats != 0 && d->ld_target_stats < d->target_stats_slots)))
+    return SD_ERR_INVALID_ARG;
+  if (d->draft_stats &&
+      (d->draft_stats_slots < 1 ||
+       (d->ld_draft_stats != 0 && d->ld_draft_stats < d->draft_stats_slots)))
+    return SD_ERR_INVALID_ARG;
+  if (d->stats_out) {
+    if (d->k != 0 || !(d->temperature > 0.f)) return SD_ERR_INVALID_ARG;
+    if (d->ld_stats_out != 0 && d->ld_stats_out < ndraw_of(d->batch, d->vocab))
+      return SD_ERR_INVALID_ARG;
+  }
   return SD_OK;
 }
 
@@ -502,6 +564,11 @@ extern "C" {
 
 size_t sd_accept_workspace_size(const sd_accept_desc *desc) { return sdv::acc::ws_size(desc); }
 
+int sd_accept_stats_slots(const sd_accept_desc *desc) {
+  if (sdv::acc::validate(desc) != SD_OK || desc->k != 0 || !(desc->temperature > 0.f)) return 0;
+  return sdv::acc::ndraw_of(desc->batch, desc->vocab);
+}
+
 sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
                     const float *draft_logits, const int32_t *draft_tokens,
                     int32_t *n_accepted, int32_t *out_tokens, int32_t *margin_flags,
@@ -530,7 +597,23 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.ndraw = ndraw_of(desc->batch, desc->vocab);
   p.rows_t = p.B * p.n_q;
   p.rows_total = p.rows_t + (sampling ? p.B * p.k : 0);
-  p.stats_chunk = stats_chunk_of(p.rows_total, desc->vocab);
+  // producer partials (sampling only; the greedy rule needs the top two of each row)
+  if (sampling && desc->target_stats) {
+    p.tstats = reinterpret_cast<const float2 *>(desc->target_stats);
+    p.tslots = desc->target_stats_slots;
+    p.tld = desc->ld_target_stats ? desc->ld_target_stats : desc->target_stats_slots;
+  }
+  if (sampling && p.k > 0 && desc->draft_stats) {
+    p.dstats = reinterpret_cast<const float2 *>(desc->draft_stats);
+    p.dslots = desc->draft_stats_slots;
+    p.dld = desc->ld_draft_stats ? desc->ld_draft_stats : desc->draft_stats_slots;
+  }
+  // rows the statistics pass still computes: target rows, then draft rows
+  const bool need_t = !(sampling && (p.k == 0 || p.tstats != nullptr));
+  const bool need_d = sampling && p.k > 0 && p.dstats == nullptr;
+  p.stats_row0 = need_t ? 0 : p.rows_t;
+  p.stats_rows = (need_t ? p.rows_t : 0) + (need_d ? p.rows_total - p.rows_t : 0);
+  p.stats_chunk = stats_chunk_of(p.stats_rows > 0 ? p.stats_rows : 1, desc->vocab);
   p.nchunks = (desc->vocab + p.stats_chunk - 1) / p.stats_chunk;
   p.T = desc->temperature;
   p.seed = desc->seed;
@@ -542,6 +625,10 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.n_acc = n_accepted;
   p.out = out_tokens;
   p.margin = margin_flags;
+  if (desc->stats_out) {
+    p.sout = reinterpret_cast<float2 *>(desc->stats_out);
+    p.sld = desc->ld_stats_out ? desc->ld_stats_out : p.ndraw;
+  }
   const size_t rows = (size_t)p.B * (p.k + 1) + (size_t)p.B * p.k;
   uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
   p.stats = reinterpret_cast<float4 *>(w8);
@@ -551,13 +638,14 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.counters = reinterpret_cast<unsigned int *>(w8);
   p.status = device_status_word();
   cudaStream_t st = (cudaStream_t)stream;
-  if (sampling && p.k == 0) {
-    // a plain draw reads no row statistics: only the per-sequence tickets need clearing (a
-    // one-block kernel: in a CUDA graph it costs less than a memset node)
+  if (p.stats_rows == 0) {
+    // every row's statistics come from elsewhere (a plain draw needs none): only the
+    // per-sequence tickets need clearing (a one-block kernel: in a CUDA graph it costs less
+    // than a memset node)
     if (launch(clear_tickets_kernel, dim3(1), dim3(kThreads), 0, st, p.counters, p.B) !=
         cudaSuccess)
       return SD_ERR_CUDA;
-  } else if (launch(accept_stats_kernel, dim3(p.rows_total, p.nchunks), dim3(kThreads), 0, st,
+  } else if (launch(accept_stats_kernel, dim3(p.stats_rows, p.nchunks), dim3(kThreads), 0, st,
                     p) != cudaSuccess) {
     return SD_ERR_CUDA;
   }
