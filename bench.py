@@ -87,6 +87,28 @@ def dram_traffic(group):
         return None
 
 
+def rank_seed(rank):
+    """Seed of a rank's synthetic inputs: every rank verifies its own batch of sequences."""
+    return 100 + 7 * rank
+
+
+def max_over_ranks(x, world, device):
+    """A per-rank time maximised over the ranks (the identity at one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, batch, n_q, steps, ms):
+    """Verified tokens per second of the whole job: each of the world ranks verifies batch x n_q
+    tokens per step, all within ms (the slowest rank's time)."""
+    return world * batch * n_q * steps / (ms / 1e3)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -113,7 +135,7 @@ class SpecStep:
         self.hq, self.hkv, self.bs = 16, 4, 16
         self.V, self.d, self.dh = 262144, 5376, 1024
         self.C, self.cs, self.top_c = 1024, 256, 32
-        seed = 100 + 7 * rank
+        seed = rank_seed(rank)
         wg = S.Workload("g", B, L, k, 16, 4, [S.AttnLayer(512), S.AttnLayer(256, 512)],
                         self.d, self.V, seed=seed, n_clusters=self.C, cluster_size=self.cs,
                         drafter_hidden=self.dh, top_c=self.top_c)
@@ -617,14 +639,10 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
     ctx_b = st.ctx.cpu().numpy()
-    if world > 1:
-        tms = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
-        ms = float(tms.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, "cuda")
     ms_step = ms / a.steps
-    value = world * st.B * st.n_q * a.steps / (ms / 1e3)
+    value = whole_job_rate(world, st.B, st.n_q, a.steps, ms)
 
     # ---- per-kernel device times: the same step captured with event nodes around each call,
     # replayed K times (synchronised per replay to read the events)
@@ -686,12 +704,8 @@ def main():
             torch.cuda.current_stream().synchronize()
         e1.record()
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tms = torch.tensor([ems], device="cuda")
-            dist.all_reduce(tms, op=dist.ReduceOp.MAX)
-            ems = float(tms.item())
-        e2e = {"value": round(world * st.B * st.n_q * a.steps / (ems / 1e3), 1), "unit": UNIT,
+        ems = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+        e2e = {"value": round(whole_job_rate(world, st.B, st.n_q, a.steps, ems), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(ems / a.steps, 4),
                "path": "public C ABI calls and the step's host transfers captured once in a "
