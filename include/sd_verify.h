@@ -306,6 +306,11 @@ const char *sd_status_string(sd_status s);
 sd_status sd_device_status_read(int *out, sd_stream stream);
 /* Resets the current device's status word to 0 (stream-ordered). */
 sd_status sd_device_status_clear(sd_stream stream);
+/* Self-test of the bounded device wait that every kernel's barrier waits use: one thread waits
+ * on a barrier that nothing completes, gives up after the wait limit (2 s) and records
+ * SD_ERR_TIMEOUT in the status word; the context stays usable.  Stream-ordered; the launch
+ * status is returned.  (No counterpart in the pages: it checks this library's failure path.) */
+sd_status sd_selftest_bounded_wait(sd_stream stream);
 /* Library version: major * 10000 + minor * 100 + patch. */
 int sd_version(void);
 

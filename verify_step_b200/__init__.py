@@ -97,6 +97,7 @@ _SIGS = {
     "sd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sd_device_status_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), _P]),
     "sd_device_status_clear": (ctypes.c_int, [_P]),
+    "sd_selftest_bounded_wait": (ctypes.c_int, [_P]),
     "sd_version": (ctypes.c_int, []),
 }
 
@@ -230,6 +231,10 @@ def sd_device_status_read(stream=None) -> int:
 
 def sd_device_status_clear(stream=None):
     _check("sd_device_status_clear", lib().sd_device_status_clear(_stream(stream)))
+
+
+def sd_selftest_bounded_wait(stream=None):
+    _check("sd_selftest_bounded_wait", lib().sd_selftest_bounded_wait(_stream(stream)))
 
 
 def sd_version() -> int:

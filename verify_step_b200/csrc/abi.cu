@@ -36,6 +36,20 @@ bool pdl_enabled() {
   return on;
 }
 
+// One thread waits on a barrier no one arrives at: the bounded wait must give up and report.
+__global__ void selftest_wait_kernel(int *status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag)) record_status(status, SD_ERR_TIMEOUT);
+}
+
 int sm_count() {
   static int cache[64];
   int dev = 0;
@@ -112,6 +126,13 @@ sd_status sd_device_status_clear(sd_stream stream) {
   int *w = sdv::device_status_word();
   if (!w) return SD_ERR_CUDA;
   return sdv::cuda_status(cudaMemsetAsync(w, 0, sizeof(int), (cudaStream_t)stream));
+}
+
+sd_status sd_selftest_bounded_wait(sd_stream stream) {
+  int *w = sdv::device_status_word();
+  if (!w) return SD_ERR_CUDA;
+  return sdv::cuda_status(sdv::launch(sdv::selftest_wait_kernel, dim3(1), dim3(32), 0,
+                                      (cudaStream_t)stream, w));
 }
 
 int sd_version(void) { return 100; }
