@@ -18,6 +18,7 @@ Inputs are synthetic and resident in HBM; every step reads ~6 GB, far more than 
 so no L2 flush is needed between steps.  Contexts grow by the accepted length each step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--k K] [--batch B] [--ctx L]   (other points of the workload range)
 
 N > 1 (under torch.distributed.run): independent replicas, one batch per GPU, no collective
 on the data path (weak scaling); time = max over ranks.
@@ -37,7 +38,11 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "spec_step_b8_ctx16384_k2"
+WORKLOAD = "spec_step_b8_ctx16384_k2"  # the default configuration
+
+
+def workload_name(batch, ctx, k):
+    return f"spec_step_b{batch}_ctx{ctx}_k{k}"
 METRIC = "verified tokens/s per verify step (B,k,ctx); HBM GB/s as % of B200 peak"
 UNIT = "verified tokens/s"
 
@@ -73,10 +78,10 @@ def source_hash(name):
     return h.hexdigest()[:16]
 
 
-def dram_traffic(group):
+def dram_traffic(group, workload=WORKLOAD):
     """DRAM bytes per launch of a kernel group from the committed ncu summary, or None when
     the summary is missing or the kernel source changed since its counters were taken."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic_%s.json" % WORKLOAD)
+    path = os.path.join(ROOT, "profiles", "dram_traffic_%s.json" % workload)
     try:
         d = json.load(open(path))
         e = d["groups"][group]
@@ -673,7 +678,8 @@ def main():
     def roof(g):
         ach = nbytes[g] / (kern_ms[g] * 1e6)
         return {"kernel": g, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
-                "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": dram_traffic(g),
+                "unit": "GB/s", "frac": round(ach / hbm, 4),
+                "traffic": dram_traffic(g, workload_name(st.B, a.ctx, st.k)),
                 "peak_source": src, "bytes_per_launch": nbytes[g],
                 "ms_per_launch": round(kern_ms[g], 4)}
     # telemetry of the acceptance rule on these (random) weights
@@ -738,7 +744,8 @@ def main():
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch": st.B, "ctx": a.ctx, "k": st.k,
+        "config": {"workload": workload_name(st.B, a.ctx, st.k), "batch": st.B, "ctx": a.ctx,
+                   "k": st.k,
                    "heads": "16q/4kv", "layers": "global D512 + sliding D256 W512",
                    "lm_head": "d5376 x V262144", "drafter": "2-step chain, 4 cross-attn "
                    "layers, clustered head 1024x256 top-32 d1024", "block_size": 16,
@@ -780,7 +787,8 @@ def run_reference(a, rank, world):
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(dt / a.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "batch": a.batch, "ctx": a.ctx, "k": a.k},
+            "config": {"workload": workload_name(a.batch, a.ctx, a.k), "batch": a.batch,
+                       "ctx": a.ctx, "k": a.k},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": blas_threads(),
                              "kind": "oracle",
                              "sample": "per step one sequence of the batch (round robin): the "

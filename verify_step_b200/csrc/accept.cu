@@ -58,14 +58,6 @@ struct Params {
   int *status;
 };
 
-// 2^x by the hardware approximation (relative error about 2^-22; arguments here are <= 0, and
-// results below 2^-126 flush to 0, far below any weight that could win a race).
-__device__ __forceinline__ float ex2_approx(float x) {
-  float r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
 // E = -ln(1 - V) for V in [0, 1): the series V + V^2/2 + ... + V^8/8 below 1/16 (truncation
 // below 3e-11 relative), else -ln(1 - V) with 1 - V formed exactly or within 2^-25 and the fast
 // logarithm (absolute error below 4e-7, i.e. below 6e-6 relative to E >= 0.0645).

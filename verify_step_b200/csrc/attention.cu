@@ -33,6 +33,7 @@ namespace sdv {
 namespace attn {
 
 constexpr int kTile = 16;
+constexpr float kRescale = 8.f;  // log2 headroom of the lazily rescaled softmax
 
 struct Params {
   int B, n_q, Hq, Hkv, G, D, bs, mbps, num_blocks, window, M, Mpad;
@@ -504,32 +505,76 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
           sc[nt][e] = x;
           mx[e >> 1] = fmaxf(mx[e >> 1], x);
         }
-      float alpha[2];
+      if constexpr (MT == 1) {
+        // one query tile: the kernel streams at the memory's pace, rescale every tile
+        float alpha[2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-        const float m_new = fmaxf(m_run[h], mx[h]);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[h] = exp2f(m_run[h] - m_use);
-        m_run[h] = m_new;
-        l_run[h] *= alpha[h];
-        mx[h] = m_use;
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
-          sc[nt][e] = pv;
-          l_run[e >> 1] += pv;
+        for (int h = 0; h < 2; ++h) {
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+          const float m_new = fmaxf(m_run[h], mx[h]);
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          alpha[h] = exp2f(m_run[h] - m_use);
+          m_run[h] = m_new;
+          l_run[h] *= alpha[h];
+          mx[h] = m_use;
         }
 #pragma unroll
-      for (int nt = 0; nt < DS / 8; ++nt) {
-        o[nt][0] *= alpha[0];
-        o[nt][1] *= alpha[0];
-        o[nt][2] *= alpha[1];
-        o[nt][3] *= alpha[1];
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+            sc[nt][e] = pv;
+            l_run[e >> 1] += pv;
+          }
+#pragma unroll
+        for (int nt = 0; nt < DS / 8; ++nt) {
+          o[nt][0] *= alpha[0];
+          o[nt][1] *= alpha[0];
+          o[nt][2] *= alpha[1];
+          o[nt][3] *= alpha[1];
+        }
+      } else {
+        // several query tiles make the kernel issue-bound: a row's exponent base moves only
+        // when a tile's maximum passes it by more than kRescale (the unscaled terms then stay
+        // below 2^kRescale), so the accumulators are rescaled on few tiles and the warp skips
+        // the rescale otherwise
+        bool grow = false;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+          grow |= mx[h] > m_run[h] + kRescale;
+        }
+        if (__any_sync(0xffffffffu, grow)) {
+          float alpha[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            alpha[h] = 1.f;
+            if (mx[h] > m_run[h] + kRescale) {  // a finite maximum always passes -inf
+              alpha[h] = m_run[h] == -INFINITY ? 0.f : ex2_approx(m_run[h] - mx[h]);
+              m_run[h] = mx[h];
+            }
+            l_run[h] *= alpha[h];
+          }
+#pragma unroll
+          for (int nt = 0; nt < DS / 8; ++nt) {
+            o[nt][0] *= alpha[0];
+            o[nt][1] *= alpha[0];
+            o[nt][2] *= alpha[1];
+            o[nt][3] *= alpha[1];
+          }
+        }
+        const float base0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
+        const float base1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float pv = ex2_approx(sc[nt][e] - ((e & 2) ? base1 : base0));
+            sc[nt][e] = pv;
+            l_run[e >> 1] += pv;
+          }
       }
       uint32_t pa[4];
       pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
@@ -891,32 +936,76 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
           sc[nt][e] = x;
           mx[e >> 1] = fmaxf(mx[e >> 1], x);
         }
-      float alpha[2];
+      if constexpr (MT == 1) {
+        // one query tile: the kernel streams at the memory's pace, rescale every tile
+        float alpha[2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-        const float m_new = fmaxf(m_run[h], mx[h]);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[h] = exp2f(m_run[h] - m_use);
-        m_run[h] = m_new;
-        l_run[h] *= alpha[h];
-        mx[h] = m_use;
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
-          sc[nt][e] = pv;
-          l_run[e >> 1] += pv;
+        for (int h = 0; h < 2; ++h) {
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+          const float m_new = fmaxf(m_run[h], mx[h]);
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          alpha[h] = exp2f(m_run[h] - m_use);
+          m_run[h] = m_new;
+          l_run[h] *= alpha[h];
+          mx[h] = m_use;
         }
 #pragma unroll
-      for (int nt = 0; nt < DS / 8; ++nt) {
-        o[nt][0] *= alpha[0];
-        o[nt][1] *= alpha[0];
-        o[nt][2] *= alpha[1];
-        o[nt][3] *= alpha[1];
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
+            sc[nt][e] = pv;
+            l_run[e >> 1] += pv;
+          }
+#pragma unroll
+        for (int nt = 0; nt < DS / 8; ++nt) {
+          o[nt][0] *= alpha[0];
+          o[nt][1] *= alpha[0];
+          o[nt][2] *= alpha[1];
+          o[nt][3] *= alpha[1];
+        }
+      } else {
+        // several query tiles make the kernel issue-bound: a row's exponent base moves only
+        // when a tile's maximum passes it by more than kRescale (the unscaled terms then stay
+        // below 2^kRescale), so the accumulators are rescaled on few tiles and the warp skips
+        // the rescale otherwise
+        bool grow = false;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+          grow |= mx[h] > m_run[h] + kRescale;
+        }
+        if (__any_sync(0xffffffffu, grow)) {
+          float alpha[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            alpha[h] = 1.f;
+            if (mx[h] > m_run[h] + kRescale) {  // a finite maximum always passes -inf
+              alpha[h] = m_run[h] == -INFINITY ? 0.f : ex2_approx(m_run[h] - mx[h]);
+              m_run[h] = mx[h];
+            }
+            l_run[h] *= alpha[h];
+          }
+#pragma unroll
+          for (int nt = 0; nt < DS / 8; ++nt) {
+            o[nt][0] *= alpha[0];
+            o[nt][1] *= alpha[0];
+            o[nt][2] *= alpha[1];
+            o[nt][3] *= alpha[1];
+          }
+        }
+        const float base0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
+        const float base1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float pv = ex2_approx(sc[nt][e] - ((e & 2) ? base1 : base0));
+            sc[nt][e] = pv;
+            l_run[e >> 1] += pv;
+          }
       }
       uint32_t pa[4];
       pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);

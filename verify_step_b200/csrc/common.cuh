@@ -252,6 +252,15 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 
+// 2^x by the hardware approximation (relative error about 2^-22; results below 2^-126 flush
+// to 0).  Used where that error is far inside the tolerance: softmax terms that are rounded to
+// bf16 next, and race weights whose decisions carry a 1e-4 margin.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
