@@ -55,7 +55,8 @@ struct Params {
   const void *v_new;
   void *k_cache;
   void *v_cache;
-  int P;         // CTAs of the persistent grid
+  int P;           // CTA groups of the persistent split-KV grid (stream-K units)
+  int row_groups;  // CTAs per group: each takes one 16-row query tile of the same tile range
   int *status;
 };
 
@@ -318,8 +319,11 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   __syncthreads();
 
   const long long T = total_tiles(p, tab);
-  const long long start = T * blockIdx.x / p.P;
-  const long long end = T * (blockIdx.x + 1) / p.P;
+  // CTAs come in groups of row_groups that stream the same tile range, one query tile each
+  // (the group's repeated reads of a tile are served by L2)
+  const int grp = blockIdx.x / p.row_groups, rg = blockIdx.x % p.row_groups;
+  const long long start = T * grp / p.P;
+  const long long end = T * (grp + 1) / p.P;
 
   if (warp == NCW) {
     // ------------------------------------------------------------------- producer warp
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
 
   // --------------------------------------------------------------------- compute warps
   const int mg = warp / NDG, dg = warp % NDG;
-  const int r0 = mg * 16 + (lane >> 2);  // rows r0 and r0 + 8 of the item
+  const int r0 = (rg * MT + mg) * 16 + (lane >> 2);  // rows r0 and r0 + 8 of the item
   const int kq = 2 * (lane & 3);         // column pair inside an 8-wide n tile
   const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(p.q);
 
@@ -649,7 +653,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
               pack_bf16x2(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
       }
     } else {
-      const size_t slot = (size_t)b * p.Hkv + g + blockIdx.x;
+      const size_t slot = (size_t)b * p.Hkv + g + grp;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int row = r0 + 8 * h;
@@ -1374,13 +1378,12 @@ struct Launcher {
   static sd_status launch(const CUtensorMap &km, const CUtensorMap &vm, const Params &p,
                           cudaStream_t st) {
     return cuda_status(
-        sdv::launch(attn_bf16_kernel<D, MT, STAGES>, dim3(p.P), dim3(C::THREADS), C::SMEM, st,
+        sdv::launch(attn_bf16_kernel<D, MT, STAGES>, dim3(p.P * p.row_groups), dim3(C::THREADS),
+                    C::SMEM, st,
                     km, vm, p));
   }
 };
 
-template <int D, int MT>
-struct Pick;
 #define SDV_STAGES(D) ((D) == 512 ? 3 : (D) == 256 ? 4 : (D) == 128 ? 6 : 8)
 
 // Persistent CTAs for a (head_dim, row tiles) pair on the current device.
@@ -1388,10 +1391,7 @@ static int persistent_ctas(int D, int MT) {
   int occ = 0;
 #define SDV_CASE(DD, MM)                                      \
   if (D == DD && MT == MM) occ = Launcher<DD, MM, SDV_STAGES(DD)>::ctas_per_sm();
-  SDV_CASE(64, 1) SDV_CASE(64, 2) SDV_CASE(64, 3) SDV_CASE(64, 4)
-  SDV_CASE(128, 1) SDV_CASE(128, 2) SDV_CASE(128, 3) SDV_CASE(128, 4)
-  SDV_CASE(256, 1) SDV_CASE(256, 2) SDV_CASE(256, 3) SDV_CASE(256, 4)
-  SDV_CASE(512, 1) SDV_CASE(512, 2) SDV_CASE(512, 3) SDV_CASE(512, 4)
+  SDV_CASE(64, 1) SDV_CASE(128, 1) SDV_CASE(256, 1) SDV_CASE(512, 1)
 #undef SDV_CASE
   const int sms = sm_count();
   if (occ <= 0 || sms <= 0) return 0;
@@ -1402,10 +1402,7 @@ static sd_status launch_bf16(int D, int MT, const CUtensorMap &km, const CUtenso
                              const Params &p, cudaStream_t st) {
 #define SDV_CASE(DD, MM) \
   if (D == DD && MT == MM) return Launcher<DD, MM, SDV_STAGES(DD)>::launch(km, vm, p, st);
-  SDV_CASE(64, 1) SDV_CASE(64, 2) SDV_CASE(64, 3) SDV_CASE(64, 4)
-  SDV_CASE(128, 1) SDV_CASE(128, 2) SDV_CASE(128, 3) SDV_CASE(128, 4)
-  SDV_CASE(256, 1) SDV_CASE(256, 2) SDV_CASE(256, 3) SDV_CASE(256, 4)
-  SDV_CASE(512, 1) SDV_CASE(512, 2) SDV_CASE(512, 3) SDV_CASE(512, 4)
+  SDV_CASE(64, 1) SDV_CASE(128, 1) SDV_CASE(256, 1) SDV_CASE(512, 1)
 #undef SDV_CASE
   return SD_ERR_UNSUPPORTED;
 }
@@ -1513,11 +1510,13 @@ static sd_status validate(const sd_attn_desc *d, bool draft) {
   return SD_OK;
 }
 
+// Stream-K groups of the split-KV kernel: the single-tile kernel's persistent CTAs, divided
+// into groups of one CTA per 16-row query tile.
 static int grid_ctas(const sd_attn_desc *d) {
   if (d->dtype != SD_BF16) return 0;
   const int G = d->h_q / d->h_kv;
   const int MT = (G * d->n_q + 15) / 16;
-  return persistent_ctas(d->head_dim, MT);
+  return persistent_ctas(d->head_dim, 1) / MT;
 }
 
 static size_t ws_size(const sd_attn_desc *d) {
@@ -1578,7 +1577,8 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
       (!draft && (!aligned16(k_new) || !aligned16(v_new))))
     return SD_ERR_INVALID_ARG;
   const int MT = p.Mpad / 16;
-  p.P = persistent_ctas(p.D, MT);
+  p.row_groups = MT;
+  p.P = grid_ctas(d);
   if (p.P <= 0) return SD_ERR_CUDA;
   const size_t need = ws_size(d);
   if (!ws || ws_bytes < need) return SD_ERR_WORKSPACE;
@@ -1609,7 +1609,7 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
     const int tiles_max = (p.window + p.n_q - 1 + kTile - 1) / kTile + 1;
     return launch_window(p.D, MT, km, vm, p, tiles_max, st);
   }
-  s = launch_bf16(p.D, MT, km, vm, p, st);
+  s = launch_bf16(p.D, 1, km, vm, p, st);
   if (s != SD_OK) return s;
   return cuda_status(
       launch(attn_combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hkv, p.M), dim3(128), 0, st, p));
