@@ -41,8 +41,8 @@ sys.path.insert(0, ROOT)
 WORKLOAD = "spec_step_b8_ctx16384_k2"  # the default configuration
 
 
-def workload_name(batch, ctx, k):
-    return f"spec_step_b{batch}_ctx{ctx}_k{k}"
+def workload_name(batch, ctx, k, drafter_layers=False):
+    return f"spec_step_b{batch}_ctx{ctx}_k{k}" + ("_drafter_layers" if drafter_layers else "")
 METRIC = "verified tokens/s per verify step (B,k,ctx); HBM GB/s as % of B200 peak"
 UNIT = "verified tokens/s"
 
@@ -58,6 +58,10 @@ def parse():
     ap.add_argument("--ctx", type=int, default=16384)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--drafter-layers", action="store_true",
+                    help="run the drafter's dense layers (input projection, 4 x (W_q, W_o, "
+                         "gated MLP, W_d), output projection) around its cross-attention, so "
+                         "the chain is driven by the committed hidden row and tokens")
     return ap.parse_args()
 
 
@@ -65,7 +69,8 @@ def parse():
 GROUP_SOURCE = {"head_dense": "lm_head.cu", "head_clustered": "lm_head.cu",
                 "verify_global": "attention.cu", "verify_sliding": "attention.cu",
                 "xattn_global": "attention.cu", "xattn_sliding": "attention.cu",
-                "accept": "accept.cu", "accept_draft": "accept.cu", "commit": "commit.cu"}
+                "accept": "accept.cu", "accept_draft": "accept.cu", "commit": "commit.cu",
+                "drafter_dense": "linear.cu"}
 
 
 def source_hash(name):
@@ -128,7 +133,7 @@ def peaks():
 class SpecStep:
     """Device buffers, descriptors and the call sequence of one speculative step."""
 
-    def __init__(self, k=2, B=8, L=16384, reserve=600, rank=0, dev="cuda"):
+    def __init__(self, k=2, B=8, L=16384, reserve=600, rank=0, dev="cuda", dense=False):
         import numpy as np
         import torch
 
@@ -137,6 +142,7 @@ class SpecStep:
         self.sd, self.np, self.torch = sd, np, torch
         self.k, self.B, self.n_q = k, B, k + 1
         self.dev = dev
+        self.dense = dense
         self.hq, self.hkv, self.bs = 16, 4, 16
         self.V, self.d, self.dh = 262144, 5376, 1024
         self.C, self.cs, self.top_c = 1024, 256, 32
@@ -164,7 +170,7 @@ class SpecStep:
             s = S.make_step_qkv(wg, layer, self.n_q)
             inp[f"q{layer}"], inp[f"kn{layer}"], inp[f"vn{layer}"] = s["q"], s["k_new"], s["v_new"]
         inp["hidden"] = S.make_hidden(wg, B * self.n_q)
-        for j in range(k):
+        for j in range(0 if dense else k):
             for layer, D in ((0, 512), (1, 256)):
                 n = 1 if layer == 0 else 3
                 inp[f"dq{j}_{layer}"] = S.bf16(S.normal(seed * 31 + 10 * j + layer,
@@ -174,7 +180,7 @@ class SpecStep:
         # all per-step inputs live in one device buffer (256-byte aligned views) ordered by
         # the phase that first reads them (drafter step 0, drafter step 1, ..., verify), so the
         # end-to-end leg moves each phase's inputs with one host-to-device copy
-        phases = [[f"dq{j}_0", f"dq{j}_1", f"dh{j}"] for j in range(k)]
+        phases = [[] if dense else [f"dq{j}_0", f"dq{j}_1", f"dh{j}"] for j in range(k)]
         phases.append([kk for kk in inp if not kk.startswith("dq") and not kk.startswith("dh")])
         offs, total, self.phase_ranges = {}, 0, []
         for keys in phases:
@@ -214,7 +220,19 @@ class SpecStep:
         self.margin = torch.zeros(B, dtype=i32, device=dev)
         self.dtok = torch.zeros((B, 1), dtype=i32, device=dev)
         self.slots = torch.zeros((B, self.n_q), dtype=i32, device=dev)
-        self.next_hidden = torch.empty((B, self.d), dtype=torch.bfloat16, device=dev)
+        self.next_hidden = g(S.make_hidden(wg, B, step=97))
+        if dense:
+            # the drafter's dense layers: link 0 reads the committed hidden row and the last
+            # emitted token of the previous step, link j > 0 the back projection of link j-1
+            # and draft j-1
+            from verify_step_b200 import drafter as VD
+            self.VD = VD
+            self.dshape = VD.DrafterShape(batch=B, d=self.dh, d_target=self.d,
+                                          ff=S.DRAFTER_FF, h_q=self.hq,
+                                          head_dims=(256, 256, 256, 512), vocab=self.V)
+            self.dwts = VD.device_weights(S.make_drafter_weights(
+                seed, self.dh, self.d, self.V, self.hq, self.dshape.head_dims), dev)
+            self.dbuf = VD.buffers(self.dshape, dev)
         # descriptors
         self.vdesc = [self._adesc(0, self.n_q), self._adesc(1, self.n_q)]
         self.xdesc = [[self._adesc(layer, 1, q_offset=j) for layer in (0, 1)] for j in range(k)]
@@ -257,12 +275,14 @@ class SpecStep:
     # kernels per call of each group on this workload (the step graph's kernel nodes are
     # counted directly where the CUDA runtime allows; this is the fallback)
     LAUNCHES = dict(xattn_sliding=1, xattn_global=2, verify_sliding=1, verify_global=3,
-                    head_dense=1, head_clustered=3, accept_draft=1, accept=2, commit=1)
+                    head_dense=1, head_clustered=3, accept_draft=1, accept=2, commit=1,
+                    drafter_dense=1)
 
     def launches_per_step(self):
         L = self.LAUNCHES
+        dense = self.VD.LAUNCHES_PER_LINK * L["drafter_dense"] if self.dense else 0
         return (self.k * (3 * L["xattn_sliding"] + L["xattn_global"] + L["head_clustered"] +
-                          L["accept_draft"]) +
+                          L["accept_draft"] + dense) +
                 L["verify_global"] + L["verify_sliding"] + L["head_dense"] + L["accept"] +
                 L["commit"])
 
@@ -288,13 +308,16 @@ class SpecStep:
             if before_phase is not None:
                 before_phase(j)
             xd0, xd1 = self.xdesc[j]
-            for r in range(3):
-                timed("xattn_sliding", lambda: sd.sd_draft_xattn(
-                    xd1, I[f"dq{j}_1"][r], c1["k"], c1["v"], c1["table"], self.ctx, None,
-                    self.xout[1], self.ws))
-            timed("xattn_global", lambda: sd.sd_draft_xattn(
-                xd0, I[f"dq{j}_0"][0], c0["k"], c0["v"], c0["table"], self.ctx, None,
-                self.xout[0], self.ws))
+            if self.dense:
+                self._dense_link(j, timed)
+            else:
+                for r in range(3):
+                    timed("xattn_sliding", lambda: sd.sd_draft_xattn(
+                        xd1, I[f"dq{j}_1"][r], c1["k"], c1["v"], c1["table"], self.ctx, None,
+                        self.xout[1], self.ws))
+                timed("xattn_global", lambda: sd.sd_draft_xattn(
+                    xd0, I[f"dq{j}_0"][0], c0["k"], c0["v"], c0["table"], self.ctx, None,
+                    self.xout[0], self.ws))
             timed("head_clustered", lambda: self._clustered(j))
             ad = self.adesc_draft[j]
             timed("accept_draft", lambda: sd.sd_accept(
@@ -316,6 +339,27 @@ class SpecStep:
         timed("commit", lambda: sd.sd_commit(self.cdesc, c0["table"], self.ctx, self.n_acc,
                                              self.slots, I["hidden"], self.next_hidden))
 
+    def _dense_link(self, j, timed):
+        sd = self.sd
+        c0, c1 = self.cache
+        xd0, xd1 = self.xdesc[j]
+
+        def attend(i, q, o):
+            if i < 3:  # sliding layers first, the global layer last
+                timed("xattn_sliding", lambda: sd.sd_draft_xattn(
+                    xd1, q, c1["k"], c1["v"], c1["table"], self.ctx, None, o, self.ws))
+            else:
+                timed("xattn_global", lambda: sd.sd_draft_xattn(
+                    xd0, q, c0["k"], c0["v"], c0["table"], self.ctx, None, o, self.ws))
+
+        if j == 0:
+            h_prev, toks, ld, sel = self.next_hidden, self.out_tokens, self.n_q, self.n_acc
+        else:
+            h_prev, toks, ld, sel = self.dbuf["h_back"], self._col_ptr(self.drafts, j - 1), \
+                self.k, None
+        self.VD.link(self.dshape, self.dwts, self.dbuf, h_prev, toks, ld, attend,
+                     token_sel=sel, wrap=lambda fn: timed("drafter_dense", fn))
+
     def _row_ptr(self, t, j):
         return t.data_ptr() + j * self.V * t.element_size()
 
@@ -324,7 +368,8 @@ class SpecStep:
 
     def _clustered(self, j):
         # logits of draft step j go to row b*k + j of draft_logits (ld_logits = k * V)
-        self.sd.sd_lm_head(self.hdesc_cl, self.inputs[f"dh{j}"], self.cl["w_cm"],
+        hidden = self.dbuf["h"] if self.dense else self.inputs[f"dh{j}"]
+        self.sd.sd_lm_head(self.hdesc_cl, hidden, self.cl["w_cm"],
                            self._row_ptr(self.draft_logits, j),
                            centroids=self.cl["centroids"],
                            cluster_tokens=self.cl["cluster_tokens"], sel_clusters=self.sel,
@@ -355,12 +400,18 @@ class SpecStep:
         out["accept"] = int((B * n_q + B * self.k) * self.V * 4)
         out["accept_draft"] = int(B * self.V * 4)
         out["commit"] = int(B * (n_q * 4 * 2 + self.d * 2 * 2))
+        if self.dense:
+            out["drafter_dense"] = int(self.VD.hbm_bytes_per_link(self.dshape) /
+                                       self.VD.LAUNCHES_PER_LINK)
         return out
 
     def calls_per_step(self):
-        return dict(xattn_sliding=3 * self.k, xattn_global=self.k, head_clustered=self.k,
-                    accept_draft=self.k, verify_global=1, verify_sliding=1, head_dense=1,
-                    accept=1, commit=1)
+        out = dict(xattn_sliding=3 * self.k, xattn_global=self.k, head_clustered=self.k,
+                   accept_draft=self.k, verify_global=1, verify_sliding=1, head_dense=1,
+                   accept=1, commit=1)
+        if self.dense:
+            out["drafter_dense"] = self.VD.LAUNCHES_PER_LINK * self.k
+        return out
 
     def reset(self):
         self.ctx.copy_(self.ctx0)
@@ -617,7 +668,9 @@ def main():
 
     # every pass below runs a.steps steps (warm-up, timed, per-kernel, e2e): reserve the blocks
     reserve = (a.warmup + 4 * a.steps + 8) * (a.k + 1) + 64
-    st = SpecStep(k=a.k, B=a.batch, L=a.ctx, reserve=reserve, rank=rank)
+    st = SpecStep(k=a.k, B=a.batch, L=a.ctx, reserve=reserve, rank=rank,
+                  dense=a.drafter_layers)
+    wname = workload_name(st.B, a.ctx, st.k, a.drafter_layers)
     L_start = st.L0.copy()
     clock = ClockSampler(local)
     for _ in range(a.warmup):
@@ -679,7 +732,7 @@ def main():
         ach = nbytes[g] / (kern_ms[g] * 1e6)
         return {"kernel": g, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
                 "unit": "GB/s", "frac": round(ach / hbm, 4),
-                "traffic": dram_traffic(g, workload_name(st.B, a.ctx, st.k)),
+                "traffic": dram_traffic(g, wname),
                 "peak_source": src, "bytes_per_launch": nbytes[g],
                 "ms_per_launch": round(kern_ms[g], 4)}
     # telemetry of the acceptance rule on these (random) weights
@@ -724,7 +777,7 @@ def main():
     del graph, graph_ev, graph_e2e
 
     cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.drafter_layers:
         t = time.perf_counter()
         nv = oracle_sample(st, [0], 0)
         dt = time.perf_counter() - t
@@ -744,14 +797,18 @@ def main():
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": workload_name(st.B, a.ctx, st.k), "batch": st.B, "ctx": a.ctx,
+        "config": {"workload": wname, "batch": st.B, "ctx": a.ctx,
                    "k": st.k,
                    "heads": "16q/4kv", "layers": "global D512 + sliding D256 W512",
                    "lm_head": "d5376 x V262144", "drafter": "2-step chain, 4 cross-attn "
                    "layers, clustered head 1024x256 top-32 d1024", "block_size": 16,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "inputs larger than L2 (~6 GB read per step)",
-                   "ctx_growth": "contexts advance by the accepted length each step"},
+                   "ctx_growth": "contexts advance by the accepted length each step",
+                   **({"drafter_layers": "per link: W_in [1024 x (5376+1024)] on the committed "
+                       "hidden row and the embedding of the last token, 4 x (RMSNorm, W_q, "
+                       "cross-attention, W_o, RMSNorm, gated GELU MLP 4096, W_d), RMSNorm, "
+                       "W_back [5376 x 1024]; synthetic weights"} if a.drafter_layers else {})},
         "gpu_launches": kernels_per_step * a.steps,
         "roofline": roof(dom),
         "roofline_attention": roof("verify_global"),

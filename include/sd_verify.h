@@ -298,6 +298,72 @@ sd_status sd_commit(const sd_commit_desc *desc, const int32_t *block_table, int3
                     void *next_hidden, sd_stream stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Drafter dense layers ("Gemma 4 MTP: drafter drafts, target verifies", section "drafter
+ * internal architecture": the drafter has a token embedder of its own and a block of 4
+ * transformer layers, and its forward pass takes the target's last-layer activation together
+ * with the drafter embedding of the last token; Gemma 4 MTP serving guide, section 4: the
+ * drafter predicts its candidates as a chain).  One call is one projection of m token rows
+ * with an optional prologue and a fused epilogue.  A drafter layer is four calls around
+ * sd_draft_xattn: W_q (normalised input), W_o (added to the residual stream), the gated MLP's
+ * gate and up rows (normalised input, gated epilogue), W_d (added to the residual stream).
+ *
+ *   input row r, k columns:
+ *     x'[r, c] = x[r, c]                        c <  k - k_gather
+ *     x'[r, c] = table[t_r, c - (k - k_gather)] c >= k - k_gather (an embedding row)
+ *     t_r = tokens[r * ld_tokens + (token_sel ? token_sel[r] : 0)]
+ *   prologue (norm_gain != NULL):
+ *     x'[r, c] <- x'[r, c] / sqrt(mean_c x'[r, c]^2 + norm_eps) * norm_gain[c]
+ *   y[r, i] = sum_c bf16(x'[r, c]) * W[i, c]    (float32 accumulation in a fixed order: the
+ *                                                result does not depend on the launch)
+ *   epilogue:
+ *     SD_EPI_STORE  out[r, i] = y[r, i]                           out_dtype f32 or bf16
+ *     SD_EPI_ADD    out[r, i] += y[r, i]                          out_dtype f32 (a residual
+ *                                                                 stream)
+ *     SD_EPI_GEGLU  out[r, f] = gelu(y[r, gate(f)]) * y[r, up(f)] out_dtype bf16, n / 2
+ *                   columns; gelu(z) = z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))); W holds
+ *                   gate and up rows in blocks of 16: rows 16t .. 16t+7 are the gate rows of
+ *                   features 8t .. 8t+7, rows 16t+8 .. 16t+15 their up rows
+ *   norm_out (nullable, needs norm_gain): bf16 [m, ld_norm_out], the normalised rows
+ *                   bf16(x') (the drafter's output row, the input of its LM head)
+ *
+ *   x      [m, ld_x] of x_dtype (f32 or bf16); its first k - k_gather columns are read
+ *   W      bf16 [n, k] row-major
+ *   table  bf16 [table_rows, ld_table]; k_gather columns of row t_r are read
+ *   tokens, token_sel   int32; token_sel[r] in [0, max(ld_tokens, 1))
+ *   out    [m, ld_out] of out_dtype
+ * Limits: 0 <= m <= 64 (m = 0 launches nothing), n a multiple of 16, k a multiple of 32,
+ * k_gather a multiple of 8 (0: no gather), ld_x and ld_table multiples of 4 elements, x, W and
+ * table 16-byte aligned; out must not overlap x, table, W or norm_out.  A token id outside
+ * [0, table_rows) or a token_sel outside its range is not dereferenced: the row reads zeros and
+ * SD_ERR_DEVICE is recorded.  No workspace: split-K partials are reduced through the shared
+ * memory of a thread-block cluster.
+ */
+typedef enum { SD_EPI_STORE = 0, SD_EPI_ADD = 1, SD_EPI_GEGLU = 2 } sd_epilogue;
+
+typedef struct {
+  int m;                  /* token rows */
+  int n;                  /* rows of W (output features; 2x the output columns for GEGLU) */
+  int k;                  /* columns of W: input width including the gathered columns */
+  sd_dtype x_dtype;       /* element type of x */
+  int64_t ld_x;           /* row stride of x (elements) */
+  int k_gather;           /* trailing input columns taken from table (0: none) */
+  int64_t ld_table;       /* row stride of table (elements) */
+  int64_t table_rows;     /* rows of table (token ids are checked against it) */
+  int64_t ld_tokens;      /* stride of tokens between rows */
+  const float *norm_gain; /* DEVICE f32 [k], or NULL for no normalisation */
+  float norm_eps;         /* e.g. 1e-6 */
+  sd_epilogue epilogue;
+  sd_dtype out_dtype;
+  int64_t ld_out;         /* row stride of out (elements) */
+  void *norm_out;         /* nullable DEVICE bf16 [m, ld_norm_out] */
+  int64_t ld_norm_out;
+} sd_linear_desc;
+
+sd_status sd_linear(const sd_linear_desc *desc, const void *x, const void *W, void *out,
+                    const void *table, const int32_t *tokens, const int32_t *token_sel,
+                    sd_stream stream);
+
+/* ---------------------------------------------------------------------------------------
  * Status.
  */
 const char *sd_status_string(sd_status s);

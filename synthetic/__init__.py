@@ -266,3 +266,35 @@ def make_logits(seed: int, rows: int, vocab: int, std: float = 1.0) -> torch.Ten
 def perturb(seed: int, z: torch.Tensor, sigma: float) -> torch.Tensor:
     """Draft logits y = z + N(0, sigma^2) noise (fp32)."""
     return z + torch.from_numpy(normal(seed, tuple(z.shape), sigma))
+
+
+# ----------------------------------------------------------------------------- drafter layers
+
+DRAFTER_FF = 4096  # gated-MLP width of the synthetic drafter layers (4 x the hidden width)
+
+
+def make_drafter_weights(seed: int, d: int, d_target: int, vocab: int, h_q: int, head_dims,
+                         ff: int = DRAFTER_FF):
+    """Synthetic drafter weights (CPU tensors): embedding E [vocab, d], input projection
+    W_in [d, d_target + d], per layer RMSNorm gains (float32, 1 + N(0, 0.1^2)) and bf16
+    projections Wq [h_q D, d], Wo [d, h_q D], Wg, Wu [ff, d], Wd [d, ff] (each ~ N(0, 1/fan_in)),
+    the output gain g_final and the back projection W_back [d_target, d]."""
+    s = 50000 + 1000 * int(seed)
+    out = {"E": bf16(normal(s, (vocab, d))),
+           "W_in": bf16(normal(s + 1, (d, d_target + d), 1 / math.sqrt(d_target + d))),
+           "g_final": torch.from_numpy(1 + normal(s + 2, (d,), 0.1)),
+           "W_back": bf16(normal(s + 3, (d_target, d), 1 / math.sqrt(d))),
+           "layers": []}
+    for i, D in enumerate(head_dims):
+        t = s + 10 * (i + 1)
+        out["layers"].append({
+            "g_attn": torch.from_numpy(1 + normal(t, (d,), 0.1)),
+            "Wq": bf16(normal(t + 1, (h_q * D, d), 1 / math.sqrt(d))),
+            "Wo": bf16(normal(t + 2, (d, h_q * D), 1 / math.sqrt(h_q * D))),
+            "g_mlp": torch.from_numpy(1 + normal(t + 3, (d,), 0.1)),
+            "Wg": bf16(normal(t + 4, (ff, d), 1 / math.sqrt(d))),
+            "Wu": bf16(normal(t + 5, (ff, d), 1 / math.sqrt(d))),
+            "Wd": bf16(normal(t + 6, (d, ff), 1 / math.sqrt(ff))),
+        })
+    return out
+

@@ -104,3 +104,70 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError):
         sd._ptr(torch.zeros(4, 4).t())
     assert d.m == 1
+
+
+def test_linear_validation(lib):
+    L = lib
+    A = 4096  # any 16-byte aligned non-null address: every case below is refused before a launch
+    assert L.sd_linear(None, None, None, None, None, None, None, None) == sd.SD_ERR_INVALID_ARG
+    d = sd.LinearDesc(m=0, n=32, k=64, x_dtype=sd.SD_BF16, ld_x=64, epilogue=sd.SD_EPI_STORE,
+                      out_dtype=sd.SD_F32, ld_out=32)
+    # an empty batch launches nothing
+    assert L.sd_linear(ctypes.byref(d), None, None, None, None, None, None, None) == sd.SD_OK
+    d.m = 8
+    assert L.sd_linear(ctypes.byref(d), None, A, A, None, None, None, None) == sd.SD_ERR_INVALID_ARG
+    for field, value, want in (("m", 65, sd.SD_ERR_UNSUPPORTED), ("n", 40, sd.SD_ERR_UNSUPPORTED),
+                               ("k", 48, sd.SD_ERR_UNSUPPORTED), ("ld_x", 62, sd.SD_ERR_INVALID_ARG),
+                               ("ld_out", 16, sd.SD_ERR_INVALID_ARG),
+                               ("x_dtype", 7, sd.SD_ERR_INVALID_ARG)):
+        e = sd.LinearDesc.from_buffer_copy(d)
+        setattr(e, field, value)
+        if field == "k":
+            e.ld_x = 48
+        assert L.sd_linear(ctypes.byref(e), A, A, A, None, None, None, None) == want, field
+    # misaligned x or W
+    assert L.sd_linear(ctypes.byref(d), A + 8, A, A, None, None, None, None) == sd.SD_ERR_INVALID_ARG
+    assert L.sd_linear(ctypes.byref(d), A, A + 2, A, None, None, None, None) == sd.SD_ERR_INVALID_ARG
+    # epilogue / output type pairs
+    e = sd.LinearDesc.from_buffer_copy(d)
+    e.epilogue, e.out_dtype = sd.SD_EPI_ADD, sd.SD_BF16
+    assert L.sd_linear(ctypes.byref(e), A, A, A, None, None, None, None) == sd.SD_ERR_INVALID_ARG
+    e.epilogue, e.out_dtype = sd.SD_EPI_GEGLU, sd.SD_F32
+    assert L.sd_linear(ctypes.byref(e), A, A, A, None, None, None, None) == sd.SD_ERR_INVALID_ARG
+    # normalised copy without a gain; gather without a table
+    e = sd.LinearDesc.from_buffer_copy(d)
+    e.norm_out, e.ld_norm_out = A, 64
+    assert L.sd_linear(ctypes.byref(e), A, A, A, None, None, None, None) == sd.SD_ERR_INVALID_ARG
+    e = sd.LinearDesc.from_buffer_copy(d)
+    e.k_gather, e.ld_x, e.ld_table, e.table_rows = 32, 32, 32, 100
+    assert L.sd_linear(ctypes.byref(e), A, A, A, None, A, None, None) == sd.SD_ERR_INVALID_ARG
+    e.k_gather = 12
+    assert L.sd_linear(ctypes.byref(e), A, A, A, A, A, None, None) == sd.SD_ERR_UNSUPPORTED
+
+
+def test_descriptor_layouts_match_the_header(tmp_path):
+    """The ctypes descriptors have the C structs' size and field offsets (gcc on the header)."""
+    structs = {"sd_attn_desc": sd.AttnDesc, "sd_head_desc": sd.HeadDesc,
+               "sd_accept_desc": sd.AcceptDesc, "sd_commit_desc": sd.CommitDesc,
+               "sd_poison_cache": sd.PoisonCache, "sd_linear_desc": sd.LinearDesc}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "sd_verify.h"',
+             'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                               check=True).stdout.splitlines():
+        cname, fname, v = line.split()
+        got[(cname, fname)] = int(v)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)

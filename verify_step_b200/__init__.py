@@ -6,7 +6,7 @@ memory and streams.  There is no fallback: if the library is missing or a call f
 binding raises.
 
 Functions carry the C names (sd_verify_attn, sd_draft_xattn, sd_lm_head, sd_accept,
-sd_commit and the *_workspace_size / status helpers).  Tensors are passed as torch CUDA
+sd_commit, sd_linear and the *_workspace_size / status helpers).  Tensors are passed as torch CUDA
 tensors (their data_ptr is used; they must be contiguous), descriptors as the ctypes
 structures below, ``stream`` as a torch.cuda.Stream (default: the current stream).
 """
@@ -73,6 +73,19 @@ class CommitDesc(ctypes.Structure):
                 ("step_ptr", ctypes.c_void_p)]
 
 
+SD_EPI_STORE, SD_EPI_ADD, SD_EPI_GEGLU = 0, 1, 2
+
+
+class LinearDesc(ctypes.Structure):
+    _fields_ = [("m", ctypes.c_int), ("n", ctypes.c_int), ("k", ctypes.c_int),
+                ("x_dtype", ctypes.c_int), ("ld_x", ctypes.c_int64), ("k_gather", ctypes.c_int),
+                ("ld_table", ctypes.c_int64), ("table_rows", ctypes.c_int64),
+                ("ld_tokens", ctypes.c_int64), ("norm_gain", ctypes.c_void_p),
+                ("norm_eps", ctypes.c_float), ("epilogue", ctypes.c_int),
+                ("out_dtype", ctypes.c_int), ("ld_out", ctypes.c_int64),
+                ("norm_out", ctypes.c_void_p), ("ld_norm_out", ctypes.c_int64)]
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -94,6 +107,7 @@ _SIGS = {
     "sd_accept_noalloc": (ctypes.c_int, [ctypes.POINTER(AcceptDesc), _P, _P, _P, _P, _P, _P,
                                          _P]),
     "sd_commit": (ctypes.c_int, [ctypes.POINTER(CommitDesc), _P, _P, _P, _P, _P, _P, _P]),
+    "sd_linear": (ctypes.c_int, [ctypes.POINTER(LinearDesc), _P, _P, _P, _P, _P, _P, _P]),
     "sd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sd_device_status_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), _P]),
     "sd_device_status_clear": (ctypes.c_int, [_P]),
@@ -220,6 +234,12 @@ def sd_commit(desc, block_table, ctx_len, n_accepted, committed_slots, hidden=No
     _check("sd_commit", lib().sd_commit(
         ctypes.byref(desc), _ptr(block_table), _ptr(ctx_len), _ptr(n_accepted),
         _ptr(committed_slots), _ptr(hidden), _ptr(next_hidden), _stream(stream)))
+
+
+def sd_linear(desc, x, w, out, table=None, tokens=None, token_sel=None, stream=None):
+    _check("sd_linear", lib().sd_linear(
+        ctypes.byref(desc), _ptr(x), _ptr(w), _ptr(out), _ptr(table), _ptr(tokens),
+        _ptr(token_sel), _stream(stream)))
 
 
 def sd_device_status_read(stream=None) -> int:
