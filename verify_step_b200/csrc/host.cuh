@@ -19,9 +19,10 @@ int *device_status_word();
 int sm_count();
 
 // 2D bf16 tensor map over a row-major matrix [outer, inner] with the given row stride in
-// bytes, box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
+// bytes, box [box_outer, box_inner], 128-byte swizzle (or none), zero fill out of bounds.
 bool encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
-                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                         bool swizzle128 = true);
 
 inline sd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_CUDA; }
 

@@ -6,12 +6,13 @@
 // drafter runs 4 transformer layers on the target's last-layer activation and its own token
 // embedding.  With B = 8 token rows a projection is a matrix-vector product in all but name:
 // 8 FLOPs per weight byte, so the weights' single pass through HBM bounds it.  The kernel
-// streams W straight from HBM into mma.sync fragments (16-byte loads, no shared-memory hop, L1
-// bypassed) and keeps the few token rows in shared memory in fragment order; the K dimension is
-// split over the CTAs of a thread-block cluster and reduced through distributed shared memory,
-// so the result needs no workspace and does not depend on the launch.
+// streams each CTA's W rows into shared memory with a few large TMA tensor copies (completing on
+// mbarriers), feeds mma.sync from there and keeps the few token rows in
+// shared memory in fragment order; the K dimension is split over the CTAs of a thread-block
+// cluster and reduced through distributed shared memory, so the result needs no workspace and
+// does not depend on the launch.
 //
-// Fragment trick: a thread's 16-byte load holds 8 consecutive columns 8q .. 8q+7 of one W row.
+// Fragment trick: a thread's 16-byte read holds 8 consecutive columns 8q .. 8q+7 of one W row.
 // The two m16n8k16 steps of a 32-column chunk take columns {8q..8q+3} and {8q+4..8q+7} as their
 // logical k indices {2q, 2q+1, 2q+8, 2q+9}; the token rows are staged with the same column
 // mapping, so each product pairs the same physical column on both sides.
@@ -27,9 +28,7 @@ constexpr int kWarpsN = 2;                 // warps along W rows (16 rows each)
 constexpr int kWarpsK = 4;                 // warps along K inside a CTA
 constexpr int kThreads = 32 * kWarpsN * kWarpsK;
 constexpr int kRows = 16 * kWarpsN;        // W rows per CTA
-constexpr int kBatch = 8;                  // chunks of 32 columns in flight per warp
 constexpr int kMaxM = 64;
-constexpr int kStageBytes = 64 * 1024;     // staged token rows per piece (upper bound)
 
 struct Params {
   int m, n, k, k_x, x_f32;
@@ -52,15 +51,6 @@ struct Params {
   int *status;
 };
 
-// 16 bytes of a weight row that is read once: no L1 allocation.
-__device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -71,32 +61,62 @@ __device__ __forceinline__ float gelu_tanh(float z) {
   return 0.5f * z * (1.f + tanhf(0.7978845608028654f * (z + 0.044715f * z * z * z)));
 }
 
-// Four consecutive input columns col .. col+3 of row r (r < m), before normalisation.
-__device__ __forceinline__ float4 input4(const Params &p, int r, int col, int tok) {
-  if (col < p.k_x) {
-    if (p.x_f32)
-      return *reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + r * p.ld_x +
-                                               col);
-    const uint2 u = *reinterpret_cast<const uint2 *>(
-        static_cast<const __nv_bfloat16 *>(p.x) + r * p.ld_x + col);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-  }
-  if (tok < 0) return make_float4(0.f, 0.f, 0.f, 0.f);
-  const uint2 u = *reinterpret_cast<const uint2 *>(p.table + tok * p.ld_table + (col - p.k_x));
+__device__ __forceinline__ float4 bf16x4_to_f4(uint2 u) {
   const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
   const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
+// Four consecutive input columns col .. col+3 of row r, before normalisation (zeros for a row
+// past m or an invalid token).  Branch-free apart from the loads' own predicates, so that a
+// thread's loads in an unrolled loop are all in flight together.
+template <bool XF32>
+__device__ __forceinline__ float4 input4(const Params &p, int r, int col, int tok) {
+  const bool in_x = r < p.m && col < p.k_x;
+  const bool in_t = r < p.m && col >= p.k_x && tok >= 0;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (XF32) {
+    if (in_x)
+      v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + r * p.ld_x + col);
+  } else if (in_x) {
+    v = bf16x4_to_f4(*reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.x) +
+                                                      r * p.ld_x + col));
+  }
+  if (in_t) v = bf16x4_to_f4(*reinterpret_cast<const uint2 *>(p.table + tok * p.ld_table +
+                                                              (col - p.k_x)));
+  return v;
+}
+
+constexpr int kLd = 8;  // input loads in flight per thread in the prologue
+
+constexpr int kGroup = 8;     // chunks per tensor-copy group (one mbarrier each)
+constexpr int kMaxPiece = 32; // chunks staged per piece
+constexpr int kMaxGroups = kMaxPiece / kGroup;
+constexpr int kGroupBytes = kRows * kGroup * 64;  // 16 KB of weights per group
+
+// Shared-memory plan of a CTA for a piece of P chunks: the weights (one 16 KB region per group
+// of 8 chunks), the token rows in fragment order, then the partial sums; the reduction buffer
+// reuses the first two regions.
+__host__ __device__ constexpr int w_bytes(int P) { return (P + kGroup - 1) / kGroup * kGroupBytes; }
+__host__ __device__ constexpr int region_a(int P, int NT) {
+  return w_bytes(P) + NT * P * 512 > kWarpsK * kRows * NT * 32 ? w_bytes(P) + NT * P * 512
+                                                               : kWarpsK * kRows * NT * 32;
+}
+
 // grid: (ceil(n / 32) row blocks) x splits CTAs, clusters of `splits` along x; NT token groups
-// of 8 (m <= 8 NT).
-template <int NT>
-__global__ void __launch_bounds__(kThreads) linear_kernel(const Params p) {
-  extern __shared__ __align__(16) uint8_t smem[];
+// of 8 (m <= 8 NT).  One thread brings the CTA's weight rows into shared memory with TMA tensor
+// copies (no multicast): a full group of 8 chunks is one [32 rows x 256 columns] box (row-major,
+// 512 bytes a row), a partial group one [32 x 32] box per chunk (64 bytes a row); each group
+// completes on its own mbarrier.  Every warp then takes a 16-row half of the rows and a quarter
+// of the chunks.  Rows past n arrive as zeros (tensor out-of-bounds fill).
+template <int NT, bool XF32>
+__global__ void __launch_bounds__(kThreads, NT <= 2 ? 2 : 1)
+    linear_kernel(const __grid_constant__ CUtensorMap wmap_big,
+                  const __grid_constant__ CUtensorMap wmap_small, const Params p) {
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_inv[kMaxM];
   __shared__ int s_tok[kMaxM];
+  __shared__ __align__(8) uint64_t s_bar[kMaxGroups];
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wr = warp % kWarpsN, wk = warp / kWarpsN;
@@ -105,13 +125,41 @@ __global__ void __launch_bounds__(kThreads) linear_kernel(const Params p) {
   const int rank = S > 1 ? (int)cluster_ctarank() : 0;
   const int rb = blockIdx.x / S;
   const int row0 = rb * kRows;
+  const int box_rows = min(kRows, p.n);  // rows of every tensor box (the map's box height)
   const int C = p.k >> 5;
   const int c_begin = (int)((long long)C * rank / S);
   const int c_end = (int)((long long)C * (rank + 1) / S);
   const int P = p.piece;
-  uint2 *xs = reinterpret_cast<uint2 *>(smem);
-  float *part = reinterpret_cast<float *>(
-      smem + (size_t)max(NT * P * 64 * 8, kWarpsK * kRows * NT * 8 * 4));
+  uint8_t *wsm = smem;
+  uint2 *xs = reinterpret_cast<uint2 *>(smem + w_bytes(P));
+  float *part = reinterpret_cast<float *>(smem + region_a(P, NT));
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMaxGroups; ++i) mbar_init(&s_bar[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // thread 0: tensor copies of the weight rows of chunks pc0 .. pc0+np-1
+  auto issue = [&](int pc0, int np) {
+    if (threadIdx.x != 0) return;
+    const int groups = (np + kGroup - 1) / kGroup;
+    for (int gi = 0; gi < groups; ++gi) {
+      const int cnt = min(kGroup, np - gi * kGroup);
+      const int col = (pc0 + gi * kGroup) * 32;
+      mbar_arrive_expect_tx(&s_bar[gi], (uint32_t)(box_rows * cnt * 64));
+      if (cnt == kGroup) {
+        tma_load_2d(wsm + gi * kGroupBytes, &wmap_big, &s_bar[gi], col, row0);
+      } else {
+        for (int c = 0; c < cnt; ++c)
+          tma_load_2d(wsm + gi * kGroupBytes + c * (kRows * 64), &wmap_small, &s_bar[gi],
+                      col + c * 32, row0);
+      }
+    }
+  };
+  // the weights are requested before anything else: the prologue below (token ids, row
+  // statistics, staging of the token rows) runs under their HBM latency
+  issue(c_begin, min(P, c_end - c_begin));
 
   // ---- token ids and row statistics
   if (threadIdx.x < p.m) {
@@ -132,10 +180,17 @@ __global__ void __launch_bounds__(kThreads) linear_kernel(const Params p) {
   __syncthreads();
   if (p.gain != nullptr) {
     for (int r = warp; r < p.m; r += kThreads / 32) {
+      const int tok = s_tok[r];
       float ss = 0.f;
-      for (int col = lane * 4; col < p.k; col += 128) {
-        const float4 v = input4(p, r, col, s_tok[r]);
-        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      for (int c0 = lane * 4; c0 < p.k; c0 += 128 * kLd) {
+        float4 v[kLd];
+#pragma unroll
+        for (int u = 0; u < kLd; ++u)
+          v[u] = c0 + 128 * u < p.k ? input4<XF32>(p, r, c0 + 128 * u, tok)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < kLd; ++u)
+          ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -146,64 +201,76 @@ __global__ void __launch_bounds__(kThreads) linear_kernel(const Params p) {
   float acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  const int wrow = row0 + wr * 16;
-  const bool active = wrow < p.n;
-  const __nv_bfloat16 *w_lo = p.W + (size_t)(wrow + g) * p.k + q * 8;
-  const __nv_bfloat16 *w_hi = w_lo + (size_t)8 * p.k;
+  const bool active = row0 + wr * 16 < p.n;
+  uint32_t parity = 0;
+  bool timed_out = false;
 
   for (int pc0 = c_begin; pc0 < c_end; pc0 += P) {
     const int np = min(P, c_end - pc0);
-    // first batch of this warp's weight chunks: issued before the staging so that the HBM
-    // latency overlaps it
-    uint4 a_lo[kBatch], a_hi[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int cc = wk + kWarpsK * u;
-      if (active && cc < np) {
-        a_lo[u] = ld_stream_u4(w_lo + (size_t)(pc0 + cc) * 32);
-        a_hi[u] = ld_stream_u4(w_hi + (size_t)(pc0 + cc) * 32);
-      }
+    if (pc0 != c_begin) {
+      __syncthreads();  // every warp is done with the previous piece's rows and fragments
+      issue(pc0, np);
     }
-    __syncthreads();  // s_inv ready; the previous piece's fragments consumed
+    __syncthreads();  // s_inv ready
     // ---- stage the token rows of chunks pc0 .. pc0+np-1 in fragment order
-    for (int idx = threadIdx.x; idx < NT * np * 64; idx += kThreads) {
-      const int ln = idx & 31, s = (idx >> 5) & 1, rest = idx >> 6;
-      const int cc = rest % np, tg = rest / np;
-      const int r = tg * 8 + (ln >> 2);
-      const int col = (pc0 + cc) * 32 + (ln & 3) * 8 + s * 4;
-      uint2 v2 = make_uint2(0u, 0u);
-      if (r < p.m) {
-        float4 v = input4(p, r, col, s_tok[r]);
-        if (p.gain != nullptr) {
-          const float inv = s_inv[r];
-          const float4 gg = *reinterpret_cast<const float4 *>(p.gain + col);
-          v = make_float4(v.x * inv * gg.x, v.y * inv * gg.y, v.z * inv * gg.z, v.w * inv * gg.w);
-        }
-        v2 = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-        if (p.norm_out != nullptr && rb == 0)
-          *reinterpret_cast<uint2 *>(p.norm_out + r * p.ld_norm_out + col) = v2;
+    const int total = NT * np * 64;
+    for (int base = threadIdx.x; base < total; base += kThreads * kLd) {
+      float4 v[kLd];
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        const int idx = base + kThreads * u;
+        const int ln = idx & 31, s = (idx >> 5) & 1, rest = idx >> 6;
+        const int cc = rest % np, tg = rest / np;
+        const int r = idx < total ? tg * 8 + (ln >> 2) : p.m;  // rows past m read nothing
+        const int col = (pc0 + cc) * 32 + (ln & 3) * 8 + s * 4;
+        v[u] = input4<XF32>(p, r, col, r < p.m ? s_tok[r] : -1);
       }
-      xs[((tg * P + cc) * 2 + s) * 32 + ln] = v2;
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        const int idx = base + kThreads * u;
+        if (idx >= total) break;
+        const int ln = idx & 31, s = (idx >> 5) & 1, rest = idx >> 6;
+        const int cc = rest % np, tg = rest / np;
+        const int r = tg * 8 + (ln >> 2);
+        const int col = (pc0 + cc) * 32 + (ln & 3) * 8 + s * 4;
+        uint2 v2 = make_uint2(0u, 0u);
+        if (r < p.m) {
+          float4 x4 = v[u];
+          if (p.gain != nullptr) {
+            const float inv = s_inv[r];
+            const float4 gg = *reinterpret_cast<const float4 *>(p.gain + col);
+            x4 = make_float4(x4.x * inv * gg.x, x4.y * inv * gg.y, x4.z * inv * gg.z,
+                             x4.w * inv * gg.w);
+          }
+          v2 = make_uint2(pack_bf16x2(x4.x, x4.y), pack_bf16x2(x4.z, x4.w));
+          if (p.norm_out != nullptr && rb == 0)
+            *reinterpret_cast<uint2 *>(p.norm_out + r * p.ld_norm_out + col) = v2;
+        }
+        xs[((tg * P + cc) * 2 + s) * 32 + ln] = v2;
+      }
     }
     __syncthreads();
-    // ---- products
-    for (int b0 = 0; b0 < np; b0 += kWarpsK * kBatch) {
-      if (b0 > 0) {
+    // ---- products: chunk cc of the piece is in group cc / 8
+    const int row = wr * 16 + g;
+    const int groups = (np + kGroup - 1) / kGroup;
+    for (int gi = 0; gi < groups; ++gi) {
+      if (!mbar_wait_timed(&s_bar[gi], parity)) timed_out = true;
+      const bool full = np - gi * kGroup >= kGroup;
+      const uint8_t *gbase = wsm + gi * kGroupBytes;
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          const int cc = b0 + wk + kWarpsK * u;
-          if (active && cc < np) {
-            a_lo[u] = ld_stream_u4(w_lo + (size_t)(pc0 + cc) * 32);
-            a_hi[u] = ld_stream_u4(w_hi + (size_t)(pc0 + cc) * 32);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int cc = b0 + wk + kWarpsK * u;
+      for (int u = 0; u < kGroup / kWarpsK; ++u) {
+        const int c8 = wk + kWarpsK * u;
+        const int cc = gi * kGroup + c8;
         if (active && cc < np) {
-          const uint32_t f0[4] = {a_lo[u].x, a_hi[u].x, a_lo[u].y, a_hi[u].y};
-          const uint32_t f1[4] = {a_lo[u].z, a_hi[u].z, a_lo[u].w, a_hi[u].w};
+          // [32 x 256] box: row r at r * 512; [32 x 32] box of chunk c8 at c8 * 2048, row r at
+          // r * 64
+          const uint8_t *w_lo = full ? gbase + row * 512 + c8 * 64 + q * 16
+                                     : gbase + c8 * (kRows * 64) + row * 64 + q * 16;
+          const int hi_off = full ? 8 * 512 : 8 * 64;
+          const uint4 lo = *reinterpret_cast<const uint4 *>(w_lo);
+          const uint4 hi = *reinterpret_cast<const uint4 *>(w_lo + hi_off);
+          const uint32_t f0[4] = {lo.x, hi.x, lo.y, hi.y};
+          const uint32_t f1[4] = {lo.z, hi.z, lo.w, hi.w};
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             const uint2 b_0 = xs[((t * P + cc) * 2 + 0) * 32 + lane];
@@ -214,7 +281,9 @@ __global__ void __launch_bounds__(kThreads) linear_kernel(const Params p) {
         }
       }
     }
+    parity ^= 1u;
   }
+  if (timed_out) record_status(p.status, SD_ERR_TIMEOUT);
 
   // ---- reduce the kWarpsK partial sums of each warp row in shared memory (fixed order)
   __syncthreads();
@@ -246,31 +315,33 @@ __global__ void __launch_bounds__(kThreads) linear_kernel(const Params p) {
   const int u0 = units * rank / S, u1 = units * (rank + 1) / S;
   const int nu = u1 - u0;
   const uint32_t part_s = smem_u32(part);
+  // sum of element idx of the partials over the cluster's CTAs, in rank order (the DSMEM loads
+  // are all issued before the first add; ranks past S add an exact zero)
+  auto cluster_sum = [&](int idx) -> float {
+    if (S == 1) return part[idx];
+    float v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      v[c] = c < S ? ld_dsmem_f32(dsmem_addr(part_s + (uint32_t)idx * 4u, c)) : 0.f;
+    float y = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) y += v[c];
+    return y;
+  };
   for (int i = threadIdx.x; i < nu * p.m; i += kThreads) {
     const int tok = i / nu, unit = u0 + i % nu;
     if (p.epi == SD_EPI_GEGLU) {
       const int f = rb * (kRows / 2) + unit;
       if (f >= p.n / 2) continue;
       const int rg = (unit >> 3) * 16 + (unit & 7), ru = rg + 8;
-      float yg = 0.f, yu = 0.f;
-      for (int c = 0; c < S; ++c) {
-        if (S > 1) {
-          yg += ld_dsmem_f32(dsmem_addr(part_s + (uint32_t)(rg * MT8 + tok) * 4u, c));
-          yu += ld_dsmem_f32(dsmem_addr(part_s + (uint32_t)(ru * MT8 + tok) * 4u, c));
-        } else {
-          yg += part[rg * MT8 + tok];
-          yu += part[ru * MT8 + tok];
-        }
-      }
+      const float yg = cluster_sum(rg * MT8 + tok);
+      const float yu = cluster_sum(ru * MT8 + tok);
       static_cast<__nv_bfloat16 *>(p.out)[tok * p.ld_out + f] =
           __float2bfloat16_rn(gelu_tanh(yg) * yu);
     } else {
       const int row = row0 + unit;
       if (row >= p.n) continue;
-      float y = 0.f;
-      for (int c = 0; c < S; ++c)
-        y += S > 1 ? ld_dsmem_f32(dsmem_addr(part_s + (uint32_t)(unit * MT8 + tok) * 4u, c))
-                   : part[unit * MT8 + tok];
+      const float y = cluster_sum(unit * MT8 + tok);
       const long long o = tok * p.ld_out + row;
       if (p.epi == SD_EPI_ADD)
         static_cast<float *>(p.out)[o] += y;
@@ -283,20 +354,20 @@ __global__ void __launch_bounds__(kThreads) linear_kernel(const Params p) {
   if (S > 1) cluster_sync();  // no CTA leaves while another still reads its partial
 }
 
-template <int NT>
+template <int NT, bool XF32>
 struct Launcher {
   static size_t smem_bytes(int piece) {
-    return (size_t)std::max(NT * piece * 64 * 8, kWarpsK * kRows * NT * 8 * 4) +
-           (size_t)kRows * NT * 8 * 4;
+    return (size_t)region_a(piece, NT) + (size_t)kRows * NT * 8 * 4;
   }
-  static sd_status launch(const Params &p, int row_blocks, cudaStream_t st) {
+  static sd_status launch(const CUtensorMap &big, const CUtensorMap &small, const Params &p,
+                          int row_blocks, cudaStream_t st) {
     const size_t smem = smem_bytes(p.piece);
     static int configured[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || configured[dev] != dev + 1) {
-      if (cudaFuncSetAttribute(linear_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem_bytes(kStageBytes / (NT * 512))) != cudaSuccess)
+      if (cudaFuncSetAttribute(linear_kernel<NT, XF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem_bytes(kMaxPiece)) != cudaSuccess)
         return SD_ERR_CUDA;
       if (dev < 64) configured[dev] = dev + 1;
     }
@@ -321,7 +392,7 @@ struct Launcher {
     }
     cfg.attrs = a;
     cfg.numAttrs = na;
-    return cuda_status(cudaLaunchKernelEx(&cfg, linear_kernel<NT>, p));
+    return cuda_status(cudaLaunchKernelEx(&cfg, linear_kernel<NT, XF32>, big, small, p));
   }
 };
 
@@ -395,12 +466,28 @@ extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const voi
   p.splits = S;
   const int NT = d->m <= 8 ? 1 : d->m <= 16 ? 2 : d->m <= 32 ? 4 : 8;
   const int per_cta = (chunks + S - 1) / S;
-  p.piece = std::max(1, std::min(per_cta, kStageBytes / (NT * 512)));
+  p.piece = std::max(1, std::min(per_cta, kMaxPiece));
+  // weight boxes: [32 rows x 256 columns] for a full group of 8 chunks, [32 x 32] for one chunk
+  CUtensorMap big, small;
+  const uint32_t box_rows = (uint32_t)std::min(kRows, d->n);
+  if (!encode_tmap_2d_bf16(&big, W, (uint64_t)d->k, (uint64_t)d->n, (uint64_t)d->k * 2,
+                           (uint32_t)std::min(kGroup * 32, d->k), box_rows, false) ||
+      !encode_tmap_2d_bf16(&small, W, (uint64_t)d->k, (uint64_t)d->n, (uint64_t)d->k * 2, 32,
+                           box_rows, false))
+    return SD_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
+  if (p.x_f32) {
+    switch (NT) {
+      case 1: return Launcher<1, true>::launch(big, small, p, row_blocks, st);
+      case 2: return Launcher<2, true>::launch(big, small, p, row_blocks, st);
+      case 4: return Launcher<4, true>::launch(big, small, p, row_blocks, st);
+      default: return Launcher<8, true>::launch(big, small, p, row_blocks, st);
+    }
+  }
   switch (NT) {
-    case 1: return Launcher<1>::launch(p, row_blocks, st);
-    case 2: return Launcher<2>::launch(p, row_blocks, st);
-    case 4: return Launcher<4>::launch(p, row_blocks, st);
-    default: return Launcher<8>::launch(p, row_blocks, st);
+    case 1: return Launcher<1, false>::launch(big, small, p, row_blocks, st);
+    case 2: return Launcher<2, false>::launch(big, small, p, row_blocks, st);
+    case 4: return Launcher<4, false>::launch(big, small, p, row_blocks, st);
+    default: return Launcher<8, false>::launch(big, small, p, row_blocks, st);
   }
 }
