@@ -13,9 +13,10 @@ Modules
   accept     lossless acceptance, correction and bonus draws (T > 0) and greedy (T = 0)
   commit     committed length, committed slots, rollback and next hidden row
   drafter    the drafter's dense layers around its cross-attention (one link of the chain)
+  target     the target's layers over the k+1 verified positions (multi-layer verify)
 
 Parity status: every function is pinned by tests/test_oracle_*.py against closed forms,
 invariants, library routines, brute-force enumeration or published known answers, except
 agreement with real Gemma 4 / vLLM / FlashInfer outputs (no weights or traces exist here).
 """
-from . import accept, attention, commit, drafter, lm_head, philox  # noqa: F401
+from . import accept, attention, commit, drafter, lm_head, philox, target  # noqa: F401
