@@ -298,3 +298,25 @@ def make_drafter_weights(seed: int, d: int, d_target: int, vocab: int, h_q: int,
         })
     return out
 
+
+
+def make_target_weights(seed: int, d: int, ff: int, h_q: int, h_kv: int, layers):
+    """Synthetic target layers (CPU tensors) for the multi-layer verify: per layer (head_dim D,
+    window W) RMSNorm gains (float32, 1 + N(0, 0.1^2)) and bf16 projections Wq [h_q D, d],
+    Wk, Wv [h_kv D, d], Wo [d, h_q D], Wg, Wu [ff, d], Wd [d, ff], each ~ N(0, 1/fan_in)."""
+    out = []
+    for i, (D, W) in enumerate(layers):
+        t = 70000 + 1000 * int(seed) + 10 * i
+        out.append({
+            "head_dim": int(D), "window": int(W),
+            "g_attn": torch.from_numpy(1 + normal(t, (d,), 0.1)),
+            "Wq": bf16(normal(t + 1, (h_q * D, d), 1 / math.sqrt(d))),
+            "Wk": bf16(normal(t + 2, (h_kv * D, d), 1 / math.sqrt(d))),
+            "Wv": bf16(normal(t + 3, (h_kv * D, d), 1 / math.sqrt(d))),
+            "Wo": bf16(normal(t + 4, (d, h_q * D), 1 / math.sqrt(h_q * D))),
+            "g_mlp": torch.from_numpy(1 + normal(t + 5, (d,), 0.1)),
+            "Wg": bf16(normal(t + 6, (ff, d), 1 / math.sqrt(d))),
+            "Wu": bf16(normal(t + 7, (ff, d), 1 / math.sqrt(d))),
+            "Wd": bf16(normal(t + 8, (d, ff), 1 / math.sqrt(ff))),
+        })
+    return out

@@ -40,6 +40,9 @@ LINEAR_CASES = [
     (24, 1024, 8192, "bf16", False, "add", "f32", 0),     # three token groups
     (64, 2048, 6400, "f32", True, "store", "bf16", 0),    # 64 rows: several staged pieces
     (33, 160, 2048, "bf16", False, "store", "f32", 2048),  # every column gathered
+    (12, 1024, 2048, "f32", True, "store", "bf16", 0),    # two token groups (B 4, k 2)
+    (16, 512, 4096, "bf16", False, "add", "f32", 0),      # two full token groups
+    (24, 2048, 1024, "f32", True, "geglu", "bf16", 0),    # three groups, gated (B 8, k 2)
 ]
 
 
