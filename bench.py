@@ -41,8 +41,9 @@ sys.path.insert(0, ROOT)
 WORKLOAD = "spec_step_b8_ctx16384_k2"  # the default configuration
 
 
-def workload_name(batch, ctx, k, drafter_layers=False):
-    return f"spec_step_b{batch}_ctx{ctx}_k{k}" + ("_drafter_layers" if drafter_layers else "")
+def workload_name(batch, ctx, k, drafter_layers=False, target_layers=False):
+    return (f"spec_step_b{batch}_ctx{ctx}_k{k}" + ("_drafter_layers" if drafter_layers else "") +
+            ("_target_layers" if target_layers else ""))
 METRIC = "verified tokens/s per verify step (B,k,ctx); HBM GB/s as % of B200 peak"
 UNIT = "verified tokens/s"
 
@@ -62,6 +63,10 @@ def parse():
                     help="run the drafter's dense layers (input projection, 4 x (W_q, W_o, "
                          "gated MLP, W_d), output projection) around its cross-attention, so "
                          "the chain is driven by the committed hidden row and tokens")
+    ap.add_argument("--target-layers", action="store_true",
+                    help="verify through two target layers with their own projections (a "
+                         "sliding and a global layer: q/k/v/o and a gated MLP 21504 wide at "
+                         "d 5376) instead of the two attention calls on given q, k, v")
     return ap.parse_args()
 
 
@@ -70,7 +75,7 @@ GROUP_SOURCE = {"head_dense": "lm_head.cu", "head_clustered": "lm_head.cu",
                 "verify_global": "attention.cu", "verify_sliding": "attention.cu",
                 "xattn_global": "attention.cu", "xattn_sliding": "attention.cu",
                 "accept": "accept.cu", "accept_draft": "accept.cu", "commit": "commit.cu",
-                "drafter_dense": "linear.cu"}
+                "drafter_dense": "linear.cu", "target_dense": "linear.cu"}
 
 
 def source_hash(name):
@@ -133,7 +138,8 @@ def peaks():
 class SpecStep:
     """Device buffers, descriptors and the call sequence of one speculative step."""
 
-    def __init__(self, k=2, B=8, L=16384, reserve=600, rank=0, dev="cuda", dense=False):
+    def __init__(self, k=2, B=8, L=16384, reserve=600, rank=0, dev="cuda", dense=False,
+                 target=False):
         import numpy as np
         import torch
 
@@ -143,6 +149,7 @@ class SpecStep:
         self.k, self.B, self.n_q = k, B, k + 1
         self.dev = dev
         self.dense = dense
+        self.target = target
         self.hq, self.hkv, self.bs = 16, 4, 16
         self.V, self.d, self.dh = 262144, 5376, 1024
         self.C, self.cs, self.top_c = 1024, 256, 32
@@ -166,9 +173,12 @@ class SpecStep:
         self.ctx0 = self.ctx.clone()
         # per-step inputs (reused every step; copied from pinned host memory in the e2e leg)
         inp = {}
-        for layer in (0, 1):
+        for layer in ((0, 1) if not target else ()):
             s = S.make_step_qkv(wg, layer, self.n_q)
             inp[f"q{layer}"], inp[f"kn{layer}"], inp[f"vn{layer}"] = s["q"], s["k_new"], s["v_new"]
+        if target:
+            # input rows of the k+1 positions (the residual stream entering the first layer)
+            inp["x0"] = torch.from_numpy(S.normal(seed * 41 + 5, (B * self.n_q, self.d)))
         inp["hidden"] = S.make_hidden(wg, B * self.n_q)
         for j in range(0 if dense else k):
             for layer, D in ((0, 512), (1, 256)):
@@ -233,6 +243,16 @@ class SpecStep:
             self.dwts = VD.device_weights(S.make_drafter_weights(
                 seed, self.dh, self.d, self.V, self.hq, self.dshape.head_dims), dev)
             self.dbuf = VD.buffers(self.dshape, dev)
+        if target:
+            # two target layers over the bench's caches: the sliding one, then the global one
+            from verify_step_b200 import target as VT
+            self.VT = VT
+            self.tshape = VT.TargetShape(batch=B, n_q=self.n_q, d=self.d, ff=4 * self.d,
+                                         h_q=self.hq, h_kv=self.hkv,
+                                         layers=((256, 512), (512, 0)))
+            self.twts = VT.device_weights(S.make_target_weights(
+                seed, self.d, 4 * self.d, self.hq, self.hkv, self.tshape.layers), dev)
+            self.tbuf = VT.buffers(self.tshape, dev)
         # descriptors
         self.vdesc = [self._adesc(0, self.n_q), self._adesc(1, self.n_q)]
         self.xdesc = [[self._adesc(layer, 1, q_offset=j) for layer in (0, 1)] for j in range(k)]
@@ -276,13 +296,14 @@ class SpecStep:
     # counted directly where the CUDA runtime allows; this is the fallback)
     LAUNCHES = dict(xattn_sliding=1, xattn_global=2, verify_sliding=1, verify_global=3,
                     head_dense=1, head_clustered=3, accept_draft=1, accept=2, commit=1,
-                    drafter_dense=1)
+                    drafter_dense=1, target_dense=1)
 
     def launches_per_step(self):
         L = self.LAUNCHES
         dense = self.VD.LAUNCHES_PER_LINK * L["drafter_dense"] if self.dense else 0
         return (self.k * (3 * L["xattn_sliding"] + L["xattn_global"] + L["head_clustered"] +
                           L["accept_draft"] + dense) +
+                (2 * self.VT.LINEAR_CALLS_PER_LAYER * L["target_dense"] if self.target else 0) +
                 L["verify_global"] + L["verify_sliding"] + L["head_dense"] + L["accept"] +
                 L["commit"])
 
@@ -325,12 +346,15 @@ class SpecStep:
                 self._col_ptr(self.drafts, j), None, self.ws))
         if before_phase is not None:
             before_phase(self.k)
-        timed("verify_global", lambda: sd.sd_verify_attn(
-            self.vdesc[0], I["q0"], I["kn0"], I["vn0"], c0["k"], c0["v"], c0["table"], self.ctx,
-            self.attn_out[0], self.ws))
-        timed("verify_sliding", lambda: sd.sd_verify_attn(
-            self.vdesc[1], I["q1"], I["kn1"], I["vn1"], c1["k"], c1["v"], c1["table"], self.ctx,
-            self.attn_out[1], self.ws))
+        if self.target:
+            self._target_layers(timed)
+        else:
+            timed("verify_global", lambda: sd.sd_verify_attn(
+                self.vdesc[0], I["q0"], I["kn0"], I["vn0"], c0["k"], c0["v"], c0["table"],
+                self.ctx, self.attn_out[0], self.ws))
+            timed("verify_sliding", lambda: sd.sd_verify_attn(
+                self.vdesc[1], I["q1"], I["kn1"], I["vn1"], c1["k"], c1["v"], c1["table"],
+                self.ctx, self.attn_out[1], self.ws))
         timed("head_dense", lambda: sd.sd_lm_head(self.hdesc_dense, I["hidden"], self.W,
                                                   self.target_logits))
         timed("accept", lambda: sd.sd_accept(self.adesc, self.target_logits, self.draft_logits,
@@ -359,6 +383,19 @@ class SpecStep:
                 self.k, None
         self.VD.link(self.dshape, self.dwts, self.dbuf, h_prev, toks, ld, attend,
                      token_sel=sel, wrap=lambda fn: timed("drafter_dense", fn))
+
+    def _target_layers(self, timed):
+        c0, c1 = self.cache
+        caches = [dict(desc=self.vdesc[1], k=c1["k"], v=c1["v"], table=c1["table"]),
+                  dict(desc=self.vdesc[0], k=c0["k"], v=c0["v"], table=c0["table"])]
+        self.tbuf["x"].copy_(self.inputs["x0"])
+        names = iter(["verify_sliding", "verify_global"])
+
+        def wrap(kind, fn):
+            timed(next(names) if kind == "attn" else "target_dense", fn)
+
+        self.VT.verify_layers(self.tshape, self.twts, self.tbuf, caches, self.ctx, self.ws,
+                              wrap=wrap)
 
     def _row_ptr(self, t, j):
         return t.data_ptr() + j * self.V * t.element_size()
@@ -403,7 +440,24 @@ class SpecStep:
         if self.dense:
             out["drafter_dense"] = int(self.VD.hbm_bytes_per_link(self.dshape) /
                                        self.VD.LAUNCHES_PER_LINK)
+        if self.target:
+            out["target_dense"] = int(self._target_dense_bytes() /
+                                      (2 * self.VT.LINEAR_CALLS_PER_LAYER))
         return out
+
+    def _target_dense_bytes(self):
+        """Algorithmic HBM bytes of the target layers' projections per step: every weight
+        once, the input rows read and the outputs written (the residual read and written)."""
+        t = self.tshape
+        m, d, F = t.batch * t.n_q, t.d, t.ff
+        total = 0
+        for D, _ in t.layers:
+            nq, nkv = t.h_q * D, t.h_kv * D
+            total += (nq + 2 * nkv) * d * 2 + 3 * m * d * 4 + m * (nq + 2 * nkv) * 2
+            total += d * nq * 2 + m * nq * 2 + 2 * m * d * 4
+            total += 2 * F * d * 2 + m * d * 4 + m * F * 2
+            total += d * F * 2 + m * F * 2 + 2 * m * d * 4
+        return total
 
     def calls_per_step(self):
         out = dict(xattn_sliding=3 * self.k, xattn_global=self.k, head_clustered=self.k,
@@ -411,6 +465,8 @@ class SpecStep:
                    accept=1, commit=1)
         if self.dense:
             out["drafter_dense"] = self.VD.LAUNCHES_PER_LINK * self.k
+        if self.target:
+            out["target_dense"] = 2 * self.VT.LINEAR_CALLS_PER_LAYER
         return out
 
     def reset(self):
@@ -669,8 +725,8 @@ def main():
     # every pass below runs a.steps steps (warm-up, timed, per-kernel, e2e): reserve the blocks
     reserve = (a.warmup + 4 * a.steps + 8) * (a.k + 1) + 64
     st = SpecStep(k=a.k, B=a.batch, L=a.ctx, reserve=reserve, rank=rank,
-                  dense=a.drafter_layers)
-    wname = workload_name(st.B, a.ctx, st.k, a.drafter_layers)
+                  dense=a.drafter_layers, target=a.target_layers)
+    wname = workload_name(st.B, a.ctx, st.k, a.drafter_layers, a.target_layers)
     L_start = st.L0.copy()
     clock = ClockSampler(local)
     for _ in range(a.warmup):
@@ -777,7 +833,8 @@ def main():
     del graph, graph_ev, graph_e2e
 
     cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.drafter_layers:
+    if (rank == 0 and world == 1 and not a.no_cpu_baseline and not a.drafter_layers and
+            not a.target_layers):
         t = time.perf_counter()
         nv = oracle_sample(st, [0], 0)
         dt = time.perf_counter() - t
@@ -808,7 +865,12 @@ def main():
                    **({"drafter_layers": "per link: W_in [1024 x (5376+1024)] on the committed "
                        "hidden row and the embedding of the last token, 4 x (RMSNorm, W_q, "
                        "cross-attention, W_o, RMSNorm, gated GELU MLP 4096, W_d), RMSNorm, "
-                       "W_back [5376 x 1024]; synthetic weights"} if a.drafter_layers else {})},
+                       "W_back [5376 x 1024]; synthetic weights"} if a.drafter_layers else {}),
+                   **({"target_layers": "verify through 2 target layers (sliding D256 W512, "
+                       "then global D512), each RMSNorm, W_q/W_k/W_v, verify attention, W_o, "
+                       "RMSNorm, gated GELU MLP 21504, W_d at d 5376; synthetic weights; the "
+                       "dense head still reads the given hidden rows"} if a.target_layers
+                      else {})},
         "gpu_launches": kernels_per_step * a.steps,
         "roofline": roof(dom),
         "roofline_attention": roof("verify_global"),
