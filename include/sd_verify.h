@@ -5,8 +5,8 @@
  * scores the k drafts plus one more position (k+1 positions) in one forward pass, accepts a
  * prefix of the drafts and emits one token of its own ("Gemma 4 MTP: drafter drafts, target
  * verifies", sections "basic structure of speculative decoding" and "drafter internal
- * architecture"; Gemma 4 MTP serving guide, section 4 "execution flow").  The five calls
- * below are the data-parallel parts of that step:
+ * architecture"; Gemma 4 MTP serving guide, section 4 "execution flow").  The calls below
+ * are the data-parallel parts of that step:
  *
  *   sd_verify_attn   k+1 causal queries per sequence over a paged bf16 KV cache (GQA,
  *                    sliding or global layer), appending the k+1 new K/V rows
@@ -14,6 +14,9 @@
  *   sd_lm_head       logits over the vocabulary, dense or two-stage clustered
  *   sd_accept        lossless acceptance, correction / bonus draw (or greedy at T = 0)
  *   sd_commit        committed length, committed slots, rollback, next hidden row
+ *   sd_linear        one dense projection of a few token rows with a normalising / gathering
+ *                    prologue and a store, residual-add or gated-GELU epilogue (the drafter's
+ *                    and the target's layers around their attention)
  *
  * Conventions shared by every call
  *   - Every data pointer is a caller-owned DEVICE buffer, densely packed in the layout
