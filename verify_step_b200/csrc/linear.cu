@@ -1,10 +1,11 @@
-// Drafter dense layers: one projection of a few token rows against a bf16 weight matrix, with
-// an RMSNorm / embedding-gather prologue and a store, residual-add or gated-GELU epilogue
-// (sm_100a).
+// Dense layers of the drafter and of the target: one projection of a few token rows against a
+// bf16 weight matrix, with an RMSNorm / embedding-gather prologue and a store, residual-add or
+// gated-GELU epilogue (sm_100a).
 //
 // "Gemma 4 MTP: drafter drafts, target verifies", section "drafter internal architecture": the
 // drafter runs 4 transformer layers on the target's last-layer activation and its own token
-// embedding.  With B = 8 token rows a projection is a matrix-vector product in all but name:
+// embedding, and the target runs its layers over the k+1 verified positions.  With B = 8 token
+// rows a projection is a matrix-vector product in all but name:
 // 8 FLOPs per weight byte, so the weights' single pass through HBM bounds it.  The kernel
 // streams each CTA's W rows into shared memory with a few large TMA tensor copies (completing on
 // mbarriers), feeds mma.sync from there and keeps the few token rows in
