@@ -638,7 +638,11 @@ def oracle_sample(step_obj, seqs, s):
                         else i for i in idx)
             return self.t[idx].to(torch.float64).numpy()
 
+    from oracle import drafter as OD
+    from oracle import target as OT
+
     st = step_obj
+    dense, target = getattr(st, "dense", False), getattr(st, "target", False)
     if st.host.get("W") is None:
         st.host["W"] = S.make_lm_head(st.w)
     k, n_q, B = st.k, st.n_q, st.B
@@ -651,30 +655,50 @@ def oracle_sample(step_obj, seqs, s):
     m = len(seqs)
     drafts = np.zeros((m, k), np.int64)
     draft_logits = np.zeros((m, k, st.V))
+    ocache = {D: dict(k=F64(c["k_cache"]), v=F64(c["v_cache"]), table=c["table"].numpy()[seqs],
+                      block_size=st.bs) for D, c in ((512, c0), (256, c1))}
+    if dense:
+        h_prev = f(st.host["h0"])[seqs]
+        tokens = np.zeros(m, np.int64)
     for j in range(k):
-        for layer, cache, D, W, n in ((1, c1, 256, 512, 3), (0, c0, 512, 0, 1)):
-            q = f(hi[f"dq{j}_{layer}"])
-            for r in range(n):
-                for b in seqs:
-                    for h in range(st.hq):
-                        OA.draft_attention_one(b, h, q[r], F64(cache["k_cache"]),
-                                               F64(cache["v_cache"]), cache["table"].numpy(), L,
-                                               L + j, W, 1 / math.sqrt(D), st.bs)
-        lg, _, _ = OH.clustered_lm_head(f(hi[f"dh{j}"])[seqs], f(cl["centroids"]),
+        if dense:
+            # the drafter's dense layers around its four cross-attentions (sequences seqs)
+            atts = [OD.cross_attend(ocache[D], st.hq, D, 512 if D == 256 else 0, L[seqs], j)
+                    for D in (256, 256, 256, 512)]
+            link = OD.drafter_step(h_prev, tokens, st.host["drafter"], atts)
+            hj, h_prev = link["h"], link["h_back"]
+        else:
+            for layer, cache, D, W, n in ((1, c1, 256, 512, 3), (0, c0, 512, 0, 1)):
+                q = f(hi[f"dq{j}_{layer}"])
+                for r in range(n):
+                    for b in seqs:
+                        for h in range(st.hq):
+                            OA.draft_attention_one(b, h, q[r], F64(cache["k_cache"]),
+                                                   F64(cache["v_cache"]),
+                                                   cache["table"].numpy(), L, L + j, W,
+                                                   1 / math.sqrt(D), st.bs)
+            hj = f(hi[f"dh{j}"])[seqs]
+        lg, _, _ = OH.clustered_lm_head(hj, f(cl["centroids"]),
                                         F64(cl["w_cm"]), cl["cluster_tokens"].numpy(), st.top_c)
         draft_logits[:, j] = lg
         r = OACC.accept(lg[:, None, :], None, np.zeros((m, 0)), 1.0, seed=7,
                         step=((j + 1) << 28) + s, purpose=OACC.PURPOSE_DRAFTER)
         drafts[:, j] = r["out_tokens"][:, 0]
-    for layer, cache, D, W in ((0, c0, 512, 0), (1, c1, 256, 512)):
-        q, kn, vn = f(hi[f"q{layer}"]), f(hi[f"kn{layer}"]), f(hi[f"vn{layer}"])
-        for b in seqs:
-            for j in range(n_q):
-                for h in range(st.hq):
-                    OA.verify_attention_one(b, j, h, q, kn, vn, F64(cache["k_cache"]),
-                                            F64(cache["v_cache"]), cache["table"].numpy(), L, W,
-                                            1 / math.sqrt(D), st.bs)
+        tokens = drafts[:, j]
     rows = np.concatenate([np.arange(b * n_q, (b + 1) * n_q) for b in seqs])
+    if target:
+        # the target's two layers with their own projections (sliding, then global)
+        OT.verify_layers(f(hi["x0"])[rows], st.host["target"], [ocache[256], ocache[512]],
+                         L[seqs], n_q, st.hq, st.hkv)
+    else:
+        for layer, cache, D, W in ((0, c0, 512, 0), (1, c1, 256, 512)):
+            q, kn, vn = f(hi[f"q{layer}"]), f(hi[f"kn{layer}"]), f(hi[f"vn{layer}"])
+            for b in seqs:
+                for j in range(n_q):
+                    for h in range(st.hq):
+                        OA.verify_attention_one(b, j, h, q, kn, vn, F64(cache["k_cache"]),
+                                                F64(cache["v_cache"]), cache["table"].numpy(),
+                                                L, W, 1 / math.sqrt(D), st.bs)
     h = f(hi["hidden"])[rows]
     Wv = F64(st.host["W"])
     z = np.empty((len(rows), st.V))
@@ -893,7 +917,7 @@ def run_reference(a, rank, world):
         return
     import torch  # noqa: F401
     os.environ.setdefault("CUDA_VISIBLE_DEVICES", "")
-    st = HostOnlyStep(a.k, a.batch, a.ctx)
+    st = HostOnlyStep(a.k, a.batch, a.ctx, dense=a.drafter_layers, target=a.target_layers)
     for s in range(a.warmup):
         oracle_sample(st, [s % st.B], s)
     t = time.perf_counter()
@@ -906,7 +930,8 @@ def run_reference(a, rank, world):
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(dt / a.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": workload_name(a.batch, a.ctx, a.k), "batch": a.batch,
+            "config": {"workload": workload_name(a.batch, a.ctx, a.k, a.drafter_layers,
+                                                 a.target_layers), "batch": a.batch,
                        "ctx": a.ctx, "k": a.k},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": blas_threads(),
                              "kind": "oracle",
@@ -920,10 +945,11 @@ def run_reference(a, rank, world):
 class HostOnlyStep:
     """The workload's host tensors only (for the CPU oracle arm)."""
 
-    def __init__(self, k, B, L, reserve=64):
-        import numpy as np  # noqa: F401
+    def __init__(self, k, B, L, reserve=64, dense=False, target=False):
+        import torch
 
         import synthetic as S
+        self.dense, self.target = dense, target
         self.k, self.B, self.n_q = k, B, k + 1
         self.hq, self.hkv, self.bs = 16, 4, 16
         self.V, self.d, self.dh = 262144, 5376, 1024
@@ -950,6 +976,21 @@ class HostOnlyStep:
         self.host_inputs = inp
         self.host["cl"] = S.make_clustered_head(self.w)
         self.host["W"] = None
+        f32 = lambda t: t.float().numpy()  # bf16 -> float32 is exact
+        if dense:
+            dw = S.make_drafter_weights(seed, self.dh, self.d, self.V, self.hq,
+                                        (256, 256, 256, 512))
+            self.host["drafter"] = {
+                "E": f32(dw["E"]), "W_in": f32(dw["W_in"]), "g_final": f32(dw["g_final"]),
+                "W_back": f32(dw["W_back"]),
+                "layers": [{kk: f32(v) for kk, v in lw.items()} for lw in dw["layers"]]}
+            self.host["h0"] = S.make_hidden(self.w, B, step=97)
+        if target:
+            tw = S.make_target_weights(seed, self.d, 4 * self.d, self.hq, self.hkv,
+                                       ((256, 512), (512, 0)))
+            self.host["target"] = [{kk: (f32(v) if hasattr(v, "float") else v)
+                                    for kk, v in lw.items()} for lw in tw]
+            inp["x0"] = torch.from_numpy(S.normal(seed * 41 + 5, (B * self.n_q, self.d)))
 
 
 if __name__ == "__main__":

@@ -66,3 +66,21 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
         sys.argv = saved
     assert bench.run_reference(args, 1, 2) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_covers_the_drafter_layer_mode(capsys):
+    """The oracle arm of the drafter-layer workload: one step of one sequence through the
+    drafter's dense layers, printed as one JSON line naming that workload."""
+    import json
+    import sys
+    saved = sys.argv
+    sys.argv = ["bench.py", "--impl", "reference", "--drafter-layers", "--steps", "1",
+                "--warmup", "0"]
+    try:
+        args = bench.parse()
+    finally:
+        sys.argv = saved
+    bench.run_reference(args, 0, 1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"]["workload"] == "spec_step_b8_ctx16384_k2_drafter_layers"
