@@ -75,7 +75,8 @@ def buffers(shape: DrafterShape, dev="cuda"):
             "h_back": torch.empty((B, shape.d_target), dtype=bf, device=dev)}
 
 
-def _desc(m, n, k, x_dtype, ld_x, epilogue, out_dtype, ld_out, **kw):
+def linear_desc(m, n, k, x_dtype, ld_x, epilogue, out_dtype, ld_out, **kw):
+    """An sd_linear descriptor with the RMSNorm epsilon of these layers."""
     return LinearDesc(m=m, n=n, k=k, x_dtype=x_dtype, ld_x=ld_x, epilogue=epilogue,
                       out_dtype=out_dtype, ld_out=ld_out, norm_eps=RMS_EPS, **kw)
 
@@ -92,28 +93,29 @@ def link(shape: DrafterShape, wts, buf, h_prev, tokens, ld_tokens, attend, token
     B, d, dt, F = shape.batch, shape.d, shape.d_target, shape.ff
     x = buf["x"]
     call = wrap if wrap is not None else (lambda fn: fn())
+    desc = linear_desc
     call(lambda: sd_linear(
-        _desc(B, d, dt + d, SD_BF16, dt, SD_EPI_STORE, SD_F32, d, k_gather=d, ld_table=d,
-              table_rows=shape.vocab, ld_tokens=ld_tokens),
+        desc(B, d, dt + d, SD_BF16, dt, SD_EPI_STORE, SD_F32, d, k_gather=d, ld_table=d,
+             table_rows=shape.vocab, ld_tokens=ld_tokens),
         h_prev, wts["W_in"], x, table=wts["E"], tokens=tokens, token_sel=token_sel,
         stream=stream))
     for i, (L, D) in enumerate(zip(wts["layers"], shape.head_dims)):
         n = shape.h_q * D
         q, o = buf["q"][i], buf["o"][i]
-        call(lambda: sd_linear(_desc(B, n, d, SD_F32, d, SD_EPI_STORE, SD_BF16, n,
-                                     norm_gain=L["g_attn"].data_ptr()),
+        call(lambda: sd_linear(desc(B, n, d, SD_F32, d, SD_EPI_STORE, SD_BF16, n,
+                                    norm_gain=L["g_attn"].data_ptr()),
                                x, L["Wq"], q, stream=stream))
         attend(i, q, o)
-        call(lambda: sd_linear(_desc(B, d, n, SD_BF16, n, SD_EPI_ADD, SD_F32, d), o, L["Wo"], x,
+        call(lambda: sd_linear(desc(B, d, n, SD_BF16, n, SD_EPI_ADD, SD_F32, d), o, L["Wo"], x,
                                stream=stream))
-        call(lambda: sd_linear(_desc(B, 2 * F, d, SD_F32, d, SD_EPI_GEGLU, SD_BF16, F,
-                                     norm_gain=L["g_mlp"].data_ptr()),
+        call(lambda: sd_linear(desc(B, 2 * F, d, SD_F32, d, SD_EPI_GEGLU, SD_BF16, F,
+                                    norm_gain=L["g_mlp"].data_ptr()),
                                x, L["Wgu"], buf["u"], stream=stream))
-        call(lambda: sd_linear(_desc(B, d, F, SD_BF16, F, SD_EPI_ADD, SD_F32, d), buf["u"],
+        call(lambda: sd_linear(desc(B, d, F, SD_BF16, F, SD_EPI_ADD, SD_F32, d), buf["u"],
                                L["Wd"], x, stream=stream))
-    call(lambda: sd_linear(_desc(B, dt, d, SD_F32, d, SD_EPI_STORE, SD_BF16, dt,
-                                 norm_gain=wts["g_final"].data_ptr(),
-                                 norm_out=buf["h"].data_ptr(), ld_norm_out=d),
+    call(lambda: sd_linear(desc(B, dt, d, SD_F32, d, SD_EPI_STORE, SD_BF16, dt,
+                                norm_gain=wts["g_final"].data_ptr(),
+                                norm_out=buf["h"].data_ptr(), ld_norm_out=d),
                            x, wts["W_back"], buf["h_back"], stream=stream))
 
 

@@ -18,9 +18,9 @@ from __future__ import annotations
 
 from dataclasses import dataclass
 
-from . import (SD_BF16, SD_EPI_ADD, SD_EPI_GEGLU, SD_EPI_STORE, SD_F32, LinearDesc,
-               sd_linear, sd_verify_attn)
-from .drafter import RMS_EPS, gate_up_blocks
+from . import (SD_BF16, SD_EPI_ADD, SD_EPI_GEGLU, SD_EPI_STORE, SD_F32, sd_linear,
+               sd_verify_attn)
+from .drafter import gate_up_blocks, linear_desc
 
 
 @dataclass
@@ -57,11 +57,6 @@ def buffers(shape: TargetShape, dev="cuda"):
             "u": mk(shape.ff)}
 
 
-def _desc(m, n, k, x_dtype, ld_x, epilogue, out_dtype, ld_out, **kw):
-    return LinearDesc(m=m, n=n, k=k, x_dtype=x_dtype, ld_x=ld_x, epilogue=epilogue,
-                      out_dtype=out_dtype, ld_out=ld_out, norm_eps=RMS_EPS, **kw)
-
-
 def verify_layers(shape: TargetShape, wts, buf, caches, ctx_len, ws, stream=None, wrap=None):
     """Run every layer on buf["x"] (the caller fills it with the k+1 positions' input rows).
 
@@ -71,23 +66,24 @@ def verify_layers(shape: TargetShape, wts, buf, caches, ctx_len, ws, stream=None
     m, d, F = shape.batch * shape.n_q, shape.d, shape.ff
     x = buf["x"]
     call = wrap if wrap is not None else (lambda kind, fn: fn())
+    desc = linear_desc
     for i, (L, (D, _W)) in enumerate(zip(wts, shape.layers)):
         nq, nkv = shape.h_q * D, shape.h_kv * D
         q, kn, vn, o = buf["q"][i], buf["k"][i], buf["v"][i], buf["o"][i]
         gain = L["g_attn"].data_ptr()
         for W, out, n in ((L["Wq"], q, nq), (L["Wk"], kn, nkv), (L["Wv"], vn, nkv)):
             call("linear", lambda: sd_linear(
-                _desc(m, n, d, SD_F32, d, SD_EPI_STORE, SD_BF16, n, norm_gain=gain), x, W, out,
+                desc(m, n, d, SD_F32, d, SD_EPI_STORE, SD_BF16, n, norm_gain=gain), x, W, out,
                 stream=stream))
         c = caches[i]
         call("attn", lambda: sd_verify_attn(c["desc"], q, kn, vn, c["k"], c["v"], c["table"],
                                             ctx_len, o, ws, stream=stream))
-        call("linear", lambda: sd_linear(_desc(m, d, nq, SD_BF16, nq, SD_EPI_ADD, SD_F32, d),
+        call("linear", lambda: sd_linear(desc(m, d, nq, SD_BF16, nq, SD_EPI_ADD, SD_F32, d),
                                          o, L["Wo"], x, stream=stream))
         call("linear", lambda: sd_linear(
-            _desc(m, 2 * F, d, SD_F32, d, SD_EPI_GEGLU, SD_BF16, F,
-                  norm_gain=L["g_mlp"].data_ptr()), x, L["Wgu"], buf["u"], stream=stream))
-        call("linear", lambda: sd_linear(_desc(m, d, F, SD_BF16, F, SD_EPI_ADD, SD_F32, d),
+            desc(m, 2 * F, d, SD_F32, d, SD_EPI_GEGLU, SD_BF16, F,
+                 norm_gain=L["g_mlp"].data_ptr()), x, L["Wgu"], buf["u"], stream=stream))
+        call("linear", lambda: sd_linear(desc(m, d, F, SD_BF16, F, SD_EPI_ADD, SD_F32, d),
                                          buf["u"], L["Wd"], x, stream=stream))
 
 
