@@ -139,9 +139,12 @@ def accept(z, y, drafts, temperature: float, seed: int, step: int,
         Vu = token_uniform_rows(seed, step, rows + n_acc, purpose, V)
         x, g = race(w, Vu)
         lnE = np.log(-np.log1p(-Vu))
-        with np.errstate(divide="ignore"):
-            g_hi = np.log(w_hi) - lnE + key_err
-            g_lo = np.log(w_lo) - lnE - key_err
+        # a token of weight exactly 0 (a -inf logit, or an empty residual entry) cannot win
+        # on either side: its key bound is -inf (its key error term may be infinite there,
+        # and -inf + inf would be NaN and hide the row's other competitors from the check)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            g_hi = np.where(w_hi > 0, np.log(w_hi) - lnE + key_err, -np.inf)
+            g_lo = np.where(w_lo > 0, np.log(w_lo) - lnE - key_err, -np.inf)
         margin |= _race_margin(g_lo, g_hi, x)
 
     out = np.full((B, n_q), -1, np.int64)
