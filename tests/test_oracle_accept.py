@@ -207,3 +207,23 @@ def test_race_picks_unique_positive_weight_and_prefers_lower_id_on_ties():
     V = np.array([[0.5, 0.5, 0.9, 0.1], [0.25, 0.25, 0.1, 0.1]])
     x, g = ACC.race(w, V)
     assert x.tolist() == [2, 0]
+
+
+def test_masked_tokens_do_not_hide_a_near_tie():
+    """A plain draw over a row whose other tokens are masked (-inf logits), with the two live
+    tokens' logits set so that their race keys differ by 1e-5 (flagged) or by 2 (not
+    flagged).  Zero-weight tokens have key -inf; an infinite key error on them must not turn
+    the row's competitor bound into NaN."""
+    from oracle.philox import token_uniform_rows
+    V, seed, step = 16, 5, 9
+    live = (3, 11)
+    u = token_uniform_rows(seed, step, [0], ACC.PURPOSE_DRAFTER, V)[0]
+    lnE = np.log(-np.log1p(-u))
+    for gap, want in ((1e-5, True), (2.0, False)):
+        z = np.full((1, 1, V), -np.inf)
+        z[0, 0, live[0]] = 0.3
+        z[0, 0, live[1]] = 0.3 + (lnE[live[1]] - lnE[live[0]]) + gap  # key difference = gap
+        r = ACC.accept(z, None, np.zeros((1, 0), np.int64), 1.0, seed=seed, step=step,
+                       purpose=ACC.PURPOSE_DRAFTER)
+        assert bool(r["margin"][0]) is want, gap
+        assert r["out_tokens"][0, 0] == live[1]
