@@ -227,3 +227,67 @@ def test_masked_tokens_do_not_hide_a_near_tie():
                        purpose=ACC.PURPOSE_DRAFTER)
         assert bool(r["margin"][0]) is want, gap
         assert r["out_tokens"][0, 0] == live[1]
+
+
+def _ratio_row(r, V=4):
+    """log p for a row with p(0) = r * q(0) under a uniform q over V tokens: token 0 gets r / V,
+    token 1 almost all the rest, the others a negligible 1e-12 each (so a residual draw after
+    a rejection at token 0 has a single token of clearly positive weight)."""
+    p = np.full(V, 1e-12)
+    p[0] = r / V
+    p[1] = 1.0 - p[0] - (V - 2) * 1e-12
+    return np.log(p)
+
+
+def test_acceptance_margin_is_the_absolute_gap_between_u_and_the_ratio():
+    """The spec margin: a decision with |u - p(d)/q(d)| < 1e-4 is flagged, one 2e-4 away
+    is not, on either side of u; the gap is absolute (a sequence whose u is small has a
+    relative gap far above 1e-4 but is still flagged); u is the uniform of the decision's own
+    row b * (k + 1) + i - 1, so a near-tie built on that row's u is seen only by that row."""
+    from oracle.philox import accept_uniform
+    seed, step, V, B = 13, 4, 4, 64
+    u = accept_uniform(seed, step, np.arange(B) * 2)
+    small = int(np.argmin(u))
+    assert u[small] < 0.05
+    cases = {small: (5e-5, True)}
+    others = [b for b in range(B) if b != small and 0.05 < u[b] < 0.95][:4]
+    for b, delta in zip(others, (5e-5, -5e-5, 2e-4, -2e-4)):
+        cases[b] = (delta, abs(delta) < 1e-4)
+    bs = sorted(cases)
+    z = np.empty((B, 2, V))
+    z[:, 0] = _ratio_row(2.0)       # sequences not under test: ratio 2, always accepted
+    z[:, 1] = [0.0, -50.0, -50.0, -50.0]   # bonus row: one token dominates the draw
+    for b in bs:
+        z[b, 0] = _ratio_row(u[b] + cases[b][0])
+    y = np.zeros((B, 1, V))         # q uniform: q(0) = 1/4
+    r = ACC.accept(z, y, np.zeros((B, 1), np.int64), 1.0, seed=seed, step=step)
+    for b in bs:
+        delta, want = cases[b]
+        assert bool(r["margin"][b]) is want, (b, u[b], delta)
+        assert r["n_accepted"][b] == (1 if delta > 0 else 0)
+    rest = [b for b in range(B) if b not in cases]
+    assert not r["margin"][rest].any()
+
+
+def test_acceptance_margin_ignores_decisions_never_taken():
+    """k = 2: a near-tie at draft 2 is flagged when draft 1 was accepted, and not flagged when
+    draft 1 was rejected (draft 2 is then never tested)."""
+    from oracle.philox import accept_uniform
+    seed, step, V, B = 21, 7, 4, 32
+    u = accept_uniform(seed, step, np.arange(B * 3)).reshape(B, 3)
+    bs = [b for b in range(B) if 0.05 < u[b, 0] < 0.95 and 0.05 < u[b, 1] < 0.95][:2]
+    assert len(bs) == 2
+    z = np.empty((B, 3, V))
+    z[:, 0] = _ratio_row(2.0)
+    z[:, 1] = _ratio_row(2.0)
+    z[:, 2] = [0.0, -50.0, -50.0, -50.0]
+    acc_b, rej_b = bs
+    z[acc_b, 0] = _ratio_row(2.0)                   # draft 1 accepted (|u - 2| > 1)
+    z[rej_b, 0] = _ratio_row(u[rej_b, 0] / 2)       # draft 1 rejected, far from the margin
+    for b in bs:
+        z[b, 1] = _ratio_row(u[b, 1] + 5e-5)        # near-tie at draft 2 (row b * 3 + 1)
+    y = np.zeros((B, 2, V))
+    r = ACC.accept(z, y, np.zeros((B, 2), np.int64), 1.0, seed=seed, step=step)
+    assert r["n_accepted"][rej_b] == 0 and not r["margin"][rej_b]
+    assert r["n_accepted"][acc_b] == 2 and r["margin"][acc_b]
+    assert r["out_tokens"][rej_b, 0] == 1          # the residual's only positive token
