@@ -140,14 +140,6 @@ typedef struct {
   int top_c;        /* 0: dense mode; else clusters kept per row (1 <= top_c <= n_clusters,
                        top_c <= 64) */
   sd_dtype dtype;   /* element type of h, w and centroids (bf16; f32 in dense mode too) */
-  /* Optional softmax partials of the logit rows for sd_accept (dense bf16 mode, m <= 64):
-   * row_stats[2 * (i * ld_stats + s)] = M, [... + 1] = S with M the largest logit / T of the
-   * vocabulary entries of slot s and S = sum of exp(logit / T - M) over them (M = -inf, S = 0
-   * for an empty slot), for s < sd_lm_head_stats_slots(desc); T = stats_temperature > 0.
-   * NULL: none. */
-  float *row_stats;
-  int ld_stats;     /* pairs between consecutive rows; 0 means the slot count */
-  float stats_temperature;
 } sd_head_desc;
 
 /*
@@ -165,9 +157,6 @@ typedef struct {
  *   sel_clusters int32 [m, top_c].
  */
 size_t sd_lm_head_workspace_size(const sd_head_desc *desc);
-/* Slots per row of row_stats for this descriptor on the current device (0 if the descriptor
- * cannot produce them). */
-int sd_lm_head_stats_slots(const sd_head_desc *desc);
 sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
                      const void *centroids, const int32_t *cluster_tokens, float *logits,
                      int32_t *sel_clusters, void *ws, size_t ws_bytes, sd_stream stream);
@@ -207,33 +196,21 @@ typedef struct {
   const uint64_t *step_ptr; /* nullable DEVICE word: when set, the step entering the counter
                                is *step_ptr + step, read when the kernels run (a decode loop
                                replayed from a CUDA graph advances it with sd_commit) */
-  /* Optional softmax partials of the rows from their producers (T > 0), in the row_stats form
-   * of sd_head_desc computed at this call's temperature: target row r = b*(k+1)+i at pairs
-   * target_stats[r * ld_target_stats + s], s < target_stats_slots; draft row b*k+i likewise.
-   * A row's statistics are the merge of its slots.  With both given the statistics pass over
-   * the logits is skipped.  NULL: computed from the logits. */
-  const float *target_stats;
-  int target_stats_slots;
-  int ld_target_stats;   /* pairs between rows; 0 means target_stats_slots */
-  const float *draft_stats;
-  int draft_stats_slots;
-  int ld_draft_stats;    /* pairs between rows; 0 means draft_stats_slots */
-  /* Plain draws (k == 0, T > 0) can also emit the drawn rows' partials in that form:
-   * stats_out pairs [b * ld_stats_out + s], s < sd_accept_stats_slots(desc).  NULL: none. */
-  float *stats_out;
-  int ld_stats_out;      /* pairs between sequences; 0 means the slot count */
 } sd_accept_desc;
 
 /*
  *   target_logits float32 rows r = b*(k+1)+i, i <= k;  draft_logits float32 rows b*k+i, i < k
  *   (unused when k == 0 or T == 0; NULL ok); draft_tokens int32 [B, k] (NULL ok if k == 0).
  *   n_accepted int32 [B]; out_tokens int32 rows of length k+1: d_1..d_a, x, then -1.
- *   margin_flags int32 [B] (nullable): 1 where a decision was within 1e-4 of flipping
- *   (|u - p/q| < 1e-4, or a draw / argmax whose two best keys differ by < 1e-4).
+ *   margin_flags int32 [B] (nullable): 1 where a decision of the sequence may have come out
+ *   differently in exact arithmetic: an acceptance test with |u - p/q| < 1e-4; a greedy
+ *   argmax whose two largest logits differ by less than 1e-4 * max(1, |largest|); a draw whose
+ *   winner's lowest possible key is not 1e-4 above every other token's highest possible key,
+ *   with each probability taken to within 1e-5 * (p + q) and each ln E and logit / T to within
+ *   1e-5 (1e-5 * (1 + |logit / T|) for a draw from p); a draw from p because every residual
+ *   weight came out 0.  Sequences not flagged are the exact rule's outcome.
  */
 size_t sd_accept_workspace_size(const sd_accept_desc *desc);
-/* Slots per row of stats_out for a plain draw with this descriptor (0 if not a plain draw). */
-int sd_accept_stats_slots(const sd_accept_desc *desc);
 sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
                     const float *draft_logits, const int32_t *draft_tokens,
                     int32_t *n_accepted, int32_t *out_tokens, int32_t *margin_flags,
@@ -249,8 +226,9 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
  * SD_ACCEPT_NOALLOC_MAX_SCRATCH bytes compiled into the library, which every GPU that loads the
  * library holds until the process exits.  A request whose sd_accept_workspace_size exceeds that
  * limit is rejected with SD_ERR_WORKSPACE before anything is launched (at V = 262144 the limit
- * covers up to 626 sequences at k = 6, 1615 at k = 2).  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * covers up to 49928 sequences, whatever k).  The first call on a device, and the first after
+ * the device's context changes (e.g. after a device reset), looks up the array's device address
+ * (cudaGetSymbolAddress), so make that first call before any stream capture.
  * All calls share the one array: calls that may overlap on the GPU (other streams, other host
  * threads) race and must be ordered by the caller.  Nothing in the array needs clearing by the
  * caller: the state that must start at zero is reset by every call.  Allocates nothing.
@@ -336,10 +314,14 @@ sd_status sd_commit(const sd_commit_desc *desc, const int32_t *block_table, int3
  *   out    [m, ld_out] of out_dtype
  * Limits: 0 <= m <= 64 (m = 0 launches nothing), n a multiple of 16, k a multiple of 32,
  * k_gather a multiple of 8 (0: no gather), ld_x and ld_table multiples of 4 elements, x, W and
- * table 16-byte aligned; out must not overlap x, table, W or norm_out.  A token id outside
- * [0, table_rows) or a token_sel outside its range is not dereferenced: the row reads zeros and
- * SD_ERR_DEVICE is recorded.  No workspace: split-K partials are reduced through the shared
- * memory of a thread-block cluster.
+ * table 16-byte aligned; out must not overlap x, table, W, norm_out or the workspace.  A token id
+ * outside [0, table_rows) or a token_sel outside its range is not dereferenced: the row reads
+ * zeros and SD_ERR_DEVICE is recorded.
+ * Workspace (desc->ws, desc->ws_bytes >= sd_linear_workspace_size(desc), 16-byte aligned, no
+ * initialisation needed): the staged bf16 input rows x', and for a K dimension split over several
+ * CTAs their partial sums and per-tile tickets.  The size depends on m, n, k and the current
+ * device's SM count.  The partial sums are added in a fixed order, so the result does not
+ * depend on the launch or the timing.
  */
 typedef enum { SD_EPI_STORE = 0, SD_EPI_ADD = 1, SD_EPI_GEGLU = 2 } sd_epilogue;
 
@@ -360,8 +342,11 @@ typedef struct {
   int64_t ld_out;         /* row stride of out (elements) */
   void *norm_out;         /* nullable DEVICE bf16 [m, ld_norm_out] */
   int64_t ld_norm_out;
+  void *ws;               /* DEVICE workspace */
+  size_t ws_bytes;
 } sd_linear_desc;
 
+size_t sd_linear_workspace_size(const sd_linear_desc *desc);
 sd_status sd_linear(const sd_linear_desc *desc, const void *x, const void *W, void *out,
                     const void *table, const int32_t *tokens, const int32_t *token_sel,
                     sd_stream stream);

@@ -43,6 +43,13 @@ LINEAR_CASES = [
     (12, 1024, 2048, "f32", True, "store", "bf16", 0),    # two token groups (B 4, k 2)
     (16, 512, 4096, "bf16", False, "add", "f32", 0),      # two full token groups
     (24, 2048, 1024, "f32", True, "geglu", "bf16", 0),    # three groups, gated (B 8, k 2)
+    # the target's projections at d 5376, MLP 21504 (B 8, k 2: 24 rows)
+    (24, 8192, 5376, "f32", True, "store", "bf16", 0),    # W_q of a global layer
+    (24, 1024, 5376, "f32", True, "store", "bf16", 0),    # W_k of a sliding layer
+    (24, 5376, 8192, "bf16", False, "add", "f32", 0),     # W_o of a global layer
+    (24, 43008, 5376, "f32", True, "geglu", "bf16", 0),   # gate and up rows of the MLP
+    (24, 5376, 21504, "bf16", False, "add", "f32", 0),    # W_d of the MLP
+    (48, 4096, 5376, "f32", True, "store", "f32", 0),     # B 8, k 5: 48 rows
 ]
 
 
@@ -99,13 +106,16 @@ def run_linear(m, n, k, x_dtype, norm, epi, out_dtype, k_gather, seed=0, bad_tok
         normed = torch.full((m, k), float("nan"), dtype=torch.bfloat16, device=DEV)
         desc.norm_out, desc.ld_norm_out = normed.data_ptr(), k
     outs = []
+    # a NaN-filled workspace: a read of a slot the call did not write fails the comparison
+    ws = torch.full((max(256, sd.sd_linear_workspace_size(desc)) // 4,), float("nan"),
+                    dtype=torch.float32, device=DEV)
     for _ in range(2):  # twice: the result must not depend on the launch
         out = to_dev(out0) if epi == "add" else torch.full((m, out_cols), float("nan"),
                                                             dtype=out_t, device=DEV)
         sd.sd_linear(desc, to_dev(x) if k_x else None, W_dev, out,
                      table=to_dev(table) if k_gather else None,
                      tokens=to_dev(toks) if k_gather else None,
-                     token_sel=to_dev(sel) if k_gather else None)
+                     token_sel=to_dev(sel) if k_gather else None, ws=ws)
         torch.cuda.synchronize()
         outs.append(out.cpu())
     assert torch.equal(outs[0], outs[1])
@@ -141,8 +151,16 @@ def test_linear_unsupported_shapes_refused():
     x = torch.zeros((65, 64), device=DEV)
     W = torch.zeros((32, 64), dtype=torch.bfloat16, device=DEV)
     out = torch.zeros((65, 32), device=DEV)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
     with pytest.raises(sd.SdError):
-        sd.sd_linear(desc, x, W, out)
+        sd.sd_linear(desc, x, W, out, ws=ws)
+    # a workspace smaller than sd_linear_workspace_size is refused before any launch
+    desc.m = 8
+    need = sd.sd_linear_workspace_size(desc)
+    assert need > 0
+    with pytest.raises(sd.SdError) as e:
+        sd.sd_linear(desc, x, W, out, ws=ws[: need - 256])
+    assert e.value.status == sd.SD_ERR_WORKSPACE
 
 
 # ----------------------------------------------------------------------------- one link

@@ -26,9 +26,13 @@ def f64(t):
     return t.detach().cpu().double().numpy()
 
 
-@pytest.mark.parametrize("B,k", [(8, 2), (4, 1)])
-def test_two_layer_verify_matches_the_oracle(B, k):
-    n_q, d, ff, hq, hkv, bs = k + 1, 2048, 4096, 16, 4, 16
+@pytest.mark.parametrize("B,k,d,ff", [(8, 2, 2048, 4096), (4, 1, 2048, 4096),
+                                      (8, 2, 5376, 21504)],
+                         ids=["b8k2-d2048", "b4k1-d2048", "b8k2-d5376-full-width"])
+def test_two_layer_verify_matches_the_oracle(B, k, d, ff):
+    """The last case is the benchmark's own width: d 5376, MLP 21504 (gate and up rows
+    n 43008, W_d k 21504)."""
+    n_q, hq, hkv, bs = k + 1, 16, 4, 16
     layers = ((256, 512), (512, 0))
     rng = np.random.default_rng(100 + B)
     L = rng.integers(300, 1200, B).astype(np.int32)

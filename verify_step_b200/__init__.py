@@ -44,8 +44,7 @@ class HeadDesc(ctypes.Structure):
     _fields_ = [("m", ctypes.c_int), ("d", ctypes.c_int), ("vocab", ctypes.c_int),
                 ("ld_logits", ctypes.c_int), ("n_clusters", ctypes.c_int),
                 ("cluster_size", ctypes.c_int), ("top_c", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("row_stats", ctypes.c_void_p),
-                ("ld_stats", ctypes.c_int), ("stats_temperature", ctypes.c_float)]
+                ("dtype", ctypes.c_int)]
 
 
 class AcceptDesc(ctypes.Structure):
@@ -53,11 +52,7 @@ class AcceptDesc(ctypes.Structure):
                 ("temperature", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("step", ctypes.c_uint64), ("purpose", ctypes.c_int),
                 ("ld_target", ctypes.c_int), ("ld_draft", ctypes.c_int),
-                ("ld_out", ctypes.c_int), ("step_ptr", ctypes.c_void_p),
-                ("target_stats", ctypes.c_void_p), ("target_stats_slots", ctypes.c_int),
-                ("ld_target_stats", ctypes.c_int), ("draft_stats", ctypes.c_void_p),
-                ("draft_stats_slots", ctypes.c_int), ("ld_draft_stats", ctypes.c_int),
-                ("stats_out", ctypes.c_void_p), ("ld_stats_out", ctypes.c_int)]
+                ("ld_out", ctypes.c_int), ("step_ptr", ctypes.c_void_p)]
 
 
 class PoisonCache(ctypes.Structure):
@@ -83,7 +78,8 @@ class LinearDesc(ctypes.Structure):
                 ("ld_tokens", ctypes.c_int64), ("norm_gain", ctypes.c_void_p),
                 ("norm_eps", ctypes.c_float), ("epilogue", ctypes.c_int),
                 ("out_dtype", ctypes.c_int), ("ld_out", ctypes.c_int64),
-                ("norm_out", ctypes.c_void_p), ("ld_norm_out", ctypes.c_int64)]
+                ("norm_out", ctypes.c_void_p), ("ld_norm_out", ctypes.c_int64),
+                ("ws", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t)]
 
 
 _lib = None
@@ -97,16 +93,15 @@ _SIGS = {
     "sd_draft_xattn": (ctypes.c_int, [ctypes.POINTER(AttnDesc), _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]),
     "sd_lm_head_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(HeadDesc)]),
-    "sd_lm_head_stats_slots": (ctypes.c_int, [ctypes.POINTER(HeadDesc)]),
     "sd_lm_head": (ctypes.c_int, [ctypes.POINTER(HeadDesc), _P, _P, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P]),
     "sd_accept_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(AcceptDesc)]),
-    "sd_accept_stats_slots": (ctypes.c_int, [ctypes.POINTER(AcceptDesc)]),
     "sd_accept": (ctypes.c_int, [ctypes.POINTER(AcceptDesc), _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.c_size_t, _P]),
     "sd_accept_noalloc": (ctypes.c_int, [ctypes.POINTER(AcceptDesc), _P, _P, _P, _P, _P, _P,
                                          _P]),
     "sd_commit": (ctypes.c_int, [ctypes.POINTER(CommitDesc), _P, _P, _P, _P, _P, _P, _P]),
+    "sd_linear_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(LinearDesc)]),
     "sd_linear": (ctypes.c_int, [ctypes.POINTER(LinearDesc), _P, _P, _P, _P, _P, _P, _P]),
     "sd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sd_device_status_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), _P]),
@@ -183,14 +178,6 @@ def sd_accept_workspace_size(desc: AcceptDesc) -> int:
     return lib().sd_accept_workspace_size(ctypes.byref(desc))
 
 
-def sd_lm_head_stats_slots(desc: HeadDesc) -> int:
-    return lib().sd_lm_head_stats_slots(ctypes.byref(desc))
-
-
-def sd_accept_stats_slots(desc: AcceptDesc) -> int:
-    return lib().sd_accept_stats_slots(ctypes.byref(desc))
-
-
 def sd_verify_attn(desc, q, k_new, v_new, k_cache, v_cache, block_table, ctx_len, out, ws,
                    stream=None):
     _check("sd_verify_attn", lib().sd_verify_attn(
@@ -236,7 +223,16 @@ def sd_commit(desc, block_table, ctx_len, n_accepted, committed_slots, hidden=No
         _ptr(committed_slots), _ptr(hidden), _ptr(next_hidden), _stream(stream)))
 
 
-def sd_linear(desc, x, w, out, table=None, tokens=None, token_sel=None, stream=None):
+def sd_linear_workspace_size(desc: LinearDesc) -> int:
+    return lib().sd_linear_workspace_size(ctypes.byref(desc))
+
+
+def sd_linear(desc, x, w, out, table=None, tokens=None, token_sel=None, stream=None, ws=None):
+    """One projection; ``ws`` (a device tensor or address), when given, is set as the
+    descriptor's workspace (its size in bytes from the tensor)."""
+    if ws is not None:
+        desc.ws = _ptr(ws)
+        desc.ws_bytes = ws.numel() * ws.element_size() if hasattr(ws, "numel") else desc.ws_bytes
     _check("sd_linear", lib().sd_linear(
         ctypes.byref(desc), _ptr(x), _ptr(w), _ptr(out), _ptr(table), _ptr(tokens),
         _ptr(token_sel), _stream(stream)))

@@ -14,18 +14,43 @@ namespace sdv {
 // Per-device status word: kernels record the first device-side error here.
 __device__ int g_status_word;
 
-int *device_status_word() {
-  static std::mutex mu;
-  static int *addr[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+static CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    addr[dev] = reinterpret_cast<int *>(p);
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+void *symbol_address(SymbolSlot &slot, const void *symbol) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= SymbolSlot::kDevices)
+    return nullptr;
+  // The context the address belongs to: a device reset or a new primary context makes a cached
+  // address stale, so the cache is keyed on the context that is current now.
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  if (get == nullptr || get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  std::lock_guard<std::mutex> lock(slot.mu);
+  if (slot.addr[dev] == nullptr || ctx == nullptr || slot.ctx[dev] != ctx) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+    slot.addr[dev] = p;
+    slot.ctx[dev] = ctx;
   }
-  return addr[dev];
+  return slot.addr[dev];
+}
+
+int *device_status_word() {
+  static SymbolSlot slot;
+  return reinterpret_cast<int *>(symbol_address(slot, &g_status_word));
 }
 
 bool pdl_enabled() {

@@ -6,11 +6,27 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <utility>
 
 #include "../../include/sd_verify.h"
 
 namespace sdv {
+
+// Cache of a __device__ variable's address per device, keyed on the CUDA context it was
+// looked up in (a device reset invalidates addresses; the next lookup then repeats).
+struct SymbolSlot {
+  static constexpr int kDevices = 64;
+  std::mutex mu;
+  void *addr[kDevices] = {};
+  void *ctx[kDevices] = {};
+};
+
+// Device address of ``symbol`` (a __device__ variable of this library) on the current device,
+// looked up with cudaGetSymbolAddress when the cache has none for the current context.  A
+// symbol's host-side name is not a device address, so kernels get this value instead.
+// nullptr if it cannot be obtained.
+void *symbol_address(SymbolSlot &slot, const void *symbol);
 
 // Device address of the current device's status word (nullptr if it cannot be obtained).
 int *device_status_word();

@@ -4,19 +4,25 @@
 //
 // "Gemma 4 MTP: drafter drafts, target verifies", section "drafter internal architecture": the
 // drafter runs 4 transformer layers on the target's last-layer activation and its own token
-// embedding, and the target runs its layers over the k+1 verified positions.  With B = 8 token
-// rows a projection is a matrix-vector product in all but name:
-// 8 FLOPs per weight byte, so the weights' single pass through HBM bounds it.  The kernel
-// streams each CTA's W rows into shared memory with a few large TMA tensor copies (completing on
-// mbarriers), feeds mma.sync from there and keeps the few token rows in
-// shared memory in fragment order; the K dimension is split over the CTAs of a thread-block
-// cluster and reduced through distributed shared memory, so the result needs no workspace and
-// does not depend on the launch.
+// embedding, and the target runs its layers over the k+1 verified positions.  With m <= 64 token
+// rows a projection reads each weight once and does 2m FLOPs with it: the weights' single pass
+// through HBM bounds it, as it bounds the LM head.
 //
-// Fragment trick: a thread's 16-byte read holds 8 consecutive columns 8q .. 8q+7 of one W row.
-// The two m16n8k16 steps of a 32-column chunk take columns {8q..8q+3} and {8q+4..8q+7} as their
-// logical k indices {2q, 2q+1, 2q+8, 2q+9}; the token rows are staged with the same column
-// mapping, so each product pairs the same physical column on both sides.
+// Two kernels per call:
+//  1. linear_stage_kernel: one CTA per token row gathers the row (the input columns and, for
+//     the drafter's first projection, an embedding row chosen by token id), normalises it
+//     (RMSNorm with gain) and writes it once as bf16 into the workspace, zero-padded to a
+//     multiple of 64 columns (x'); it also clears the split tickets of kernel 2.
+//  2. linear_umma_kernel<N>: the product on the tensor cores with the operands swapped so the
+//     streamed weights are the MMA's M side, as in the dense LM head: A = a 128-row tile of W
+//     [128 x 64] per pipeline stage, B = x' [N x 64] (N = m rounded up to 16, zero rows past m),
+//     D = y^T tile [128 x N] float32 in tensor memory (two buffers).  Warp 0 issues the TMA
+//     copies (no multicast; W evict-first, x' evict-last), warp 1 issues tcgen05.mma from one
+//     thread, warps 2-5 read the accumulator (thread = output row).  Persistent: one CTA per
+//     SM walks the work units (tile, K split); the K dimension is split so that the units
+//     spread evenly over the SMs.  A split writes its [128 x m] partial to the workspace; the
+//     last split of a tile to finish (atomic ticket, no waiting) adds the partials in split
+//     order, so the result does not depend on the timing, and applies the epilogue.
 #include <algorithm>
 
 #include "common.cuh"
@@ -25,38 +31,35 @@
 namespace sdv {
 namespace lin {
 
-constexpr int kWarpsN = 2;                 // warps along W rows (16 rows each)
-constexpr int kWarpsK = 4;                 // warps along K inside a CTA
-constexpr int kThreads = 32 * kWarpsN * kWarpsK;
-constexpr int kRows = 16 * kWarpsN;        // W rows per CTA
+constexpr int BM = 128;      // weight rows per tile (UMMA M)
+constexpr int BK = 64;       // K elements per stage (128-byte rows)
 constexpr int kMaxM = 64;
+constexpr int kMaxSplits = 32;
+constexpr int kStageThreads = 256;
 
 struct Params {
-  int m, n, k, k_x, x_f32;
+  // input rows
+  int m, n, k, k64, k_x, x_f32;
   long long ld_x;
   const void *x;
-  const __nv_bfloat16 *W;
   const __nv_bfloat16 *table;
   long long ld_table, table_rows, ld_tokens;
   const int32_t *tokens;
   const int32_t *token_sel;
   const float *gain;
   float eps;
+  __nv_bfloat16 *norm_out;
+  long long ld_norm_out;
+  __nv_bfloat16 *xp;  // x' [m][k64] bf16 (workspace)
+  // product
+  int tiles, kblocks, splits, kb_per_split, units;
   int epi, out_f32;
   long long ld_out;
   void *out;
-  __nv_bfloat16 *norm_out;
-  long long ld_norm_out;
-  int splits;        // CTAs per cluster, each taking a contiguous share of the k chunks
-  int piece;         // chunks staged per piece
+  float *part;              // [units][N][BM] partial sums (splits > 1)
+  unsigned int *tickets;    // [tiles]
   int *status;
 };
-
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
 
 __device__ __forceinline__ float gelu_tanh(float z) {
   return 0.5f * z * (1.f + tanhf(0.7978845608028654f * (z + 0.044715f * z * z * z)));
@@ -68,103 +71,33 @@ __device__ __forceinline__ float4 bf16x4_to_f4(uint2 u) {
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
-// Four consecutive input columns col .. col+3 of row r, before normalisation (zeros for a row
-// past m or an invalid token).  Branch-free apart from the loads' own predicates, so that a
-// thread's loads in an unrolled loop are all in flight together.
-template <bool XF32>
+// Four consecutive input columns col .. col+3 of row r before normalisation (zeros for an
+// invalid token).
 __device__ __forceinline__ float4 input4(const Params &p, int r, int col, int tok) {
-  const bool in_x = r < p.m && col < p.k_x;
-  const bool in_t = r < p.m && col >= p.k_x && tok >= 0;
-  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (XF32) {
-    if (in_x)
-      v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + r * p.ld_x + col);
-  } else if (in_x) {
-    v = bf16x4_to_f4(*reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.x) +
-                                                      r * p.ld_x + col));
+  if (col < p.k_x) {
+    if (p.x_f32)
+      return *reinterpret_cast<const float4 *>(static_cast<const float *>(p.x) + r * p.ld_x +
+                                               col);
+    return bf16x4_to_f4(*reinterpret_cast<const uint2 *>(
+        static_cast<const __nv_bfloat16 *>(p.x) + r * p.ld_x + col));
   }
-  if (in_t) v = bf16x4_to_f4(*reinterpret_cast<const uint2 *>(p.table + tok * p.ld_table +
-                                                              (col - p.k_x)));
-  return v;
+  if (tok < 0) return make_float4(0.f, 0.f, 0.f, 0.f);
+  return bf16x4_to_f4(
+      *reinterpret_cast<const uint2 *>(p.table + tok * p.ld_table + (col - p.k_x)));
 }
 
-constexpr int kLd = 8;  // input loads in flight per thread in the prologue
+// ------------------------------------------------------------------------------ staging
 
-constexpr int kGroup = 8;     // chunks per tensor-copy group (one mbarrier each)
-constexpr int kMaxPiece = 32; // chunks staged per piece
-constexpr int kMaxGroups = kMaxPiece / kGroup;
-constexpr int kGroupBytes = kRows * kGroup * 64;  // 16 KB of weights per group
-
-// Shared-memory plan of a CTA for a piece of P chunks: the weights (one 16 KB region per group
-// of 8 chunks), the token rows in fragment order, then the partial sums; the reduction buffer
-// reuses the first two regions.
-__host__ __device__ constexpr int w_bytes(int P) { return (P + kGroup - 1) / kGroup * kGroupBytes; }
-__host__ __device__ constexpr int region_a(int P, int NT) {
-  return w_bytes(P) + NT * P * 512 > kWarpsK * kRows * NT * 32 ? w_bytes(P) + NT * P * 512
-                                                               : kWarpsK * kRows * NT * 32;
-}
-
-// grid: (ceil(n / 32) row blocks) x splits CTAs, clusters of `splits` along x; NT token groups
-// of 8 (m <= 8 NT).  One thread brings the CTA's weight rows into shared memory with TMA tensor
-// copies (no multicast): a full group of 8 chunks is one [32 rows x 256 columns] box (row-major,
-// 512 bytes a row), a partial group one [32 x 32] box per chunk (64 bytes a row); each group
-// completes on its own mbarrier.  Every warp then takes a 16-row half of the rows and a quarter
-// of the chunks.  Rows past n arrive as zeros (tensor out-of-bounds fill).
-template <int NT, bool XF32>
-__global__ void __launch_bounds__(kThreads, NT <= 2 ? 2 : 1)
-    linear_kernel(const __grid_constant__ CUtensorMap wmap_big,
-                  const __grid_constant__ CUtensorMap wmap_small, const Params p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float s_inv[kMaxM];
-  __shared__ int s_tok[kMaxM];
-  __shared__ __align__(8) uint64_t s_bar[kMaxGroups];
+__global__ void __launch_bounds__(kStageThreads) linear_stage_kernel(const Params p) {
+  __shared__ int s_tok;
+  __shared__ float s_red[kStageThreads / 32];
+  __shared__ float s_inv;
   pdl_wait();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wr = warp % kWarpsN, wk = warp / kWarpsN;
-  const int g = lane >> 2, q = lane & 3;
-  const int S = p.splits;
-  const int rank = S > 1 ? (int)cluster_ctarank() : 0;
-  const int rb = blockIdx.x / S;
-  const int row0 = rb * kRows;
-  const int box_rows = min(kRows, p.n);  // rows of every tensor box (the map's box height)
-  const int C = p.k >> 5;
-  const int c_begin = (int)((long long)C * rank / S);
-  const int c_end = (int)((long long)C * (rank + 1) / S);
-  const int P = p.piece;
-  uint8_t *wsm = smem;
-  uint2 *xs = reinterpret_cast<uint2 *>(smem + w_bytes(P));
-  float *part = reinterpret_cast<float *>(smem + region_a(P, NT));
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxGroups; ++i) mbar_init(&s_bar[i], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  // thread 0: tensor copies of the weight rows of chunks pc0 .. pc0+np-1
-  auto issue = [&](int pc0, int np) {
-    if (threadIdx.x != 0) return;
-    const int groups = (np + kGroup - 1) / kGroup;
-    for (int gi = 0; gi < groups; ++gi) {
-      const int cnt = min(kGroup, np - gi * kGroup);
-      const int col = (pc0 + gi * kGroup) * 32;
-      mbar_arrive_expect_tx(&s_bar[gi], (uint32_t)(box_rows * cnt * 64));
-      if (cnt == kGroup) {
-        tma_load_2d(wsm + gi * kGroupBytes, &wmap_big, &s_bar[gi], col, row0);
-      } else {
-        for (int c = 0; c < cnt; ++c)
-          tma_load_2d(wsm + gi * kGroupBytes + c * (kRows * 64), &wmap_small, &s_bar[gi],
-                      col + c * 32, row0);
-      }
-    }
-  };
-  // the weights are requested before anything else: the prologue below (token ids, row
-  // statistics, staging of the token rows) runs under their HBM latency
-  issue(c_begin, min(P, c_end - c_begin));
-
-  // ---- token ids and row statistics
-  if (threadIdx.x < p.m) {
-    const int r = threadIdx.x;
+  const int r = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (r == 0 && p.splits > 1)
+    for (int t = tid; t < p.tiles; t += blockDim.x) p.tickets[t] = 0u;
+  if (tid == 0) {
     int t = -1;
     if (p.k_x < p.k) {
       int sel = 0;
@@ -176,235 +109,339 @@ __global__ void __launch_bounds__(kThreads, NT <= 2 ? 2 : 1)
       }
       if (t < 0) record_status(p.status, SD_ERR_DEVICE);
     }
-    s_tok[threadIdx.x] = t;
+    s_tok = t;
   }
   __syncthreads();
+  const int tok = s_tok;
+  float inv = 1.f;
   if (p.gain != nullptr) {
-    for (int r = warp; r < p.m; r += kThreads / 32) {
-      const int tok = s_tok[r];
-      float ss = 0.f;
-      for (int c0 = lane * 4; c0 < p.k; c0 += 128 * kLd) {
-        float4 v[kLd];
-#pragma unroll
-        for (int u = 0; u < kLd; ++u)
-          v[u] = c0 + 128 * u < p.k ? input4<XF32>(p, r, c0 + 128 * u, tok)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int u = 0; u < kLd; ++u)
-          ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (lane == 0) s_inv[r] = rsqrtf(ss / (float)p.k + p.eps);
+    float ss = 0.f;
+    for (int c = tid * 4; c < p.k; c += kStageThreads * 4) {
+      const float4 v = input4(p, r, c, tok);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
     }
-  }
-
-  float acc[NT][4];
 #pragma unroll
-  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-  const bool active = row0 + wr * 16 < p.n;
-  uint32_t parity = 0;
-  bool timed_out = false;
-
-  for (int pc0 = c_begin; pc0 < c_end; pc0 += P) {
-    const int np = min(P, c_end - pc0);
-    if (pc0 != c_begin) {
-      __syncthreads();  // every warp is done with the previous piece's rows and fragments
-      issue(pc0, np);
-    }
-    __syncthreads();  // s_inv ready
-    // ---- stage the token rows of chunks pc0 .. pc0+np-1 in fragment order
-    const int total = NT * np * 64;
-    for (int base = threadIdx.x; base < total; base += kThreads * kLd) {
-      float4 v[kLd];
-#pragma unroll
-      for (int u = 0; u < kLd; ++u) {
-        const int idx = base + kThreads * u;
-        const int ln = idx & 31, s = (idx >> 5) & 1, rest = idx >> 6;
-        const int cc = rest % np, tg = rest / np;
-        const int r = idx < total ? tg * 8 + (ln >> 2) : p.m;  // rows past m read nothing
-        const int col = (pc0 + cc) * 32 + (ln & 3) * 8 + s * 4;
-        v[u] = input4<XF32>(p, r, col, r < p.m ? s_tok[r] : -1);
-      }
-#pragma unroll
-      for (int u = 0; u < kLd; ++u) {
-        const int idx = base + kThreads * u;
-        if (idx >= total) break;
-        const int ln = idx & 31, s = (idx >> 5) & 1, rest = idx >> 6;
-        const int cc = rest % np, tg = rest / np;
-        const int r = tg * 8 + (ln >> 2);
-        const int col = (pc0 + cc) * 32 + (ln & 3) * 8 + s * 4;
-        uint2 v2 = make_uint2(0u, 0u);
-        if (r < p.m) {
-          float4 x4 = v[u];
-          if (p.gain != nullptr) {
-            const float inv = s_inv[r];
-            const float4 gg = *reinterpret_cast<const float4 *>(p.gain + col);
-            x4 = make_float4(x4.x * inv * gg.x, x4.y * inv * gg.y, x4.z * inv * gg.z,
-                             x4.w * inv * gg.w);
-          }
-          v2 = make_uint2(pack_bf16x2(x4.x, x4.y), pack_bf16x2(x4.z, x4.w));
-          if (p.norm_out != nullptr && rb == 0)
-            *reinterpret_cast<uint2 *>(p.norm_out + r * p.ld_norm_out + col) = v2;
-        }
-        xs[((tg * P + cc) * 2 + s) * 32 + ln] = v2;
-      }
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s_red[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      float t = 0.f;
+      for (int w = 0; w < kStageThreads / 32; ++w) t += s_red[w];
+      s_inv = rsqrtf(t / (float)p.k + p.eps);
     }
     __syncthreads();
-    // ---- products: chunk cc of the piece is in group cc / 8
-    const int row = wr * 16 + g;
-    const int groups = (np + kGroup - 1) / kGroup;
-    for (int gi = 0; gi < groups; ++gi) {
-      if (!mbar_wait_timed(&s_bar[gi], parity)) timed_out = true;
-      const bool full = np - gi * kGroup >= kGroup;
-      const uint8_t *gbase = wsm + gi * kGroupBytes;
-#pragma unroll
-      for (int u = 0; u < kGroup / kWarpsK; ++u) {
-        const int c8 = wk + kWarpsK * u;
-        const int cc = gi * kGroup + c8;
-        if (active && cc < np) {
-          // [32 x 256] box: row r at r * 512; [32 x 32] box of chunk c8 at c8 * 2048, row r at
-          // r * 64
-          const uint8_t *w_lo = full ? gbase + row * 512 + c8 * 64 + q * 16
-                                     : gbase + c8 * (kRows * 64) + row * 64 + q * 16;
-          const int hi_off = full ? 8 * 512 : 8 * 64;
-          const uint4 lo = *reinterpret_cast<const uint4 *>(w_lo);
-          const uint4 hi = *reinterpret_cast<const uint4 *>(w_lo + hi_off);
-          const uint32_t f0[4] = {lo.x, hi.x, lo.y, hi.y};
-          const uint32_t f1[4] = {lo.z, hi.z, lo.w, hi.w};
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            const uint2 b_0 = xs[((t * P + cc) * 2 + 0) * 32 + lane];
-            const uint2 b_1 = xs[((t * P + cc) * 2 + 1) * 32 + lane];
-            mma_bf16_16816(acc[t], f0, b_0.x, b_0.y);
-            mma_bf16_16816(acc[t], f1, b_1.x, b_1.y);
-          }
-        }
+    inv = s_inv;
+  }
+  for (int c = tid * 4; c < p.k64; c += kStageThreads * 4) {
+    uint2 v2 = make_uint2(0u, 0u);
+    if (c < p.k) {
+      float4 x4 = input4(p, r, c, tok);
+      if (p.gain != nullptr) {
+        const float4 g = *reinterpret_cast<const float4 *>(p.gain + c);
+        x4 = make_float4(x4.x * inv * g.x, x4.y * inv * g.y, x4.z * inv * g.z, x4.w * inv * g.w);
       }
+      v2 = make_uint2(pack_bf16x2(x4.x, x4.y), pack_bf16x2(x4.z, x4.w));
+      if (p.norm_out != nullptr)
+        *reinterpret_cast<uint2 *>(p.norm_out + r * p.ld_norm_out + c) = v2;
     }
-    parity ^= 1u;
+    *reinterpret_cast<uint2 *>(p.xp + (size_t)r * p.k64 + c) = v2;
   }
-  if (timed_out) record_status(p.status, SD_ERR_TIMEOUT);
-
-  // ---- reduce the kWarpsK partial sums of each warp row in shared memory (fixed order)
-  __syncthreads();
-  float *red = reinterpret_cast<float *>(smem);  // [kWarpsK][kRows][NT * 8]
-  constexpr int MT8 = NT * 8;
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    float *base = red + ((size_t)wk * kRows + wr * 16) * MT8 + t * 8 + 2 * q;
-    base[g * MT8] = acc[t][0];
-    base[g * MT8 + 1] = acc[t][1];
-    base[(g + 8) * MT8] = acc[t][2];
-    base[(g + 8) * MT8 + 1] = acc[t][3];
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kRows * MT8; i += kThreads) {
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarpsK; ++w) v += red[(size_t)w * kRows * MT8 + i];
-    part[i] = v;
-  }
-  if (S > 1)
-    cluster_sync();  // every CTA's partial is complete and visible to the cluster
-  else
-    __syncthreads();
-
-  // ---- sum over the cluster in rank order and apply the epilogue; CTA `rank` takes a
-  // contiguous share of the output units (rows, or gated features)
-  const int units = p.epi == SD_EPI_GEGLU ? kRows / 2 : kRows;
-  const int u0 = units * rank / S, u1 = units * (rank + 1) / S;
-  const int nu = u1 - u0;
-  const uint32_t part_s = smem_u32(part);
-  // sum of element idx of the partials over the cluster's CTAs, in rank order (the DSMEM loads
-  // are all issued before the first add; ranks past S add an exact zero)
-  auto cluster_sum = [&](int idx) -> float {
-    if (S == 1) return part[idx];
-    float v[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      v[c] = c < S ? ld_dsmem_f32(dsmem_addr(part_s + (uint32_t)idx * 4u, c)) : 0.f;
-    float y = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) y += v[c];
-    return y;
-  };
-  for (int i = threadIdx.x; i < nu * p.m; i += kThreads) {
-    const int tok = i / nu, unit = u0 + i % nu;
-    if (p.epi == SD_EPI_GEGLU) {
-      const int f = rb * (kRows / 2) + unit;
-      if (f >= p.n / 2) continue;
-      const int rg = (unit >> 3) * 16 + (unit & 7), ru = rg + 8;
-      const float yg = cluster_sum(rg * MT8 + tok);
-      const float yu = cluster_sum(ru * MT8 + tok);
-      static_cast<__nv_bfloat16 *>(p.out)[tok * p.ld_out + f] =
-          __float2bfloat16_rn(gelu_tanh(yg) * yu);
-    } else {
-      const int row = row0 + unit;
-      if (row >= p.n) continue;
-      const float y = cluster_sum(unit * MT8 + tok);
-      const long long o = tok * p.ld_out + row;
-      if (p.epi == SD_EPI_ADD)
-        static_cast<float *>(p.out)[o] += y;
-      else if (p.out_f32)
-        static_cast<float *>(p.out)[o] = y;
-      else
-        static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(y);
-    }
-  }
-  if (S > 1) cluster_sync();  // no CTA leaves while another still reads its partial
 }
 
-template <int NT, bool XF32>
-struct Launcher {
-  static size_t smem_bytes(int piece) {
-    return (size_t)region_a(piece, NT) + (size_t)kRows * NT * 8 * 4;
-  }
-  static sd_status launch(const CUtensorMap &big, const CUtensorMap &small, const Params &p,
-                          int row_blocks, cudaStream_t st) {
-    const size_t smem = smem_bytes(p.piece);
-    static int configured[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || configured[dev] != dev + 1) {
-      if (cudaFuncSetAttribute(linear_kernel<NT, XF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem_bytes(kMaxPiece)) != cudaSuccess)
-        return SD_ERR_CUDA;
-      if (dev < 64) configured[dev] = dev + 1;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(row_blocks * p.splits);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute a[2];
-    int na = 0;
-    if (p.splits > 1) {
-      a[na].id = cudaLaunchAttributeClusterDimension;
-      a[na].val.clusterDim.x = p.splits;
-      a[na].val.clusterDim.y = 1;
-      a[na].val.clusterDim.z = 1;
-      ++na;
-    }
-    if (pdl_enabled()) {
-      a[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      a[na].val.programmaticStreamSerializationAllowed = 1;
-      ++na;
-    }
-    cfg.attrs = a;
-    cfg.numAttrs = na;
-    return cuda_status(cudaLaunchKernelEx(&cfg, linear_kernel<NT, XF32>, big, small, p));
-  }
+// ------------------------------------------------------------------------------ product
+
+template <int N>
+struct UCfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = N * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (192 * 1024 / STAGE_BYTES) < 8 ? (192 * 1024 / STAGE_BYTES) : 8;
+  static constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : 128;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 8 * (2 * STAGES + 4) + 64;
+  static constexpr int THREADS = 192;
 };
 
-}  // namespace lin
-}  // namespace sdv
+// The epilogue of one output row i (this thread's) for token r: y = the row's product.  The
+// gated form pairs row i (a gate row: i % 16 < 8) with row i + 8 of the same warp (lane + 8);
+// every lane of the warp calls it for the same r.
+__device__ __forceinline__ void apply_epilogue(const Params &p, int i, int r, float y, int lane) {
+  if (p.epi == SD_EPI_GEGLU) {
+    const float yu = __shfl_down_sync(0xffffffffu, y, 8);
+    if ((lane & 8) == 0 && r < p.m) {
+      const int f = (i >> 4) * 8 + (i & 7);
+      if (f < p.n / 2)
+        static_cast<__nv_bfloat16 *>(p.out)[r * p.ld_out + f] =
+            __float2bfloat16_rn(gelu_tanh(y) * yu);
+    }
+    return;
+  }
+  if (r >= p.m || i >= p.n) return;
+  const long long o = r * p.ld_out + i;
+  if (p.epi == SD_EPI_ADD)
+    static_cast<float *>(p.out)[o] += y;
+  else if (p.out_f32)
+    static_cast<float *>(p.out)[o] = y;
+  else
+    static_cast<__nv_bfloat16 *>(p.out)[o] = __float2bfloat16_rn(y);
+}
 
-extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const void *W, void *out,
-                               const void *table, const int32_t *tokens,
-                               const int32_t *token_sel, sd_stream stream) {
-  using namespace sdv;
-  using namespace sdv::lin;
+template <int N>
+__global__ void __launch_bounds__(192, 1)
+    linear_umma_kernel(const __grid_constant__ CUtensorMap wmap,
+                       const __grid_constant__ CUtensorMap xmap, const Params p) {
+  using C = UCfg<N>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)STAGES * C::STAGE_BYTES);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;   // [2] accumulator ready
+  uint64_t *tempty = tfull + 2;       // [2] accumulator drained
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *s_last = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // x' comes from the staging kernel
+
+  if (warp == 0) {
+    // ----------------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&wmap);
+      tma_prefetch_desc(&xmap);
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
+      uint32_t g = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        const int tile = u / p.splits, split = u % p.splits;
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
+          const int stage = g % STAGES;
+          const uint32_t ph = (g / STAGES) & 1;
+          if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) {
+            record_status(p.status, SD_ERR_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t *a = smem + (size_t)stage * C::STAGE_BYTES;
+          uint8_t *b = a + C::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d_hint(a, &wmap, &full[stage], kb * BK, tile * BM, pol_w);
+          tma_load_2d_hint(b, &xmap, &full[stage], kb * BK, 0, pol_x);
+        }
+      }
+      if (!ok) {
+        for (uint32_t j = (g > (uint32_t)STAGES ? g - STAGES : 0); j < g; ++j)
+          mbar_wait_timed(&full[j % STAGES], (j / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, N);
+      uint32_t g = 0, i = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++i) {
+        const int split = u % p.splits;
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        const uint32_t buf = i & 1, tph = (i >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], tph ^ 1, abort_flag)) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * N;
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
+          const int stage = g % STAGES;
+          const uint32_t ph = (g / STAGES) & 1;
+          if (!mbar_wait(&full[stage], ph, abort_flag)) {
+            record_status(p.status, SD_ERR_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + (size_t)stage * C::STAGE_BYTES);
+          const uint32_t b = a + C::A_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks)
+            umma_bf16(d_tmem, umma_desc_sw128(a + ks * 32), umma_desc_sw128(b + ks * 32), idesc,
+                      (kb != kb0 || ks != 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+        }
+        if (ok) umma_commit(&tfull[buf]);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------------------- epilogue
+    // Every epilogue warp runs the same number of unit iterations and named barriers whatever
+    // happens, so an abort cannot leave a warp waiting at a barrier: after a failed wait the
+    // warp skips the work (later waits return at once) but keeps the barriers.
+    const int quad = warp & 3;  // tensor-memory lanes 32*quad .. 32*quad+31
+    const int row_in_tile = quad * 32 + lane;
+    uint32_t i = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++i) {
+      const int tile = u / p.splits;
+      const uint32_t buf = i & 1, tph = (i >> 1) & 1;
+      bool ok = *abort_flag == 0 && mbar_wait(&tfull[buf], tph, abort_flag);
+      if (!ok && *abort_flag == 0) {
+        record_status(p.status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      tc_fence_after();
+      const int row = tile * BM + row_in_tile;
+      float y[N];
+      if (ok) {
+        const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * N;
+#pragma unroll
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          uint32_t rr[16];
+          tmem_ld16(taddr + c0, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) y[c0 + e] = __uint_as_float(rr[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < N; ++e) y[e] = 0.f;
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+      if (p.splits == 1) {
+        if (ok) {
+#pragma unroll
+          for (int r = 0; r < N; ++r) apply_epilogue(p, row, r, y[r], lane);
+        }
+        continue;
+      }
+      // ---- split K: partial to the workspace; the tile's last split reduces
+      if (ok) {
+        float *dst = p.part + (size_t)u * N * BM + row_in_tile;
+#pragma unroll
+        for (int r = 0; r < N; ++r)
+          if (r < p.m) dst[(size_t)r * BM] = y[r];
+        __threadfence();
+      }
+      named_barrier(1, 128);
+      if (threadIdx.x == 64) {
+        int last = 0;
+        if (*abort_flag == 0) {
+          const unsigned int t = atomicAdd(&p.tickets[tile], 1u);
+          last = t == (unsigned int)(p.splits - 1);
+        }
+        *s_last = last;
+      }
+      named_barrier(1, 128);
+      if (*s_last) {
+        __threadfence();
+        const int s0 = u - u % p.splits;  // first unit of the tile
+#pragma unroll 1
+        for (int r = 0; r < N; ++r) {
+          float acc = 0.f;
+          if (r < p.m) {
+            for (int s = 0; s < p.splits; ++s)
+              acc += __ldcg(p.part + ((size_t)(s0 + s) * N + r) * BM + row_in_tile);
+          }
+          apply_epilogue(p, row, r, acc, lane);
+        }
+        if (threadIdx.x == 64) p.tickets[tile] = 0u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    if (*abort_flag) {
+      // let MMAs already issued drain before the tensor memory is released
+      const unsigned long long t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 1000000ull) {
+      }
+    }
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------ host side
+
+struct Shape {
+  int N, tiles, kblocks, splits, kb_per_split, units, grid;
+};
+
+static int n_of(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 48 ? 48 : 64; }
+
+// Work split of a call: S splits of the K blocks per 128-row tile, chosen to minimise the
+// K blocks of the busiest SM (ceil(tiles S / SMs) units of ceil(kblocks / S) blocks), a split
+// costing about one K block more (its partial write and the reduction).
+static Shape shape_of(int m, int n, int k) {
+  Shape s;
+  s.N = n_of(m);
+  s.tiles = (n + BM - 1) / BM;
+  s.kblocks = (k + BK - 1) / BK;
+  const int sms = std::max(sm_count(), 1);
+  long long best = -1;
+  int best_s = 1;
+  for (int S = 1; S <= std::min(kMaxSplits, s.kblocks); ++S) {
+    const int kps = (s.kblocks + S - 1) / S;
+    const int S_eff = (s.kblocks + kps - 1) / kps;  // every split non-empty
+    if (S_eff != S) continue;
+    const long long units = (long long)s.tiles * S;
+    const long long cost = (units + sms - 1) / sms * (long long)kps + (S > 1 ? 1 : 0);
+    if (best < 0 || cost < best) {
+      best = cost;
+      best_s = S;
+    }
+  }
+  s.splits = best_s;
+  s.kb_per_split = (s.kblocks + best_s - 1) / best_s;
+  s.units = s.tiles * best_s;
+  s.grid = std::min(s.units, sms);
+  return s;
+}
+
+struct Layout {
+  size_t xp, part, tickets, total;
+};
+
+static Layout layout_of(const sd_linear_desc *d, const Shape &s) {
+  Layout l;
+  const size_t k64 = (size_t)s.kblocks * BK;
+  l.xp = 0;
+  l.part = round_up((size_t)d->m * k64 * 2, 256);
+  const size_t part_bytes = s.splits > 1 ? (size_t)s.units * s.N * BM * 4 : 0;
+  l.tickets = l.part + round_up(part_bytes, 256);
+  l.total = l.tickets + round_up((size_t)s.tiles * 4, 256);
+  return l;
+}
+
+static sd_status validate(const sd_linear_desc *d, const void *x, const void *W, void *out,
+                          const void *table, const int32_t *tokens) {
   if (!d) return SD_ERR_INVALID_ARG;
   if (d->m < 0 || d->n < 1 || d->k < 1 || d->k_gather < 0 || d->k_gather > d->k)
     return SD_ERR_INVALID_ARG;
@@ -432,16 +469,57 @@ extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const voi
   if (d->norm_out && (d->ld_norm_out < d->k || d->ld_norm_out % 4 != 0 ||
                       (reinterpret_cast<uintptr_t>(d->norm_out) & 7u) != 0))
     return SD_ERR_INVALID_ARG;
+  return SD_OK;
+}
+
+template <int N>
+static sd_status launch_product(const CUtensorMap &wm, const CUtensorMap &xm, const Params &p,
+                                int grid, cudaStream_t st) {
+  using C = UCfg<N>;
+  static int configured[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64 || configured[dev] != dev + 1) {
+    if (cudaFuncSetAttribute(linear_umma_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C::SMEM) != cudaSuccess)
+      return SD_ERR_CUDA;
+    if (dev < 64) configured[dev] = dev + 1;
+  }
+  return cuda_status(
+      launch(linear_umma_kernel<N>, dim3(grid), dim3(C::THREADS), C::SMEM, st, wm, xm, p));
+}
+
+}  // namespace lin
+}  // namespace sdv
+
+extern "C" size_t sd_linear_workspace_size(const sd_linear_desc *d) {
+  using namespace sdv::lin;
+  if (!d || d->m < 1 || d->m > kMaxM || d->n < 1 || d->n % 16 || d->k < 1 || d->k % 32)
+    return 0;
+  return layout_of(d, shape_of(d->m, d->n, d->k)).total;
+}
+
+extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const void *W, void *out,
+                               const void *table, const int32_t *tokens,
+                               const int32_t *token_sel, sd_stream stream) {
+  using namespace sdv;
+  using namespace sdv::lin;
+  sd_status s = validate(d, x, W, out, table, tokens);
+  if (s != SD_OK || d->m == 0) return s;
+  const Shape sh = shape_of(d->m, d->n, d->k);
+  const Layout lay = layout_of(d, sh);
+  if (!d->ws || d->ws_bytes < lay.total || !aligned16(d->ws)) return SD_ERR_WORKSPACE;
+  uint8_t *ws = static_cast<uint8_t *>(d->ws);
 
   Params p{};
   p.m = d->m;
   p.n = d->n;
   p.k = d->k;
-  p.k_x = k_x;
+  p.k64 = sh.kblocks * BK;
+  p.k_x = d->k - d->k_gather;
   p.x_f32 = d->x_dtype == SD_F32;
   p.ld_x = d->ld_x;
   p.x = x;
-  p.W = static_cast<const __nv_bfloat16 *>(W);
   p.table = static_cast<const __nv_bfloat16 *>(table);
   p.ld_table = d->ld_table;
   p.table_rows = d->table_rows;
@@ -450,45 +528,36 @@ extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const voi
   p.token_sel = token_sel;
   p.gain = d->norm_gain;
   p.eps = d->norm_eps;
+  p.norm_out = static_cast<__nv_bfloat16 *>(d->norm_out);
+  p.ld_norm_out = d->ld_norm_out;
+  p.xp = reinterpret_cast<__nv_bfloat16 *>(ws + lay.xp);
+  p.tiles = sh.tiles;
+  p.kblocks = sh.kblocks;
+  p.splits = sh.splits;
+  p.kb_per_split = sh.kb_per_split;
+  p.units = sh.units;
   p.epi = d->epilogue;
   p.out_f32 = d->out_dtype == SD_F32;
   p.ld_out = d->ld_out;
   p.out = out;
-  p.norm_out = static_cast<__nv_bfloat16 *>(d->norm_out);
-  p.ld_norm_out = d->ld_norm_out;
+  p.part = reinterpret_cast<float *>(ws + lay.part);
+  p.tickets = reinterpret_cast<unsigned int *>(ws + lay.tickets);
   p.status = device_status_word();
 
-  // Split K over a cluster until the grid covers about two CTAs per SM.
-  const int row_blocks = (d->n + kRows - 1) / kRows;
-  const int chunks = d->k / 32;
-  const int target = 2 * std::max(sm_count(), 1);
-  int S = 1;
-  while (S < 8 && row_blocks * S * 2 <= target + target / 4 && chunks >= 8 * S) S *= 2;
-  p.splits = S;
-  const int NT = d->m <= 8 ? 1 : d->m <= 16 ? 2 : d->m <= 32 ? 4 : 8;
-  const int per_cta = (chunks + S - 1) / S;
-  p.piece = std::max(1, std::min(per_cta, kMaxPiece));
-  // weight boxes: [32 rows x 256 columns] for a full group of 8 chunks, [32 x 32] for one chunk
-  CUtensorMap big, small;
-  const uint32_t box_rows = (uint32_t)std::min(kRows, d->n);
-  if (!encode_tmap_2d_bf16(&big, W, (uint64_t)d->k, (uint64_t)d->n, (uint64_t)d->k * 2,
-                           (uint32_t)std::min(kGroup * 32, d->k), box_rows, false) ||
-      !encode_tmap_2d_bf16(&small, W, (uint64_t)d->k, (uint64_t)d->n, (uint64_t)d->k * 2, 32,
-                           box_rows, false))
+  // weights: [128 rows x 64 columns] boxes, 128-byte swizzle (rows past n and columns past k
+  // arrive as zeros); x': [N rows x 64 columns] boxes of the m staged rows (rows past m zero)
+  CUtensorMap wm, xm;
+  if (!encode_tmap_2d_bf16(&wm, W, (uint64_t)d->k, (uint64_t)d->n, (uint64_t)d->k * 2, BK, BM) ||
+      !encode_tmap_2d_bf16(&xm, p.xp, (uint64_t)p.k64, (uint64_t)d->m, (uint64_t)p.k64 * 2, BK,
+                           (uint32_t)sh.N))
     return SD_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  if (p.x_f32) {
-    switch (NT) {
-      case 1: return Launcher<1, true>::launch(big, small, p, row_blocks, st);
-      case 2: return Launcher<2, true>::launch(big, small, p, row_blocks, st);
-      case 4: return Launcher<4, true>::launch(big, small, p, row_blocks, st);
-      default: return Launcher<8, true>::launch(big, small, p, row_blocks, st);
-    }
-  }
-  switch (NT) {
-    case 1: return Launcher<1, false>::launch(big, small, p, row_blocks, st);
-    case 2: return Launcher<2, false>::launch(big, small, p, row_blocks, st);
-    case 4: return Launcher<4, false>::launch(big, small, p, row_blocks, st);
-    default: return Launcher<8, false>::launch(big, small, p, row_blocks, st);
+  if (launch(linear_stage_kernel, dim3(d->m), dim3(kStageThreads), 0, st, p) != cudaSuccess)
+    return SD_ERR_CUDA;
+  switch (sh.N) {
+    case 16: return launch_product<16>(wm, xm, p, sh.grid, st);
+    case 32: return launch_product<32>(wm, xm, p, sh.grid, st);
+    case 48: return launch_product<48>(wm, xm, p, sh.grid, st);
+    default: return launch_product<64>(wm, xm, p, sh.grid, st);
   }
 }

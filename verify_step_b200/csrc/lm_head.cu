@@ -36,9 +36,6 @@ struct Params {
   int num_tiles, kblocks;
   float *logits;
   int *status;
-  float2 *stats;  // optional softmax partials [M][stats_ld]: slot 4 * CTA + epilogue warp
-  int stats_ld;
-  float inv_t;    // 1 / temperature of the partials
 };
 
 template <int N>
@@ -163,17 +160,6 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ----------------------------------------------------------------------- epilogue
     const int quad = warp & 3;  // tensor-memory lanes 32*quad .. 32*quad+31
-    // Optional softmax partials: this thread's running (max, sum exp(x - max)) of logit / T
-    // over its vocabulary rows, per batch row (N <= 64 keeps them in registers).
-    constexpr int NS = N <= 64 ? N : 1;
-    constexpr float L2E = 1.4426950408889634f;
-    const bool want_stats = N <= 64 && p.stats != nullptr;
-    float st_m[NS], st_s[NS];
-#pragma unroll
-    for (int e = 0; e < NS; ++e) {
-      st_m[e] = -INFINITY;
-      st_s[e] = 0.f;
-    }
     uint32_t i = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
       const uint32_t buf = i & 1, tph = (i >> 1) & 1;
@@ -196,48 +182,10 @@ __global__ void __launch_bounds__(192, 1)
             const int m = c0 + e;
             if (m < p.M) p.logits[(size_t)m * p.ld + v] = __uint_as_float(r[e]);
           }
-          if constexpr (N <= 64) {
-            if (want_stats) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int m = c0 + e;
-                if (m < p.M) {
-                  const float x = __uint_as_float(r[e]) * p.inv_t;
-                  if (x > st_m[m]) {
-                    st_s[m] = st_s[m] * exp2f((st_m[m] - x) * L2E) + 1.f;
-                    st_m[m] = x;
-                  } else {
-                    st_s[m] += exp2f((x - st_m[m]) * L2E);
-                  }
-                }
-              }
-            }
-          }
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
-    }
-    if constexpr (N <= 64) {
-      if (want_stats) {
-        // merge over the warp's 32 vocabulary rows; one slot per (CTA, epilogue warp)
-#pragma unroll
-        for (int m = 0; m < NS; ++m) {
-          if (m >= p.M) break;
-          float mm = st_m[m], ss = st_s[m];
-          for (int off = 16; off > 0; off >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, mm, off);
-            const float s2 = __shfl_xor_sync(0xffffffffu, ss, off);
-            const float mx = fmaxf(mm, m2);
-            if (mx != -INFINITY) {
-              ss = ss * exp2f((mm - mx) * L2E) + s2 * exp2f((m2 - mx) * L2E);
-              mm = mx;
-            }
-          }
-          if (lane == 0)
-            p.stats[(size_t)m * p.stats_ld + blockIdx.x * 4 + quad] = make_float2(mm, ss);
-        }
-      }
     }
   }
   tc_fence_before();
@@ -691,8 +639,7 @@ static int umma_grid(int V) {
 
 template <int N>
 static sd_status launch_umma(const void *h, const void *w, int M, int d, int V, float *logits,
-                             int ld, cudaStream_t st, float2 *stats = nullptr,
-                             int stats_ld = 0, float inv_t = 1.f) {
+                             int ld, cudaStream_t st) {
   using C = UCfg<N>;
   static bool attr_set[64];
   int dev = 0;
@@ -716,24 +663,19 @@ static sd_status launch_umma(const void *h, const void *w, int M, int d, int V, 
   p.kblocks = d / BK;
   p.logits = logits;
   p.status = device_status_word();
-  p.stats = stats;
-  p.stats_ld = stats_ld;
-  p.inv_t = inv_t;
   const int grid = umma_grid(V);
   if (grid <= 0) return SD_ERR_CUDA;
   return cuda_status(
       launch(lm_head_umma_kernel<N>, dim3(grid), dim3(C::THREADS), C::SMEM, st, wm, hm, p));
 }
 
-// Dense bf16 projection of up to 256 rows (softmax partials for up to 64).
+// Dense bf16 projection of up to 256 rows.
 static sd_status dense_bf16(const void *h, const void *w, int M, int d, int V, float *logits,
-                            int ld, cudaStream_t st, float2 *stats = nullptr, int stats_ld = 0,
-                            float inv_t = 1.f) {
-  if (M <= 16) return launch_umma<16>(h, w, M, d, V, logits, ld, st, stats, stats_ld, inv_t);
-  if (M <= 32) return launch_umma<32>(h, w, M, d, V, logits, ld, st, stats, stats_ld, inv_t);
-  if (M <= 48) return launch_umma<48>(h, w, M, d, V, logits, ld, st, stats, stats_ld, inv_t);
-  if (M <= 64) return launch_umma<64>(h, w, M, d, V, logits, ld, st, stats, stats_ld, inv_t);
-  if (stats) return SD_ERR_UNSUPPORTED;
+                            int ld, cudaStream_t st) {
+  if (M <= 16) return launch_umma<16>(h, w, M, d, V, logits, ld, st);
+  if (M <= 32) return launch_umma<32>(h, w, M, d, V, logits, ld, st);
+  if (M <= 48) return launch_umma<48>(h, w, M, d, V, logits, ld, st);
+  if (M <= 64) return launch_umma<64>(h, w, M, d, V, logits, ld, st);
   if (M <= 96) return launch_umma<96>(h, w, M, d, V, logits, ld, st);
   if (M <= 128) return launch_umma<128>(h, w, M, d, V, logits, ld, st);
   if (M <= 192) return launch_umma<192>(h, w, M, d, V, logits, ld, st);
@@ -756,11 +698,6 @@ static sd_status validate(const sd_head_desc *d) {
   }
   if (d->dtype == SD_BF16 && d->d % 64) return SD_ERR_UNSUPPORTED;
   if (d->dtype == SD_BF16 && (long long)d->vocab >= (1ll << 31)) return SD_ERR_UNSUPPORTED;
-  if (d->row_stats) {
-    if (d->top_c != 0 || d->dtype != SD_BF16 || d->m > 64) return SD_ERR_UNSUPPORTED;
-    if (!(d->stats_temperature > 0.f) || d->stats_temperature > 1e30f) return SD_ERR_INVALID_ARG;
-    if (d->ld_stats != 0 && d->ld_stats < 4 * umma_grid(d->vocab)) return SD_ERR_INVALID_ARG;
-  }
   return SD_OK;
 }
 
@@ -776,13 +713,6 @@ static size_t ws_size(const sd_head_desc *d) {
 extern "C" {
 
 size_t sd_lm_head_workspace_size(const sd_head_desc *desc) { return sdv::head::ws_size(desc); }
-
-int sd_lm_head_stats_slots(const sd_head_desc *desc) {
-  if (!desc || desc->top_c != 0 || desc->dtype != SD_BF16 || desc->m < 1 || desc->m > 64 ||
-      desc->vocab < 1)
-    return 0;
-  return 4 * sdv::head::umma_grid(desc->vocab);
-}
 
 sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
                      const void *centroids, const int32_t *cluster_tokens, float *logits,
@@ -806,12 +736,6 @@ sd_status sd_lm_head(const sd_head_desc *desc, const void *h, const void *w,
   }
   if (!aligned16(h) || !aligned16(w)) return SD_ERR_INVALID_ARG;
   const size_t hrow = (size_t)desc->d * 2;
-  if (desc->top_c == 0 && desc->row_stats) {  // m <= 64: one launch
-    const int slots = 4 * umma_grid(desc->vocab);
-    return dense_bf16(h, w, desc->m, desc->d, desc->vocab, logits, ld, st,
-                      reinterpret_cast<float2 *>(desc->row_stats),
-                      desc->ld_stats ? desc->ld_stats : slots, 1.f / desc->stats_temperature);
-  }
   if (desc->top_c == 0) {
     for (int m0 = 0; m0 < desc->m; m0 += 256) {
       const int mm = desc->m - m0 < 256 ? desc->m - m0 : 256;

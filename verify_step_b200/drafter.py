@@ -23,7 +23,7 @@ from __future__ import annotations
 from dataclasses import dataclass
 
 from . import (SD_BF16, SD_EPI_ADD, SD_EPI_GEGLU, SD_EPI_STORE, SD_F32, LinearDesc,
-               sd_linear)
+               sd_linear, sd_linear_workspace_size)
 
 RMS_EPS = 1e-6
 
@@ -62,12 +62,30 @@ def device_weights(host, dev="cuda"):
     return out
 
 
+def call_shapes(shape: DrafterShape):
+    """(m, n, k) of the link's sd_linear calls."""
+    B, d, dt, F = shape.batch, shape.d, shape.d_target, shape.ff
+    out = [(B, d, dt + d)]
+    for D in shape.head_dims:
+        n = shape.h_q * D
+        out += [(B, n, d), (B, d, n), (B, 2 * F, d), (B, d, F)]
+    out.append((B, dt, d))
+    return out
+
+
+def workspace_bytes(shapes):
+    """The largest sd_linear workspace over calls of the given (m, n, k) shapes."""
+    return max(sd_linear_workspace_size(LinearDesc(m=m, n=n, k=k)) for m, n, k in shapes)
+
+
 def buffers(shape: DrafterShape, dev="cuda"):
-    """Activation buffers of one link (reused by every link)."""
+    """Activation buffers of one link (reused by every link) and the sd_linear workspace."""
     import torch
     B = shape.batch
     bf, f32 = torch.bfloat16, torch.float32
-    return {"x": torch.empty((B, shape.d), dtype=f32, device=dev),
+    return {"ws": torch.empty(max(256, workspace_bytes(call_shapes(shape))), dtype=torch.uint8,
+                              device=dev),
+            "x": torch.empty((B, shape.d), dtype=f32, device=dev),
             "q": [torch.empty((B, shape.h_q * D), dtype=bf, device=dev) for D in shape.head_dims],
             "o": [torch.empty((B, shape.h_q * D), dtype=bf, device=dev) for D in shape.head_dims],
             "u": torch.empty((B, shape.ff), dtype=bf, device=dev),
@@ -93,27 +111,34 @@ def link(shape: DrafterShape, wts, buf, h_prev, tokens, ld_tokens, attend, token
     B, d, dt, F = shape.batch, shape.d, shape.d_target, shape.ff
     x = buf["x"]
     call = wrap if wrap is not None else (lambda fn: fn())
+    ws = buf.get("ws")
+
+    def sd_linear_ws(*args, **kw):
+        return sd_linear(*args, ws=ws, **kw)
+
     desc = linear_desc
-    call(lambda: sd_linear(
+    call(lambda: sd_linear_ws(
         desc(B, d, dt + d, SD_BF16, dt, SD_EPI_STORE, SD_F32, d, k_gather=d, ld_table=d,
              table_rows=shape.vocab, ld_tokens=ld_tokens),
         h_prev, wts["W_in"], x, table=wts["E"], tokens=tokens, token_sel=token_sel,
         stream=stream))
+    # each call's arguments are bound when its closure is made, so a wrap that defers the call
+    # still issues this layer's projection
     for i, (L, D) in enumerate(zip(wts["layers"], shape.head_dims)):
         n = shape.h_q * D
         q, o = buf["q"][i], buf["o"][i]
-        call(lambda: sd_linear(desc(B, n, d, SD_F32, d, SD_EPI_STORE, SD_BF16, n,
-                                    norm_gain=L["g_attn"].data_ptr()),
-                               x, L["Wq"], q, stream=stream))
+        call(lambda L=L, n=n, q=q: sd_linear_ws(desc(B, n, d, SD_F32, d, SD_EPI_STORE, SD_BF16, n,
+                                                  norm_gain=L["g_attn"].data_ptr()),
+                                             x, L["Wq"], q, stream=stream))
         attend(i, q, o)
-        call(lambda: sd_linear(desc(B, d, n, SD_BF16, n, SD_EPI_ADD, SD_F32, d), o, L["Wo"], x,
-                               stream=stream))
-        call(lambda: sd_linear(desc(B, 2 * F, d, SD_F32, d, SD_EPI_GEGLU, SD_BF16, F,
-                                    norm_gain=L["g_mlp"].data_ptr()),
-                               x, L["Wgu"], buf["u"], stream=stream))
-        call(lambda: sd_linear(desc(B, d, F, SD_BF16, F, SD_EPI_ADD, SD_F32, d), buf["u"],
-                               L["Wd"], x, stream=stream))
-    call(lambda: sd_linear(desc(B, dt, d, SD_F32, d, SD_EPI_STORE, SD_BF16, dt,
+        call(lambda L=L, n=n, o=o: sd_linear_ws(desc(B, d, n, SD_BF16, n, SD_EPI_ADD, SD_F32, d),
+                                             o, L["Wo"], x, stream=stream))
+        call(lambda L=L: sd_linear_ws(desc(B, 2 * F, d, SD_F32, d, SD_EPI_GEGLU, SD_BF16, F,
+                                        norm_gain=L["g_mlp"].data_ptr()),
+                                   x, L["Wgu"], buf["u"], stream=stream))
+        call(lambda L=L: sd_linear_ws(desc(B, d, F, SD_BF16, F, SD_EPI_ADD, SD_F32, d), buf["u"],
+                                   L["Wd"], x, stream=stream))
+    call(lambda: sd_linear_ws(desc(B, dt, d, SD_F32, d, SD_EPI_STORE, SD_BF16, dt,
                                 norm_gain=wts["g_final"].data_ptr(),
                                 norm_out=buf["h"].data_ptr(), ld_norm_out=d),
                            x, wts["W_back"], buf["h_back"], stream=stream))
