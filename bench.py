@@ -1,24 +1,41 @@
 #!/usr/bin/env python
 """Benchmark of the speculative-decoding verify step on B200.
 
-One step is one pass of the whole hot path for a batch of B = 8 sequences with 16384 committed
-tokens and k = 2 drafts (the global-layer verify configuration at its reference point, with
-the drafter's pass over the same shared cache):
+The default workload (``spec_step``) is one pass of the whole hot path for a batch of B = 8
+sequences with 16384 committed tokens and k = 2 drafts -- the global-layer verify
+configuration at its reference point, with the drafter's pass over the same shared cache:
 
   drafter chain, j = 0..k-1:   3 x sd_draft_xattn (sliding, D256, W512) + 1 x sd_draft_xattn
                                (global, D512) on the target cache, the clustered LM head
                                (1024 clusters x 256 tokens, d 1024, top 32) and the drafter's
-                               own draw (sd_accept, k = 0, purpose 2)
+                               own draw of draft j (sd_accept, k = 0, purpose 2)
   verify:                      sd_verify_attn on the global (D512) and sliding (D256, W512)
                                layers (k+1 = 3 positions, 16q/4kv, block 16), the dense LM head
                                (d 5376, V 262144), sd_accept (T = 1), sd_commit
 
+The draft distribution q that the drafter samples from and the acceptance tests against is, by
+default, the target's own logits perturbed by the tuned noise of the synthetic recipe (standard
+deviation 1.446 at draft 1 and 1.318 after it, which makes the closed-form acceptance 0.47 and
+then 0.51, the serving guide's measured per-position rates).  Random drafter weights give a q
+unrelated to p, which rejects almost every draft; the drafter's kernels still run at full size
+and their logits are written, but the draws read the tuned q (``--random-q`` draws from the
+drafter's clustered logits instead).  The tuned q is device-resident, like the weights: it
+stands in for the drafter's device output.
+
+Other workloads (``--workload``), one JSON line each: ``tiny_fp32`` (B 1, ctx 256, fp32,
+d 256, V 1024), ``edge`` (B 1, ctx 4096, sliding D256 W512, d 2560), ``global`` (B 8, ctx 16384,
+global D512 only, k swept by --k), ``drafter`` (the 4-layer drafter pass with its dense layers
+chained for 4 drafts; drafted tokens/s) and ``serving`` (B 64, ragged contexts in
+[1024, 16384], shuffled block tables, a sliding and a global layer).  Workloads without a
+drafter pass draw their k drafts from q in one sd_accept call (k = 0, purpose 2) each step.
+
 The metric is verified positions per second, B * (k+1) per step, over the whole job.
-Inputs are synthetic and resident in HBM; every step reads ~6 GB, far more than the 126 MB L2,
-so no L2 flush is needed between steps.  Contexts grow by the accepted length each step.
+Inputs are synthetic and resident in HBM; the large workloads read far more than the 126 MB L2
+per step, so no L2 flush is needed between steps (the line says which).  Contexts grow by the
+accepted length each step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--k K] [--batch B] [--ctx L]   (other points of the workload range)
+                  [--workload NAME] [--k K] [--batch B] [--ctx L]
 
 N > 1 (under torch.distributed.run): independent replicas, one batch per GPU, no collective
 on the data path (weak scaling); time = max over ranks.
@@ -34,40 +51,145 @@ import statistics
 import subprocess
 import sys
 import time
+from dataclasses import dataclass, field, replace
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "spec_step_b8_ctx16384_k2"  # the default configuration
-
-
-def workload_name(batch, ctx, k, drafter_layers=False, target_layers=False):
-    return (f"spec_step_b{batch}_ctx{ctx}_k{k}" + ("_drafter_layers" if drafter_layers else "") +
-            ("_target_layers" if target_layers else ""))
 METRIC = "verified tokens/s per verify step (B,k,ctx); HBM GB/s as % of B200 peak"
 UNIT = "verified tokens/s"
+NOISE_FILE = os.path.join(ROOT, "tests", "golden", "draft_noise.json")
 
 
-def parse():
+# --------------------------------------------------------------------------------- workloads
+
+@dataclass
+class Cfg:
+    """One benchmark workload."""
+    kind: str                      # workload family (see WORKLOADS)
+    B: int
+    L: object                      # committed context: int, or (lo, hi) ragged
+    k: int                         # drafts per sequence
+    verify_layers: tuple           # ((head_dim, window), ...) of the verify
+    hq: int = 16
+    hkv: int = 4
+    d: int = 5376                  # target width (dense head input)
+    V: int = 262144
+    dtype: str = "bf16"
+    shuffle: bool = False
+    chain: int = 0                 # drafter chain links per step (0: no drafter pass)
+    xlayers: tuple = ()            # drafter layers' cache ((D, W), ...)
+    dh: int = 1024                 # drafter width
+    C: int = 1024
+    cs: int = 256
+    top_c: int = 32
+    drafter_dense: bool = False    # the drafter's projections around its cross-attention
+    target_layers: bool = False    # verify through two target layers with their projections
+    q_mode: str = "tuned"          # "tuned": q = softmax((z + noise) / T); "drafter": its logits
+    sigmas: tuple = ()             # noise std of draft position 0, 1, ...
+    T: float = 1.0
+    verify: bool = True
+    seed_base: int = 100
+
+    @property
+    def n_q(self):
+        return self.k + 1
+
+    @property
+    def cache_layers(self):
+        """Distinct (D, W) layers of the target cache, in first-use order."""
+        out = []
+        for lay in tuple(self.verify_layers) + tuple(self.xlayers):
+            if lay not in out:
+                out.append(lay)
+        return out
+
+    def name(self):
+        ctx = self.L if isinstance(self.L, int) else "%d-%d" % tuple(self.L)
+        base = {"spec_step": "spec_step", "tiny_fp32": "tiny_fp32", "edge": "edge_verify",
+                "global": "global_verify", "drafter": "drafter_pass",
+                "serving": "serving_verify"}[self.kind]
+        n = f"{base}_b{self.B}_ctx{ctx}_k{self.k}"
+        if self.drafter_dense and self.kind == "spec_step":
+            n += "_drafter_layers"
+        if self.target_layers:
+            n += "_target_layers"
+        if self.kind in ("spec_step",) and self.q_mode == "drafter":
+            n += "_random_q"
+        return n
+
+    @property
+    def unit(self):
+        return UNIT if self.verify else "drafted tokens/s"
+
+
+def _sigmas(k):
+    try:
+        d = json.load(open(NOISE_FILE))
+        s0, s1 = float(d["sigma_pos0"]), float(d["sigma_later"])
+    except Exception:
+        s0, s1 = 1.4458, 1.3183
+    return tuple([s0] + [s1] * max(0, k - 1))
+
+
+def make_cfg(a) -> Cfg:
+    """The workload named by --workload, with --k / --batch / --ctx applied where they fit."""
+    kind = a.workload
+    SL, GL = (256, 512), (512, 0)
+    if kind == "spec_step":
+        k = a.k
+        c = Cfg("spec_step", a.batch, a.ctx, k, (GL, SL), chain=k, xlayers=(SL, SL, SL, GL),
+                drafter_dense=a.drafter_layers, target_layers=a.target_layers,
+                q_mode="drafter" if a.random_q else "tuned", sigmas=_sigmas(k))
+    elif kind == "tiny_fp32":
+        # configuration 1: draft q = softmax(z + N(0, 1.5)) (1.5 a variance)
+        c = Cfg("tiny_fp32", 1, 256, 2, ((64, 0),), hq=4, hkv=1, d=256, V=1024, dtype="f32",
+                sigmas=(math.sqrt(1.5),) * 2, seed_base=1)
+    elif kind == "edge":
+        c = Cfg("edge", 1, 4096, 2, (SL,), hq=8, hkv=2, d=2560, sigmas=_sigmas(2), seed_base=2)
+    elif kind == "global":
+        c = Cfg("global", 8, 16384, a.k, (GL,), sigmas=_sigmas(a.k), seed_base=3)
+    elif kind == "drafter":
+        c = Cfg("drafter", 8, 16384, 4, (), chain=4, xlayers=(SL, SL, SL, GL),
+                drafter_dense=True, q_mode="drafter", verify=False, seed_base=4)
+    elif kind == "serving":
+        c = Cfg("serving", 64, (1024, 16384), 2, (SL, GL), shuffle=True, sigmas=_sigmas(2),
+                seed_base=5)
+    else:
+        raise SystemExit(f"unknown workload {kind}")
+    return c
+
+
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--k", type=int, default=2)
-    ap.add_argument("--batch", type=int, default=8)
-    ap.add_argument("--ctx", type=int, default=16384)
+    ap.add_argument("--workload", default="spec_step",
+                    choices=["spec_step", "tiny_fp32", "edge", "global", "drafter", "serving"])
+    ap.add_argument("--k", type=int, default=2, help="drafts (spec_step, global)")
+    ap.add_argument("--batch", type=int, default=8, help="sequences (spec_step)")
+    ap.add_argument("--ctx", type=int, default=16384, help="committed tokens (spec_step)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--telemetry-steps", type=int, default=64,
+                    help="untimed steps after the timed region whose acceptance outcomes are "
+                         "read back for the telemetry")
+    ap.add_argument("--random-q", action="store_true",
+                    help="spec_step: draw and accept against the drafter's clustered logits "
+                         "(random weights) instead of the tuned q")
     ap.add_argument("--drafter-layers", action="store_true",
-                    help="run the drafter's dense layers (input projection, 4 x (W_q, W_o, "
-                         "gated MLP, W_d), output projection) around its cross-attention, so "
-                         "the chain is driven by the committed hidden row and tokens")
+                    help="spec_step: run the drafter's dense layers (input projection, 4 x "
+                         "(W_q, W_o, gated MLP, W_d), output projection) around its "
+                         "cross-attention, so the chain is driven by the committed hidden row "
+                         "and tokens")
     ap.add_argument("--target-layers", action="store_true",
-                    help="verify through two target layers with their own projections (a "
-                         "sliding and a global layer: q/k/v/o and a gated MLP 21504 wide at "
-                         "d 5376) instead of the two attention calls on given q, k, v")
-    return ap.parse_args()
+                    help="spec_step: verify through two target layers with their own "
+                         "projections (a sliding and a global layer: q/k/v/o and a gated MLP "
+                         "21504 wide at d 5376) instead of the two attention calls on given "
+                         "q, k, v")
+    return ap.parse_args(argv)
 
 
 # kernel group -> the CUDA source whose ncu counters a committed profile summary holds
@@ -88,18 +210,20 @@ def source_hash(name):
     return h.hexdigest()[:16]
 
 
-def dram_traffic(group, workload=WORKLOAD):
-    """DRAM bytes per launch of a kernel group from the committed ncu summary, or None when
-    the summary is missing or the kernel source changed since its counters were taken."""
+def dram_traffic(group, workload):
+    """DRAM bytes per launch of a kernel group from the committed ncu summary, with the source
+    hash it was taken at, or (None, None) when the summary is missing or the kernel source
+    changed since its counters were taken."""
     path = os.path.join(ROOT, "profiles", "dram_traffic_%s.json" % workload)
     try:
         d = json.load(open(path))
         e = d["groups"][group]
-        if e["source_sha"] != source_hash(GROUP_SOURCE[group]):
-            return None
-        return int(e["dram_bytes_per_launch"])
+        sha = source_hash(GROUP_SOURCE[group])
+        if e["source_sha"] != sha:
+            return None, None
+        return int(e["dram_bytes_per_launch"]), sha
     except Exception:
-        return None
+        return None, None
 
 
 def rank_seed(rank):
@@ -133,186 +257,250 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-# --------------------------------------------------------------------------------- workload
+# --------------------------------------------------------------------------------- the step
 
 class SpecStep:
-    """Device buffers, descriptors and the call sequence of one speculative step."""
+    """Host inputs, device buffers, descriptors and the call sequence of one step of a
+    workload.  dev=None builds the host side only (the CPU oracle arm)."""
 
-    def __init__(self, k=2, B=8, L=16384, reserve=600, rank=0, dev="cuda", dense=False,
-                 target=False):
+    def __init__(self, cfg: Cfg, reserve=600, rank=0, dev="cuda"):
         import numpy as np
         import torch
 
         import synthetic as S
-        import verify_step_b200 as sd
-        self.sd, self.np, self.torch = sd, np, torch
-        self.k, self.B, self.n_q = k, B, k + 1
+        self.cfg, self.np, self.torch, self.S = cfg, np, torch, S
         self.dev = dev
-        self.dense = dense
-        self.target = target
-        self.hq, self.hkv, self.bs = 16, 4, 16
-        self.V, self.d, self.dh = 262144, 5376, 1024
-        self.C, self.cs, self.top_c = 1024, 256, 32
-        seed = rank_seed(rank)
-        wg = S.Workload("g", B, L, k, 16, 4, [S.AttnLayer(512), S.AttnLayer(256, 512)],
-                        self.d, self.V, seed=seed, n_clusters=self.C, cluster_size=self.cs,
-                        drafter_hidden=self.dh, top_c=self.top_c)
+        c = cfg
+        self.k, self.B, self.n_q = c.k, c.B, c.n_q
+        self.hq, self.hkv, self.bs = c.hq, c.hkv, 16
+        self.V, self.d, self.dh = c.V, c.d, c.dh
+        self.C, self.cs, self.top_c = c.C, c.cs, c.top_c
+        self.dense, self.target = c.drafter_dense, c.target_layers
+        self.f32 = c.dtype == "f32"
+        seed = c.seed_base + 7 * rank if c.kind == "spec_step" else c.seed_base + 1000 * rank
+        self.seed = seed
+        lay = [S.AttnLayer(D, W) for D, W in c.cache_layers]
+        wg = S.Workload(c.kind, c.B, c.L, c.k, c.hq, c.hkv, lay, c.d, c.V, dtype=c.dtype,
+                        shuffle=c.shuffle, seed=seed, n_clusters=c.C, cluster_size=c.cs,
+                        drafter_hidden=c.dh, top_c=c.top_c)
         self.w = wg
         self.L0 = S.contexts(wg)
-        self.host = {}
-        g = lambda t: t.contiguous().to(dev)
+        self.li = {lw: i for i, lw in enumerate(c.cache_layers)}
         mb = int((self.L0.max() + reserve + self.bs - 1) // self.bs)
-        # target cache: layer 0 global D512, layer 1 sliding D256 W512
-        self.cache = []
-        for layer in (0, 1):
-            c = S.make_cache(wg, layer, self.L0, reserve=reserve, max_blocks=mb)
-            self.host[f"cache{layer}"] = c
-            self.cache.append(dict(k=g(c["k_cache"]), v=g(c["v_cache"]), table=g(c["table"]),
-                                   nb=c["num_blocks"], mb=c["max_blocks"]))
+        self.host = {"caches": [S.make_cache(wg, i, self.L0, reserve=reserve, max_blocks=mb)
+                                for i in range(len(c.cache_layers))]}
+        # per-step inputs (copied from pinned host memory in the end-to-end leg)
+        inp = {}
+        if c.verify and not c.target_layers:
+            for D, W in c.verify_layers:
+                i = self.li[(D, W)]
+                s = S.make_step_qkv(wg, i, self.n_q)
+                inp[f"q{i}"], inp[f"kn{i}"], inp[f"vn{i}"] = s["q"], s["k_new"], s["v_new"]
+        if c.verify and c.target_layers:
+            # input rows of the k+1 positions (the residual stream entering the first layer)
+            inp["x0"] = torch.from_numpy(S.normal(seed * 41 + 5, (c.B * self.n_q, c.d)))
+        if c.verify:
+            inp["hidden"] = S.make_hidden(wg, c.B * self.n_q)
+        for j in range(0 if c.drafter_dense else c.chain):
+            for i, (D, W) in enumerate(c.xlayers):
+                inp[f"dq{j}_{i}"] = S.bf16(S.normal(seed * 31 + 10 * j + i, (c.B, 1, c.hq, D),
+                                                    1 / math.sqrt(D)))
+            inp[f"dh{j}"] = S.bf16(S.normal(seed * 37 + j, (c.B, c.dh)))
+        if c.drafter_dense and not c.verify:
+            # the drafter pass alone: the target's last activation and the last token enter
+            # from the host every step
+            inp["h0"] = S.make_hidden(wg, c.B, step=97)
+            inp["tok0"] = torch.from_numpy(
+                np.random.default_rng([seed, 0x70]).integers(0, c.V, c.B).astype(np.int32))
+        self.host_inputs = inp
+        # phases: drafter link j reads its own block, the verify the last one
+        self.phases = [[kk for kk in inp if kk.startswith((f"dq{j}_", f"dh{j}")) or
+                        (j == 0 and kk in ("h0", "tok0"))] for j in range(c.chain)]
+        if c.verify:
+            self.phases.append([kk for kk in inp if not kk.startswith(("dq", "dh"))])
+        self.host["W"] = None  # regenerated on demand for the CPU oracle
+        if c.chain > 0:
+            self.host["cl"] = S.make_clustered_head(wg)
+        if c.drafter_dense:
+            self.host["drafter_w"] = S.make_drafter_weights(
+                seed, c.dh, c.d, c.V, c.hq, tuple(D for D, _ in c.xlayers))
+            self.host["h0"] = S.make_hidden(wg, c.B, step=97)
+        if c.target_layers:
+            self.host["target_w"] = S.make_target_weights(
+                seed, c.d, 4 * c.d, c.hq, c.hkv, ((256, 512), (512, 0)))
+        if dev is not None:
+            self._device(reserve)
+
+    # ------------------------------------------------------------------ device side
+    def _device(self, reserve):
+        np, torch, S, c = self.np, self.torch, self.S, self.cfg
+        import verify_step_b200 as sd
+        self.sd = sd
+        dev, B, k = self.dev, self.B, self.k
+        g = lambda t: t.contiguous().to(dev)
+        sdt = sd.SD_F32 if self.f32 else sd.SD_BF16
+        self.sdt = sdt
+        self.cache = [dict(k=g(h["k_cache"]), v=g(h["v_cache"]), table=g(h["table"]),
+                           nb=h["num_blocks"], mb=h["max_blocks"]) for h in self.host["caches"]]
         self.ctx = g(torch.from_numpy(self.L0))
         self.ctx0 = self.ctx.clone()
-        # per-step inputs (reused every step; copied from pinned host memory in the e2e leg)
-        inp = {}
-        for layer in ((0, 1) if not target else ()):
-            s = S.make_step_qkv(wg, layer, self.n_q)
-            inp[f"q{layer}"], inp[f"kn{layer}"], inp[f"vn{layer}"] = s["q"], s["k_new"], s["v_new"]
-        if target:
-            # input rows of the k+1 positions (the residual stream entering the first layer)
-            inp["x0"] = torch.from_numpy(S.normal(seed * 41 + 5, (B * self.n_q, self.d)))
-        inp["hidden"] = S.make_hidden(wg, B * self.n_q)
-        for j in range(0 if dense else k):
-            for layer, D in ((0, 512), (1, 256)):
-                n = 1 if layer == 0 else 3
-                inp[f"dq{j}_{layer}"] = S.bf16(S.normal(seed * 31 + 10 * j + layer,
-                                                        (n, B, 1, self.hq, D), 1 / math.sqrt(D)))
-            inp[f"dh{j}"] = S.bf16(S.normal(seed * 37 + j, (B, self.dh)))
-        self.host_inputs = inp
-        # all per-step inputs live in one device buffer (256-byte aligned views) ordered by
-        # the phase that first reads them (drafter step 0, drafter step 1, ..., verify), so the
-        # end-to-end leg moves each phase's inputs with one host-to-device copy
-        phases = [[] if dense else [f"dq{j}_0", f"dq{j}_1", f"dh{j}"] for j in range(k)]
-        phases.append([kk for kk in inp if not kk.startswith("dq") and not kk.startswith("dh")])
+        # all per-step inputs in one device buffer (256-byte aligned views), ordered by phase
         offs, total, self.phase_ranges = {}, 0, []
-        for keys in phases:
+        for keys in self.phases:
             start = total
             for kk in keys:
-                v = inp[kk]
+                v = self.host_inputs[kk]
                 offs[kk] = total
                 total += (v.numel() * v.element_size() + 255) // 256 * 256
             self.phase_ranges.append((start, total))
-        self.input_buf = torch.empty(total, dtype=torch.uint8, device=dev)
+        self.input_buf = torch.empty(max(total, 256), dtype=torch.uint8, device=dev)
         self.input_offs = offs
         self.inputs = {}
-        for kk, v in inp.items():
+        for kk, v in self.host_inputs.items():
             n = v.numel() * v.element_size()
             view = self.input_buf[offs[kk]:offs[kk] + n].view(v.dtype).view(v.shape)
             view.copy_(v.contiguous().to(dev))
             self.inputs[kk] = view
-        self.W = g(S.make_lm_head(wg))
-        self.host["W"] = None  # regenerated on demand for the CPU baseline
-        cl = S.make_clustered_head(wg)
-        self.host["cl"] = cl
-        self.cl = {kk: g(v) for kk, v in cl.items()}
-        # outputs and scratch
         f32, i32 = torch.float32, torch.int32
-        self.attn_out = [torch.empty((B, self.n_q, self.hq, D), dtype=torch.bfloat16, device=dev)
-                         for D in (512, 256)]
-        self.xout = [torch.empty((B, 1, self.hq, D), dtype=torch.bfloat16, device=dev)
-                     for D in (512, 256)]
-        self.draft_logits = torch.empty((B, k, self.V), dtype=f32, device=dev)
-        self.target_logits = torch.empty((B * self.n_q, self.V), dtype=f32, device=dev)
-        self.sel = torch.empty((B, self.top_c), dtype=i32, device=dev)
-        self.drafts = torch.zeros((B, k), dtype=i32, device=dev)
+        if c.verify:
+            self.W = g(S.make_lm_head(self.w))
+            self.attn_out = {lw: torch.empty((B, self.n_q, self.hq, lw[0]),
+                                             dtype=torch.float32 if self.f32 else torch.bfloat16,
+                                             device=dev) for lw in c.verify_layers}
+            self.target_logits = torch.empty((B * self.n_q, self.V), dtype=f32, device=dev)
+        if c.chain > 0:
+            self.cl = {kk: g(v) for kk, v in self.host["cl"].items()}
+            self.xout = {lw: torch.empty((B, 1, self.hq, lw[0]), dtype=torch.bfloat16,
+                                         device=dev) for lw in set(c.xlayers)}
+            self.draft_logits = torch.empty((B, c.chain, self.V), dtype=f32, device=dev)
+            self.sel = torch.empty((B, self.top_c), dtype=i32, device=dev)
+        self.drafts = torch.zeros((B, max(k, c.chain)), dtype=i32, device=dev)
         # the step's results, read back to the host as one block: n_accepted then out_tokens
         self.results = torch.zeros(B * (1 + self.n_q), dtype=i32, device=dev)
         self.n_acc = self.results[:B]
         self.out_tokens = self.results[B:].view(B, self.n_q)
         self.margin = torch.zeros(B, dtype=i32, device=dev)
-        self.dtok = torch.zeros((B, 1), dtype=i32, device=dev)
-        self.slots = torch.zeros((B, self.n_q), dtype=i32, device=dev)
-        self.next_hidden = g(S.make_hidden(wg, B, step=97))
-        if dense:
-            # the drafter's dense layers: link 0 reads the committed hidden row and the last
-            # emitted token of the previous step, link j > 0 the back projection of link j-1
-            # and draft j-1
+        hid_dt = torch.float32 if self.f32 else torch.bfloat16
+        self.next_hidden = torch.zeros((B, self.d), dtype=hid_dt, device=dev)
+        if c.drafter_dense:
             from verify_step_b200 import drafter as VD
             self.VD = VD
             self.dshape = VD.DrafterShape(batch=B, d=self.dh, d_target=self.d,
                                           ff=S.DRAFTER_FF, h_q=self.hq,
-                                          head_dims=(256, 256, 256, 512), vocab=self.V)
-            self.dwts = VD.device_weights(S.make_drafter_weights(
-                seed, self.dh, self.d, self.V, self.hq, self.dshape.head_dims), dev)
+                                          head_dims=tuple(D for D, _ in c.xlayers),
+                                          vocab=self.V)
+            self.dwts = VD.device_weights(self.host["drafter_w"], dev)
             self.dbuf = VD.buffers(self.dshape, dev)
-        if target:
-            # two target layers over the bench's caches: the sliding one, then the global one
+            self.next_hidden.copy_(g(self.host["h0"]))
+        if c.target_layers:
             from verify_step_b200 import target as VT
             self.VT = VT
             self.tshape = VT.TargetShape(batch=B, n_q=self.n_q, d=self.d, ff=4 * self.d,
                                          h_q=self.hq, h_kv=self.hkv,
                                          layers=((256, 512), (512, 0)))
-            self.twts = VT.device_weights(S.make_target_weights(
-                seed, self.d, 4 * self.d, self.hq, self.hkv, self.tshape.layers), dev)
+            self.twts = VT.device_weights(self.host["target_w"], dev)
             self.tbuf = VT.buffers(self.tshape, dev)
         # descriptors
-        self.vdesc = [self._adesc(0, self.n_q), self._adesc(1, self.n_q)]
-        self.xdesc = [[self._adesc(layer, 1, q_offset=j) for layer in (0, 1)] for j in range(k)]
-        self.hdesc_dense = sd.HeadDesc(m=B * self.n_q, d=self.d, vocab=self.V, dtype=sd.SD_BF16)
-        self.hdesc_cl = sd.HeadDesc(m=B, d=self.dh, vocab=self.V, ld_logits=k * self.V,
-                                    n_clusters=self.C, cluster_size=self.cs, top_c=self.top_c,
-                                    dtype=sd.SD_BF16)
+        self.vdesc = {lw: self._adesc(lw, self.n_q) for lw in c.verify_layers}
+        if c.target_layers:
+            for lw in ((256, 512), (512, 0)):
+                self.vdesc[lw] = self._adesc(lw, self.n_q)
+        self.xdesc = [{lw: self._adesc(lw, 1, q_offset=j) for lw in set(c.xlayers)}
+                      for j in range(c.chain)]
+        if c.verify:
+            self.hdesc_dense = sd.HeadDesc(m=B * self.n_q, d=self.d, vocab=self.V, dtype=sdt)
+        if c.chain > 0:
+            self.hdesc_cl = sd.HeadDesc(m=B, d=self.dh, vocab=self.V, ld_logits=c.chain * self.V,
+                                        n_clusters=self.C, cluster_size=self.cs,
+                                        top_c=self.top_c, dtype=sd.SD_BF16)
         # step counter on the device: the acceptance draws of step s use counter value s (the
         # drafter's chain step j adds (j+1) << 28 to keep its uniforms apart); sd_commit
         # advances it, so a step captured once in a CUDA graph draws fresh numbers each replay
         self.step_dev = torch.zeros(1, dtype=torch.int64, device=dev)
         sp = self.step_dev.data_ptr()
-        self.adesc_draft = [sd.AcceptDesc(batch=B, k=0, vocab=self.V, temperature=1.0, seed=7,
-                                          step=(j + 1) << 28, purpose=2, ld_target=k * self.V,
-                                          ld_out=k, step_ptr=sp)
-                            for j in range(k)]
-        self.adesc = sd.AcceptDesc(batch=B, k=k, vocab=self.V, temperature=1.0, seed=7, step=0,
-                                   purpose=1, step_ptr=sp)
-        self.cdesc = sd.CommitDesc(batch=B, k=k, block_size=self.bs,
-                                   max_blocks_per_seq=self.cache[0]["mb"],
-                                   num_blocks=self.cache[0]["nb"], d=self.d,
-                                   hidden_dtype=sd.SD_BF16, step_ptr=sp)
-        wsz = max([sd.sd_verify_attn_workspace_size(x) for x in self.vdesc] +
-                  [sd.sd_draft_xattn_workspace_size(x) for row in self.xdesc for x in row] +
-                  [sd.sd_lm_head_workspace_size(self.hdesc_cl),
-                   sd.sd_accept_workspace_size(self.adesc)] +
-                  [sd.sd_accept_workspace_size(x) for x in self.adesc_draft])
-        self.ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        qrows = c.chain if c.q_mode == "drafter" else k
+        self.adesc_draft = [sd.AcceptDesc(batch=B, k=0, vocab=self.V, temperature=c.T, seed=7,
+                                          step=(j + 1) << 28, purpose=2,
+                                          ld_target=qrows * self.V, ld_out=self.drafts.shape[1],
+                                          step_ptr=sp)
+                            for j in range(c.chain)]
+        # workloads without a drafter pass draw all k drafts from q in one call
+        self.adesc_draws = sd.AcceptDesc(batch=B * k, k=0, vocab=self.V, temperature=c.T, seed=7,
+                                         step=1 << 28, purpose=2, step_ptr=sp)
+        if c.verify:
+            self.adesc = sd.AcceptDesc(batch=B, k=k, vocab=self.V, temperature=c.T, seed=7,
+                                       step=0, purpose=1, ld_draft=self.V,
+                                       ld_out=self.n_q, step_ptr=sp)
+            cc = self.cache[self.commit_layer()]
+            self.cdesc = sd.CommitDesc(batch=B, k=k, block_size=self.bs,
+                                       max_blocks_per_seq=cc["mb"], num_blocks=cc["nb"], d=self.d,
+                                       hidden_dtype=sdt, step_ptr=sp)
+            self.ctable = self.cache[self.commit_layer()]["table"]
+        wsz = [sd.sd_verify_attn_workspace_size(x) for x in self.vdesc.values()]
+        wsz += [sd.sd_draft_xattn_workspace_size(x) for row in self.xdesc for x in row.values()]
+        if c.chain > 0:
+            wsz.append(sd.sd_lm_head_workspace_size(self.hdesc_cl))
+        wsz += [sd.sd_accept_workspace_size(x) for x in self.adesc_draft]
+        if c.verify:
+            wsz += [sd.sd_accept_workspace_size(self.adesc),
+                    sd.sd_accept_workspace_size(self.adesc_draws)]
+        self.ws = torch.empty(max([256] + wsz), dtype=torch.uint8, device=dev)
+        # the draft distribution: the tuned noise on the target's own logits (the hidden rows,
+        # hence the logits, are the same every step)
+        if c.q_mode == "tuned" and c.verify:
+            sd.sd_lm_head(self.hdesc_dense, self.inputs["hidden"], self.W, self.target_logits)
+            torch.cuda.synchronize()
+            z = self.target_logits.view(B, self.n_q, self.V)[:, :k].cpu()
+            self.q_tuned = g(z + self.tuned_noise(range(B)))
+            self.host["z_gpu"] = z
         torch.cuda.synchronize()
 
-    def _adesc(self, layer, n_q, q_offset=0):
-        D, W = (512, 0) if layer == 0 else (256, 512)
-        c = self.cache[layer]
+    def commit_layer(self):
+        """Cache layer whose block table gives the committed slots: the first global layer."""
+        for i, (D, W) in enumerate(self.cfg.cache_layers):
+            if W == 0:
+                return i
+        return 0
+
+    def tuned_noise(self, seqs):
+        """Noise of the tuned draft logits, [len(seqs), k, V] float32 (position i has standard
+        deviation sigmas[i]); the same values for the GPU and the oracle arm."""
+        np, torch, S, c = self.np, self.torch, self.S, self.cfg
+        out = np.empty((len(seqs), self.k, self.V), np.float32)
+        for n, b in enumerate(seqs):
+            for i in range(self.k):
+                out[n, i] = S.normal(self.seed * 53 + 1000 * b + i, (self.V,), c.sigmas[i])
+        return torch.from_numpy(out)
+
+    def _adesc(self, lw, n_q, q_offset=0):
+        D, W = lw
+        c = self.cache[self.li[lw]]
         return self.sd.AttnDesc(batch=self.B, n_q=n_q, h_q=self.hq, h_kv=self.hkv, head_dim=D,
                                 block_size=self.bs, max_blocks_per_seq=c["mb"],
                                 num_blocks=c["nb"], window=W, scale=1 / math.sqrt(D),
-                                dtype=self.sd.SD_BF16, q_offset=q_offset)
+                                dtype=self.sdt, q_offset=q_offset)
 
-    # kernels launched per call (bf16 paths)
-    # kernels per call of each group on this workload (the step graph's kernel nodes are
-    # counted directly where the CUDA runtime allows; this is the fallback)
+    @staticmethod
+    def group(kind, lw):
+        return f"{kind}_{'global' if lw[1] == 0 else 'sliding'}"
+
+    # kernels per call of each group (fallback when the graph's kernel nodes cannot be counted)
     LAUNCHES = dict(xattn_sliding=1, xattn_global=2, verify_sliding=1, verify_global=3,
-                    head_dense=1, head_clustered=3, accept_draft=1, accept=2, commit=1,
+                    head_dense=1, head_clustered=3, accept_draft=2, accept=2, commit=1,
                     drafter_dense=1, target_dense=1)
 
     def launches_per_step(self):
-        L = self.LAUNCHES
-        dense = self.VD.LAUNCHES_PER_LINK * L["drafter_dense"] if self.dense else 0
-        return (self.k * (3 * L["xattn_sliding"] + L["xattn_global"] + L["head_clustered"] +
-                          L["accept_draft"] + dense) +
-                (2 * self.VT.LINEAR_CALLS_PER_LAYER * L["target_dense"] if self.target else 0) +
-                L["verify_global"] + L["verify_sliding"] + L["head_dense"] + L["accept"] +
-                L["commit"])
+        return sum(self.LAUNCHES[g] * n for g, n in self.calls_per_step().items())
+
+    def q_source(self):
+        return self.q_tuned if self.cfg.q_mode == "tuned" else self.draft_logits
 
     def run(self, ev=None, before_phase=None):
         """Issue one step on the current stream.  ev (used while capturing a CUDA graph) maps a
         kernel group to a list that receives (start, end) events recorded as graph nodes
-        around each call of that group.  before_phase(j) is called before drafter step j
-        (j < k) and before the verify (j = k)."""
-        sd, I = self.sd, self.inputs
+        around each call of that group.  before_phase(j) is called before drafter link j
+        (j < chain) and before the verify (j = chain)."""
+        sd, I, c = self.sd, self.inputs, self.cfg
 
         def timed(name, fn):
             if ev is None or name not in ev:
@@ -324,70 +512,78 @@ class SpecStep:
             record_external(b)
             ev[name].append((a, b))
 
-        c0, c1 = self.cache
-        for j in range(self.k):
+        for j in range(c.chain):
             if before_phase is not None:
                 before_phase(j)
-            xd0, xd1 = self.xdesc[j]
             if self.dense:
                 self._dense_link(j, timed)
             else:
-                for r in range(3):
-                    timed("xattn_sliding", lambda: sd.sd_draft_xattn(
-                        xd1, I[f"dq{j}_1"][r], c1["k"], c1["v"], c1["table"], self.ctx, None,
-                        self.xout[1], self.ws))
-                timed("xattn_global", lambda: sd.sd_draft_xattn(
-                    xd0, I[f"dq{j}_0"][0], c0["k"], c0["v"], c0["table"], self.ctx, None,
-                    self.xout[0], self.ws))
+                for i, lw in enumerate(c.xlayers):
+                    cc = self.cache[self.li[lw]]
+                    timed(self.group("xattn", lw), lambda i=i, lw=lw, cc=cc: sd.sd_draft_xattn(
+                        self.xdesc[j][lw], I[f"dq{j}_{i}"], cc["k"], cc["v"], cc["table"],
+                        self.ctx, None, self.xout[lw], self.ws))
             timed("head_clustered", lambda: self._clustered(j))
             ad = self.adesc_draft[j]
             timed("accept_draft", lambda: sd.sd_accept(
-                ad, self._row_ptr(self.draft_logits, j), None, None, self.n_acc,
+                ad, self._row_ptr(self.q_source(), j), None, None, self.n_acc,
                 self._col_ptr(self.drafts, j), None, self.ws))
+        if not c.verify:
+            return
         if before_phase is not None:
-            before_phase(self.k)
+            before_phase(c.chain)
+        if c.chain == 0:
+            timed("accept_draft", lambda: sd.sd_accept(
+                self.adesc_draws, self.q_tuned, None, None, self.n_acc, self.drafts, None,
+                self.ws))
         if self.target:
             self._target_layers(timed)
         else:
-            timed("verify_global", lambda: sd.sd_verify_attn(
-                self.vdesc[0], I["q0"], I["kn0"], I["vn0"], c0["k"], c0["v"], c0["table"],
-                self.ctx, self.attn_out[0], self.ws))
-            timed("verify_sliding", lambda: sd.sd_verify_attn(
-                self.vdesc[1], I["q1"], I["kn1"], I["vn1"], c1["k"], c1["v"], c1["table"],
-                self.ctx, self.attn_out[1], self.ws))
+            for lw in c.verify_layers:
+                i, cc = self.li[lw], self.cache[self.li[lw]]
+                timed(self.group("verify", lw), lambda i=i, lw=lw, cc=cc: sd.sd_verify_attn(
+                    self.vdesc[lw], I[f"q{i}"], I[f"kn{i}"], I[f"vn{i}"], cc["k"], cc["v"],
+                    cc["table"], self.ctx, self.attn_out[lw], self.ws))
         timed("head_dense", lambda: sd.sd_lm_head(self.hdesc_dense, I["hidden"], self.W,
                                                   self.target_logits))
-        timed("accept", lambda: sd.sd_accept(self.adesc, self.target_logits, self.draft_logits,
+        timed("accept", lambda: sd.sd_accept(self.adesc, self.target_logits, self.q_source(),
                                              self.drafts, self.n_acc, self.out_tokens,
                                              self.margin, self.ws))
-        timed("commit", lambda: sd.sd_commit(self.cdesc, c0["table"], self.ctx, self.n_acc,
-                                             self.slots, I["hidden"], self.next_hidden))
+        timed("commit", lambda: sd.sd_commit(self.cdesc, self.ctable, self.ctx, self.n_acc,
+                                             self.slots_buf(), I["hidden"], self.next_hidden))
+
+    def slots_buf(self):
+        if not hasattr(self, "_slots"):
+            self._slots = self.torch.zeros((self.B, self.n_q), dtype=self.torch.int32,
+                                           device=self.dev)
+        return self._slots
 
     def _dense_link(self, j, timed):
-        sd = self.sd
-        c0, c1 = self.cache
-        xd0, xd1 = self.xdesc[j]
+        sd, c = self.sd, self.cfg
 
         def attend(i, q, o):
-            if i < 3:  # sliding layers first, the global layer last
-                timed("xattn_sliding", lambda: sd.sd_draft_xattn(
-                    xd1, q, c1["k"], c1["v"], c1["table"], self.ctx, None, o, self.ws))
-            else:
-                timed("xattn_global", lambda: sd.sd_draft_xattn(
-                    xd0, q, c0["k"], c0["v"], c0["table"], self.ctx, None, o, self.ws))
+            lw = c.xlayers[i]
+            cc = self.cache[self.li[lw]]
+            timed(self.group("xattn", lw), lambda: sd.sd_draft_xattn(
+                self.xdesc[j][lw], q, cc["k"], cc["v"], cc["table"], self.ctx, None, o,
+                self.ws))
 
         if j == 0:
-            h_prev, toks, ld, sel = self.next_hidden, self.out_tokens, self.n_q, self.n_acc
+            if c.verify:  # the committed hidden row and the last emitted token of the last step
+                h_prev, toks, ld, sel = self.next_hidden, self.out_tokens, self.n_q, self.n_acc
+            else:         # drafter pass alone: the row and token copied in for this step
+                h_prev, toks, ld, sel = self.inputs["h0"], self.inputs["tok0"], 1, None
         else:
-            h_prev, toks, ld, sel = self.dbuf["h_back"], self._col_ptr(self.drafts, j - 1), \
-                self.k, None
+            h_prev, toks, ld, sel = (self.dbuf["h_back"], self._col_ptr(self.drafts, j - 1),
+                                     self.drafts.shape[1], None)
         self.VD.link(self.dshape, self.dwts, self.dbuf, h_prev, toks, ld, attend,
                      token_sel=sel, wrap=lambda fn: timed("drafter_dense", fn))
 
     def _target_layers(self, timed):
-        c0, c1 = self.cache
-        caches = [dict(desc=self.vdesc[1], k=c1["k"], v=c1["v"], table=c1["table"]),
-                  dict(desc=self.vdesc[0], k=c0["k"], v=c0["v"], table=c0["table"])]
+        caches = []
+        for lw in ((256, 512), (512, 0)):
+            cc = self.cache[self.li[lw]]
+            caches.append(dict(desc=self.vdesc[lw], k=cc["k"], v=cc["v"], table=cc["table"]))
         self.tbuf["x"].copy_(self.inputs["x0"])
         names = iter(["verify_sliding", "verify_global"])
 
@@ -404,7 +600,7 @@ class SpecStep:
         return t.data_ptr() + j * t.element_size()
 
     def _clustered(self, j):
-        # logits of draft step j go to row b*k + j of draft_logits (ld_logits = k * V)
+        # logits of chain link j go to row b*chain + j of draft_logits (ld_logits = chain * V)
         hidden = self.dbuf["h"] if self.dense else self.inputs[f"dh{j}"]
         self.sd.sd_lm_head(self.hdesc_cl, hidden, self.cl["w_cm"],
                            self._row_ptr(self.draft_logits, j),
@@ -415,28 +611,40 @@ class SpecStep:
     # --------------------------------------------------------------- algorithmic bytes
     def bytes_per_call(self, L):
         """Algorithmic HBM bytes of one call of each kernel group at committed lengths L."""
-        np = self.np
+        np, c = self.np, self.cfg
         B, hkv, n_q, hq = self.B, self.hkv, self.n_q, self.hq
-        L = np.asarray(L, np.int64)
+        es = 4 if self.f32 else 2
+        L = np.asarray(L, np.float64)
         out = {}
-        # verify: K and V of every key read once per (sequence, kv head), new rows written,
-        # queries read, outputs written
-        for name, D, W in (("verify_global", 512, 0), ("verify_sliding", 256, 512)):
+        verify_layers = (((256, 512), (512, 0)) if self.target else c.verify_layers) \
+            if c.verify else ()
+        for lw in verify_layers:
+            D, W = lw
+            # K and V of every key read once per (sequence, kv head), new rows written,
+            # queries read, outputs written
             keys = (L + n_q) if W == 0 else np.minimum(L + n_q, W + n_q - 1)
-            out[name] = int(keys.sum() * hkv * D * 2 * 2 + B * n_q * hkv * D * 2 * 2 * 2 +
-                            2 * B * n_q * hq * D * 2)
-        for name, D, W in (("xattn_global", 512, 0), ("xattn_sliding", 256, 512)):
-            # chain step j queries position L + j: the committed keys in its window
-            keys = L if W == 0 else np.mean([np.minimum(L, W - 1 - j) for j in range(self.k)],
+            out[self.group("verify", lw)] = int(keys.sum() * hkv * D * es * 2 +
+                                                B * n_q * hkv * D * es * 2 * 2 +
+                                                2 * B * n_q * hq * D * es)
+        for lw in set(c.xlayers):
+            D, W = lw
+            # chain link j queries position L + j: the committed keys in its window
+            keys = L if W == 0 else np.mean([np.minimum(L, W - 1 - j) for j in range(c.chain)],
                                             axis=0)
-            out[name] = int(keys.sum() * hkv * D * 2 * 2 + 2 * B * hq * D * 2)
-        out["head_dense"] = int(self.V * self.d * 2 + B * n_q * self.d * 2 +
-                                B * n_q * self.V * 4)
-        out["head_clustered"] = int(self.C * self.dh * 2 + B * self.dh * 2 +
-                                    B * self.top_c * self.cs * self.dh * 2 + B * self.V * 4)
-        out["accept"] = int((B * n_q + B * self.k) * self.V * 4)
-        out["accept_draft"] = int(B * self.V * 4)
-        out["commit"] = int(B * (n_q * 4 * 2 + self.d * 2 * 2))
+            out[self.group("xattn", lw)] = int(keys.sum() * hkv * D * 2 * 2 +
+                                               2 * B * hq * D * 2)
+        if c.verify:
+            out["head_dense"] = int(self.V * self.d * es + B * n_q * self.d * es +
+                                    B * n_q * self.V * 4)
+            out["accept"] = int((B * n_q + B * self.k) * self.V * 4)
+            out["commit"] = int(B * (n_q * 4 * 2 + self.d * es * 2))
+        if c.chain > 0:
+            out["head_clustered"] = int(self.C * self.dh * 2 + B * self.dh * 2 +
+                                        B * self.top_c * self.cs * self.dh * 2 +
+                                        B * self.V * 4)
+            out["accept_draft"] = int(B * self.V * 4)
+        elif c.verify:
+            out["accept_draft"] = int(B * self.k * self.V * 4)
         if self.dense:
             out["drafter_dense"] = int(self.VD.hbm_bytes_per_link(self.dshape) /
                                        self.VD.LAUNCHES_PER_LINK)
@@ -460,14 +668,34 @@ class SpecStep:
         return total
 
     def calls_per_step(self):
-        out = dict(xattn_sliding=3 * self.k, xattn_global=self.k, head_clustered=self.k,
-                   accept_draft=self.k, verify_global=1, verify_sliding=1, head_dense=1,
-                   accept=1, commit=1)
+        c = self.cfg
+        out = {}
+        for lw in c.xlayers:
+            g = self.group("xattn", lw)
+            out[g] = out.get(g, 0) + c.chain
+        if c.chain > 0:
+            out["head_clustered"] = c.chain
+            out["accept_draft"] = c.chain
+        if c.verify:
+            if c.chain == 0:
+                out["accept_draft"] = 1
+            layers = ((256, 512), (512, 0)) if self.target else c.verify_layers
+            for lw in layers:
+                g = self.group("verify", lw)
+                out[g] = out.get(g, 0) + 1
+            out.update(head_dense=1, accept=1, commit=1)
         if self.dense:
-            out["drafter_dense"] = self.VD.LAUNCHES_PER_LINK * self.k
+            out["drafter_dense"] = self.VD.LAUNCHES_PER_LINK * c.chain
         if self.target:
             out["target_dense"] = 2 * self.VT.LINEAR_CALLS_PER_LAYER
         return out
+
+    def positions_per_step(self):
+        """Verified positions (or drafted tokens for the drafter pass alone) per step."""
+        return self.B * (self.n_q if self.cfg.verify else self.cfg.chain)
+
+    def input_bytes(self):
+        return sum(v.numel() * v.element_size() for v in self.host_inputs.values())
 
     def reset(self):
         self.ctx.copy_(self.ctx0)
@@ -480,24 +708,26 @@ class SpecStep:
         return g
 
     def capture_e2e(self, pinned, res_h):
-        """The step with its host transfers as graph nodes: the first drafter step's inputs
-        are copied on the step's stream before it starts; the later phases' inputs are copied
-        on a second stream meanwhile, each phase waiting only for its own block; the results
-        are copied back to pinned host memory at the end."""
+        """The step with its host transfers as graph nodes: the first phase's inputs are copied
+        on the step's stream before it starts; the later phases' inputs are copied on a second
+        stream meanwhile, each phase waiting only for its own block; the results are copied
+        back to pinned host memory at the end."""
         torch = self.torch
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
         with torch.cuda.graph(g):
             cur = torch.cuda.current_stream()
             s0, e0 = self.phase_ranges[0]
-            self.input_buf[s0:e0].copy_(pinned[s0:e0], non_blocking=True)
+            if e0 > s0:
+                self.input_buf[s0:e0].copy_(pinned[s0:e0], non_blocking=True)
             fork = torch.cuda.Event()
             fork.record(cur)
             side.wait_event(fork)
             ready = []
             with torch.cuda.stream(side):
                 for s, e in self.phase_ranges[1:]:
-                    self.input_buf[s:e].copy_(pinned[s:e], non_blocking=True)
+                    if e > s:
+                        self.input_buf[s:e].copy_(pinned[s:e], non_blocking=True)
                     ev = torch.cuda.Event()
                     ev.record(side)
                     ready.append(ev)
@@ -507,6 +737,10 @@ class SpecStep:
                     cur.wait_event(ready[j - 1])
 
             self.run(before_phase=before_phase)
+            if not ready:  # a single phase: nothing else to wait for
+                cur.wait_event(fork)
+            else:
+                cur.wait_event(ready[-1])
             res_h.copy_(self.results, non_blocking=True)
         return g
 
@@ -614,10 +848,11 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------------- oracle
 
-def oracle_sample(step_obj, seqs, s):
-    """The CPU oracle on sequences ``seqs`` of the batch: the full step for them (drafter
-    chain, verify on both layers, dense LM head over the full vocabulary, acceptance,
-    commit).  Returns the number of verified positions."""
+def oracle_sample(st, seqs, s):
+    """The CPU oracle on sequences ``seqs`` of the batch: the full step of the workload for
+    them (drafter chain, verify on every layer, dense LM head over the full vocabulary,
+    acceptance, commit).  Returns the number of verified positions (drafted tokens for the
+    drafter pass alone)."""
     import numpy as np
     import torch
 
@@ -625,7 +860,9 @@ def oracle_sample(step_obj, seqs, s):
     from oracle import accept as OACC
     from oracle import attention as OA
     from oracle import commit as OC
+    from oracle import drafter as OD
     from oracle import lm_head as OH
+    from oracle import target as OT
 
     class F64:
         def __init__(self, t):
@@ -638,78 +875,105 @@ def oracle_sample(step_obj, seqs, s):
                         else i for i in idx)
             return self.t[idx].to(torch.float64).numpy()
 
-    from oracle import drafter as OD
-    from oracle import target as OT
-
-    st = step_obj
-    dense, target = getattr(st, "dense", False), getattr(st, "target", False)
-    if st.host.get("W") is None:
-        st.host["W"] = S.make_lm_head(st.w)
-    k, n_q, B = st.k, st.n_q, st.B
+    c = st.cfg
+    k, n_q, B, V = st.k, st.n_q, st.B, st.V
     hi = st.host_inputs
     f = lambda t: t.to(torch.float64).numpy()
+    f32 = lambda t: t.float().numpy()
     L = st.L0.copy()
-    c0, c1 = st.host["cache0"], st.host["cache1"]
-    cl = st.host["cl"]
     seqs = list(seqs)
     m = len(seqs)
-    drafts = np.zeros((m, k), np.int64)
-    draft_logits = np.zeros((m, k, st.V))
-    ocache = {D: dict(k=F64(c["k_cache"]), v=F64(c["v_cache"]), table=c["table"].numpy()[seqs],
-                      block_size=st.bs) for D, c in ((512, c0), (256, c1))}
-    if dense:
-        h_prev = f(st.host["h0"])[seqs]
-        tokens = np.zeros(m, np.int64)
-    for j in range(k):
-        if dense:
-            # the drafter's dense layers around its four cross-attentions (sequences seqs)
-            atts = [OD.cross_attend(ocache[D], st.hq, D, 512 if D == 256 else 0, L[seqs], j)
-                    for D in (256, 256, 256, 512)]
-            link = OD.drafter_step(h_prev, tokens, st.host["drafter"], atts)
+    caches = {lw: st.host["caches"][st.li[lw]] for lw in c.cache_layers}
+    ocache = {lw: dict(k=F64(h["k_cache"]), v=F64(h["v_cache"]), table=h["table"].numpy()[seqs],
+                       block_size=st.bs) for lw, h in caches.items()}
+    rows = np.concatenate([np.arange(b * n_q, (b + 1) * n_q) for b in seqs]) if c.verify \
+        else np.zeros(0, np.int64)
+    z = None
+    if c.verify:
+        if st.host.get("W") is None:
+            st.host["W"] = S.make_lm_head(st.w)
+        h = f(hi["hidden"])[rows]
+        Wv = F64(st.host["W"])
+        z = np.empty((len(rows), V))
+        chunk = 16384
+        for v0 in range(0, V, chunk):
+            z[:, v0:v0 + chunk] = OH.lm_head(h, Wv, np.arange(v0, min(V, v0 + chunk)))
+        z = z.astype(np.float32).astype(np.float64).reshape(m, n_q, V)
+    q_tuned = None
+    if c.q_mode == "tuned" and c.verify:
+        q_tuned = (z[:, :k].astype(np.float32) + st.tuned_noise(seqs).numpy()).astype(np.float64)
+    drafts = np.zeros((m, max(k, c.chain)), np.int64)
+    draft_logits = np.zeros((m, c.chain, V))
+    if c.drafter_dense:
+        dw = st.host["drafter_w"]
+        wts = {"E": f32(dw["E"]), "W_in": f32(dw["W_in"]), "g_final": f32(dw["g_final"]),
+               "W_back": f32(dw["W_back"]),
+               "layers": [{kk: f32(v) for kk, v in lw.items()} for lw in dw["layers"]]}
+        if c.verify:
+            h_prev = f(st.host["h0"])[seqs]
+            tokens = np.zeros(m, np.int64)
+        else:
+            h_prev = f(hi["h0"])[seqs]
+            tokens = hi["tok0"].numpy()[seqs].astype(np.int64)
+    for j in range(c.chain):
+        if c.drafter_dense:
+            atts = [OD.cross_attend(ocache[lw], st.hq, lw[0], lw[1], L[seqs], j)
+                    for lw in c.xlayers]
+            link = OD.drafter_step(h_prev, tokens, wts, atts)
             hj, h_prev = link["h"], link["h_back"]
         else:
-            for layer, cache, D, W, n in ((1, c1, 256, 512, 3), (0, c0, 512, 0, 1)):
-                q = f(hi[f"dq{j}_{layer}"])
-                for r in range(n):
-                    for b in seqs:
-                        for h in range(st.hq):
-                            OA.draft_attention_one(b, h, q[r], F64(cache["k_cache"]),
-                                                   F64(cache["v_cache"]),
-                                                   cache["table"].numpy(), L, L + j, W,
-                                                   1 / math.sqrt(D), st.bs)
+            for i, (D, W) in enumerate(c.xlayers):
+                cache = caches[(D, W)]
+                q = f(hi[f"dq{j}_{i}"])
+                for b in seqs:
+                    for hh in range(st.hq):
+                        OA.draft_attention_one(b, hh, q, F64(cache["k_cache"]),
+                                               F64(cache["v_cache"]), cache["table"].numpy(),
+                                               L, L + j, W, 1 / math.sqrt(D), st.bs)
             hj = f(hi[f"dh{j}"])[seqs]
-        lg, _, _ = OH.clustered_lm_head(hj, f(cl["centroids"]),
-                                        F64(cl["w_cm"]), cl["cluster_tokens"].numpy(), st.top_c)
+        cl = st.host["cl"]
+        lg, _, _ = OH.clustered_lm_head(hj, f(cl["centroids"]), F64(cl["w_cm"]),
+                                        cl["cluster_tokens"].numpy(), st.top_c)
         draft_logits[:, j] = lg
-        r = OACC.accept(lg[:, None, :], None, np.zeros((m, 0)), 1.0, seed=7,
+        qj = q_tuned[:, j] if q_tuned is not None else lg
+        r = OACC.accept(qj[:, None, :], None, np.zeros((m, 0)), c.T, seed=7,
                         step=((j + 1) << 28) + s, purpose=OACC.PURPOSE_DRAFTER)
         drafts[:, j] = r["out_tokens"][:, 0]
         tokens = drafts[:, j]
-    rows = np.concatenate([np.arange(b * n_q, (b + 1) * n_q) for b in seqs])
-    if target:
-        # the target's two layers with their own projections (sliding, then global)
-        OT.verify_layers(f(hi["x0"])[rows], st.host["target"], [ocache[256], ocache[512]],
+    if not c.verify:
+        return m * c.chain
+    if c.chain == 0:  # the k drafts drawn from q in one call (rows b * k + i)
+        r = OACC.accept(q_tuned.reshape(m * k, 1, V), None, np.zeros((m * k, 0)), c.T, seed=7,
+                        step=(1 << 28) + s, purpose=OACC.PURPOSE_DRAFTER)
+        drafts[:, :k] = r["out_tokens"][:, 0].reshape(m, k)
+    if c.target_layers:
+        OT.verify_layers(f(hi["x0"])[rows], st.host["target_w_f32"] if "target_w_f32" in st.host
+                         else _target_f32(st), [ocache[(256, 512)], ocache[(512, 0)]],
                          L[seqs], n_q, st.hq, st.hkv)
     else:
-        for layer, cache, D, W in ((0, c0, 512, 0), (1, c1, 256, 512)):
-            q, kn, vn = f(hi[f"q{layer}"]), f(hi[f"kn{layer}"]), f(hi[f"vn{layer}"])
+        for lw in c.verify_layers:
+            D, W = lw
+            i = st.li[lw]
+            cache = caches[lw]
+            q, kn, vn = f(hi[f"q{i}"]), f(hi[f"kn{i}"]), f(hi[f"vn{i}"])
             for b in seqs:
                 for j in range(n_q):
-                    for h in range(st.hq):
-                        OA.verify_attention_one(b, j, h, q, kn, vn, F64(cache["k_cache"]),
+                    for hh in range(st.hq):
+                        OA.verify_attention_one(b, j, hh, q, kn, vn, F64(cache["k_cache"]),
                                                 F64(cache["v_cache"]), cache["table"].numpy(),
                                                 L, W, 1 / math.sqrt(D), st.bs)
-    h = f(hi["hidden"])[rows]
-    Wv = F64(st.host["W"])
-    z = np.empty((len(rows), st.V))
-    chunk = 16384
-    for v0 in range(0, st.V, chunk):
-        z[:, v0:v0 + chunk] = OH.lm_head(h, Wv, np.arange(v0, min(st.V, v0 + chunk)))
-    z = z.astype(np.float32).astype(np.float64).reshape(m, n_q, st.V)
-    r = OACC.accept(z, draft_logits, drafts, 1.0, seed=7, step=s)
-    OC.commit(L[seqs], r["n_accepted"], c0["table"].numpy()[seqs], st.bs, n_q,
-              f(hi["hidden"]).reshape(B, n_q, -1)[seqs])
+    y = q_tuned if q_tuned is not None else draft_logits
+    r = OACC.accept(z, y, drafts[:, :k], c.T, seed=7, step=s)
+    OC.commit(L[seqs], r["n_accepted"], caches[c.cache_layers[0]]["table"].numpy()[seqs], st.bs,
+              n_q, f(hi["hidden"]).reshape(B, n_q, -1)[seqs])
     return m * n_q
+
+
+def _target_f32(st):
+    tw = st.host["target_w"]
+    st.host["target_w_f32"] = [{kk: (v.float().numpy() if hasattr(v, "float") else v)
+                                for kk, v in lw.items()} for lw in tw]
+    return st.host["target_w_f32"]
 
 
 def blas_threads():
@@ -722,6 +986,76 @@ def blas_threads():
 
 
 # --------------------------------------------------------------------------------- main
+
+def config_line(st, a, world):
+    c = st.cfg
+    desc = {
+        "spec_step": "drafter chain (4 cross-attention layers, clustered head 1024x256 top-32 "
+                     "d1024, draw) per draft + verify on a global D512 and a sliding D256 W512 "
+                     "layer, dense head d5376 x V262144, acceptance T=1, commit",
+        "tiny_fp32": "fp32: global D64 4q/1kv verify, dense head d256 x V1024, drafts drawn "
+                     "from q, acceptance T=1, commit",
+        "edge": "sliding D256 W512 8q/2kv verify, dense head d2560 x V262144, drafts drawn from "
+                "q, acceptance T=1, commit",
+        "global": "global D512 16q/4kv verify, dense head d5376 x V262144, drafts drawn from "
+                  "q, acceptance T=1, commit",
+        "drafter": "drafter pass alone: 4 links, each W_in, 4 x (RMSNorm, W_q, cross-attention "
+                   "into the target cache (3 sliding D256 W512, 1 global D512), W_o, gated "
+                   "MLP 4096, W_d), W_back, clustered head 1024x256 top-32, draw",
+        "serving": "ragged contexts U[1024,16384], shuffled block tables, sliding D256 W512 "
+                   "and global D512 verify, dense head d5376 x V262144, drafts drawn from q, "
+                   "acceptance T=1, commit and rollback",
+    }[c.kind]
+    big = c.kind != "tiny_fp32" and c.kind != "edge"
+    out = {"workload": c.name(), "batch": c.B, "ctx": c.L if isinstance(c.L, int) else list(c.L),
+           "k": c.k, "heads": f"{c.hq}q/{c.hkv}kv", "block_size": 16, "step": desc,
+           "parallelism": "replicas" if world > 1 else "single",
+           "l2": "inputs larger than L2 (GBs read per step)" if big else
+                 "inputs smaller than L2, not flushed: the step reads its weights once "
+                 "(tiny/edge workloads are latency-bound)",
+           "shuffled_block_tables": c.shuffle}
+    if c.verify:
+        out["draft_q"] = ("tuned noise on the target's logits, std " +
+                          "/".join("%.3f" % s for s in c.sigmas) + " per draft position "
+                          "(closed-form acceptance 0.47, then 0.51); device-resident")\
+            if c.q_mode == "tuned" else "the drafter's clustered-head logits (random weights)"
+        out["ctx_growth"] = "contexts advance by the accepted length each step"
+    if c.drafter_dense and c.kind == "spec_step":
+        out["drafter_layers"] = ("per link: W_in [1024 x (5376+1024)] on the committed hidden "
+                                 "row and the embedding of the last token, 4 x (RMSNorm, W_q, "
+                                 "cross-attention, W_o, RMSNorm, gated GELU MLP 4096, W_d), "
+                                 "RMSNorm, W_back [5376 x 1024]; synthetic weights")
+    if c.target_layers:
+        out["target_layers"] = ("verify through 2 target layers (sliding D256 W512, then global "
+                                "D512), each RMSNorm, W_q/W_k/W_v, verify attention, W_o, "
+                                "RMSNorm, gated GELU MLP 21504, W_d at d 5376; synthetic "
+                                "weights; the dense head still reads the given hidden rows")
+    return out
+
+
+def telemetry(st, graph, steps):
+    """Acceptance outcomes of ``steps`` untimed replays, read back after each: realised
+    acceptance per position (cumulative P(a >= i)), mean accepted length (MAL = 1 + E[a]),
+    overall acceptance E[a] / k and the count of margin-flagged sequences."""
+    import numpy as np
+    torch = st.torch
+    acc = []
+    flags = 0
+    for _ in range(steps):
+        graph.replay()
+        torch.cuda.synchronize()
+        acc.append(st.n_acc.cpu().numpy().copy())
+        flags += int(st.margin.cpu().numpy().sum())
+    a = np.concatenate(acc).astype(np.float64)
+    k = st.k
+    return {"sequences": int(a.size),
+            "accept_cumulative": [round(float((a >= i).mean()), 4) for i in range(1, k + 1)],
+            "mal": round(1.0 + float(a.mean()), 4),
+            "acceptance_overall": round(float(a.mean()) / k, 4) if k else None,
+            "margin_flagged": flags,
+            "window": f"{steps} untimed steps after the timed region, n_accepted and "
+                      "margin_flags read back after each"}
+
 
 def main():
     a = parse()
@@ -746,12 +1080,12 @@ def main():
     import verify_step_b200 as sd
     sd.lib()
 
-    # every pass below runs a.steps steps (warm-up, timed, per-kernel, e2e): reserve the blocks
-    reserve = (a.warmup + 4 * a.steps + 8) * (a.k + 1) + 64
-    st = SpecStep(k=a.k, B=a.batch, L=a.ctx, reserve=reserve, rank=rank,
-                  dense=a.drafter_layers, target=a.target_layers)
-    wname = workload_name(st.B, a.ctx, st.k, a.drafter_layers, a.target_layers)
-    L_start = st.L0.copy()
+    cfg = make_cfg(a)
+    # every pass below runs a.steps steps (warm-up, timed, per-kernel, e2e, telemetry): reserve
+    # the blocks the contexts grow into
+    reserve = (a.warmup + 4 * a.steps + a.telemetry_steps + 8) * (cfg.k + 1) + 64
+    st = SpecStep(cfg, reserve=reserve, rank=rank)
+    wname = cfg.name()
     clock = ClockSampler(local)
     for _ in range(a.warmup):
         st.run()
@@ -780,7 +1114,8 @@ def main():
     ctx_b = st.ctx.cpu().numpy()
     ms = max_over_ranks(t0.elapsed_time(t1), world, "cuda")
     ms_step = ms / a.steps
-    value = whole_job_rate(world, st.B, st.n_q, a.steps, ms)
+    per_step = st.positions_per_step()
+    value = world * per_step * a.steps / (ms / 1e3)
 
     # ---- per-kernel device times: the same step captured with event nodes around each call,
     # replayed K times (synchronised per replay to read the events)
@@ -809,14 +1144,16 @@ def main():
     dom = max(groups, key=lambda g: kern_ms[g] * cps[g])
 
     def roof(g):
+        if g not in kern_ms or not kern_ms[g]:
+            return None
         ach = nbytes[g] / (kern_ms[g] * 1e6)
+        traffic, sha = dram_traffic(g, wname)
         return {"kernel": g, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
-                "unit": "GB/s", "frac": round(ach / hbm, 4),
-                "traffic": dram_traffic(g, wname),
+                "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": traffic,
+                "traffic_source": (f"committed ncu summary profiles/dram_traffic_{wname}.json, "
+                                   f"kernel source sha {sha}") if traffic else None,
                 "peak_source": src, "bytes_per_launch": nbytes[g],
                 "ms_per_launch": round(kern_ms[g], 4)}
-    # telemetry of the acceptance rule on these (random) weights
-    mean_acc = float(((ctx_b - ctx_a) - a.steps).sum()) / max(1, a.steps * st.B)
 
     # ---- end-to-end: every step copies its inputs from pinned host memory, replays the step
     # and reads the accepted counts and tokens back to the host
@@ -829,7 +1166,7 @@ def main():
             pinned[st.input_offs[kk]:st.input_offs[kk] + n].view(v.dtype).copy_(
                 v.contiguous().view(-1))
         res_h = torch.empty(st.results.numel(), dtype=torch.int32).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in st.host_inputs.values())
+        h2d = st.input_bytes()
         d2h = res_h.numel() * 4
         if world > 1:
             dist.barrier()
@@ -844,29 +1181,33 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
-        e2e = {"value": round(whole_job_rate(world, st.B, st.n_q, a.steps, ems), 1), "unit": UNIT,
+        e2e = {"value": round(world * per_step * a.steps / (ems / 1e3), 1), "unit": cfg.unit,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(ems / a.steps, 4),
                "path": "public C ABI calls and the step's host transfers captured once in a "
                        "CUDA graph; per step: H2D of the step inputs from pinned memory in one "
-                       "block per phase (drafter step 0 first; drafter step 1 and the verify "
-                       "inputs on a second stream while the drafter runs), the kernels, one "
-                       "D2H of n_accepted and out_tokens, stream synchronise"}
+                       "block per phase (later phases on a second stream while the earlier "
+                       "ones run), the kernels, one D2H of n_accepted and out_tokens, stream "
+                       "synchronise"}
+    # ---- acceptance telemetry (untimed)
+    tele = None
+    if cfg.verify and a.telemetry_steps > 0:
+        tele = telemetry(st, graph, a.telemetry_steps)
+        tele["emitted_tokens_per_s"] = round(world * st.B * tele["mal"] / (ms_step / 1e3), 1)
     clocks = clock.stop()
     status = sd.sd_device_status_read()
     del graph, graph_ev, graph_e2e
 
     cpu = None
-    if (rank == 0 and world == 1 and not a.no_cpu_baseline and not a.drafter_layers and
-            not a.target_layers):
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
         t = time.perf_counter()
         nv = oracle_sample(st, [0], 0)
         dt = time.perf_counter() - t
-        cpu = {"value": round(nv / dt, 4), "unit": UNIT, "cores": blas_threads(),
+        cpu = {"value": round(nv / dt, 4), "unit": cfg.unit, "cores": blas_threads(),
                "kind": "oracle",
-               "sample": "sequence 0 of the batch: full step (drafter chain, verify on both "
-                         "layers, dense LM head over all 262144 tokens, acceptance, commit) "
-                         "in float64 on the host; %.1f s for %d verified positions" % (dt, nv)}
+               "sample": "sequence 0 of the batch: the workload's full step for it in float64 "
+                         "on the host; %.1f s for %d %s" %
+                         (dt, nv, "verified positions" if cfg.verify else "drafted tokens")}
 
     if world > 1:
         dist.barrier()
@@ -874,37 +1215,27 @@ def main():
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": round(value, 1), "unit": cfg.unit, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": wname, "batch": st.B, "ctx": a.ctx,
-                   "k": st.k,
-                   "heads": "16q/4kv", "layers": "global D512 + sliding D256 W512",
-                   "lm_head": "d5376 x V262144", "drafter": "2-step chain, 4 cross-attn "
-                   "layers, clustered head 1024x256 top-32 d1024", "block_size": 16,
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (~6 GB read per step)",
-                   "ctx_growth": "contexts advance by the accepted length each step",
-                   **({"drafter_layers": "per link: W_in [1024 x (5376+1024)] on the committed "
-                       "hidden row and the embedding of the last token, 4 x (RMSNorm, W_q, "
-                       "cross-attention, W_o, RMSNorm, gated GELU MLP 4096, W_d), RMSNorm, "
-                       "W_back [5376 x 1024]; synthetic weights"} if a.drafter_layers else {}),
-                   **({"target_layers": "verify through 2 target layers (sliding D256 W512, "
-                       "then global D512), each RMSNorm, W_q/W_k/W_v, verify attention, W_o, "
-                       "RMSNorm, gated GELU MLP 21504, W_d at d 5376; synthetic weights; the "
-                       "dense head still reads the given hidden rows"} if a.target_layers
-                      else {})},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if cfg.dtype == "f32" else "bf16", "data": "synthetic",
+        "config": config_line(st, a, world),
         "gpu_launches": kernels_per_step * a.steps,
         "roofline": roof(dom),
-        "roofline_attention": roof("verify_global"),
+        "roofline_attention": roof("verify_global") or roof("verify_sliding")
+        or roof("xattn_global"),
         "roofline_lm_head": roof("head_dense"),
         "kernels": per_kernel,
         "kernel_busy_ms_per_step": round(busy_ms, 4),
+        "kernel_times_note": "per-kernel times come from a second capture of the step with an "
+                             "event node around every call; those nodes add time, so the sum "
+                             "exceeds ms_per_step and the per-kernel fractions read slightly low",
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "mean_accepted": round(mean_acc, 4),
+        "telemetry": tele,
+        "mean_accepted": round(float(((ctx_b - ctx_a) - a.steps).sum()) /
+                               max(1, a.steps * st.B), 4) if cfg.verify else None,
         "device_status": status,
     }
     print(json.dumps(line))
@@ -917,7 +1248,8 @@ def run_reference(a, rank, world):
         return
     import torch  # noqa: F401
     os.environ.setdefault("CUDA_VISIBLE_DEVICES", "")
-    st = HostOnlyStep(a.k, a.batch, a.ctx, dense=a.drafter_layers, target=a.target_layers)
+    cfg = make_cfg(a)
+    st = SpecStep(cfg, reserve=64, dev=None)
     for s in range(a.warmup):
         oracle_sample(st, [s % st.B], s)
     t = time.perf_counter()
@@ -926,71 +1258,19 @@ def run_reference(a, rank, world):
         nv += oracle_sample(st, [s % st.B], a.warmup + s)
     dt = time.perf_counter() - t
     value = nv / dt
-    line = {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+    line = {"metric": METRIC, "value": round(value, 4), "unit": cfg.unit, "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(dt / a.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": workload_name(a.batch, a.ctx, a.k, a.drafter_layers,
-                                                 a.target_layers), "batch": a.batch,
-                       "ctx": a.ctx, "k": a.k},
-            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": blas_threads(),
+            "config": {"workload": cfg.name(), "batch": cfg.B,
+                       "ctx": cfg.L if isinstance(cfg.L, int) else list(cfg.L), "k": cfg.k},
+            "cpu_baseline": {"value": round(value, 4), "unit": cfg.unit, "cores": blas_threads(),
                              "kind": "oracle",
                              "sample": "per step one sequence of the batch (round robin): the "
-                                       "full step for it in float64 on the host"},
-            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                                       "workload's full step for it in float64 on the host"},
+            "e2e": {"value": round(value, 4), "unit": cfg.unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
-
-
-class HostOnlyStep:
-    """The workload's host tensors only (for the CPU oracle arm)."""
-
-    def __init__(self, k, B, L, reserve=64, dense=False, target=False):
-        import torch
-
-        import synthetic as S
-        self.dense, self.target = dense, target
-        self.k, self.B, self.n_q = k, B, k + 1
-        self.hq, self.hkv, self.bs = 16, 4, 16
-        self.V, self.d, self.dh = 262144, 5376, 1024
-        self.C, self.cs, self.top_c = 1024, 256, 32
-        seed = 100
-        self.w = S.Workload("g", B, L, k, 16, 4, [S.AttnLayer(512), S.AttnLayer(256, 512)],
-                            self.d, self.V, seed=seed, n_clusters=self.C, cluster_size=self.cs,
-                            drafter_hidden=self.dh, top_c=self.top_c)
-        self.L0 = S.contexts(self.w)
-        mb = int((self.L0.max() + reserve + self.bs - 1) // self.bs)
-        self.host = {f"cache{layer}": S.make_cache(self.w, layer, self.L0, reserve=reserve,
-                                                   max_blocks=mb) for layer in (0, 1)}
-        inp = {}
-        for layer in (0, 1):
-            s = S.make_step_qkv(self.w, layer, self.n_q)
-            inp[f"q{layer}"], inp[f"kn{layer}"], inp[f"vn{layer}"] = s["q"], s["k_new"], s["v_new"]
-        inp["hidden"] = S.make_hidden(self.w, B * self.n_q)
-        for j in range(k):
-            for layer, D in ((0, 512), (1, 256)):
-                n = 1 if layer == 0 else 3
-                inp[f"dq{j}_{layer}"] = S.bf16(S.normal(seed * 31 + 10 * j + layer,
-                                                        (n, B, 1, self.hq, D), 1 / math.sqrt(D)))
-            inp[f"dh{j}"] = S.bf16(S.normal(seed * 37 + j, (B, self.dh)))
-        self.host_inputs = inp
-        self.host["cl"] = S.make_clustered_head(self.w)
-        self.host["W"] = None
-        f32 = lambda t: t.float().numpy()  # bf16 -> float32 is exact
-        if dense:
-            dw = S.make_drafter_weights(seed, self.dh, self.d, self.V, self.hq,
-                                        (256, 256, 256, 512))
-            self.host["drafter"] = {
-                "E": f32(dw["E"]), "W_in": f32(dw["W_in"]), "g_final": f32(dw["g_final"]),
-                "W_back": f32(dw["W_back"]),
-                "layers": [{kk: f32(v) for kk, v in lw.items()} for lw in dw["layers"]]}
-            self.host["h0"] = S.make_hidden(self.w, B, step=97)
-        if target:
-            tw = S.make_target_weights(seed, self.d, 4 * self.d, self.hq, self.hkv,
-                                       ((256, 512), (512, 0)))
-            self.host["target"] = [{kk: (f32(v) if hasattr(v, "float") else v)
-                                    for kk, v in lw.items()} for lw in tw]
-            inp["x0"] = torch.from_numpy(S.normal(seed * 41 + 5, (B * self.n_q, self.d)))
 
 
 if __name__ == "__main__":
