@@ -6,24 +6,22 @@
 // u_i < p_i(d_i) / q_i(d_i); at the first rejection emit x ~ norm(max(0, p_i - q_i)); if all
 // are accepted emit the bonus x ~ p_{k+1}.  T = 0: accept iff d_i == argmax, emit argmax.
 //
-// Two kernels:
-//  1. accept_decide: one thread-block cluster per sequence.  CTA c of the cluster streams
-//     token slice c of every logit row the sequence needs (its k+1 target rows and, for
-//     T > 0, its k draft rows) from HBM into shared memory with bulk copies (a 3-stage ring)
-//     and reduces each row slice: online max / sum of exp(x / T) (T > 0) or the top two values
-//     and the argmax (T = 0).  CTA 0 merges the slices' partials through distributed shared
-//     memory in rank order and takes the acceptance decisions; at T = 0 it writes the outputs,
-//     at T > 0 it writes the sequence's decision record (accepted count, margin flag, the
-//     normalisers of the draw row) for the draw kernel.
-//  2. accept_draw: one CTA per (sequence, token chunk), one wave of CTAs.  Exponential race of
-//     the draw row over the chunk: key_v = ln w_v - ln(-ln(1 - V_v)), V_v the token's Philox
-//     uniform, for the residual weights max(0, p - q) and for p (the bonus draw, and the
-//     fallback when the residual is empty).  Each race keeps its winner, the winner's lowest
-//     possible key and the highest possible key of every other token under the float32 error
-//     model of the margin rule.  The last CTA of a sequence (atomic ticket; no waiting) merges
-//     the chunk winners (lowest token id first on equal keys) and writes the outputs.
-//  A plain draw (k = 0, T > 0, the drafter sampling its own token) runs the draw kernel alone:
-//  its race keys are unnormalised logits / T, so no row statistics are needed.
+// Three kernels (a plain draw, k = 0 at T > 0, runs only the last):
+//  1. accept_stats: one CTA per (logit row, token chunk) over every row the sequences need (the
+//     k+1 target rows and, for T > 0, the k draft rows), sized to one wave of CTAs: online max /
+//     sum of exp(x / T) of the chunk (T > 0), or its top two values and the argmax (T = 0),
+//     with 16-byte loads kept in flight.
+//  2. accept_decide: one CTA per sequence merges the chunks of each row (a warp per row, fixed
+//     order), tests the k drafts lane-parallel and writes the sequence's decision record
+//     (accepted count, acceptance margin flag, the normalisers of the draw row); at T = 0 it
+//     writes the outputs itself.
+//  3. accept_draw: one CTA per (sequence, token chunk), one wave of CTAs.  Exponential race of
+//     the draw row over the chunk: key_v = log2 w_v - log2(-ln(1 - V_v)), V_v the token's
+//     Philox uniform, for the residual weights max(0, p - q) after a rejection or for p (the
+//     bonus draw, a plain draw).  The race keeps its winner, the winner's lowest possible key
+//     and the highest possible key of every other token under the float32 error model of the
+//     margin rule.  The last CTA of a sequence (atomic ticket; no waiting) merges the chunk
+//     winners (lowest token id first on equal keys) and writes the outputs.
 #include <cfloat>
 
 #include "common.cuh"
@@ -33,15 +31,19 @@
 namespace sdv {
 namespace acc {
 
-constexpr int kDecideThreads = 512;
-constexpr int kPiece = 16384;       // floats per bulk copy of the decision pass (64 KB)
-constexpr int kStages = 3;          // bulk-copy ring depth of the decision pass
+constexpr int kStatThreads = 256;
+constexpr int kChunk = 8192;        // tokens per statistics CTA at least
+constexpr int kDecideThreads = 256;
 constexpr int kMaxRows = 31;        // rows per sequence: 2k + 1 with k <= 15
 constexpr int kDrawSlots = 592;     // draw CTAs aimed at: one wave at 4 CTAs on each of 148 SMs
 constexpr int kDrawThreads = 256;
 constexpr float kMargin = 1e-4f;    // spec margin on |u - p/q|; also for draws, argmaxes
 constexpr float kRelP = 1e-5f;      // float32 error bound assumed on a probability p_v or q_v
 constexpr float kAbsKey = 1e-5f;    // float32 error bound assumed on ln E_v and z_v / T
+constexpr float kLog2e = 1.4426950408889634f;
+// the race keys are kept in log2 units: the natural-log margin and bounds scaled by log2(e)
+constexpr float kMargin2 = kMargin * kLog2e;
+constexpr float kAbsKey2 = kAbsKey * kLog2e;
 
 // Decision record of one sequence (T > 0): written by the decision kernel, read by the draw.
 struct Record {
@@ -55,10 +57,8 @@ struct Record {
 
 struct Params {
   int B, k, V, n_q, ld_t, ld_d, ld_o, purpose;
-  int rps;           // rows per sequence read by the decision pass
-  int cl;            // CTAs per sequence (the cluster) of the decision pass
-  int slice;         // tokens per CTA of the decision pass (a multiple of 4)
-  int npieces;       // bulk copies per row slice
+  int rps;           // rows per sequence read by the statistics pass
+  int nchunks, stats_chunk;
   int ndraw, draw_chunk;
   float T;
   unsigned long long seed;
@@ -70,6 +70,7 @@ struct Params {
   int32_t *n_acc;
   int32_t *out;
   int32_t *margin;
+  float4 *stats;           // [B * rps][nchunks] chunk partials
   Record *rec;             // [B]
   float4 *cand;            // [B][ndraw][3]
   unsigned int *counters;  // [B]
@@ -179,7 +180,7 @@ __device__ __forceinline__ Race race_shfl(const Race &c, int off) {
   return o;
 }
 
-__device__ __forceinline__ bool race_flag(const Race &r) { return r.hi2 > r.lo1 - kMargin; }
+__device__ __forceinline__ bool race_flag(const Race &r) { return r.hi2 > r.lo1 - kMargin2; }
 
 // (max, sum exp(x - max)) pairs
 __device__ __forceinline__ void ms_merge(float &m, float &s, float m2, float s2) {
@@ -198,175 +199,126 @@ __device__ __forceinline__ uint32_t counter_step(const Params &p) {
   return (uint32_t)(p.step + (p.step_ptr != nullptr ? *p.step_ptr : 0ull));
 }
 
+// ------------------------------------------------------------------ statistics kernel
+
+__global__ void __launch_bounds__(kStatThreads) accept_stats_kernel(const Params p) {
+  pdl_wait();  // many waves: no early trigger, so the next kernel does not take their slots
+  const int rr = blockIdx.x, c = blockIdx.y;
+  const int b = rr / p.rps, ri = rr - b * p.rps;
+  const float *row = seq_row(p, b, ri);
+  const int v0 = c * p.stats_chunk;
+  const int v1 = min(p.V, v0 + p.stats_chunk);
+  const float4 *row4 = reinterpret_cast<const float4 *>(row + v0);
+  const int n4 = max(0, v1 - v0) >> 2;
+  __shared__ float4 red[kStatThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (p.T > 0.f) {
+    // a batch of PER independent loads per thread, then their max, then the sum, merged
+    // online across batches
+    constexpr int PER = 8;
+    const float inv_t = 1.f / p.T;
+    float m = -INFINITY, s = 0.f;
+    for (int base = 0; base < n4; base += PER * kStatThreads) {
+      float4 x[PER];
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int i = base + threadIdx.x + u * kStatThreads;
+        x[u] = i < n4 ? __ldg(row4 + i)
+                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+      if (p.T != 1.f) {
+#pragma unroll
+        for (int u = 0; u < PER; ++u)
+          x[u] = make_float4(x[u].x * inv_t, x[u].y * inv_t, x[u].z * inv_t, x[u].w * inv_t);
+      }
+      float mb = -INFINITY, sb = 0.f;
+#pragma unroll
+      for (int u = 0; u < PER; ++u)
+        mb = fmaxf(mb, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
+      if (mb != -INFINITY) {
+        const float ml = mb * kLog2e;
+#pragma unroll
+        for (int u = 0; u < PER; ++u)
+          sb += (exp2f(fmaf(x[u].x, kLog2e, -ml)) + exp2f(fmaf(x[u].y, kLog2e, -ml))) +
+                (exp2f(fmaf(x[u].z, kLog2e, -ml)) + exp2f(fmaf(x[u].w, kLog2e, -ml)));
+      }
+      ms_merge(m, s, mb, sb);
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+      const float s2 = __shfl_xor_sync(0xffffffffu, s, off);
+      ms_merge(m, s, m2, s2);
+    }
+    if (lane == 0) red[warp] = make_float4(m, s, 0.f, 0.f);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float M = red[0].x, S = red[0].y;
+      for (int w = 1; w < kStatThreads / 32; ++w) ms_merge(M, S, red[w].x, red[w].y);
+      p.stats[(size_t)rr * p.nchunks + c] = make_float4(M, S, 0.f, 0.f);
+    }
+  } else {
+    Top2 cd{-INFINITY, -INFINITY, -1};
+    for (int i = threadIdx.x; i < n4; i += kStatThreads) {
+      const float4 x4 = __ldg(row4 + i);
+      const int v = v0 + 4 * i;
+      top2_push(cd, x4.x, v);
+      top2_push(cd, x4.y, v + 1);
+      top2_push(cd, x4.z, v + 2);
+      top2_push(cd, x4.w, v + 3);
+    }
+    for (int off = 16; off > 0; off >>= 1) cd = top2_merge(cd, top2_shfl(cd, off));
+    if (lane == 0) red[warp] = make_float4(cd.g1, __int_as_float(cd.v1), cd.g2, 0.f);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      Top2 t{red[0].x, red[0].z, __float_as_int(red[0].y)};
+      for (int w = 1; w < kStatThreads / 32; ++w)
+        t = top2_merge(t, Top2{red[w].x, red[w].z, __float_as_int(red[w].y)});
+      p.stats[(size_t)rr * p.nchunks + c] = make_float4(t.g1, __int_as_float(t.v1), t.g2, 0.f);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ decision kernel
 
-__global__ void __launch_bounds__(kDecideThreads, 1) accept_decide_kernel(const Params p) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  float *ring = reinterpret_cast<float *>(smem_raw);  // [kStages][piece]
-  __shared__ uint64_t full[kStages];
-  __shared__ float4 s_wpart[kMaxRows][kDecideThreads / 32];
-  __shared__ float4 s_part[kMaxRows];   // this CTA's slice partial of each row
-  __shared__ float4 s_row[kMaxRows];    // merged rows (CTA 0)
-  __shared__ int s_abort;
+__global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Params p) {
+  __shared__ float4 s_row[kMaxRows];  // merged rows
   __shared__ uint32_t s_step;
   pdl_wait();
-  const uint32_t rank = cluster_ctarank();
-  const int ncl = p.cl;       // CTAs per sequence: the cluster
-  const int b = blockIdx.x / ncl;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
-  const int v0 = (int)rank * p.slice;
-  const int v1 = min(p.V, v0 + p.slice);
-  const int n = max(0, v1 - v0);
-  const int piece = (n + p.npieces - 1) / p.npieces;
-  const int piece4 = (piece + 3) & ~3;
-  const int units = p.rps * p.npieces;
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool sampling = p.T > 0.f;
-
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
-    fence_mbar_init();
-    s_abort = 0;
-    if (rank == 0) s_step = counter_step(p);
+  if (threadIdx.x == 0) {
+    s_step = counter_step(p);
+    if (sampling) p.counters[b] = 0u;  // tickets of the draw kernel
+  }
+  // merge the chunks of each row (one warp per row, lanes over chunks, fixed order)
+  for (int ri = warp; ri < p.rps; ri += kDecideThreads / 32) {
+    const float4 *st = p.stats + (size_t)(b * p.rps + ri) * p.nchunks;
+    float4 v;
+    if (sampling) {
+      float M = -INFINITY, S = 0.f;
+      for (int c = lane; c < p.nchunks; c += 32) ms_merge(M, S, st[c].x, st[c].y);
+      for (int off = 16; off > 0; off >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, M, off);
+        const float s2 = __shfl_xor_sync(0xffffffffu, S, off);
+        ms_merge(M, S, m2, s2);
+      }
+      v = make_float4(M, S, 0.f, 0.f);
+    } else {
+      Top2 t{-INFINITY, -INFINITY, -1};
+      for (int c = lane; c < p.nchunks; c += 32)
+        t = top2_merge(t, Top2{st[c].x, st[c].z, __float_as_int(st[c].y)});
+      for (int off = 16; off > 0; off >>= 1) t = top2_merge(t, top2_shfl(t, off));
+      v = make_float4(t.g1, __int_as_float(t.v1), t.g2, 0.f);
+    }
+    if (lane == 0) s_row[ri] = v;
   }
   __syncthreads();
-  // unit u = (row u / npieces, piece u % npieces); its tokens [v0 + piece4 * pc, ...)
-  auto unit_range = [&](int u, int &ri, int &t0, int &cnt) {
-    ri = u / p.npieces;
-    const int pc = u - ri * p.npieces;
-    t0 = v0 + pc * piece4;
-    cnt = max(0, min(v1, t0 + piece4) - t0);
-  };
-  auto issue = [&](int u) {
-    int ri, t0, cnt;
-    unit_range(u, ri, t0, cnt);
-    const int s = u % kStages;
-    if (cnt > 0) {
-      mbar_arrive_expect_tx(&full[s], (uint32_t)cnt * 4u);
-      bulk_load(ring + (size_t)s * piece4, seq_row(p, b, ri) + t0, (uint32_t)cnt * 4u, &full[s]);
-    } else {
-      mbar_arrive(&full[s]);
-    }
-  };
-  if (tid == 0)
-    for (int u = 0; u < kStages && u < units; ++u) issue(u);
-
-  constexpr float L2E = 1.4426950408889634f;
-  const float inv_t = sampling ? 1.f / p.T : 1.f;
-  // per-warp partial of the current row, merged over its pieces
-  float wm = -INFINITY, ws = 0.f;
-  Top2 wt{-INFINITY, -INFINITY, -1};
-  int last_issued = min(kStages, units) - 1;  // (thread 0) the latest unit copied
-  for (int u = 0; u < units; ++u) {
-    const int s = u % kStages;
-    int ri, t0, cnt;
-    unit_range(u, ri, t0, cnt);
-    if (s_abort == 0 && !mbar_wait(&full[s], (u / kStages) & 1, &s_abort)) {
-      record_status(p.status, SD_ERR_TIMEOUT);
-      s_abort = 1;
-    }
-    if (s_abort == 0) {
-      const float *buf = ring + (size_t)s * piece4;
-      const int n4 = cnt >> 2;
-      const float4 *buf4 = reinterpret_cast<const float4 *>(buf);
-      if (sampling) {
-        float m = -INFINITY, sm = 0.f;
-        for (int i = tid; i < n4; i += blockDim.x) {
-          float4 x = buf4[i];
-          if (p.T != 1.f) x = make_float4(x.x * inv_t, x.y * inv_t, x.z * inv_t, x.w * inv_t);
-          const float mb = fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w));
-          if (mb == -INFINITY) continue;
-          if (mb > m) {
-            sm *= exp2f((m - mb) * L2E);
-            m = mb;
-          }
-          sm += (exp2f((x.x - m) * L2E) + exp2f((x.y - m) * L2E)) +
-                (exp2f((x.z - m) * L2E) + exp2f((x.w - m) * L2E));
-        }
-        for (int off = 16; off > 0; off >>= 1) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
-          const float s2 = __shfl_xor_sync(0xffffffffu, sm, off);
-          ms_merge(m, sm, m2, s2);
-        }
-        ms_merge(wm, ws, m, sm);
-      } else {
-        Top2 c{-INFINITY, -INFINITY, -1};
-        for (int i = tid; i < n4; i += blockDim.x) {
-          const float4 x = buf4[i];
-          const int v = t0 + 4 * i;
-          top2_push(c, x.x, v);
-          top2_push(c, x.y, v + 1);
-          top2_push(c, x.z, v + 2);
-          top2_push(c, x.w, v + 3);
-        }
-        for (int off = 16; off > 0; off >>= 1) c = top2_merge(c, top2_shfl(c, off));
-        wt = top2_merge(wt, c);
-      }
-    }
-    const bool row_end = (u + 1) % p.npieces == 0;
-    if (row_end && lane == 0) {
-      s_wpart[ri][warp] = sampling ? make_float4(wm, ws, 0.f, 0.f)
-                                   : make_float4(wt.g1, __int_as_float(wt.v1), wt.g2, 0.f);
-    }
-    if (row_end) {
-      wm = -INFINITY;
-      ws = 0.f;
-      wt = Top2{-INFINITY, -INFINITY, -1};
-    }
-    __syncthreads();  // every thread is done with stage s: refill it
-    if (tid == 0 && u + kStages < units && s_abort == 0) {
-      issue(u + kStages);
-      last_issued = u + kStages;
-    }
-  }
-  if (s_abort != 0 && tid == 0) {
-    // drain the copies still in flight (the latest one per stage) before the shared memory is
-    // released
-    for (int j = max(0, last_issued - kStages + 1); j <= last_issued; ++j)
-      mbar_wait_timed(&full[j % kStages], (j / kStages) & 1);
-  }
-  // this CTA's partial of each row (warps merged in order)
-  if (tid < p.rps) {
-    float4 r = s_wpart[tid][0];
-    for (int w = 1; w < nwarps; ++w) {
-      const float4 o = s_wpart[tid][w];
-      if (sampling) {
-        ms_merge(r.x, r.y, o.x, o.y);
-      } else {
-        const Top2 t = top2_merge(Top2{r.x, r.z, __float_as_int(r.y)},
-                                  Top2{o.x, o.z, __float_as_int(o.y)});
-        r = make_float4(t.g1, __int_as_float(t.v1), t.g2, 0.f);
-      }
-    }
-    s_part[tid] = r;
-  }
-  cluster_sync();  // every CTA's partials are visible to CTA 0
-  if (rank == 0) {
-    // merge the slices of row w in rank order (one warp per row)
-    for (int ri = warp; ri < p.rps; ri += nwarps) {
-      float4 v = lane < ncl ? ld_dsmem_f4(dsmem_addr(smem_u32(&s_part[ri]), lane))
-                            : (sampling ? make_float4(-INFINITY, 0.f, 0.f, 0.f)
-                                        : make_float4(-INFINITY, __int_as_float(-1), -INFINITY,
-                                                      0.f));
-      if (sampling) {
-        for (int off = 16; off > 0; off >>= 1) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, v.x, off);
-          const float s2 = __shfl_xor_sync(0xffffffffu, v.y, off);
-          ms_merge(v.x, v.y, m2, s2);
-        }
-      } else {
-        Top2 t{v.x, v.z, __float_as_int(v.y)};
-        for (int off = 16; off > 0; off >>= 1) t = top2_merge(t, top2_shfl(t, off));
-        v = make_float4(t.g1, __int_as_float(t.v1), t.g2, 0.f);
-      }
-      if (lane == 0) s_row[ri] = v;
-    }
-  }
-  cluster_sync();  // CTA 0 has read the other CTAs' shared memory: they may exit
-  if (rank != 0 || warp != 0) return;
+  if (warp != 0) return;
 
   // ---- decisions (one warp): lane i-1 tests draft i; the first rejection stops the scan
   const uint32_t step = s_step;
+  const float inv_t = sampling ? 1.f / p.T : 1.f;
   bool acc = true;
   int flag = 0;
   if (lane < p.k) {
@@ -416,118 +368,153 @@ __global__ void __launch_bounds__(kDecideThreads, 1) accept_decide_kernel(const 
   r.my = sy.x;
   r.isy = 1.f / sy.y;
   p.rec[b] = r;
-  p.counters[b] = 0u;  // tickets of the draw kernel
 }
 
 // ------------------------------------------------------------------ draw kernel
 
-__global__ void __launch_bounds__(kDrawThreads) accept_draw_kernel(const Params p) {
+// One token of the race: adds its key and bounds to the race state (log2 units).
+//   draw from p (resid == false): key = zt log2(e) - lg2 E, bounds key -/+ 1e-5 (1 + |zt|)
+//   residual (resid == true): key = lg2 w - lg2 E (w = max(0, p - q) > 0), its lower bound from
+//   w - s and the upper bound of every token from w + s, s = 1e-5 (p + q), each -/+ 1e-5;
+//   pb, the bare p race without bounds, keeps a fallback winner for an empty residual.
+__device__ __forceinline__ void race_token(bool resid, float zt, float w, float sl, float lgE,
+                                           int v, Race &cr, Race &pb) {
+  if (!resid) {
+    if (zt == -INFINITY) return;
+    const float g = fmaf(zt, kLog2e, -lgE);
+    const float err = kAbsKey2 * (1.f + fabsf(zt));
+    race_push(cr, g, g - err, g + err, v);
+    return;
+  }
+  if (zt != -INFINITY) {
+    const float g = fmaf(zt, kLog2e, -lgE);
+    if (g > pb.g1) {
+      pb.g1 = g;
+      pb.v1 = v;
+    }
+  }
+  if (w + sl > 0.f) {
+    const float hi = __log2f(w + sl) - lgE + kAbsKey2;
+    const float g = w > 0.f ? __log2f(w) - lgE : -INFINITY;
+    if (g > cr.g1) {
+      const float wl = w - sl;
+      race_push(cr, g, wl > 0.f ? __log2f(wl) - lgE - kAbsKey2 : -INFINITY, hi, v);
+    } else {
+      cr.hi2 = fmaxf(cr.hi2, hi);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kDrawThreads, 4) accept_draw_kernel(const Params p) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x, c = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __shared__ Record s_rec;
   __shared__ Race s_red[2][kDrawThreads / 32];
   __shared__ int s_last;
 
-  if (threadIdx.x == 0) {
-    if (p.k == 0) {  // plain draw: no decisions, unnormalised keys
-      s_rec = Record{0, 0, counter_step(p), 0, 0.f, 1.f, 0.f, 1.f};
-    } else {
-      s_rec = p.rec[b];
-    }
+  // every thread reads the record itself (one broadcast load): no barrier before the loads
+  Record rec;
+  if (p.k == 0) {  // plain draw: no decisions, unnormalised keys
+    rec = Record{0, 0, 0u, 0, 0.f, 1.f, 0.f, 1.f};
+  } else {
+    rec = p.rec[b];
   }
-  __syncthreads();
-  const int a = s_rec.a;
-  const uint32_t step = s_rec.step;
+  const int a = rec.a;
   const bool resid = a < p.k;
   const int rt = b * p.n_q + a;
   const float *zr = p.z + (size_t)rt * p.ld_t;
   const float *yr = resid ? p.y + ((size_t)b * p.k + a) * p.ld_d : nullptr;
-  const float isz = s_rec.isz, isy = s_rec.isy;
   const int v0 = c * p.draw_chunk;
   const int v1 = min(p.V, v0 + p.draw_chunk);
   const int n4 = max(0, v1 - v0) >> 2;
-  Race cp = race_empty(), cr = race_empty();
-  // Keys in float32 with fast exp2 / log where the error (<~1e-6 absolute on a key, <~1e-6
-  // relative on p and q) is far inside the error model the bounds assume (1e-5); the log1p of
-  // the uniform stays accurate because small uniforms decide the winners.
-  constexpr float L2E = 1.4426950408889634f;
+  // Keys in float32 with fast exp2 / log2 where the error (<~1e-6 absolute on a key, <~1e-6
+  // relative on p and q) is far inside the error model the bounds assume (1e-5); the -ln(1 - V)
+  // of the uniform stays accurate because small uniforms decide the winners.
   const bool unit_t = p.T == 1.f;
   const float inv_t = 1.f / p.T;
-  const float mzl = s_rec.mz * L2E, myl = s_rec.my * L2E;
-  for (int i = threadIdx.x; i < n4; i += kDrawThreads) {
-    const int v = v0 + 4 * i;
-    const float4 z4 = __ldg(reinterpret_cast<const float4 *>(zr + v));
-    float4 y4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (resid) y4 = __ldg(reinterpret_cast<const float4 *>(yr + v));
-    const float zz[4] = {z4.x, z4.y, z4.z, z4.w};
-    const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
-    float zt[4], w[4], sl[4];
-    bool any = false;
+  const float isz = rec.isz, isy = rec.isy;
+  const float mzl = rec.mz * kLog2e, myl = rec.my * kLog2e;
+  Race cr = race_empty();
+  Race pb = race_empty();  // bare p race (residual fallback), g1 / v1 only
+  constexpr int PER = 2;   // float4 groups whose loads are issued together
+  uint32_t step = rec.step;
+  bool have_step = p.k != 0;
+  for (int base = 0; base < n4; base += PER * kDrawThreads) {
+    float4 z4[PER], y4[PER];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      zt[e] = unit_t ? zz[e] : zz[e] * inv_t;
-      w[e] = 0.f;
-      sl[e] = 0.f;
-      if (resid) {
-        const float yt = unit_t ? yy[e] : yy[e] * inv_t;
-        const float pv = ex2_approx(fmaf(zt[e], L2E, -mzl)) * isz;
-        const float qv = ex2_approx(fmaf(yt, L2E, -myl)) * isy;
-        w[e] = fmaxf(pv - qv, 0.f);
-        sl[e] = kRelP * (pv + qv);
-      }
-      any |= zt[e] != -INFINITY || w[e] + sl[e] > 0.f;
+    for (int u = 0; u < PER; ++u) {
+      const int i = base + threadIdx.x + u * kDrawThreads;
+      z4[u] = i < n4 ? __ldg(reinterpret_cast<const float4 *>(zr + v0) + i)
+                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      y4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (resid && i < n4) y4[u] = __ldg(reinterpret_cast<const float4 *>(yr + v0) + i);
     }
-    if (!any) continue;  // no token of the group has any weight: no uniforms needed
-    float U[4];
-    token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1), U[0],
-                       U[1]);
-    token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1) + 1u,
-                       U[2], U[3]);
+    if (!have_step) {  // a plain draw reads the step counter behind its first loads
+      step = counter_step(p);
+      have_step = true;
+    }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float lnE = __logf(neg_log1m(U[e]));  // E == 0 gives -inf: that token wins
-      if (zt[e] != -INFINITY) {
-        const float g = zt[e] - lnE;
-        const float err = kAbsKey * (1.f + fabsf(zt[e]));
-        race_push(cp, g, g - err, g + err, v + e);
-      }
-      if (resid && w[e] + sl[e] > 0.f) {
-        const float hi = __logf(w[e] + sl[e]) - lnE + kAbsKey;
-        const float g = w[e] > 0.f ? __logf(w[e]) - lnE : -INFINITY;
-        if (g > cr.g1) {
-          const float wl = w[e] - sl[e];
-          race_push(cr, g, wl > 0.f ? __logf(wl) - lnE - kAbsKey : -INFINITY, hi, v + e);
+    for (int u = 0; u < PER; ++u) {
+      const int i = base + threadIdx.x + u * kDrawThreads;
+      if (i >= n4) break;
+      const int v = v0 + 4 * i;
+      const float zz[4] = {z4[u].x, z4[u].y, z4[u].z, z4[u].w};
+      const float yy[4] = {y4[u].x, y4[u].y, y4[u].z, y4[u].w};
+      float zt[4], w[4], sl[4];
+      bool any = false;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        zt[e] = unit_t ? zz[e] : zz[e] * inv_t;
+        w[e] = 0.f;
+        sl[e] = 0.f;
+        if (resid) {
+          const float yt = unit_t ? yy[e] : yy[e] * inv_t;
+          const float pv = ex2_approx(fmaf(zt[e], kLog2e, -mzl)) * isz;
+          const float qv = ex2_approx(fmaf(yt, kLog2e, -myl)) * isy;
+          w[e] = fmaxf(pv - qv, 0.f);
+          sl[e] = kRelP * (pv + qv);
+          any |= w[e] + sl[e] > 0.f;
         } else {
-          cr.hi2 = fmaxf(cr.hi2, hi);
+          any |= zt[e] != -INFINITY;
         }
+      }
+      if (!any) continue;  // no token of the group has any weight: no uniforms needed
+      float U[4];
+      token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1),
+                         U[0], U[1]);
+      token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose,
+                         (uint32_t)(v >> 1) + 1u, U[2], U[3]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lgE = __log2f(neg_log1m(U[e]));  // E == 0 gives -inf: that token wins
+        race_token(resid, zt[e], w[e], sl[e], lgE, v + e, cr, pb);
       }
     }
   }
   for (int off = 16; off > 0; off >>= 1) {
-    const Race o1 = race_shfl(cp, off);
-    cp = (lane & off) ? race_merge(o1, cp) : race_merge(cp, o1);
+    const Race o1 = race_shfl(cr, off);
+    cr = (lane & off) ? race_merge(o1, cr) : race_merge(cr, o1);
     if (resid) {
-      const Race o2 = race_shfl(cr, off);
-      cr = (lane & off) ? race_merge(o2, cr) : race_merge(cr, o2);
+      const Race o2 = race_shfl(pb, off);
+      pb = (lane & off) ? race_merge(o2, pb) : race_merge(pb, o2);
     }
   }
   if (lane == 0) {
-    s_red[0][warp] = cp;
-    s_red[1][warp] = cr;
+    s_red[0][warp] = cr;
+    s_red[1][warp] = pb;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    Race tp = s_red[0][0], tr = s_red[1][0];
+    Race tr = s_red[0][0], tp = s_red[1][0];
     for (int w = 1; w < kDrawThreads / 32; ++w) {
-      tp = race_merge(tp, s_red[0][w]);
-      tr = race_merge(tr, s_red[1][w]);
+      tr = race_merge(tr, s_red[0][w]);
+      tp = race_merge(tp, s_red[1][w]);
     }
     float4 *slot = p.cand + ((size_t)b * p.ndraw + c) * 3;
-    slot[0] = make_float4(tp.g1, tp.lo1, tp.hi1, tp.hi2);
-    slot[1] = make_float4(tr.g1, tr.lo1, tr.hi1, tr.hi2);
-    slot[2] = make_float4(__int_as_float(tp.v1), __int_as_float(tr.v1), 0.f, 0.f);
+    slot[0] = make_float4(tr.g1, tr.lo1, tr.hi1, tr.hi2);
+    slot[1] = make_float4(tp.g1, tp.lo1, tp.hi1, tp.hi2);
+    slot[2] = make_float4(__int_as_float(tr.v1), __int_as_float(tp.v1), 0.f, 0.f);
     __threadfence();
     const unsigned int ticket = atomicAdd(&p.counters[b], 1u);
     s_last = ticket == (unsigned int)(p.ndraw - 1);
@@ -538,31 +525,29 @@ __global__ void __launch_bounds__(kDrawThreads) accept_draw_kernel(const Params 
   // ---- last CTA of the sequence: merge the chunk winners (order-independent: equal keys go to
   // the lower token id), one warp
   if (threadIdx.x >= 32) return;
-  const volatile float4 *cv = reinterpret_cast<const volatile float4 *>(p.cand) +
-                              (size_t)b * p.ndraw * 3;
-  Race tp = race_empty(), tr = race_empty();
+  const float4 *cv = p.cand + (size_t)b * p.ndraw * 3;
+  Race tr = race_empty(), tp = race_empty();
   for (int cc = lane; cc < p.ndraw; cc += 32) {
-    const float4 a0 = make_float4(cv[3 * cc].x, cv[3 * cc].y, cv[3 * cc].z, cv[3 * cc].w);
-    const float4 a1 =
-        make_float4(cv[3 * cc + 1].x, cv[3 * cc + 1].y, cv[3 * cc + 1].z, cv[3 * cc + 1].w);
-    const float ix = cv[3 * cc + 2].x, iy = cv[3 * cc + 2].y;
-    tp = race_merge(tp, Race{a0.x, a0.y, a0.z, a0.w, __float_as_int(ix)});
-    tr = race_merge(tr, Race{a1.x, a1.y, a1.z, a1.w, __float_as_int(iy)});
+    const float4 a0 = __ldcg(cv + 3 * cc);
+    const float4 a1 = __ldcg(cv + 3 * cc + 1);
+    const float4 id = __ldcg(cv + 3 * cc + 2);
+    tr = race_merge(tr, Race{a0.x, a0.y, a0.z, a0.w, __float_as_int(id.x)});
+    tp = race_merge(tp, Race{a1.x, a1.y, a1.z, a1.w, __float_as_int(id.y)});
   }
   for (int off = 16; off > 0; off >>= 1) {
-    tp = race_merge(tp, race_shfl(tp, off));
     tr = race_merge(tr, race_shfl(tr, off));
+    tp = race_merge(tp, race_shfl(tp, off));
   }
   if (lane != 0) return;
-  // the residual race unless every residual weight came out 0 (then p, and the draw is flagged:
-  // a residual too small for float32 may still be positive)
-  const bool use_r = resid && tr.v1 >= 0;
-  const Race &w = use_r ? tr : tp;
-  int flag = s_rec.flag;
-  if (race_flag(w) || (resid && !use_r)) flag = 1;
+  // the residual race unless every residual weight came out 0: then the bare race over p, and
+  // the draw is flagged (a residual too small for float32 may still be positive)
+  const bool empty = resid && tr.v1 < 0;
+  const int x = empty ? tp.v1 : tr.v1;
+  int flag = rec.flag;
+  if (empty || race_flag(tr)) flag = 1;
   int32_t *o = p.out + (size_t)b * p.ld_o;
   for (int j = 0; j < p.n_q; ++j)
-    o[j] = j < a ? p.drafts[(size_t)b * p.k + j] : (j == a ? w.v1 : -1);
+    o[j] = j < a ? p.drafts[(size_t)b * p.k + j] : (j == a ? x : -1);
   p.n_acc[b] = a;
   if (p.margin) p.margin[b] = flag;
   p.counters[b] = 0u;
@@ -602,82 +587,38 @@ static int ndraw_of(int B, int V) {
   return (V + c - 1) / c;
 }
 
-// Clusters of each size (1, 2, 4, 8, 16 CTAs per sequence) the device holds at once for the
-// decision kernel at one CTA per SM (looked up once per device; 0 where a size cannot run).
-static const int *active_clusters(size_t smem) {
-  static int cache[64][5];
-  static bool done[64];
+static int nchunks_of(int V) { return (V + kChunk - 1) / kChunk; }
+
+// Tokens per CTA of the statistics pass: kChunk, or more (multiples of 1024) when the rows
+// times kChunk-token chunks would not fit in one wave of CTAs.  Never more chunks per row than
+// nchunks_of(V), which sizes the workspace.
+static int stats_chunk_of(int rows, int V) {
+  static int occ_cache[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (done[dev]) return cache[dev];
-  cudaFuncSetAttribute(accept_decide_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  cudaFuncSetAttribute(accept_decide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)smem);
-  for (int i = 0; i < 5; ++i) {
-    const int cl = 1 << i;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cl, 1, 1);
-    cfg.blockDim = dim3(kDecideThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, accept_decide_kernel, &cfg) != cudaSuccess) n = 0;
-    cache[dev][i] = n;
+  cudaGetDevice(&dev);
+  int occ = dev >= 0 && dev < 64 ? occ_cache[dev] : 0;
+  if (occ <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, accept_stats_kernel, kStatThreads,
+                                                      0) != cudaSuccess ||
+        occ <= 0)
+      occ = 1;
+    if (dev >= 0 && dev < 64) occ_cache[dev] = occ;
   }
-  cudaGetLastError();
-  done[dev] = true;
-  return cache[dev];
-}
-
-// Launch shape of the decision pass: cluster size (CTAs per sequence), tokens per CTA, bulk
-// copies per row slice and the thread count.  As many CTAs per sequence as keep B x cluster
-// within one CTA per SM (every CTA streams with a 3 x 64 KB ring), at least 1024 tokens each.
-struct DecideShape {
-  int cl, slice, npieces, threads;
-  size_t smem;
-};
-
-static DecideShape decide_shape(int B, int V) {
-  DecideShape s;
-  const size_t full_smem = (size_t)kStages * kPiece * 4;
-  // cluster size: fewest waves of clusters per CTA-slice of the vocabulary, i.e. the smallest
-  // ceil(B / resident clusters) / cl; at least 1024 tokens per CTA
-  const int *act = active_clusters(full_smem);
-  int cl = 1;
-  double best = -1.0;
-  for (int i = 0; i < 5; ++i) {
-    const int c = 1 << i;
-    if (c > 1 && (V + c - 1) / c < 1024) break;
-    const int n = act != nullptr ? act[i] : (c == 1 ? 1 : 0);
-    if (n <= 0) continue;
-    const double cost = (double)((B + n - 1) / n) / c;
-    if (best < 0.0 || cost <= best) {
-      best = cost;
-      cl = c;
-    }
-  }
-  s.cl = cl;
-  int slice = (V + cl - 1) / cl;
-  slice = (slice + 3) & ~3;
-  s.slice = slice;
-  s.npieces = (slice + kPiece - 1) / kPiece;
-  const int piece = ((slice + s.npieces - 1) / s.npieces + 3) & ~3;
-  // threads: enough for one float4 per thread of a piece, 32 .. kDecideThreads
-  int th = (piece / 4 + 31) / 32 * 32;
-  s.threads = th < 32 ? 32 : (th > kDecideThreads ? kDecideThreads : th);
-  s.smem = (size_t)kStages * piece * 4;
-  return s;
+  const int sms = sm_count();
+  const long long slots = (long long)occ * (sms > 0 ? sms : 148);
+  long long n = slots / (rows > 0 ? rows : 1);
+  if (n < 1) n = 1;
+  if (n > nchunks_of(V)) n = nchunks_of(V);
+  int chunk = (int)((V + n - 1) / n);
+  chunk = (chunk + 1023) / 1024 * 1024;
+  return chunk < kChunk ? kChunk : chunk;
 }
 
 static size_t ws_size(const sd_accept_desc *d) {
   if (validate(d) != SD_OK) return 0;
-  return round_up((size_t)d->batch * sizeof(Record), 256) +
+  const size_t rows = (size_t)d->batch * (2 * d->k + 1);
+  return round_up(rows * nchunks_of(d->vocab) * 16, 256) +
+         round_up((size_t)d->batch * sizeof(Record), 256) +
          round_up((size_t)d->batch * ndraw_of(d->batch, d->vocab) * 48, 256) +
          round_up((size_t)d->batch * 4, 256);
 }
@@ -727,6 +668,8 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.out = out_tokens;
   p.margin = margin_flags;
   uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
+  p.stats = reinterpret_cast<float4 *>(w8);
+  w8 += round_up((size_t)p.B * (2 * p.k + 1) * nchunks_of(p.V) * 16, 256);
   p.rec = reinterpret_cast<Record *>(w8);
   w8 += round_up((size_t)p.B * sizeof(Record), 256);
   p.cand = reinterpret_cast<float4 *>(w8);
@@ -740,25 +683,13 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
         cudaSuccess)
       return SD_ERR_CUDA;
   } else {
-    const DecideShape ds = decide_shape(p.B, p.V);
-    p.cl = ds.cl;
-    p.slice = ds.slice;
-    p.npieces = ds.npieces;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ds.cl * p.B, 1, 1);
-    cfg.blockDim = dim3(ds.threads, 1, 1);
-    cfg.dynamicSmemBytes = ds.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = ds.cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    if (cudaLaunchKernelEx(&cfg, accept_decide_kernel, p) != cudaSuccess) return SD_ERR_CUDA;
+    p.stats_chunk = stats_chunk_of(p.B * p.rps, p.V);
+    p.nchunks = (p.V + p.stats_chunk - 1) / p.stats_chunk;
+    if (launch(accept_stats_kernel, dim3(p.B * p.rps, p.nchunks), dim3(kStatThreads), 0, st,
+               p) != cudaSuccess)
+      return SD_ERR_CUDA;
+    if (launch(accept_decide_kernel, dim3(p.B), dim3(kDecideThreads), 0, st, p) != cudaSuccess)
+      return SD_ERR_CUDA;
     if (!sampling) return SD_OK;  // greedy: the decision pass wrote the outputs
   }
   return cuda_status(
