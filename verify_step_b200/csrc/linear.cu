@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(kStageThreads) linear_stage_kernel(const Param
   __shared__ int s_tok;
   __shared__ float s_red[kStageThreads / 32];
   __shared__ float s_inv;
+  pdl_trigger();  // the product kernel may start its weight copies meanwhile
   pdl_wait();
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -223,7 +224,11 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // x' comes from the staging kernel
+  // x' and the tickets come from the staging kernel, which this kernel may overlap (it is
+  // launched as its programmatic dependent): every role waits for it before touching global
+  // memory, except that the producer first requests the weights of its first stages (the
+  // weights are not written by the staging kernel)
+  if (warp != 0) pdl_wait();
 
   if (warp == 0) {
     // ----------------------------------------------------------------------- producer
@@ -232,6 +237,25 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch_desc(&xmap);
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
+      // the first STAGES stages (fresh barriers: no wait for a free stage): weights now,
+      // x' rows once the staging kernel is done
+      int pre_kb[STAGES];
+      uint32_t pre = 0;
+      for (int u = blockIdx.x; u < p.units && pre < (uint32_t)STAGES; u += gridDim.x) {
+        const int tile = u / p.splits, split = u % p.splits;
+        const int kb0 = split * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1 && pre < (uint32_t)STAGES; ++kb, ++pre) {
+          uint8_t *a = smem + (size_t)pre * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
+          tma_load_2d_hint(a, &wmap, &full[pre], kb * BK, tile * BM, pol_w);
+          pre_kb[pre] = kb;
+        }
+      }
+      pdl_wait();
+      for (uint32_t j = 0; j < pre; ++j)
+        tma_load_2d_hint(smem + (size_t)j * C::STAGE_BYTES + C::A_BYTES, &xmap, &full[j],
+                         pre_kb[j] * BK, 0, pol_x);
       uint32_t g = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
@@ -239,6 +263,7 @@ __global__ void __launch_bounds__(192, 1)
         const int kb0 = split * p.kb_per_split;
         const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb, ++g) {
+          if (g < pre) continue;  // requested above
           const int stage = g % STAGES;
           const uint32_t ph = (g / STAGES) & 1;
           if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) {
@@ -472,6 +497,8 @@ static sd_status validate(const sd_linear_desc *d, const void *x, const void *W,
   return SD_OK;
 }
 
+// The product is launched as a programmatic dependent of the staging kernel (always: the two
+// are one call), so its launch, set-up and first weight copies overlap the staging.
 template <int N>
 static sd_status launch_product(const CUtensorMap &wm, const CUtensorMap &xm, const Params &p,
                                 int grid, cudaStream_t st) {
@@ -485,8 +512,17 @@ static sd_status launch_product(const CUtensorMap &wm, const CUtensorMap &xm, co
       return SD_ERR_CUDA;
     if (dev < 64) configured[dev] = dev + 1;
   }
-  return cuda_status(
-      launch(linear_umma_kernel<N>, dim3(grid), dim3(C::THREADS), C::SMEM, st, wm, xm, p));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, linear_umma_kernel<N>, wm, xm, p));
 }
 
 }  // namespace lin
