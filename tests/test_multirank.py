@@ -32,7 +32,7 @@ def _worker(rank, world, port, out):
 
 def test_time_is_the_slowest_rank_and_rate_counts_every_rank():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork after threads have started
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     for rank in range(world):
         ms, rate = out[rank]

@@ -1304,49 +1304,115 @@ __global__ void append_kv_kernel(const Params p, const T *k_new, const T *v_new,
 }
 
 // float32 path: one warp per (sequence, query position, head).
-__global__ void attn_f32_kernel(const Params p, const float *k_cache, const float *v_cache) {
+// One CTA per query row; warp w takes the row's keys lo + w, lo + w + kF32Warps, ... with the
+// lanes over the head dimension.  The block ids of the next 32 keys of a warp are fetched
+// lane-parallel, and the K and V rows of kF32Unroll keys are loaded together, so a warp has
+// several keys' loads in flight.  Each warp keeps its own online softmax; the warps' (m, l, o)
+// are merged in warp order through shared memory.
+constexpr int kF32Warps = 8;
+constexpr int kF32Unroll = 4;
+
+__global__ void __launch_bounds__(32 * kF32Warps) attn_f32_kernel(const Params p,
+                                                                  const float *k_cache,
+                                                                  const float *v_cache) {
+  __shared__ float s_ml[kF32Warps][2];
+  __shared__ float s_o[kF32Warps][512];
   pdl_wait();
-  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int total = p.B * p.n_q * p.Hq;
-  if (wid >= total) return;
-  const int h = wid % p.Hq;
-  const int j = (wid / p.Hq) % p.n_q;
-  const int b = wid / (p.Hq * p.n_q);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row_id = blockIdx.x;  // (b, j, h)
+  const int h = row_id % p.Hq;
+  const int j = (row_id / p.Hq) % p.n_q;
+  const int b = row_id / (p.Hq * p.n_q);
   const int g = h / p.G;
-  const SeqRange s = seq_range(p, b, lane == 0);
+  const SeqRange s = seq_range(p, b, threadIdx.x == 0);
   int lo, hi;
   row_range(p, s, b, j * p.G + (h % p.G), lo, hi);
   constexpr int MAXE = 16;  // D <= 512
   const int per = p.D / 32;
-  const float *qv = reinterpret_cast<const float *>(p.q) + (((size_t)b * p.n_q + j) * p.Hq + h) * p.D;
+  const float *qv =
+      reinterpret_cast<const float *>(p.q) + (((size_t)b * p.n_q + j) * p.Hq + h) * p.D;
   float qr[MAXE], acc[MAXE];
+#pragma unroll
   for (int e = 0; e < MAXE; ++e) {
     qr[e] = e < per ? qv[lane + 32 * e] : 0.f;
     acc[e] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  for (int pos = lo; pos <= hi; ++pos) {
-    const int blk = p.table[(size_t)b * p.mbps + pos / p.bs];
-    if (blk < 0 || blk >= p.num_blocks) {
-      if (lane == 0) record_status(p.status, SD_ERR_DEVICE);
-      continue;
+  const int nk = hi >= lo ? hi - lo + 1 : 0;
+  const int mine = nk > warp ? (nk - warp + kF32Warps - 1) / kF32Warps : 0;  // this warp's keys
+  for (int base = 0; base < mine; base += 32) {
+    // block ids of keys base .. base + 31 of this warp, one per lane
+    int blk_l = -1;
+    if (base + lane < mine) {
+      const int pos = lo + warp + kF32Warps * (base + lane);
+      blk_l = p.table[(size_t)b * p.mbps + pos / p.bs];
+      if (blk_l < 0 || blk_l >= p.num_blocks) {
+        record_status(p.status, SD_ERR_DEVICE);
+        blk_l = -1;
+      }
     }
-    const size_t row = (((size_t)blk * p.Hkv + g) * p.bs + pos % p.bs) * p.D;
-    float dot = 0.f;
-    for (int e = 0; e < per; ++e) dot = fmaf(qr[e], k_cache[row + lane + 32 * e], dot);
-    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    const float x = dot * p.scale;
-    const float m_new = fmaxf(m, x);
-    const float alpha = expf(m - m_new);
-    const float w = expf(x - m_new);
-    l = l * alpha + w;
-    for (int e = 0; e < per; ++e) acc[e] = acc[e] * alpha + w * v_cache[row + lane + 32 * e];
-    m = m_new;
+    const int cnt = min(32, mine - base);
+    for (int i0 = 0; i0 < cnt; i0 += kF32Unroll) {
+      float kr[kF32Unroll][MAXE], vr[kF32Unroll][MAXE];
+      bool valid[kF32Unroll];
+#pragma unroll
+      for (int u = 0; u < kF32Unroll; ++u) {
+        const int i = i0 + u;
+        const int blk = __shfl_sync(0xffffffffu, blk_l, i < cnt ? i : 0);
+        valid[u] = i < cnt && blk >= 0;
+        const int pos = lo + warp + kF32Warps * (base + i);
+        const size_t row = valid[u] ? (((size_t)blk * p.Hkv + g) * p.bs + pos % p.bs) * p.D : 0;
+#pragma unroll
+        for (int e = 0; e < MAXE; ++e) {
+          kr[u][e] = (valid[u] && e < per) ? k_cache[row + lane + 32 * e] : 0.f;
+          vr[u][e] = (valid[u] && e < per) ? v_cache[row + lane + 32 * e] : 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kF32Unroll; ++u) {
+        if (!valid[u]) continue;  // warp-uniform
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < MAXE; ++e) dot = fmaf(qr[e], kr[u][e], dot);
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        const float x = dot * p.scale;
+        const float m_new = fmaxf(m, x);
+        const float alpha = expf(m - m_new);
+        const float w = expf(x - m_new);
+        l = l * alpha + w;
+#pragma unroll
+        for (int e = 0; e < MAXE; ++e) acc[e] = acc[e] * alpha + w * vr[u][e];
+        m = m_new;
+      }
+    }
+  }
+  // merge the warps in order
+  if (lane == 0) {
+    s_ml[warp][0] = m;
+    s_ml[warp][1] = l;
+  }
+#pragma unroll
+  for (int e = 0; e < MAXE; ++e)
+    if (e < per) s_o[warp][lane + 32 * e] = acc[e];
+  __syncthreads();
+  if (warp != 0) return;
+  float M = -INFINITY;
+  for (int w = 0; w < kF32Warps; ++w) M = fmaxf(M, s_ml[w][0]);
+  float L = 0.f, o[MAXE];
+#pragma unroll
+  for (int e = 0; e < MAXE; ++e) o[e] = 0.f;
+  for (int w = 0; w < kF32Warps; ++w) {
+    const float sc = s_ml[w][0] == -INFINITY ? 0.f : expf(s_ml[w][0] - M);
+    L += s_ml[w][1] * sc;
+#pragma unroll
+    for (int e = 0; e < MAXE; ++e)
+      if (e < per) o[e] += s_o[w][lane + 32 * e] * sc;
   }
   float *ov = reinterpret_cast<float *>(p.out) + (((size_t)b * p.n_q + j) * p.Hq + h) * p.D;
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  for (int e = 0; e < per; ++e) ov[lane + 32 * e] = acc[e] * inv;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int e = 0; e < MAXE; ++e)
+    if (e < per) ov[lane + 32 * e] = o[e] * inv;
 }
 
 // ------------------------------------------------------------------------------- host side
@@ -1567,9 +1633,8 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
                  (float *)v_cache) != cudaSuccess)
         return SD_ERR_CUDA;
     }
-    const int warps = p.B * p.n_q * p.Hq;
-    return cuda_status(launch(attn_f32_kernel, dim3((warps + 3) / 4), dim3(128), 0, st, p,
-                              (const float *)k_cache, (const float *)v_cache));
+    return cuda_status(launch(attn_f32_kernel, dim3(p.B * p.n_q * p.Hq), dim3(32 * kF32Warps),
+                              0, st, p, (const float *)k_cache, (const float *)v_cache));
   }
 
   // bf16

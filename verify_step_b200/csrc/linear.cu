@@ -385,16 +385,28 @@ __global__ void __launch_bounds__(192, 1)
       named_barrier(1, 128);
       if (*s_last) {
         __threadfence();
-        const int s0 = u - u % p.splits;  // first unit of the tile
-#pragma unroll 1
-        for (int r = 0; r < N; ++r) {
-          float acc = 0.f;
-          if (r < p.m) {
-            for (int s = 0; s < p.splits; ++s)
-              acc += __ldcg(p.part + ((size_t)(s0 + s) * N + r) * BM + row_in_tile);
+        const int own = u % p.splits;
+        const int s0 = u - own;  // first unit of the tile
+        // partials added in split order; each split's N loads are issued together (this
+        // split's own partial is still in registers)
+        float acc[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) acc[r] = 0.f;
+        for (int sp = 0; sp < p.splits; ++sp) {
+          if (sp == own) {
+#pragma unroll
+            for (int r = 0; r < N; ++r) acc[r] += y[r];
+            continue;
           }
-          apply_epilogue(p, row, r, acc, lane);
+          const float *src = p.part + (size_t)(s0 + sp) * N * BM + row_in_tile;
+          float v[N];
+#pragma unroll
+          for (int r = 0; r < N; ++r) v[r] = r < p.m ? __ldcg(src + (size_t)r * BM) : 0.f;
+#pragma unroll
+          for (int r = 0; r < N; ++r) acc[r] += v[r];
         }
+#pragma unroll
+        for (int r = 0; r < N; ++r) apply_epilogue(p, row, r, acc[r], lane);
         if (threadIdx.x == 64) p.tickets[tile] = 0u;
       }
     }
@@ -421,24 +433,28 @@ struct Shape {
 
 static int n_of(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 48 ? 48 : 64; }
 
-// Work split of a call: S splits of the K blocks per 128-row tile, chosen to minimise the
-// K blocks of the busiest SM (ceil(tiles S / SMs) units of ceil(kblocks / S) blocks), a split
-// costing about one K block more (its partial write and the reduction).
+// Work split of a call: S splits of the K blocks per 128-row tile, chosen to minimise a time
+// model of the busiest SM: ceil(tiles S / SMs) units, each its K blocks at about 0.36 us (16 KB
+// of weights and 4 KB of x' at a fair share of the HBM rate) plus, when split, about 2.5 us of
+// partial write, fence and ticket; and the reductions the SM finishes (ceil(tiles / SMs) tiles,
+// about 0.5 us per split read back).
 static Shape shape_of(int m, int n, int k) {
   Shape s;
   s.N = n_of(m);
   s.tiles = (n + BM - 1) / BM;
   s.kblocks = (k + BK - 1) / BK;
   const int sms = std::max(sm_count(), 1);
-  long long best = -1;
+  double best = -1.0;
   int best_s = 1;
   for (int S = 1; S <= std::min(kMaxSplits, s.kblocks); ++S) {
     const int kps = (s.kblocks + S - 1) / S;
     const int S_eff = (s.kblocks + kps - 1) / kps;  // every split non-empty
     if (S_eff != S) continue;
     const long long units = (long long)s.tiles * S;
-    const long long cost = (units + sms - 1) / sms * (long long)kps + (S > 1 ? 1 : 0);
-    if (best < 0 || cost < best) {
+    const double per_unit = kps * 0.36 + (S > 1 ? 2.5 : 0.0);
+    double cost = (double)((units + sms - 1) / sms) * per_unit;
+    if (S > 1) cost += (double)((s.tiles + sms - 1) / sms) * 0.5 * S;
+    if (best < 0.0 || cost < best) {
       best = cost;
       best_s = S;
     }
