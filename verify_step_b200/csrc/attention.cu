@@ -15,11 +15,14 @@
 //    [num_blocks, h_kv, block_size, D] layout) into shared memory once, by TMA
 //    (cp.async.bulk.tensor, 128-byte swizzle, no multicast), through an mbarrier ring.
 //  * The tile is reused by every query row of the item: the G query heads of the kv head times
-//    the n_q verify positions (M = G * n_q rows, padded to 16-row MMA tiles).
-//  * Compute warps own (16-row tile, D slice of 128 columns).  Q K^T partials over the slices
-//    are summed through shared memory (fixed order, so every warp of a row tile gets the same
-//    scores); the online softmax and P V run in registers on bf16 mma.sync tensor cores with
-//    float32 accumulation.
+//    the n_q verify positions (M = G * n_q rows, up to 24 per CTA in 8-row blocks; larger items
+//    take groups of CTAs streaming the same tiles).
+//  * Compute warps own a D slice of 128 columns.  Keys are the M side of the bf16 mma.sync
+//    tensor-core products (S^T = K Q^T, O^T += V^T P^T, float32 accumulation) and query rows
+//    the N side, so few rows cost little padding.  S^T partials over the slices are summed
+//    through shared memory (fixed order, so every warp gets the same scores); the online
+//    softmax runs in registers, masking only the tiles at a row's range ends and rescaling only
+//    when a row maximum grows by more than 2^8.
 //  * Items split across CTAs leave (m, l, o) partials in the workspace; a combine kernel merges
 //    them in CTA order (deterministic).  Items one CTA finishes are written directly.
 //
@@ -36,7 +39,8 @@ constexpr int kTile = 16;
 constexpr float kRescale = 8.f;  // log2 headroom of the lazily rescaled softmax
 
 struct Params {
-  int B, n_q, Hq, Hkv, G, D, bs, mbps, num_blocks, window, M, Mpad;
+  int B, n_q, Hq, Hkv, G, D, bs, mbps, num_blocks, window, M;
+  int Mpad;          // rows of a workspace slot (split-KV kernel)
   int is_draft;
   int q_offset;      // query position ctx_len[b] + q_offset when q_pos is null
   float scale_log2;  // scale * log2(e)
@@ -56,7 +60,7 @@ struct Params {
   void *k_cache;
   void *v_cache;
   int P;           // CTA groups of the persistent split-KV grid (stream-K units)
-  int row_groups;  // CTAs per group: each takes one 16-row query tile of the same tile range
+  int row_groups;  // CTAs per group: each takes one row group of the item, same tile range
   int *status;
 };
 
@@ -266,27 +270,44 @@ __device__ __forceinline__ bool patch_new_rows(const Params &p, int b, int g, in
   return true;
 }
 
-template <int D, int MT, int STAGES>
+// Split-KV tile shape: query rows are the MMA's N dimension in blocks of 8 (NB blocks per CTA),
+// keys its M dimension (one 16-key tile), so an item of up to 24 rows (k + 1 = 6 positions at
+// G = 4) is one CTA's work and needs no padding beyond the next multiple of 8.
+template <int D, int NB, int STAGES>
 struct Cfg {
   static constexpr int DS = D >= 128 ? 128 : 64;
-  static constexpr int NDG = D / DS;
-  static constexpr int NCW = MT * NDG;
+  static constexpr int NDG = D / DS;  // compute warps, one D slice each
+  static constexpr int NCW = NDG;
   static constexpr int THREADS = 32 * (NCW + 1);
+  static constexpr int ROWS = 8 * NB;
   static constexpr int TILE_BYTES = kTile * D * 2;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int RED_FLOATS = 2 * NCW * 32 * 8;
+  static constexpr int RED_FLOATS = NDG > 1 ? 2 * NCW * 32 * 4 * NB : 4;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + RED_FLOATS * 4 +
                                  16 * STAGES + 16 + 4 * (1 + STAGES) + 64 + sizeof(SeqTab) + 16;
-  // two independent tile pipelines per SM where registers allow (one CTA's per-tile chain
-  // of waits, MMAs and the cross-warp score exchange is latency-bound on its own)
-  static constexpr int MIN_CTAS = NCW <= 4 ? 2 : 1;
+  // two independent tile pipelines per SM (one CTA's per-tile chain of waits, MMAs and the
+  // cross-warp score exchange is latency-bound on its own)
+  static constexpr int MIN_CTAS = 2;
 };
 
-template <int D, int MT, int STAGES>
-__global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES>::MIN_CTAS)
+// Rows per CTA group for an item of M query rows: groups of at most 24 rows (three 8-row
+// blocks), R groups of NB blocks each.
+struct RowSplit {
+  int R, NB;
+};
+__host__ __device__ inline RowSplit row_split(int M) {
+  RowSplit s;
+  s.R = (M + 23) / 24;
+  const int per = (M + s.R - 1) / s.R;
+  s.NB = (per + 7) / 8;
+  return s;
+}
+
+template <int D, int NB, int STAGES>
+__global__ void __launch_bounds__(Cfg<D, NB, STAGES>::THREADS, Cfg<D, NB, STAGES>::MIN_CTAS)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const Params p) {
-  using C = Cfg<D, MT, STAGES>;
+  using C = Cfg<D, NB, STAGES>;
   constexpr int DS = C::DS, NDG = C::NDG, NCW = C::NCW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -319,7 +340,7 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   __syncthreads();
 
   const long long T = total_tiles(p, tab);
-  // CTAs come in groups of row_groups that stream the same tile range, one query tile each
+  // CTAs come in groups of row_groups that stream the same tile range, one row group each
   // (the group's repeated reads of a tile are served by L2)
   const int grp = blockIdx.x / p.row_groups, rg = blockIdx.x % p.row_groups;
   const long long start = T * grp / p.P;
@@ -388,9 +409,15 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
   }
 
   // --------------------------------------------------------------------- compute warps
-  const int mg = warp / NDG, dg = warp % NDG;
-  const int r0 = (rg * MT + mg) * 16 + (lane >> 2);  // rows r0 and r0 + 8 of the item
-  const int kq = 2 * (lane & 3);         // column pair inside an 8-wide n tile
+  // Per tile the warp computes S^T = K Q^T over its D slice (keys as M = 16, the CTA's query
+  // rows as N in 8-row blocks), the slices are summed through shared memory, and
+  // O^T += V^T P^T over the slice (D columns as M, rows as N, the tile's keys as K).  In the
+  // accumulator layout a lane holds keys kr and kr + 8 (S^T) or D columns kr and kr + 8 (O^T),
+  // each for query rows rq and rq + 1 of every 8-row block.
+  const int dg = warp;
+  const int kr = lane >> 2;
+  const int rq = 2 * (lane & 3);
+  const int row0 = rg * C::ROWS;  // first query row of the item this CTA takes
   const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(p.q);
 
   Cursor c;
@@ -407,38 +434,56 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     const bool whole = (t_begin == 0 && seg_n == c.s.n);
     const SeqRange s = c.s;
 
-    uint32_t qa[DS / 16][4];
+    // Q^T as the B operand: block nb holds query row row0 + nb*8 + kr, columns rq, rq + 1
+    // (and + 8) of each 16-column step
+    uint32_t qb[DS / 16][NB][2];
 #pragma unroll
-    for (int ks = 0; ks < DS / 16; ++ks) {
+    for (int ks = 0; ks < DS / 16; ++ks)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = r0 + ((e & 1) ? 8 : 0);
-        const int col = dg * DS + ks * 16 + kq + ((e & 2) ? 8 : 0);
-        uint32_t v = 0;
-        if (row < p.M) {
-          const int j = row / p.G, hh = row % p.G;
-          const size_t off = (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D + col;
-          v = *reinterpret_cast<const uint32_t *>(qg + off);
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int row = row0 + nb * 8 + kr;
+          const int col = dg * DS + ks * 16 + rq + 8 * h;
+          uint32_t v = 0;
+          if (row < p.M) {
+            const int j = row / p.G, hh = row % p.G;
+            const size_t off =
+                (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D + col;
+            v = *reinterpret_cast<const uint32_t *>(qg + off);
+          }
+          qb[ks][nb][h] = v;
         }
-        qa[ks][e] = v;
+    // keys every real row of this CTA may read: tiles inside [lo_all, hi_all] need no mask
+    int lo_all = 1, hi_all = 0;
+    {
+      const int r_last = min(row0 + C::ROWS, p.M) - 1;
+      if (r_last >= row0) {
+        int lo_a, hi_a, lo_b, hi_b;
+        row_range(p, s, b, row0, lo_a, hi_a);
+        row_range(p, s, b, r_last, lo_b, hi_b);
+        lo_all = max(lo_a, lo_b);
+        hi_all = min(hi_a, hi_b);
       }
     }
-    int lo0, hi0, lo1, hi1;
-    row_range(p, s, b, r0, lo0, hi0);
-    row_range(p, s, b, r0 + 8, lo1, hi1);
 
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.f, 0.f};
-    float o[DS / 8][4];
+    float m_run[NB][2], l_run[NB][2];
+    float o[DS / 16][NB][4];
 #pragma unroll
-    for (int nt = 0; nt < DS / 8; ++nt)
+    for (int nb = 0; nb < NB; ++nb) {
+      m_run[nb][0] = m_run[nb][1] = -INFINITY;
+      l_run[nb][0] = l_run[nb][1] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+      for (int mb = 0; mb < DS / 16; ++mb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[mb][nb][e] = 0.f;
+    }
 
     for (int t = 0; t < seg_n; ++t) {
       const int stage = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
-      if (!mbar_wait(&full[stage], ph, abort_flag)) {
+      // (the warp leaves together: its later shuffles and votes need every lane)
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], ph, abort_flag))) {
         record_status(p.status, SD_ERR_TIMEOUT);
         *abort_flag = 1;
         ok = false;
@@ -449,142 +494,127 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
       const uint32_t vbase = kbase + C::TILE_BYTES;
       const int p0 = (s.tf + t_begin + t) * kTile;
 
-      // ---- partial S = Q K^T over this warp's D slice
-      float sp[2][4];
+      // ---- partial S^T = K Q^T over this warp's D slice
+      float sc[NB][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sp[nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) sc[nb][e] = 0.f;
+      {
+        const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int coff = (lane >> 4) * 8;
 #pragma unroll
-      for (int ks = 0; ks < DS / 16; ++ks) {
-        const int d0 = dg * DS + ks * 16;
-        uint32_t kb[4];
-        const int key = ((lane >> 4) << 3) + (lane & 7);
-        const int col = d0 + ((lane >> 3) & 1) * 8;
-        ldsm_x4(kb, kbase + swz(key, col));
-        mma_bf16_16816(sp[0], qa[ks], kb[0], kb[1]);
-        mma_bf16_16816(sp[1], qa[ks], kb[2], kb[3]);
-      }
-      float *myred = red + ((size_t)(buf * NCW + warp) * 32 + lane) * 8;
-      reinterpret_cast<float4 *>(myred)[0] = make_float4(sp[0][0], sp[0][1], sp[0][2], sp[0][3]);
-      reinterpret_cast<float4 *>(myred)[1] = make_float4(sp[1][0], sp[1][1], sp[1][2], sp[1][3]);
-      mbar_arrive(&red_bar[buf]);
-      if (!mbar_wait(&red_bar[buf], (it >> 1) & 1, abort_flag)) {
-        record_status(p.status, SD_ERR_TIMEOUT);
-        *abort_flag = 1;
-        ok = false;
-        break;
-      }
-      float sc[2][4];
+        for (int ks = 0; ks < DS / 16; ++ks) {
+          uint32_t ka[4];
+          ldsm_x4(ka, kbase + swz(key, dg * DS + ks * 16 + coff));
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-#pragma unroll
-      for (int dd = 0; dd < NDG; ++dd) {
-        const float *src = red + ((size_t)(buf * NCW + mg * NDG + dd) * 32 + lane) * 8;
-        const float4 a = reinterpret_cast<const float4 *>(src)[0];
-        const float4 bq = reinterpret_cast<const float4 *>(src)[1];
-        sc[0][0] += a.x;
-        sc[0][1] += a.y;
-        sc[0][2] += a.z;
-        sc[0][3] += a.w;
-        sc[1][0] += bq.x;
-        sc[1][1] += bq.y;
-        sc[1][2] += bq.z;
-        sc[1][3] += bq.w;
-      }
-      buf ^= 1;
-
-      // ---- mask, online softmax (base-2 exponent with the scale folded in)
-      float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int pos = p0 + nt * 8 + kq + (e & 1);
-          const int lo = (e & 2) ? lo1 : lo0, hi = (e & 2) ? hi1 : hi0;
-          const bool valid = !is_bad && pos >= lo && pos <= hi;
-          const float x = valid ? sc[nt][e] * p.scale_log2 : -INFINITY;
-          sc[nt][e] = x;
-          mx[e >> 1] = fmaxf(mx[e >> 1], x);
+          for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(sc[nb], ka, qb[ks][nb][0], qb[ks][nb][1]);
         }
-      if constexpr (MT == 1) {
-        // one query tile: the kernel streams at the memory's pace, rescale every tile
-        float alpha[2];
+      }
+      if constexpr (NDG > 1) {
+        float4 *myred = reinterpret_cast<float4 *>(red) + ((buf * NCW + warp) * 32 + lane) * NB;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-          const float m_new = fmaxf(m_run[h], mx[h]);
-          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          alpha[h] = exp2f(m_run[h] - m_use);
-          m_run[h] = m_new;
-          l_run[h] *= alpha[h];
-          mx[h] = m_use;
+        for (int nb = 0; nb < NB; ++nb)
+          myred[nb] = make_float4(sc[nb][0], sc[nb][1], sc[nb][2], sc[nb][3]);
+        mbar_arrive(&red_bar[buf]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&red_bar[buf], (it >> 1) & 1, abort_flag))) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+          break;
         }
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float pv = exp2f(sc[nt][e] - mx[e >> 1]);
-            sc[nt][e] = pv;
-            l_run[e >> 1] += pv;
+          for (int e = 0; e < 4; ++e) sc[nb][e] = 0.f;
+#pragma unroll
+        for (int dd = 0; dd < NDG; ++dd) {
+          const float4 *src = reinterpret_cast<const float4 *>(red) + ((buf * NCW + dd) * 32 + lane) * NB;
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const float4 a = src[nb];
+            sc[nb][0] += a.x;
+            sc[nb][1] += a.y;
+            sc[nb][2] += a.z;
+            sc[nb][3] += a.w;
           }
-#pragma unroll
-        for (int nt = 0; nt < DS / 8; ++nt) {
-          o[nt][0] *= alpha[0];
-          o[nt][1] *= alpha[0];
-          o[nt][2] *= alpha[1];
-          o[nt][3] *= alpha[1];
         }
+        buf ^= 1;
+      }
+
+      // ---- scale (base-2 exponent), mask on the tiles that need it
+      if (!is_bad && p0 >= lo_all && p0 + kTile - 1 <= hi_all) {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nb][e] *= p.scale_log2;
       } else {
-        // several query tiles make the kernel issue-bound: a row's exponent base moves only
-        // when a tile's maximum passes it by more than kRescale (the unscaled terms then stay
-        // below 2^kRescale), so the accumulators are rescaled on few tiles and the warp skips
-        // the rescale otherwise
-        bool grow = false;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-          mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-          grow |= mx[h] > m_run[h] + kRescale;
-        }
-        if (__any_sync(0xffffffffu, grow)) {
-          float alpha[2];
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            alpha[h] = 1.f;
-            if (mx[h] > m_run[h] + kRescale) {  // a finite maximum always passes -inf
-              alpha[h] = m_run[h] == -INFINITY ? 0.f : ex2_approx(m_run[h] - mx[h]);
-              m_run[h] = mx[h];
+            int lo, hi;
+            row_range(p, s, b, row0 + nb * 8 + rq + h, lo, hi);
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const int pos = p0 + kr + 8 * kk;
+              const bool valid = !is_bad && pos >= lo && pos <= hi;
+              sc[nb][2 * kk + h] = valid ? sc[nb][2 * kk + h] * p.scale_log2 : -INFINITY;
             }
-            l_run[h] *= alpha[h];
-          }
-#pragma unroll
-          for (int nt = 0; nt < DS / 8; ++nt) {
-            o[nt][0] *= alpha[0];
-            o[nt][1] *= alpha[0];
-            o[nt][2] *= alpha[1];
-            o[nt][3] *= alpha[1];
-          }
-        }
-        const float base0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
-        const float base1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float pv = ex2_approx(sc[nt][e] - ((e & 2) ? base1 : base0));
-            sc[nt][e] = pv;
-            l_run[e >> 1] += pv;
           }
       }
-      uint32_t pa[4];
-      pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
-      pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
-      pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
-      pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+
+      // ---- online softmax, rescaled lazily: a row's exponent base moves only when a tile's
+      // maximum passes it by more than kRescale (the unscaled terms then stay below
+      // 2^kRescale), so the accumulators are rescaled on few tiles
+      {
+        float xm[NB][2];
+        bool grow = false;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            xm[nb][h] = fmaxf(sc[nb][h], sc[nb][h + 2]);
+            grow |= xm[nb][h] > m_run[nb][h] + kRescale;
+          }
+        if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float x = xm[nb][h];
+              x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+              x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+              x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+              if (x > m_run[nb][h] + kRescale) {  // a finite maximum always passes -inf
+                const float alpha =
+                    m_run[nb][h] == -INFINITY ? 0.f : ex2_approx(m_run[nb][h] - x);
+                m_run[nb][h] = x;
+                l_run[nb][h] *= alpha;
+#pragma unroll
+                for (int mb = 0; mb < DS / 16; ++mb) {
+                  o[mb][nb][h] *= alpha;
+                  o[mb][nb][h + 2] *= alpha;
+                }
+              }
+            }
+        }
+      }
+      uint32_t pb[NB][2];
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        float pv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float base = m_run[nb][e & 1] == -INFINITY ? 0.f : m_run[nb][e & 1];
+          pv[e] = ex2_approx(sc[nb][e] - base);
+          l_run[nb][e & 1] += pv[e];
+        }
+        // P^T (keys x rows, this lane: keys kr / kr + 8, rows rq, rq + 1) transposed in
+        // registers into the B operand (keys rq, rq + 1 / + 8, row kr)
+        pb[nb][0] = movmatrix_trans(pack_bf16x2(pv[0], pv[1]));
+        pb[nb][1] = movmatrix_trans(pack_bf16x2(pv[2], pv[3]));
+      }
 
       // ---- V rows no query of the item may read can hold anything (rolled-back or never
       // written slots, NaN included); zero this warp's slice of them so 0 * V stays 0.
@@ -612,16 +642,17 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
         }
       }
 
-      // ---- O += P V over this warp's D slice
+      // ---- O^T += V^T P^T over this warp's D slice
+      {
+        const int key = (lane & 7) + (lane >> 4) * 8;
+        const int coff = ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int np = 0; np < DS / 16; ++np) {
-        const int d0 = dg * DS + np * 16;
-        uint32_t vb[4];
-        const int key = ((lane >> 3) & 1) * 8 + (lane & 7);
-        const int col = d0 + (lane >> 4) * 8;
-        ldsm_x4_trans(vb, vbase + swz(key, col));
-        mma_bf16_16816(o[2 * np], pa, vb[0], vb[1]);
-        mma_bf16_16816(o[2 * np + 1], pa, vb[2], vb[3]);
+        for (int mb = 0; mb < DS / 16; ++mb) {
+          uint32_t va[4];
+          ldsm_x4_trans(va, vbase + swz(key, dg * DS + mb * 16 + coff));
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(o[mb][nb], va, pb[nb][0], pb[nb][1]);
+        }
       }
       mbar_arrive(&empty[stage]);
       ++it;
@@ -629,44 +660,54 @@ __global__ void __launch_bounds__(Cfg<D, MT, STAGES>::THREADS, Cfg<D, MT, STAGES
     if (!ok) break;
 
     // ---- segment end: final rows or a partial for the combine kernel
-    float l_tot[2];
+    float l_tot[NB][2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float l = l_run[h];
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      l_tot[h] = l;
-    }
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float l = l_run[nb][h];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        l_tot[nb][h] = l;
+      }
     if (whole) {
       __nv_bfloat16 *outg = reinterpret_cast<__nv_bfloat16 *>(p.out);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = r0 + 8 * h;
-        if (row >= p.M) continue;
-        const int j = row / p.G, hh = row % p.G;
-        const float inv = l_tot[h] > 0.f ? 1.f / l_tot[h] : 0.f;
-        __nv_bfloat16 *dst =
-            outg + (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D + dg * DS + kq;
+      for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int nt = 0; nt < DS / 8; ++nt)
-          *reinterpret_cast<uint32_t *>(dst + nt * 8) =
-              pack_bf16x2(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
-      }
+        for (int h = 0; h < 2; ++h) {
+          const int row = row0 + nb * 8 + rq + h;
+          if (row >= p.M) continue;
+          const int j = row / p.G, hh = row % p.G;
+          const float inv = l_tot[nb][h] > 0.f ? 1.f / l_tot[nb][h] : 0.f;
+          __nv_bfloat16 *dst =
+              outg + (((size_t)b * p.n_q + j) * p.Hq + (size_t)g * p.G + hh) * D + dg * DS + kr;
+#pragma unroll
+          for (int mb = 0; mb < DS / 16; ++mb) {
+            dst[mb * 16] = __float2bfloat16_rn(o[mb][nb][h] * inv);
+            dst[mb * 16 + 8] = __float2bfloat16_rn(o[mb][nb][h + 2] * inv);
+          }
+        }
     } else {
       const size_t slot = (size_t)b * p.Hkv + g + grp;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = r0 + 8 * h;
-        if (row >= p.M) continue;
-        float *dst = p.ws_o + (slot * p.Mpad + row) * D + dg * DS + kq;
+      for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int nt = 0; nt < DS / 8; ++nt)
-          *reinterpret_cast<float2 *>(dst + nt * 8) = make_float2(o[nt][2 * h], o[nt][2 * h + 1]);
-        if (dg == 0 && (lane & 3) == 0) {
-          p.ws_ml[(slot * p.Mpad + row) * 2 + 0] = m_run[h];
-          p.ws_ml[(slot * p.Mpad + row) * 2 + 1] = l_tot[h];
+        for (int h = 0; h < 2; ++h) {
+          const int row = row0 + nb * 8 + rq + h;
+          if (row >= p.M) continue;
+          float *dst = p.ws_o + (slot * p.Mpad + row) * D + dg * DS + kr;
+#pragma unroll
+          for (int mb = 0; mb < DS / 16; ++mb) {
+            dst[mb * 16] = o[mb][nb][h];
+            dst[mb * 16 + 8] = o[mb][nb][h + 2];
+          }
+          if (dg == 0 && kr == 0) {
+            p.ws_ml[(slot * p.Mpad + row) * 2 + 0] = m_run[nb][h];
+            p.ws_ml[(slot * p.Mpad + row) * 2 + 1] = l_tot[nb][h];
+          }
         }
-      }
     }
     c.tau += seg_n;
     c.left -= seg_n;
@@ -1417,22 +1458,22 @@ __global__ void __launch_bounds__(32 * kF32Warps) attn_f32_kernel(const Params p
 
 // ------------------------------------------------------------------------------- host side
 
-template <int D, int MT, int STAGES>
+template <int D, int NB, int STAGES>
 struct Launcher {
-  using C = Cfg<D, MT, STAGES>;
+  using C = Cfg<D, NB, STAGES>;
   static int ctas_per_sm() {
     static int dev_cache[64];
     static int occ_cache[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && dev_cache[dev] == dev + 1) return occ_cache[dev];
-    cudaFuncSetAttribute(attn_bf16_kernel<D, MT, STAGES>,
+    cudaFuncSetAttribute(attn_bf16_kernel<D, NB, STAGES>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    cudaFuncSetAttribute(attn_bf16_kernel<D, MT, STAGES>,
+    cudaFuncSetAttribute(attn_bf16_kernel<D, NB, STAGES>,
                          cudaFuncAttributePreferredSharedMemoryCarveout,
                          (int)cudaSharedmemCarveoutMaxShared);
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_bf16_kernel<D, MT, STAGES>,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_bf16_kernel<D, NB, STAGES>,
                                                       C::THREADS, C::SMEM) != cudaSuccess)
       occ = 0;
     if (dev < 64) {
@@ -1444,7 +1485,7 @@ struct Launcher {
   static sd_status launch(const CUtensorMap &km, const CUtensorMap &vm, const Params &p,
                           cudaStream_t st) {
     return cuda_status(
-        sdv::launch(attn_bf16_kernel<D, MT, STAGES>, dim3(p.P * p.row_groups), dim3(C::THREADS),
+        sdv::launch(attn_bf16_kernel<D, NB, STAGES>, dim3(p.P * p.row_groups), dim3(C::THREADS),
                     C::SMEM, st,
                     km, vm, p));
   }
@@ -1452,23 +1493,27 @@ struct Launcher {
 
 #define SDV_STAGES(D) ((D) == 512 ? 3 : (D) == 256 ? 4 : (D) == 128 ? 6 : 8)
 
-// Persistent CTAs for a (head_dim, row tiles) pair on the current device.
-static int persistent_ctas(int D, int MT) {
+// Persistent CTAs for a (head_dim, 8-row blocks) pair on the current device.
+static int persistent_ctas(int D, int NB) {
   int occ = 0;
-#define SDV_CASE(DD, MM)                                      \
-  if (D == DD && MT == MM) occ = Launcher<DD, MM, SDV_STAGES(DD)>::ctas_per_sm();
+#define SDV_CASE(DD, NN) \
+  if (D == DD && NB == NN) occ = Launcher<DD, NN, SDV_STAGES(DD)>::ctas_per_sm();
   SDV_CASE(64, 1) SDV_CASE(128, 1) SDV_CASE(256, 1) SDV_CASE(512, 1)
+  SDV_CASE(64, 2) SDV_CASE(128, 2) SDV_CASE(256, 2) SDV_CASE(512, 2)
+  SDV_CASE(64, 3) SDV_CASE(128, 3) SDV_CASE(256, 3) SDV_CASE(512, 3)
 #undef SDV_CASE
   const int sms = sm_count();
   if (occ <= 0 || sms <= 0) return 0;
   return occ * sms;
 }
 
-static sd_status launch_bf16(int D, int MT, const CUtensorMap &km, const CUtensorMap &vm,
+static sd_status launch_bf16(int D, int NB, const CUtensorMap &km, const CUtensorMap &vm,
                              const Params &p, cudaStream_t st) {
-#define SDV_CASE(DD, MM) \
-  if (D == DD && MT == MM) return Launcher<DD, MM, SDV_STAGES(DD)>::launch(km, vm, p, st);
+#define SDV_CASE(DD, NN) \
+  if (D == DD && NB == NN) return Launcher<DD, NN, SDV_STAGES(DD)>::launch(km, vm, p, st);
   SDV_CASE(64, 1) SDV_CASE(128, 1) SDV_CASE(256, 1) SDV_CASE(512, 1)
+  SDV_CASE(64, 2) SDV_CASE(128, 2) SDV_CASE(256, 2) SDV_CASE(512, 2)
+  SDV_CASE(64, 3) SDV_CASE(128, 3) SDV_CASE(256, 3) SDV_CASE(512, 3)
 #undef SDV_CASE
   return SD_ERR_UNSUPPORTED;
 }
@@ -1576,20 +1621,19 @@ static sd_status validate(const sd_attn_desc *d, bool draft) {
   return SD_OK;
 }
 
-// Stream-K groups of the split-KV kernel: the single-tile kernel's persistent CTAs, divided
-// into groups of one CTA per 16-row query tile.
+// Stream-K groups of the split-KV kernel: its persistent CTAs, divided into groups of one CTA
+// per row group of the item.
 static int grid_ctas(const sd_attn_desc *d) {
   if (d->dtype != SD_BF16) return 0;
-  const int G = d->h_q / d->h_kv;
-  const int MT = (G * d->n_q + 15) / 16;
-  return persistent_ctas(d->head_dim, 1) / MT;
+  const RowSplit rs = row_split(d->h_q / d->h_kv * d->n_q);
+  return persistent_ctas(d->head_dim, rs.NB) / rs.R;
 }
 
 static size_t ws_size(const sd_attn_desc *d) {
   if (validate(d, false) != SD_OK && validate(d, true) != SD_OK) return 0;
   if (d->dtype != SD_BF16) return 0;
-  const int G = d->h_q / d->h_kv;
-  const int Mpad = (G * d->n_q + 15) / 16 * 16;
+  const RowSplit rs = row_split(d->h_q / d->h_kv * d->n_q);
+  const int Mpad = rs.R * 8 * rs.NB;
   const size_t slots = (size_t)d->batch * d->h_kv + (size_t)grid_ctas(d);
   return round_up(slots * Mpad * d->head_dim * 4, 256) + round_up(slots * Mpad * 2 * 4, 256);
 }
@@ -1614,7 +1658,6 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   p.num_blocks = d->num_blocks;
   p.window = d->window > 0 ? d->window : 0;
   p.M = p.G * p.n_q;
-  p.Mpad = (p.M + 15) / 16 * 16;
   p.is_draft = draft ? 1 : 0;
   p.q_offset = d->q_offset;
   p.scale = d->scale;
@@ -1641,8 +1684,10 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
       (!draft && (!aligned16(k_new) || !aligned16(v_new))))
     return SD_ERR_INVALID_ARG;
-  const int MT = p.Mpad / 16;
-  p.row_groups = MT;
+  const int MT = (p.M + 15) / 16;  // 16-row query tiles of the cluster (sliding-window) kernel
+  const RowSplit rs = row_split(p.M);
+  p.row_groups = rs.R;
+  p.Mpad = rs.R * 8 * rs.NB;
   p.P = grid_ctas(d);
   if (p.P <= 0) return SD_ERR_CUDA;
   const size_t need = ws_size(d);
@@ -1674,7 +1719,7 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
     const int tiles_max = (p.window + p.n_q - 1 + kTile - 1) / kTile + 1;
     return launch_window(p.D, MT, km, vm, p, tiles_max, st);
   }
-  s = launch_bf16(p.D, 1, km, vm, p, st);
+  s = launch_bf16(p.D, rs.NB, km, vm, p, st);
   if (s != SD_OK) return s;
   return cuda_status(
       launch(attn_combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hkv, p.M), dim3(128), 0, st, p));
