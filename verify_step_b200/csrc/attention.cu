@@ -273,12 +273,22 @@ __device__ __forceinline__ bool patch_new_rows(const Params &p, int b, int g, in
 // Split-KV tile shape: query rows are the MMA's N dimension in blocks of 8 (NB blocks per CTA),
 // keys its M dimension (one 16-key tile), so an item of up to 24 rows (k + 1 = 6 positions at
 // G = 4) is one CTA's work and needs no padding beyond the next multiple of 8.
-template <int D, int NB, int STAGES>
+template <int D, int NB, int STAGES, bool SPLIT>
 struct Cfg {
   static constexpr int DS = D >= 128 ? 128 : 64;
   static constexpr int NDG = D / DS;  // compute warps, one D slice each
   static constexpr int NCW = NDG;
-  static constexpr int THREADS = 32 * (NCW + 1);
+  // Two or three row blocks at D 512 need more registers per compute thread than 10 warps per SM
+  // leave (168): the CTA is then two warpgroups, the copy warp's group handing registers to the
+  // four compute warps (setmaxnreg: 4 x 32 x kRegCopy + 4 x 32 x kRegMath = 256 threads x 128
+  // registers at launch, checked on the host before the first launch).
+  static constexpr bool WS = SPLIT;
+  static constexpr int THREADS = WS ? 256 : 32 * (NCW + 1);
+  static constexpr int COPY_WARP = WS ? 0 : NCW;   // the warp issuing the tile copies
+  static constexpr int MATH_WARP0 = WS ? 4 : 0;    // first compute warp
+  static constexpr int kRegLaunch = 128, kRegCopy = 24, kRegMath = 232;
+  static_assert(!WS || 128 * kRegCopy + 128 * kRegMath == THREADS * kRegLaunch,
+                "register split must equal the launch total");
   static constexpr int ROWS = 8 * NB;
   static constexpr int TILE_BYTES = kTile * D * 2;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
@@ -291,23 +301,28 @@ struct Cfg {
 };
 
 // Rows per CTA group for an item of M query rows: groups of at most 24 rows (three 8-row
-// blocks), R groups of NB blocks each.
+// blocks), R groups of NB blocks each.  At D 512 a single group of two or three blocks takes
+// the warpgroup register split; groups of a larger item do better without it (measured at
+// 28 rows, two groups of two blocks: 288 against 331 us).
 struct RowSplit {
   int R, NB;
+  bool split;
 };
-__host__ __device__ inline RowSplit row_split(int M) {
+__host__ __device__ inline RowSplit row_split(int M, int D) {
   RowSplit s;
   s.R = (M + 23) / 24;
   const int per = (M + s.R - 1) / s.R;
   s.NB = (per + 7) / 8;
+  s.split = D == 512 && s.NB >= 2 && s.R == 1;
   return s;
 }
 
-template <int D, int NB, int STAGES>
-__global__ void __launch_bounds__(Cfg<D, NB, STAGES>::THREADS, Cfg<D, NB, STAGES>::MIN_CTAS)
+template <int D, int NB, int STAGES, bool SPLIT>
+__global__ void __launch_bounds__(Cfg<D, NB, STAGES, SPLIT>::THREADS,
+                                  Cfg<D, NB, STAGES, SPLIT>::MIN_CTAS)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const Params p) {
-  using C = Cfg<D, NB, STAGES>;
+  using C = Cfg<D, NB, STAGES, SPLIT>;
   constexpr int DS = C::DS, NDG = C::NDG, NCW = C::NCW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -346,7 +361,15 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES>::THREADS, Cfg<D, NB, STAGES
   const long long start = T * grp / p.P;
   const long long end = T * (grp + 1) / p.P;
 
-  if (warp == NCW) {
+  if constexpr (C::WS) {
+    if (warp < 4) {
+      setmaxnreg_dec<C::kRegCopy>();
+      if (warp != C::COPY_WARP) return;
+    } else {
+      setmaxnreg_inc<C::kRegMath>();
+    }
+  }
+  if (warp == C::COPY_WARP) {
     // ------------------------------------------------------------------- producer warp
     // The whole warp walks the cursor; its lanes fetch the block-table entries of the next 32
     // tiles of the current sequence at once (off the per-tile path), lane 0 issues the copies.
@@ -414,7 +437,7 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES>::THREADS, Cfg<D, NB, STAGES
   // O^T += V^T P^T over the slice (D columns as M, rows as N, the tile's keys as K).  In the
   // accumulator layout a lane holds keys kr and kr + 8 (S^T) or D columns kr and kr + 8 (O^T),
   // each for query rows rq and rq + 1 of every 8-row block.
-  const int dg = warp;
+  const int dg = warp - C::MATH_WARP0;
   const int kr = lane >> 2;
   const int rq = 2 * (lane & 3);
   const int row0 = rg * C::ROWS;  // first query row of the item this CTA takes
@@ -512,7 +535,7 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES>::THREADS, Cfg<D, NB, STAGES
         }
       }
       if constexpr (NDG > 1) {
-        float4 *myred = reinterpret_cast<float4 *>(red) + ((buf * NCW + warp) * 32 + lane) * NB;
+        float4 *myred = reinterpret_cast<float4 *>(red) + ((buf * NCW + dg) * 32 + lane) * NB;
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
           myred[nb] = make_float4(sc[nb][0], sc[nb][1], sc[nb][2], sc[nb][3]);
@@ -1458,24 +1481,31 @@ __global__ void __launch_bounds__(32 * kF32Warps) attn_f32_kernel(const Params p
 
 // ------------------------------------------------------------------------------- host side
 
-template <int D, int NB, int STAGES>
+template <int D, int NB, int STAGES, bool SPLIT>
 struct Launcher {
-  using C = Cfg<D, NB, STAGES>;
+  using C = Cfg<D, NB, STAGES, SPLIT>;
   static int ctas_per_sm() {
     static int dev_cache[64];
     static int occ_cache[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && dev_cache[dev] == dev + 1) return occ_cache[dev];
-    cudaFuncSetAttribute(attn_bf16_kernel<D, NB, STAGES>,
+    cudaFuncSetAttribute(attn_bf16_kernel<D, NB, STAGES, SPLIT>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    cudaFuncSetAttribute(attn_bf16_kernel<D, NB, STAGES>,
+    cudaFuncSetAttribute(attn_bf16_kernel<D, NB, STAGES, SPLIT>,
                          cudaFuncAttributePreferredSharedMemoryCarveout,
                          (int)cudaSharedmemCarveoutMaxShared);
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_bf16_kernel<D, NB, STAGES>,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_bf16_kernel<D, NB, STAGES, SPLIT>,
                                                       C::THREADS, C::SMEM) != cudaSuccess)
       occ = 0;
+    if constexpr (C::WS) {
+      // the warpgroups' register split must match the registers the kernel launches with
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, attn_bf16_kernel<D, NB, STAGES, SPLIT>) != cudaSuccess ||
+          fa.numRegs != C::kRegLaunch)
+        occ = 0;
+    }
     if (dev < 64) {
       occ_cache[dev] = occ;
       dev_cache[dev] = dev + 1;
@@ -1485,7 +1515,7 @@ struct Launcher {
   static sd_status launch(const CUtensorMap &km, const CUtensorMap &vm, const Params &p,
                           cudaStream_t st) {
     return cuda_status(
-        sdv::launch(attn_bf16_kernel<D, NB, STAGES>, dim3(p.P * p.row_groups), dim3(C::THREADS),
+        sdv::launch(attn_bf16_kernel<D, NB, STAGES, SPLIT>, dim3(p.P * p.row_groups), dim3(C::THREADS),
                     C::SMEM, st,
                     km, vm, p));
   }
@@ -1493,27 +1523,31 @@ struct Launcher {
 
 #define SDV_STAGES(D) ((D) == 512 ? 3 : (D) == 256 ? 4 : (D) == 128 ? 6 : 8)
 
-// Persistent CTAs for a (head_dim, 8-row blocks) pair on the current device.
-static int persistent_ctas(int D, int NB) {
+// Persistent CTAs for a (head_dim, 8-row blocks, register split) case on the current device.
+static int persistent_ctas(int D, const RowSplit &rs) {
   int occ = 0;
-#define SDV_CASE(DD, NN) \
-  if (D == DD && NB == NN) occ = Launcher<DD, NN, SDV_STAGES(DD)>::ctas_per_sm();
-  SDV_CASE(64, 1) SDV_CASE(128, 1) SDV_CASE(256, 1) SDV_CASE(512, 1)
-  SDV_CASE(64, 2) SDV_CASE(128, 2) SDV_CASE(256, 2) SDV_CASE(512, 2)
-  SDV_CASE(64, 3) SDV_CASE(128, 3) SDV_CASE(256, 3) SDV_CASE(512, 3)
+#define SDV_CASE(DD, NN, SS) \
+  if (D == DD && rs.NB == NN && rs.split == SS) \
+    occ = Launcher<DD, NN, SDV_STAGES(DD), SS>::ctas_per_sm();
+  SDV_CASE(64, 1, false) SDV_CASE(128, 1, false) SDV_CASE(256, 1, false) SDV_CASE(512, 1, false)
+  SDV_CASE(64, 2, false) SDV_CASE(128, 2, false) SDV_CASE(256, 2, false) SDV_CASE(512, 2, false)
+  SDV_CASE(64, 3, false) SDV_CASE(128, 3, false) SDV_CASE(256, 3, false) SDV_CASE(512, 3, false)
+  SDV_CASE(512, 2, true) SDV_CASE(512, 3, true)
 #undef SDV_CASE
   const int sms = sm_count();
   if (occ <= 0 || sms <= 0) return 0;
   return occ * sms;
 }
 
-static sd_status launch_bf16(int D, int NB, const CUtensorMap &km, const CUtensorMap &vm,
-                             const Params &p, cudaStream_t st) {
-#define SDV_CASE(DD, NN) \
-  if (D == DD && NB == NN) return Launcher<DD, NN, SDV_STAGES(DD)>::launch(km, vm, p, st);
-  SDV_CASE(64, 1) SDV_CASE(128, 1) SDV_CASE(256, 1) SDV_CASE(512, 1)
-  SDV_CASE(64, 2) SDV_CASE(128, 2) SDV_CASE(256, 2) SDV_CASE(512, 2)
-  SDV_CASE(64, 3) SDV_CASE(128, 3) SDV_CASE(256, 3) SDV_CASE(512, 3)
+static sd_status launch_bf16(int D, const RowSplit &rs, const CUtensorMap &km,
+                             const CUtensorMap &vm, const Params &p, cudaStream_t st) {
+#define SDV_CASE(DD, NN, SS)                            \
+  if (D == DD && rs.NB == NN && rs.split == SS)         \
+    return Launcher<DD, NN, SDV_STAGES(DD), SS>::launch(km, vm, p, st);
+  SDV_CASE(64, 1, false) SDV_CASE(128, 1, false) SDV_CASE(256, 1, false) SDV_CASE(512, 1, false)
+  SDV_CASE(64, 2, false) SDV_CASE(128, 2, false) SDV_CASE(256, 2, false) SDV_CASE(512, 2, false)
+  SDV_CASE(64, 3, false) SDV_CASE(128, 3, false) SDV_CASE(256, 3, false) SDV_CASE(512, 3, false)
+  SDV_CASE(512, 2, true) SDV_CASE(512, 3, true)
 #undef SDV_CASE
   return SD_ERR_UNSUPPORTED;
 }
@@ -1625,14 +1659,14 @@ static sd_status validate(const sd_attn_desc *d, bool draft) {
 // per row group of the item.
 static int grid_ctas(const sd_attn_desc *d) {
   if (d->dtype != SD_BF16) return 0;
-  const RowSplit rs = row_split(d->h_q / d->h_kv * d->n_q);
-  return persistent_ctas(d->head_dim, rs.NB) / rs.R;
+  const RowSplit rs = row_split(d->h_q / d->h_kv * d->n_q, d->head_dim);
+  return persistent_ctas(d->head_dim, rs) / rs.R;
 }
 
 static size_t ws_size(const sd_attn_desc *d) {
   if (validate(d, false) != SD_OK && validate(d, true) != SD_OK) return 0;
   if (d->dtype != SD_BF16) return 0;
-  const RowSplit rs = row_split(d->h_q / d->h_kv * d->n_q);
+  const RowSplit rs = row_split(d->h_q / d->h_kv * d->n_q, d->head_dim);
   const int Mpad = rs.R * 8 * rs.NB;
   const size_t slots = (size_t)d->batch * d->h_kv + (size_t)grid_ctas(d);
   return round_up(slots * Mpad * d->head_dim * 4, 256) + round_up(slots * Mpad * 2 * 4, 256);
@@ -1685,7 +1719,7 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
       (!draft && (!aligned16(k_new) || !aligned16(v_new))))
     return SD_ERR_INVALID_ARG;
   const int MT = (p.M + 15) / 16;  // 16-row query tiles of the cluster (sliding-window) kernel
-  const RowSplit rs = row_split(p.M);
+  const RowSplit rs = row_split(p.M, p.D);
   p.row_groups = rs.R;
   p.Mpad = rs.R * 8 * rs.NB;
   p.P = grid_ctas(d);
@@ -1719,7 +1753,7 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
     const int tiles_max = (p.window + p.n_q - 1 + kTile - 1) / kTile + 1;
     return launch_window(p.D, MT, km, vm, p, tiles_max, st);
   }
-  s = launch_bf16(p.D, rs.NB, km, vm, p, st);
+  s = launch_bf16(p.D, rs, km, vm, p, st);
   if (s != SD_OK) return s;
   return cuda_status(
       launch(attn_combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hkv, p.M), dim3(128), 0, st, p));

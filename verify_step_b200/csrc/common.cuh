@@ -262,6 +262,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return r;
 }
 
+// Register hand-over between the warpgroups of a CTA (all threads of the warpgroup execute
+// it): the per-thread register count of the calling warpgroup becomes N.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Transposes an 8x8 matrix of 16-bit elements held one 32-bit pair per lane (lane l: row l/4,
 // columns 2(l%4), 2(l%4)+1) into the same layout of its transpose.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
