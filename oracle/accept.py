@@ -24,22 +24,28 @@ target verifies", section "basic structure of speculative decoding"):
 
 Readings of points the pages leave open:
   * q(d) = 0 accepts iff p(d) > 0 (the ratio is +inf).
-  * Categorical draws are exponential races: x = argmin_v E_v / w_v over w_v > 0 with
-    E_v = -ln(1 - V_v), V_v the per-token Philox uniform of the draw's row and purpose;
-    lowest v wins ties.  This is an exact categorical draw needing no normalisation.
-    Implemented as argmax of ln w_v - ln E_v.
+  * Categorical draws are exponential races taken in two levels.  The row's tokens fall in
+    groups of GROUP = 512 consecutive ids (the last group ragged).  Level 1 races the groups:
+    g* = argmax_g ln W_g - ln E_g over W_g > 0, W_g the sum of the group's weights and
+    E_g = -ln(1 - V_g), V_g the group's Philox uniform (philox.group_uniform_rows).  Level 2
+    races the tokens of g*: x = argmax ln w_v - ln E_v over w_v > 0, E_v from the per-token
+    Philox uniform V_v of the draw's row and purpose.  Lowest index wins ties at both levels.
+    An exponential race is an exact categorical draw needing no normalisation, and so is the
+    pair: P(g*) = W_g* / W and P(x | g*) = w_x / W_g*.
   * Margins (decisions a float32 implementation may take differently): an acceptance
-    with |u - p/q| < MARGIN; a draw whose winner's lowest possible key does not beat every
-    other token's highest possible key by MARGIN, the key bounds taking each weight as
-    w +- REL_P * (p + q) (the float32 error of p - q) and ln E, z / T to within ABS_KEY;
-    a greedy argmax whose top two logits differ by less than MARGIN * max(1, |top|).
+    with |u - p/q| < MARGIN; a race whose winner's lowest possible key does not beat every
+    other competitor's highest possible key by MARGIN, at either level, the key bounds taking
+    each weight as w +- REL_P * (p + q) (the float32 error of p - q) and ln E, z / T to within
+    ABS_KEY (a group's sums of the token bounds, its key error the largest of its weighted
+    tokens'); a greedy argmax whose top two logits differ by less than MARGIN * max(1, |top|).
 """
 from __future__ import annotations
 
 import numpy as np
 
-from .philox import accept_uniform, token_uniform_rows
+from .philox import accept_uniform, group_uniform_rows, token_uniform_at
 
+GROUP = 512            # tokens per group of the two-level race
 MARGIN = 1e-4          # north-star margin on |u - p/q|; reused for draws and argmaxes
 REL_P = 1e-5           # assumed float32 relative error bound on a probability p_v or q_v
 ABS_KEY = 1e-5         # assumed float32 absolute error bound on ln E_v and z_v / T
@@ -72,6 +78,45 @@ def _race_margin(g_lo: np.ndarray, g_hi: np.ndarray, x: np.ndarray) -> np.ndarra
     hi = g_hi.copy()
     hi[np.arange(R), x] = -np.inf
     return hi.max(axis=-1) > g_lo[np.arange(R), x] - MARGIN
+
+
+def _group_sum(a: np.ndarray, n_groups: int, reduce=np.sum) -> np.ndarray:
+    R, V = a.shape
+    pad = np.zeros((R, n_groups * GROUP - V))
+    return reduce(np.concatenate([a, pad], axis=1).reshape(R, n_groups, GROUP), axis=-1)
+
+
+def two_level_race(w, w_lo, w_hi, key_err, seed: int, step: int, rows, purpose: int):
+    """Two-level exponential race per row of the weights w [R, V] (bounds w_lo, w_hi and the
+    per-token key error key_err for the margin).  Returns (winner ids, margin flags)."""
+    w, w_lo, w_hi, key_err = (np.asarray(a, np.float64) for a in (w, w_lo, w_hi, key_err))
+    R, V = w.shape
+    NG = (V + GROUP - 1) // GROUP
+    rows = np.asarray(rows)
+    # level 1: the groups
+    W, W_lo, W_hi = (_group_sum(a, NG) for a in (w, w_lo, w_hi))
+    kerr = _group_sum(np.where(w_hi > 0, key_err, 0.0), NG, np.max)
+    lnEg = np.log(-np.log1p(-group_uniform_rows(seed, step, rows, purpose, NG)))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        G = np.where(W > 0, np.log(W) - lnEg, -np.inf)
+        G_hi = np.where(W_hi > 0, np.log(W_hi) - lnEg + kerr, -np.inf)
+        G_lo = np.where(W_lo > 0, np.log(W_lo) - lnEg - kerr, -np.inf)
+    gs = np.argmax(G, axis=-1)
+    margin = _race_margin(G_lo, G_hi, gs)
+    # level 2: the tokens of the winning group (ids past the vocabulary carry weight 0)
+    ids = gs[:, None] * GROUP + np.arange(min(GROUP, V))[None, :]
+    live = ids < V
+    idc = np.minimum(ids, V - 1)
+    take = lambda a: np.where(live, np.take_along_axis(a, idc, axis=1), 0.0)
+    wg, wg_lo, wg_hi, kg = take(w), take(w_lo), take(w_hi), take(key_err)
+    lnE = np.log(-np.log1p(-token_uniform_at(seed, step, rows, purpose, ids)))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        g = np.where(wg > 0, np.log(wg) - lnE, -np.inf)
+        g_hi = np.where(wg_hi > 0, np.log(wg_hi) - lnE + kg, -np.inf)
+        g_lo = np.where(wg_lo > 0, np.log(wg_lo) - lnE - kg, -np.inf)
+    j = np.argmax(g, axis=-1)
+    margin |= _race_margin(g_lo, g_hi, j)
+    return gs * GROUP + j, margin
 
 
 def greedy_gap(z: np.ndarray) -> np.ndarray:
@@ -136,16 +181,12 @@ def accept(z, y, drafts, temperature: float, seed: int, step: int,
         else:
             w = w_hi = w_lo = pa
             key_err = ABS_KEY * (1.0 + np.abs(za))
-        Vu = token_uniform_rows(seed, step, rows + n_acc, purpose, V)
-        x, g = race(w, Vu)
-        lnE = np.log(-np.log1p(-Vu))
         # a token of weight exactly 0 (a -inf logit, or an empty residual entry) cannot win
         # on either side: its key bound is -inf (its key error term may be infinite there,
         # and -inf + inf would be NaN and hide the row's other competitors from the check)
-        with np.errstate(divide="ignore", invalid="ignore"):
-            g_hi = np.where(w_hi > 0, np.log(w_hi) - lnE + key_err, -np.inf)
-            g_lo = np.where(w_lo > 0, np.log(w_lo) - lnE - key_err, -np.inf)
-        margin |= _race_margin(g_lo, g_hi, x)
+        key_err = np.where(w_hi > 0, np.broadcast_to(key_err, w.shape), 0.0)
+        x, m = two_level_race(w, w_lo, w_hi, key_err, seed, step, rows + n_acc, purpose)
+        margin |= m
 
     out = np.full((B, n_q), -1, np.int64)
     for b in range(B):

@@ -19,6 +19,8 @@ Uniforms used by the acceptance rule (the pages state no generator; this build's
       V  = 0 when x = 0.
   V keeps 24 significant bits at every scale, so it is exactly representable in float32
   and float64 and both sides of a parity test see the same number.
+  group uniform of token group g (tokens 512 g .. 512 g + 511) on row r for a draw with
+  purpose P: the token uniform's construction with purpose P + 16 and g in place of v.
 """
 from __future__ import annotations
 
@@ -91,6 +93,18 @@ def token_uniform(seed: int, step: int, row: int, purpose: int, vocab_ids) -> np
     return _float_uniform((hi << S32) | lo)
 
 
+def token_uniform_at(seed: int, step: int, rows, purpose: int, ids) -> np.ndarray:
+    """Token uniforms of tokens ``ids`` [R, n] on rows ``rows`` [R]: shape [R, n]."""
+    k0, k1 = _key(seed)
+    rows = np.asarray(rows, dtype=np.uint64)[:, None]
+    v = np.asarray(ids, dtype=np.uint64)
+    ws = philox4x32_10(v >> np.uint64(1), rows, int(step) & 0xFFFFFFFF, int(purpose), k0, k1)
+    odd = np.broadcast_to((v & np.uint64(1)).astype(bool), ws[0].shape)
+    lo = np.where(odd, ws[2], ws[0])
+    hi = np.where(odd, ws[3], ws[1])
+    return _float_uniform((hi << S32) | lo)
+
+
 def token_uniform_rows(seed: int, step: int, rows, purpose: int, vocab: int) -> np.ndarray:
     """Token uniforms for several rows at once: shape [len(rows), vocab]."""
     k0, k1 = _key(seed)
@@ -101,3 +115,11 @@ def token_uniform_rows(seed: int, step: int, rows, purpose: int, vocab: int) -> 
     lo = np.where(odd, ws[2], ws[0])
     hi = np.where(odd, ws[3], ws[1])
     return _float_uniform((hi << S32) | lo)
+
+
+GROUP_PURPOSE_OFFSET = 16
+
+
+def group_uniform_rows(seed: int, step: int, rows, purpose: int, n_groups: int) -> np.ndarray:
+    """Uniforms of the token groups of a two-level draw, shape [len(rows), n_groups]."""
+    return token_uniform_rows(seed, step, rows, int(purpose) + GROUP_PURPOSE_OFFSET, n_groups)

@@ -291,3 +291,78 @@ def test_acceptance_margin_ignores_decisions_never_taken():
     assert r["n_accepted"][rej_b] == 0 and not r["margin"][rej_b]
     assert r["n_accepted"][acc_b] == 2 and r["margin"][acc_b]
     assert r["out_tokens"][rej_b, 0] == 1          # the residual's only positive token
+
+
+def test_two_level_draw_is_exact_over_several_groups():
+    """A plain draw over 700 tokens: two groups of the two-level race (512 and a ragged 188),
+    the second holding most of the mass.  The Philox-driven frequencies of 60 000 draws (one
+    logit row each) follow p: a group weight that dropped a term, a wrong group boundary or a
+    lost ragged tail would bias whole groups."""
+    V, n = 700, 60_000
+    rng = np.random.default_rng(7)
+    logp = rng.standard_normal(V) * 0.5
+    logp[512:] += 1.5                      # group 1 (188 tokens) carries about 60 % of p
+    p = np.exp(logp) / np.exp(logp).sum()
+    assert 0.5 < p[512:].sum() < 0.8
+    z = np.broadcast_to(logp, (n, 1, V))
+    r = ACC.accept(z, None, np.zeros((n, 0), np.int64), 1.0, seed=11, step=3,
+                   purpose=ACC.PURPOSE_DRAFTER)
+    counts = np.bincount(r["out_tokens"][:, 0], minlength=V)
+    assert stats.chisquare(counts, p * n).pvalue > 0.01
+    # the group split alone: group 1's share is binomial around its mass
+    share = counts[512:].sum() / n
+    assert abs(share - p[512:].sum()) < 4 * np.sqrt(p[512:].sum() * (1 - p[512:].sum()) / n)
+
+
+def test_residual_draw_over_several_groups_follows_the_residual():
+    """k = 1 over 1100 tokens (groups of 512, 512, 76): among the rejected sequences the
+    emitted token follows norm(max(0, p - q)), whose mass sits in different groups than p's."""
+    V, n = 1100, 40_000
+    rng = np.random.default_rng(3)
+    zp = rng.standard_normal(V)
+    zq = zp.copy()
+    zq[:600] += 1.0                        # q over-weights the first groups: residual elsewhere
+    p = np.exp(zp) / np.exp(zp).sum()
+    q = np.exp(zq) / np.exp(zq).sum()
+    resid = np.maximum(0.0, p - q)
+    resid /= resid.sum()
+    z = np.empty((n, 2, V))
+    z[:, 0] = zp
+    z[:, 1] = zp
+    y = np.broadcast_to(zq, (n, 1, V))
+    drafts = rng.choice(V, size=(n, 1), p=q)
+    r = ACC.accept(z, y, drafts, 1.0, seed=23, step=1)
+    rej = r["n_accepted"] == 0
+    assert rej.sum() > 5000
+    counts = np.bincount(r["out_tokens"][rej, 0], minlength=V)
+    exp = resid * rej.sum()
+    big = exp >= 5
+    obs = np.append(counts[big], counts[~big].sum())
+    ex = np.append(exp[big], exp[~big].sum())
+    assert stats.chisquare(obs, ex).pvalue > 0.01
+
+
+def test_group_level_near_tie_is_flagged():
+    """Two groups of equal-weight tokens whose level-1 keys differ by 1e-5 (flagged) or by 2
+    (not flagged); the winning group is the one with the larger key either way."""
+    from oracle.philox import group_uniform_rows
+    V, seed, step = 1024, 5, 9
+    ug = group_uniform_rows(seed, step, [0], ACC.PURPOSE_DRAFTER, 2)[0]
+    lnEg = np.log(-np.log1p(-ug))
+    for gap, want in ((1e-5, True), (2.0, False)):
+        # ln W_1 - lnE_1 = ln W_0 - lnE_0 + gap, tokens equal inside each group
+        lnW0 = 0.0
+        lnW1 = lnW0 + lnEg[1] - lnEg[0] + gap
+        z = np.empty((1, 1, V))
+        z[0, 0, :512] = lnW0 - np.log(512)
+        z[0, 0, 512:] = lnW1 - np.log(512)
+        r = ACC.accept(z, None, np.zeros((1, 0), np.int64), 1.0, seed=seed, step=step,
+                       purpose=ACC.PURPOSE_DRAFTER)
+        assert 512 <= r["out_tokens"][0, 0] < 1024
+        if want:
+            assert r["margin"][0]
+        else:
+            # not flagged by level 1; level 2 over 512 equal weights rarely ties within 1e-4
+            G = np.log(np.exp(z[0, 0]).reshape(2, 512).sum(-1)) - lnEg
+            assert G[1] - G[0] > 1.9
+            assert not r["margin"][0]
