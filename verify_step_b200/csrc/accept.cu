@@ -6,7 +6,7 @@
 // u_i < p_i(d_i) / q_i(d_i); at the first rejection emit x ~ norm(max(0, p_i - q_i)); if all
 // are accepted emit the bonus x ~ p_{k+1}.  T = 0: accept iff d_i == argmax, emit argmax.
 //
-// Three kernels (a plain draw, k = 0 at T > 0, runs only the last):
+// Three kernels (a plain draw, k = 0 at T > 0, runs a ticket clear and the last):
 //  1. accept_stats: one CTA per (logit row, token chunk) over every row the sequences need (the
 //     k+1 target rows and, for T > 0, the k draft rows), sized to one wave of CTAs: online max /
 //     sum of exp(x / T) of the chunk (T > 0), or its top two values and the argmax (T = 0),
@@ -15,13 +15,15 @@
 //     order), tests the k drafts lane-parallel and writes the sequence's decision record
 //     (accepted count, acceptance margin flag, the normalisers of the draw row); at T = 0 it
 //     writes the outputs itself.
-//  3. accept_draw: one CTA per (sequence, token chunk), one wave of CTAs.  Exponential race of
-//     the draw row over the chunk: key_v = log2 w_v - log2(-ln(1 - V_v)), V_v the token's
-//     Philox uniform, for the residual weights max(0, p - q) after a rejection or for p (the
-//     bonus draw, a plain draw).  The race keeps its winner, the winner's lowest possible key
-//     and the highest possible key of every other token under the float32 error model of the
-//     margin rule.  The last CTA of a sequence (atomic ticket; no waiting) merges the chunk
-//     winners (lowest token id first on equal keys) and writes the outputs.
+//  3. accept_mass: the categorical draw as a two-level exponential race.  CTAs per (sequence,
+//     run of 512-token groups), one wave of them, reduce each group of the draw row to its mass
+//     (max(0, p - q) after a rejection; p for the bonus draw and plain draws) with the sums the
+//     margin bounds need.  The last CTA of a sequence (atomic ticket; no waiting) races the
+//     groups, key_g = log2 W_g - log2(-ln(1 - V_g)) with the group's Philox uniform, then the
+//     winning group's 512 tokens, key_v = log2 w_v - log2(-ln(1 - V_v)), keeping at each level
+//     the winner's lowest possible key and the highest possible key of every other competitor
+//     under the float32 error model of the margin rule, and writes the outputs.  The generator
+//     runs for the groups and one group's tokens instead of every token of the row.
 #include <cfloat>
 
 #include "common.cuh"
@@ -35,8 +37,10 @@ constexpr int kStatThreads = 256;
 constexpr int kChunk = 8192;        // tokens per statistics CTA at least
 constexpr int kDecideThreads = 256;
 constexpr int kMaxRows = 31;        // rows per sequence: 2k + 1 with k <= 15
-constexpr int kDrawSlots = 592;     // draw CTAs aimed at: one wave at 4 CTAs on each of 148 SMs
-constexpr int kDrawThreads = 256;
+constexpr int kMassSlots = 592;     // group-mass CTAs aimed at: one wave at 4 CTAs per SM
+constexpr int kMassThreads = 256;   // the last CTA races 2 groups / 2 tokens per thread
+constexpr int kGroup = 512;         // tokens per group of the two-level race
+constexpr uint32_t kGroupPurpose = 16;  // group uniforms: the draw's purpose + 16
 constexpr float kMargin = 1e-4f;    // spec margin on |u - p/q|; also for draws, argmaxes
 constexpr float kRelP = 1e-5f;      // float32 error bound assumed on a probability p_v or q_v
 constexpr float kAbsKey = 1e-5f;    // float32 error bound assumed on ln E_v and z_v / T
@@ -59,7 +63,8 @@ struct Params {
   int B, k, V, n_q, ld_t, ld_d, ld_o, purpose;
   int rps;           // rows per sequence read by the statistics pass
   int nchunks, stats_chunk;
-  int ndraw, draw_chunk;
+  int ngroups;       // token groups of a row, ceil(V / kGroup)
+  int nmass, mass_groups;  // group-mass CTAs per sequence, groups per CTA
   float T;
   unsigned long long seed;
   unsigned long long step;
@@ -72,7 +77,7 @@ struct Params {
   int32_t *margin;
   float4 *stats;           // [B * rps][nchunks] chunk partials
   Record *rec;             // [B]
-  float4 *cand;            // [B][ndraw][3]
+  float4 *gm;              // [B][ngroups] group masses of the draw row
   unsigned int *counters;  // [B]
   int *status;
 };
@@ -370,28 +375,20 @@ __global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Par
   p.rec[b] = r;
 }
 
-// ------------------------------------------------------------------ draw kernel
+// ------------------------------------------------------------------ group masses and the race
 
-// One token of the race: adds its key and bounds to the race state (log2 units).
+// Level-2 token of the race (log2 units):
 //   draw from p (resid == false): key = zt log2(e) - lg2 E, bounds key -/+ 1e-5 (1 + |zt|)
 //   residual (resid == true): key = lg2 w - lg2 E (w = max(0, p - q) > 0), its lower bound from
-//   w - s and the upper bound of every token from w + s, s = 1e-5 (p + q), each -/+ 1e-5;
-//   pb, the bare p race without bounds, keeps a fallback winner for an empty residual.
+//   w - s and the upper bound of every token from w + s, s = 1e-5 (p + q), each -/+ 1e-5.
 __device__ __forceinline__ void race_token(bool resid, float zt, float w, float sl, float lgE,
-                                           int v, Race &cr, Race &pb) {
+                                           int v, Race &cr) {
   if (!resid) {
     if (zt == -INFINITY) return;
     const float g = fmaf(zt, kLog2e, -lgE);
     const float err = kAbsKey2 * (1.f + fabsf(zt));
     race_push(cr, g, g - err, g + err, v);
     return;
-  }
-  if (zt != -INFINITY) {
-    const float g = fmaf(zt, kLog2e, -lgE);
-    if (g > pb.g1) {
-      pb.g1 = g;
-      pb.v1 = v;
-    }
   }
   if (w + sl > 0.f) {
     const float hi = __log2f(w + sl) - lgE + kAbsKey2;
@@ -405,12 +402,34 @@ __device__ __forceinline__ void race_token(bool resid, float zt, float w, float 
   }
 }
 
-__global__ void __launch_bounds__(kDrawThreads, 4) accept_draw_kernel(const Params p) {
+// Reduces a race over the CTA (lowest index first on equal keys); every thread gets the result.
+__device__ __forceinline__ Race race_block(Race r, Race *s_red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int off = 16; off > 0; off >>= 1) {
+    const Race o = race_shfl(r, off);
+    r = (lane & off) ? race_merge(o, r) : race_merge(r, o);
+  }
+  __syncthreads();  // s_red may still be read from an earlier reduction
+  if (lane == 0) s_red[warp] = r;
+  __syncthreads();
+  Race t = s_red[0];
+  for (int w = 1; w < kMassThreads / 32; ++w) t = race_merge(t, s_red[w]);
+  return t;
+}
+
+// One CTA per (sequence, run of token groups).  Each warp reduces whole 512-token groups of the
+// draw row (16 tokens a lane, 16-byte loads issued together):
+//   draw from p:   (m_g, s_g, A_g) = group max of z / T, sum of exp(z / T - m_g), max |z / T|
+//   residual:      (W_g, S_g, P_g) = sums of max(0, p - q), of 1e-5 (p + q), and of p
+// The last CTA of the sequence (atomic ticket, no waiting) races the groups (level 1, group
+// uniforms), then the 512 tokens of the winning group (level 2, token uniforms), and writes the
+// outputs.  An empty residual falls back to the race over p (flagged).
+__global__ void __launch_bounds__(kMassThreads) accept_mass_kernel(const Params p) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x, c = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __shared__ Race s_red[2][kDrawThreads / 32];
+  __shared__ Race s_red[kMassThreads / 32];
   __shared__ int s_last;
 
   // every thread reads the record itself (one broadcast load): no barrier before the loads
@@ -425,126 +444,183 @@ __global__ void __launch_bounds__(kDrawThreads, 4) accept_draw_kernel(const Para
   const int rt = b * p.n_q + a;
   const float *zr = p.z + (size_t)rt * p.ld_t;
   const float *yr = resid ? p.y + ((size_t)b * p.k + a) * p.ld_d : nullptr;
-  const int v0 = c * p.draw_chunk;
-  const int v1 = min(p.V, v0 + p.draw_chunk);
-  const int n4 = max(0, v1 - v0) >> 2;
-  // Keys in float32 with fast exp2 / log2 where the error (<~1e-6 absolute on a key, <~1e-6
-  // relative on p and q) is far inside the error model the bounds assume (1e-5); the -ln(1 - V)
-  // of the uniform stays accurate because small uniforms decide the winners.
   const bool unit_t = p.T == 1.f;
   const float inv_t = 1.f / p.T;
   const float isz = rec.isz, isy = rec.isy;
   const float mzl = rec.mz * kLog2e, myl = rec.my * kLog2e;
-  Race cr = race_empty();
-  Race pb = race_empty();  // bare p race (residual fallback), g1 / v1 only
-  constexpr int PER = 2;   // float4 groups whose loads are issued together
-  uint32_t step = rec.step;
-  bool have_step = p.k != 0;
-  for (int base = 0; base < n4; base += PER * kDrawThreads) {
-    float4 z4[PER], y4[PER];
+  float4 *gm = p.gm + (size_t)b * p.ngroups;
+
+  const int g_end = min(p.ngroups, (c + 1) * p.mass_groups);
+  for (int g = c * p.mass_groups + warp; g < g_end; g += kMassThreads / 32) {
+    const int v0 = g * kGroup;
+    const int n4 = min(kGroup, p.V - v0) >> 2;
+    const float4 *z4 = reinterpret_cast<const float4 *>(zr + v0);
+    const float4 *y4 = resid ? reinterpret_cast<const float4 *>(yr + v0) : nullptr;
+    float4 zz[4], yy[4];
 #pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int i = base + threadIdx.x + u * kDrawThreads;
-      z4[u] = i < n4 ? __ldg(reinterpret_cast<const float4 *>(zr + v0) + i)
-                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      y4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (resid && i < n4) y4[u] = __ldg(reinterpret_cast<const float4 *>(yr + v0) + i);
+    for (int u = 0; u < 4; ++u) {
+      const int i = lane + 32 * u;
+      zz[u] = i < n4 ? __ldg(z4 + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      yy[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (resid && i < n4) yy[u] = __ldg(y4 + i);
     }
-    if (!have_step) {  // a plain draw reads the step counter behind its first loads
-      step = counter_step(p);
-      have_step = true;
-    }
+    float4 out;
+    if (!resid) {
+      float m = -INFINITY, A = 0.f;
 #pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int i = base + threadIdx.x + u * kDrawThreads;
-      if (i >= n4) break;
-      const int v = v0 + 4 * i;
-      const float zz[4] = {z4[u].x, z4[u].y, z4[u].z, z4[u].w};
-      const float yy[4] = {y4[u].x, y4[u].y, y4[u].z, y4[u].w};
-      float zt[4], w[4], sl[4];
-      bool any = false;
+      for (int u = 0; u < 4; ++u) {
+        float *x = reinterpret_cast<float *>(&zz[u]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        zt[e] = unit_t ? zz[e] : zz[e] * inv_t;
-        w[e] = 0.f;
-        sl[e] = 0.f;
-        if (resid) {
-          const float yt = unit_t ? yy[e] : yy[e] * inv_t;
-          const float pv = ex2_approx(fmaf(zt[e], kLog2e, -mzl)) * isz;
-          const float qv = ex2_approx(fmaf(yt, kLog2e, -myl)) * isy;
-          w[e] = fmaxf(pv - qv, 0.f);
-          sl[e] = kRelP * (pv + qv);
-          any |= w[e] + sl[e] > 0.f;
-        } else {
-          any |= zt[e] != -INFINITY;
+        for (int e = 0; e < 4; ++e) {
+          if (!unit_t) x[e] *= inv_t;
+          m = fmaxf(m, x[e]);
+          if (x[e] != -INFINITY) A = fmaxf(A, fabsf(x[e]));
         }
       }
-      if (!any) continue;  // no token of the group has any weight: no uniforms needed
-      float U[4];
-      token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1),
-                         U[0], U[1]);
-      token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose,
-                         (uint32_t)(v >> 1) + 1u, U[2], U[3]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float lgE = __log2f(neg_log1m(U[e]));  // E == 0 gives -inf: that token wins
-        race_token(resid, zt[e], w[e], sl[e], lgE, v + e, cr, pb);
+      for (int off = 16; off > 0; off >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        A = fmaxf(A, __shfl_xor_sync(0xffffffffu, A, off));
       }
+      float s = 0.f;
+      if (m != -INFINITY) {
+        const float ml = m * kLog2e;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float *x = reinterpret_cast<const float *>(&zz[u]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s += ex2_approx(fmaf(x[e], kLog2e, -ml));
+        }
+      }
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      out = make_float4(m, s, A, 0.f);
+    } else {
+      float W = 0.f, S = 0.f, P = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (lane + 32 * u >= n4) continue;  // past the row's end
+        const float *zx = reinterpret_cast<const float *>(&zz[u]);
+        const float *yx = reinterpret_cast<const float *>(&yy[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float zt = unit_t ? zx[e] : zx[e] * inv_t;
+          const float yt = unit_t ? yx[e] : yx[e] * inv_t;
+          const float pv = ex2_approx(fmaf(zt, kLog2e, -mzl)) * isz;
+          const float qv = ex2_approx(fmaf(yt, kLog2e, -myl)) * isy;
+          W += fmaxf(pv - qv, 0.f);
+          S += kRelP * (pv + qv);
+          P += pv;
+        }
+      }
+      for (int off = 16; off > 0; off >>= 1) {
+        W += __shfl_xor_sync(0xffffffffu, W, off);
+        S += __shfl_xor_sync(0xffffffffu, S, off);
+        P += __shfl_xor_sync(0xffffffffu, P, off);
+      }
+      out = make_float4(W, S, P, 0.f);
     }
-  }
-  for (int off = 16; off > 0; off >>= 1) {
-    const Race o1 = race_shfl(cr, off);
-    cr = (lane & off) ? race_merge(o1, cr) : race_merge(cr, o1);
-    if (resid) {
-      const Race o2 = race_shfl(pb, off);
-      pb = (lane & off) ? race_merge(o2, pb) : race_merge(pb, o2);
-    }
-  }
-  if (lane == 0) {
-    s_red[0][warp] = cr;
-    s_red[1][warp] = pb;
+    if (lane == 0) gm[g] = out;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    Race tr = s_red[0][0], tp = s_red[1][0];
-    for (int w = 1; w < kDrawThreads / 32; ++w) {
-      tr = race_merge(tr, s_red[0][w]);
-      tp = race_merge(tp, s_red[1][w]);
-    }
-    float4 *slot = p.cand + ((size_t)b * p.ndraw + c) * 3;
-    slot[0] = make_float4(tr.g1, tr.lo1, tr.hi1, tr.hi2);
-    slot[1] = make_float4(tp.g1, tp.lo1, tp.hi1, tp.hi2);
-    slot[2] = make_float4(__int_as_float(tr.v1), __int_as_float(tp.v1), 0.f, 0.f);
     __threadfence();
     const unsigned int ticket = atomicAdd(&p.counters[b], 1u);
-    s_last = ticket == (unsigned int)(p.ndraw - 1);
+    s_last = ticket == (unsigned int)(p.nmass - 1);
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // ---- last CTA of the sequence: merge the chunk winners (order-independent: equal keys go to
-  // the lower token id), one warp
-  if (threadIdx.x >= 32) return;
-  const float4 *cv = p.cand + (size_t)b * p.ndraw * 3;
-  Race tr = race_empty(), tp = race_empty();
-  for (int cc = lane; cc < p.ndraw; cc += 32) {
-    const float4 a0 = __ldcg(cv + 3 * cc);
-    const float4 a1 = __ldcg(cv + 3 * cc + 1);
-    const float4 id = __ldcg(cv + 3 * cc + 2);
-    tr = race_merge(tr, Race{a0.x, a0.y, a0.z, a0.w, __float_as_int(id.x)});
-    tp = race_merge(tp, Race{a1.x, a1.y, a1.z, a1.w, __float_as_int(id.y)});
+
+  // ---- last CTA of the sequence.  Level 1: the groups (thread t takes the group pair
+  // 2t, 2t + 1: one Philox call)
+  const uint32_t step = p.k == 0 ? counter_step(p) : rec.step;
+  const uint32_t gpurpose = (uint32_t)p.purpose + kGroupPurpose;
+  Race cr = race_empty();
+  Race pb = race_empty();  // residual fallback: the race over the groups' p mass, g1 / v1 only
+  for (int gp = threadIdx.x; 2 * gp < p.ngroups; gp += kMassThreads) {
+    float U[2];
+    token_uniform_pair(p.seed, step, (uint32_t)rt, gpurpose, (uint32_t)gp, U[0], U[1]);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int g = 2 * gp + e;
+      if (g >= p.ngroups) break;
+      const float4 q = __ldcg(gm + g);
+      const float lgE = __log2f(neg_log1m(U[e]));
+      if (!resid) {
+        if (q.x == -INFINITY || !(q.y > 0.f)) continue;
+        const float key = __log2f(q.y) + q.x * kLog2e - lgE;
+        const float err = kAbsKey2 * (1.f + q.z);
+        race_push(cr, key, key - err, key + err, g);
+      } else {
+        if (q.z > 0.f) {
+          const float kp = __log2f(q.z) - lgE;
+          if (kp > pb.g1) {
+            pb.g1 = kp;
+            pb.v1 = g;
+          }
+        }
+        if (q.x + q.y > 0.f) {
+          const float hi = __log2f(q.x + q.y) - lgE + kAbsKey2;
+          const float key = q.x > 0.f ? __log2f(q.x) - lgE : -INFINITY;
+          if (key > cr.g1) {
+            const float wl = q.x - q.y;
+            race_push(cr, key, wl > 0.f ? __log2f(wl) - lgE - kAbsKey2 : -INFINITY, hi, g);
+          } else {
+            cr.hi2 = fmaxf(cr.hi2, hi);
+          }
+        }
+      }
+    }
   }
-  for (int off = 16; off > 0; off >>= 1) {
-    tr = race_merge(tr, race_shfl(tr, off));
-    tp = race_merge(tp, race_shfl(tp, off));
-  }
-  if (lane != 0) return;
-  // the residual race unless every residual weight came out 0: then the bare race over p, and
-  // the draw is flagged (a residual too small for float32 may still be positive)
-  const bool empty = resid && tr.v1 < 0;
-  const int x = empty ? tp.v1 : tr.v1;
+  cr = race_block(cr, s_red);
+  if (resid) pb = race_block(pb, s_red);
+  // the residual race unless every residual weight came out 0: then the race over p, flagged
+  // (a residual too small for float32 may still be positive)
+  const bool empty = resid && cr.v1 < 0;
   int flag = rec.flag;
-  if (empty || race_flag(tr)) flag = 1;
+  if (empty || race_flag(cr)) flag = 1;
+  int gsel = empty ? pb.v1 : cr.v1;
+  if (gsel < 0) {  // no positive weight in the row at all
+    gsel = 0;
+    flag = 1;
+  }
+  const bool tok_resid = resid && !empty;
+
+  // ---- level 2: the tokens of group gsel (thread t takes tokens 2t, 2t + 1)
+  Race tr = race_empty();
+  {
+    const int v = gsel * kGroup + 2 * threadIdx.x;
+    if (v < p.V) {  // V is a multiple of 4: both tokens exist
+      float U[2];
+      token_uniform_pair(p.seed, step, (uint32_t)rt, (uint32_t)p.purpose, (uint32_t)(v >> 1),
+                         U[0], U[1]);
+      const float2 z2 = __ldg(reinterpret_cast<const float2 *>(zr + v));
+      const float2 y2 = tok_resid ? __ldg(reinterpret_cast<const float2 *>(yr + v))
+                                  : make_float2(0.f, 0.f);
+      const float zz[2] = {z2.x, z2.y}, yy[2] = {y2.x, y2.y};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float zt = unit_t ? zz[e] : zz[e] * inv_t;
+        float w = 0.f, sl = 0.f;
+        if (tok_resid) {
+          const float yt = unit_t ? yy[e] : yy[e] * inv_t;
+          const float pv = ex2_approx(fmaf(zt, kLog2e, -mzl)) * isz;
+          const float qv = ex2_approx(fmaf(yt, kLog2e, -myl)) * isy;
+          w = fmaxf(pv - qv, 0.f);
+          sl = kRelP * (pv + qv);
+        }
+        const float lgE = __log2f(neg_log1m(U[e]));  // E == 0 gives -inf: that token wins
+        race_token(tok_resid, zt, w, sl, lgE, v + e, tr);
+      }
+    }
+  }
+  tr = race_block(tr, s_red);
+  if (threadIdx.x != 0) return;
+  if (race_flag(tr)) flag = 1;
+  int x = tr.v1;
+  if (x < 0) {
+    x = gsel * kGroup;
+    flag = 1;
+  }
   int32_t *o = p.out + (size_t)b * p.ld_o;
   for (int j = 0; j < p.n_q; ++j)
     o[j] = j < a ? p.drafts[(size_t)b * p.k + j] : (j == a ? x : -1);
@@ -573,18 +649,21 @@ static sd_status validate(const sd_accept_desc *d) {
   return SD_OK;
 }
 
-// Tokens per draw CTA: the race of one sequence is split so that all B sequences together give
-// about one wave of CTAs; multiples of 1024 tokens.
-static int draw_chunk_of(int B, int V) {
-  int per_seq = kDrawSlots / (B > 0 ? B : 1);
+// Token groups per group-mass CTA: the groups of one sequence are split so that all B sequences
+// together give about one wave of CTAs, at least one group per warp.
+static int ngroups_of(int V) { return (V + kGroup - 1) / kGroup; }
+static int mass_groups_of(int B, int V) {
+  int per_seq = kMassSlots / (B > 0 ? B : 1);
   if (per_seq < 1) per_seq = 1;
-  int chunk = (V + per_seq - 1) / per_seq;
-  chunk = (chunk + 1023) / 1024 * 1024;
-  return chunk;
+  const int ng = ngroups_of(V);
+  int m = (ng + per_seq - 1) / per_seq;
+  constexpr int W = kMassThreads / 32;
+  m = (m + W - 1) / W * W;
+  return m;
 }
-static int ndraw_of(int B, int V) {
-  const int c = draw_chunk_of(B, V);
-  return (V + c - 1) / c;
+static int nmass_of(int B, int V) {
+  const int m = mass_groups_of(B, V);
+  return (ngroups_of(V) + m - 1) / m;
 }
 
 static int nchunks_of(int V) { return (V + kChunk - 1) / kChunk; }
@@ -619,7 +698,7 @@ static size_t ws_size(const sd_accept_desc *d) {
   const size_t rows = (size_t)d->batch * (2 * d->k + 1);
   return round_up(rows * nchunks_of(d->vocab) * 16, 256) +
          round_up((size_t)d->batch * sizeof(Record), 256) +
-         round_up((size_t)d->batch * ndraw_of(d->batch, d->vocab) * 48, 256) +
+         round_up((size_t)d->batch * ngroups_of(d->vocab) * 16, 256) +
          round_up((size_t)d->batch * 4, 256);
 }
 
@@ -654,8 +733,9 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   p.ld_d = desc->ld_draft ? desc->ld_draft : desc->vocab;
   p.ld_o = desc->ld_out ? desc->ld_out : desc->k + 1;
   p.purpose = desc->purpose;
-  p.draw_chunk = draw_chunk_of(desc->batch, desc->vocab);
-  p.ndraw = ndraw_of(desc->batch, desc->vocab);
+  p.ngroups = ngroups_of(desc->vocab);
+  p.mass_groups = mass_groups_of(desc->batch, desc->vocab);
+  p.nmass = nmass_of(desc->batch, desc->vocab);
   p.rps = p.n_q + (sampling ? p.k : 0);
   p.T = desc->temperature;
   p.seed = desc->seed;
@@ -672,14 +752,14 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   w8 += round_up((size_t)p.B * (2 * p.k + 1) * nchunks_of(p.V) * 16, 256);
   p.rec = reinterpret_cast<Record *>(w8);
   w8 += round_up((size_t)p.B * sizeof(Record), 256);
-  p.cand = reinterpret_cast<float4 *>(w8);
-  w8 += round_up((size_t)p.B * p.ndraw * 48, 256);
+  p.gm = reinterpret_cast<float4 *>(w8);
+  w8 += round_up((size_t)p.B * p.ngroups * 16, 256);
   p.counters = reinterpret_cast<unsigned int *>(w8);
   p.status = device_status_word();
   cudaStream_t st = (cudaStream_t)stream;
   const bool plain = sampling && p.k == 0;
   if (plain) {
-    if (launch(clear_tickets_kernel, dim3(1), dim3(kDrawThreads), 0, st, p.counters, p.B) !=
+    if (launch(clear_tickets_kernel, dim3(1), dim3(kMassThreads), 0, st, p.counters, p.B) !=
         cudaSuccess)
       return SD_ERR_CUDA;
   } else {
@@ -693,7 +773,7 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
     if (!sampling) return SD_OK;  // greedy: the decision pass wrote the outputs
   }
   return cuda_status(
-      launch(accept_draw_kernel, dim3(p.B, p.ndraw), dim3(kDrawThreads), 0, st, p));
+      launch(accept_mass_kernel, dim3(p.B, p.nmass), dim3(kMassThreads), 0, st, p));
 }
 
 }  // extern "C"

@@ -7,7 +7,8 @@ rotated over more than L2 where they are large), for micro-benchmarks and profil
     python -m verify_step_b200.probe head --m 24 --d 5376 --vocab 65536
     python -m verify_step_b200.probe attn --batch 2 --ctx 16384 --head-dim 512 --k 2
 
---reps 1 --warmup 1 runs the call twice (one warm-up) for a profiler capture.  Inputs are
+--reps 1 --warmup 1 runs the call twice (one warm-up), eagerly, for a profiler capture; more
+repetitions are timed as replays of a CUDA graph holding them.  Inputs are
 random (torch on the device); nothing is checked here: the tests hold the parity checks.
 Prints one line per shape: microseconds per call and the weight / logit / KV stream rate.
 """
@@ -25,16 +26,33 @@ def _events(torch):
 
 
 def _time(torch, fn, reps, warmup):
+    """Microseconds per call.  With more than one repetition the calls are captured once in a
+    CUDA graph and the graph is replayed, so that host launch overhead does not set the time of
+    short calls; with one (a profiler capture) they run eagerly."""
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
     e0, e1 = _events(torch)
+    if reps <= 1:
+        e0.record()
+        for i in range(reps):
+            fn(warmup + i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / max(reps, 1) * 1e3
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            fn(warmup + i)
+    g.replay()
+    torch.cuda.synchronize()
+    replays = 3
     e0.record()
-    for i in range(reps):
-        fn(warmup + i)
+    for _ in range(replays):
+        g.replay()
     e1.record()
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / max(reps, 1) * 1e3
+    return e0.elapsed_time(e1) / (replays * reps) * 1e3
 
 
 def run_accept(a, torch, sd):
