@@ -294,7 +294,18 @@ __global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Par
   const bool sampling = p.T > 0.f;
   if (threadIdx.x == 0) {
     s_step = counter_step(p);
-    if (sampling) p.counters[b] = 0u;  // tickets of the draw kernel
+    if (sampling) p.counters[b] = 0u;  // tickets of the group-mass kernel
+  }
+  // the drafts and their logits, loaded before the merge so that their round trips overlap it
+  // (warp 0, lane i - 1 for draft i)
+  int d = -1;
+  float zd = 0.f, yd = 0.f;
+  if (warp == 0 && lane < p.k) {
+    d = p.drafts[(size_t)b * p.k + lane];
+    if (sampling && d >= 0 && d < p.V) {
+      zd = p.z[(size_t)(b * p.n_q + lane) * p.ld_t + d];
+      yd = p.y[((size_t)b * p.k + lane) * p.ld_d + d];
+    }
   }
   // merge the chunks of each row (one warp per row, lanes over chunks, fixed order)
   for (int ri = warp; ri < p.rps; ri += kDecideThreads / 32) {
@@ -327,7 +338,6 @@ __global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Par
   bool acc = true;
   int flag = 0;
   if (lane < p.k) {
-    const int d = p.drafts[(size_t)b * p.k + lane];
     const int rt = b * p.n_q + lane;
     const float4 sz = s_row[lane];
     if (d < 0 || d >= p.V) {
@@ -335,8 +345,8 @@ __global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Par
       acc = false;
     } else if (sampling) {
       const float4 sy = s_row[p.n_q + lane];
-      const float pd = expf(p.z[(size_t)rt * p.ld_t + d] * inv_t - sz.x) / sz.y;
-      const float qd = expf(p.y[((size_t)b * p.k + lane) * p.ld_d + d] * inv_t - sy.x) / sy.y;
+      const float pd = expf(zd * inv_t - sz.x) / sz.y;
+      const float qd = expf(yd * inv_t - sy.x) / sy.y;
       const float ratio = qd > 0.f ? pd / qd : (pd > 0.f ? INFINITY : 0.f);
       const float u = accept_uniform(p.seed, step, (uint32_t)rt);
       flag = fabsf(u - ratio) < kMargin;
