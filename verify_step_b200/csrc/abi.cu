@@ -122,6 +122,21 @@ bool encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_tmap_kv_chunks_bf16(CUtensorMap *map, const void *base, uint64_t D, uint64_t rows,
+                                uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || D % 64) return false;
+  // (64 columns, rows, D / 64 column chunks): one box = box_rows rows of every chunk, laid
+  // out chunk-major in shared memory, each chunk's rows 128 bytes with the 128-byte swizzle
+  const cuuint64_t dims[3] = {64, rows, D / 64};
+  const cuuint64_t strides[2] = {D * 2, 128};
+  const cuuint32_t box[3] = {64, box_rows, (cuuint32_t)(D / 64)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace sdv
 
 extern "C" {

@@ -38,8 +38,7 @@ namespace attn {
 
 constexpr int kTile = 16;
 constexpr float kRescale = 8.f;  // log2 headroom of the lazily rescaled softmax
-constexpr int kCombineThreads = 256;
-constexpr int kMaxGroups = 1024;  // stream-K groups of the split-KV grid at most (combine slots)
+constexpr int kMaxGroups = 1024;  // stream-K groups of the split-KV grid at most
 
 struct Params {
   int B, n_q, Hq, Hkv, G, D, bs, mbps, num_blocks, window, M;
@@ -62,6 +61,7 @@ struct Params {
   const void *v_new;
   void *k_cache;
   void *v_cache;
+  int kv3d;        // the K / V tensor maps are the 3D chunk view (one box per tile)
   int P;           // CTA groups of the persistent split-KV grid (stream-K units)
   int row_groups;  // CTAs per group: each takes one row group of the item, same tile range
   int *status;
@@ -414,10 +414,15 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES, SPLIT>::THREADS,
           uint8_t *kd = stages + (size_t)stage * C::STAGE_BYTES;
           uint8_t *vd = kd + C::TILE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          if (p.kv3d) {  // one box per tile brings every column chunk
+            tma_load_3d(kd, &kmap, &full[stage], 0, row, 0);
+            tma_load_3d(vd, &vmap, &full[stage], 0, row, 0);
+          } else {
 #pragma unroll
-          for (int ch = 0; ch < D / 64; ++ch) {
-            tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
-            tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+            for (int ch = 0; ch < D / 64; ++ch) {
+              tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
+              tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+            }
           }
         }
       }
@@ -869,10 +874,15 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
           uint8_t *kd = stages + (size_t)stage * C::STAGE_BYTES;
           uint8_t *vd = kd + C::TILE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          if (p.kv3d) {  // one box per tile brings every column chunk
+            tma_load_3d(kd, &kmap, &full[stage], 0, row, 0);
+            tma_load_3d(vd, &vmap, &full[stage], 0, row, 0);
+          } else {
 #pragma unroll
-          for (int ch = 0; ch < D / 64; ++ch) {
-            tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
-            tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+            for (int ch = 0; ch < D / 64; ++ch) {
+              tma_load_2d(kd + ch * (kTile * 128), &kmap, &full[stage], ch * 64, row);
+              tma_load_2d(vd + ch * (kTile * 128), &vmap, &full[stage], ch * 64, row);
+            }
           }
         }
       }
@@ -1220,18 +1230,16 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
 // Merges the partials of items that several CTAs shared, in CTA order; writes zero rows for
 // drafter items with an empty key range.  One CTA per (item, query row).
 template <typename T>
-__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const Params p) {
-  constexpr int kWarps = kCombineThreads / 32;
+__global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
+  constexpr int kChunk = 512;
   __shared__ long long s_F, s_Fl, s_T;
   __shared__ int s_n;
-  __shared__ float s_w[kMaxGroups];
-  __shared__ float2 s_red[kWarps];
-  __shared__ float4 s_part[kWarps][128];  // per-warp partial rows, D <= 512
+  __shared__ float s_w[kChunk];
+  __shared__ float s_red[4];
   pdl_trigger();
   pdl_wait();
   const int item = blockIdx.x, row = blockIdx.y;
   const int b = item / p.Hkv, g = item % p.Hkv;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x < 32) {  // tile counts of all sequences, one warp
     long long pre = 0, T_all = 0;
     int n = 0;
@@ -1266,100 +1274,76 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const Par
   const int c_last = (int)(((Fl + 1) * p.P - 1) / T_all);
   if (c_first == c_last) return;  // written directly by its only CTA
   const size_t slot0 = (size_t)b * p.Hkv + g;
-  // CTA group c holds tiles [T*c/P, T*(c+1)/P); with fewer tiles than groups some hold none
-  // and wrote no partial for this item.
+  // CTA c holds tiles [T*c/P, T*(c+1)/P); with fewer tiles than CTAs some hold none and
+  // wrote no partial for this item.
   auto holds = [&](int c) {
     const long long s_c = T_all * c / p.P, e_c = T_all * (c + 1) / p.P;
     return e_c > F && s_c <= Fl && e_c > s_c;
   };
-  const int S = c_last - c_first + 1;  // at most P <= kMaxGroups
-  // (max, sum of 2^(m - max) l) over the slots, one pass, merged in a fixed order
-  float M = -INFINITY, L = 0.f;
-  for (int t = threadIdx.x; t < S; t += blockDim.x) {
-    if (!holds(c_first + t)) continue;
-    const size_t sl = (slot0 + c_first + t) * p.Mpad + row;
-    const float m = __ldcg(p.ws_ml + sl * 2), l = __ldcg(p.ws_ml + sl * 2 + 1);
-    if (m == -INFINITY) continue;
-    const float mm = fmaxf(M, m);
-    L = L * exp2f(M - mm) + l * exp2f(m - mm);
-    M = mm;
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, M, o);
-    const float l2 = __shfl_xor_sync(0xffffffffu, L, o);
-    const float mm = fmaxf(M, m2);
-    if (mm != -INFINITY) {
-      L = L * exp2f(M - mm) + l2 * exp2f(m2 - mm);
-      M = mm;
+  auto block_reduce = [&](float v, bool is_max) {
+    for (int o = 16; o > 0; o >>= 1) {
+      const float u = __shfl_xor_sync(0xffffffffu, v, o);
+      v = is_max ? fmaxf(v, u) : v + u;
     }
-  }
-  if (lane == 0) s_red[warp] = make_float2(M, L);
-  __syncthreads();
-  float mmax = -INFINITY, den = 0.f;
-  for (int w = 0; w < kWarps; ++w) {
-    const float2 r = s_red[w];
-    const float mm = fmaxf(mmax, r.x);
-    if (mm == -INFINITY) continue;
-    den = den * exp2f(mmax - mm) + r.y * exp2f(r.x - mm);
-    mmax = mm;
-  }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = s_red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = is_max ? fmaxf(r, s_red[w]) : r + s_red[w];
+    return r;
+  };
+  const int S = c_last - c_first + 1;
+  float mloc = -INFINITY;
+  for (int t = threadIdx.x; t < S; t += blockDim.x)
+    if (holds(c_first + t))
+      mloc = fmaxf(mloc, p.ws_ml[((slot0 + c_first + t) * p.Mpad + row) * 2]);
+  const float mmax = block_reduce(mloc, true);
+  float den_loc = 0.f;
+  if (mmax != -INFINITY)
+    for (int t = threadIdx.x; t < S; t += blockDim.x)
+      if (holds(c_first + t)) {
+        const size_t sl = (slot0 + c_first + t) * p.Mpad + row;
+        den_loc += exp2f(p.ws_ml[sl * 2] - mmax) * p.ws_ml[sl * 2 + 1];
+      }
+  const float den = block_reduce(den_loc, false);
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  for (int t = threadIdx.x; t < S; t += blockDim.x) {
-    const int c = c_first + t;
-    s_w[t] = (mmax != -INFINITY && holds(c))
-                 ? exp2f(__ldcg(p.ws_ml + ((slot0 + c) * p.Mpad + row) * 2) - mmax)
-                 : 0.f;
-  }
-  __syncthreads();
-  // weighted sum of the partial rows: warp w takes slots w, w + kWarps, ...; lane l columns
-  // 4 (l + 32 e), e < D / 128, as 16-byte loads, two slots' loads in flight together
-  const int n4 = p.D / 4;
-  float4 acc[4];
+  // weighted sum of the partial rows, slots in CTA order, kChunk slots at a time; the loads
+  // of 8 slots are issued before their multiply-adds (they are independent L2 reads)
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // D <= 512 with 128 threads
+  for (int t0 = 0; t0 < S; t0 += kChunk) {
+    const int n = min(kChunk, S - t0);
+    __syncthreads();
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+      const int c = c_first + t0 + t;
+      s_w[t] = (mmax != -INFINITY && holds(c))
+                   ? exp2f(p.ws_ml[((slot0 + c) * p.Mpad + row) * 2] - mmax)
+                   : 0.f;
+    }
+    __syncthreads();
+    for (int u0 = 0; u0 < n; u0 += 8) {
+      float v[8][4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int t0 = warp; t0 < S; t0 += 2 * kWarps) {
-    float4 v[2][4];
-    float w[2];
+      for (int u = 0; u < 8; ++u) {
+        const float w = u0 + u < n ? s_w[u0 + u] : 0.f;
+        const float *o = p.ws_o + ((slot0 + c_first + t0 + u0 + u) * p.Mpad + row) * p.D;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int t = t0 + u * kWarps;
-      w[u] = t < S ? s_w[t] : 0.f;
-      const float4 *o = reinterpret_cast<const float4 *>(
-          p.ws_o + ((slot0 + c_first + t) * p.Mpad + row) * p.D);
+        for (int e = 0; e < 4; ++e) {
+          const int d = threadIdx.x + e * 128;
+          v[u][e] = (w != 0.f && d < p.D) ? __ldcg(o + d) : 0.f;
+        }
+      }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c4 = lane + 32 * e;
-        v[u][e] = (w[u] != 0.f && c4 < n4) ? __ldcg(o + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 8; ++u) {
+        const float w = u0 + u < n ? s_w[u0 + u] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
       }
     }
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[e].x = fmaf(w[u], v[u][e].x, acc[e].x);
-        acc[e].y = fmaf(w[u], v[u][e].y, acc[e].y);
-        acc[e].z = fmaf(w[u], v[u][e].z, acc[e].z);
-        acc[e].w = fmaf(w[u], v[u][e].w, acc[e].w);
-      }
   }
 #pragma unroll
-  for (int e = 0; e < 4; ++e)
-    if (lane + 32 * e < n4) s_part[warp][lane + 32 * e] = acc[e];
-  __syncthreads();
-  // the warps' partials summed in warp order
-  for (int c4 = threadIdx.x; c4 < n4; c4 += blockDim.x) {
-    float4 r = s_part[0][c4];
-    for (int w = 1; w < kWarps; ++w) {
-      const float4 q = s_part[w][c4];
-      r.x += q.x;
-      r.y += q.y;
-      r.z += q.z;
-      r.w += q.w;
-    }
-    dst[4 * c4 + 0] = T(r.x * inv);
-    dst[4 * c4 + 1] = T(r.y * inv);
-    dst[4 * c4 + 2] = T(r.z * inv);
-    dst[4 * c4 + 3] = T(r.w * inv);
+  for (int e = 0; e < 4; ++e) {
+    const int d = threadIdx.x + e * 128;
+    if (d < p.D) dst[d] = T(acc[e] * inv);
   }
 }
 
@@ -1761,8 +1745,11 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
                                       round_up(slots * p.Mpad * p.D * 4, 256));
   CUtensorMap km, vm;
   const uint64_t rows = (uint64_t)p.num_blocks * p.Hkv * p.bs;
-  if (!encode_tmap_2d_bf16(&km, k_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile) ||
-      !encode_tmap_2d_bf16(&vm, v_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile))
+  p.kv3d = encode_tmap_kv_chunks_bf16(&km, k_cache, p.D, rows, kTile) &&
+           encode_tmap_kv_chunks_bf16(&vm, v_cache, p.D, rows, kTile);
+  if (!p.kv3d &&
+      (!encode_tmap_2d_bf16(&km, k_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile) ||
+       !encode_tmap_2d_bf16(&vm, v_cache, p.D, rows, (uint64_t)p.D * 2, 64, kTile)))
     return SD_ERR_CUDA;
   const bool window = p.window > 0 && p.window <= kWinMax && MT <= 2;
   if (!draft && window && MT == 1) {
@@ -1785,8 +1772,7 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   s = launch_bf16(p.D, rs, km, vm, p, st);
   if (s != SD_OK) return s;
   return cuda_status(
-      launch(attn_combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hkv, p.M), dim3(kCombineThreads), 0,
-             st, p));
+      launch(attn_combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hkv, p.M), dim3(128), 0, st, p));
 }
 
 }  // namespace attn

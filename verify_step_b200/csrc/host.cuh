@@ -40,6 +40,13 @@ bool encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uin
                          uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                          bool swizzle128 = true);
 
+// A [rows x D] bf16 matrix viewed as (64 columns, rows, D / 64 chunks), so that one 3D box of
+// box_rows rows brings all of a row block's column chunks at once, chunk-major with the 128-byte
+// swizzle (the layout of box_rows x 64 2D boxes stored one after another).  False if the driver
+// refuses the view.
+bool encode_tmap_kv_chunks_bf16(CUtensorMap *map, const void *base, uint64_t D, uint64_t rows,
+                                uint32_t box_rows);
+
 inline sd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_CUDA; }
 
 // Programmatic dependent launch: off unless the environment sets SDV_PDL=1 (read once per

@@ -5,7 +5,8 @@ rotated over more than L2 where they are large), for micro-benchmarks and profil
     python -m verify_step_b200.probe linear --m 24 --n 43008 --kdim 5376 [--epilogue geglu]
                                             [--x f32|bf16] [--norm] [--out f32|bf16]
     python -m verify_step_b200.probe head --m 24 --d 5376 --vocab 65536
-    python -m verify_step_b200.probe attn --batch 2 --ctx 16384 --head-dim 512 --k 2
+    python -m verify_step_b200.probe head --m 8 --d 1024 --clusters 1024 [--top-c 32]
+    python -m verify_step_b200.probe attn --batch 2 --ctx 16384 --head-dim 512 --k 2 [--draft]
 
 --reps 1 --warmup 1 runs the call twice (one warm-up), eagerly, for a profiler capture; more
 repetitions are timed as replays of a CUDA graph holding them.  Inputs are
@@ -109,7 +110,34 @@ def run_linear(a, torch, sd):
           f"{n * k * 2 / (us * 1e3):.0f} GB/s of weights")
 
 
+def run_head_clustered(a, torch, sd):
+    """The clustered head: centroid scores, top-c selection, exact logits of the kept clusters
+    (cluster-major weights; random cluster membership, as the benchmark's drafter head)."""
+    m, d, V, C = a.m, a.d, a.vocab, a.clusters
+    cs = V // C
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    h = torch.randn(m, d, device="cuda", generator=g).to(torch.bfloat16)
+    w_cm = (torch.randn(C, cs, d, device="cuda", generator=g) / math.sqrt(d)).to(torch.bfloat16)
+    cent = w_cm.float().mean(dim=1).to(torch.bfloat16)
+    tokens = torch.randperm(V, device="cuda", generator=g).to(torch.int32).reshape(C, cs)
+    out = torch.empty(m, V, device="cuda")
+    sel = torch.empty(m, a.top_c, dtype=torch.int32, device="cuda")
+    desc = sd.HeadDesc(m=m, d=d, vocab=V, n_clusters=C, cluster_size=cs, top_c=a.top_c,
+                       dtype=sd.SD_BF16)
+    ws = torch.empty(max(256, sd.sd_lm_head_workspace_size(desc)), dtype=torch.uint8,
+                     device="cuda")
+    us = _time(torch, lambda i: sd.sd_lm_head(desc, h, w_cm, out, centroids=cent,
+                                              cluster_tokens=tokens, sel_clusters=sel, ws=ws),
+               a.reps, a.warmup)
+    gb = (C * d * 2 + m * a.top_c * cs * d * 2 + m * V * 4) / 1e9
+    print(f"clustered head m{m} d{d} V{V} C{C} top{a.top_c}: {us:.1f} us, "
+          f"{gb / (us * 1e-6):.0f} GB/s (centroids, kept clusters' weights, logit rows)")
+
+
 def run_head(a, torch, sd):
+    if a.clusters:
+        return run_head_clustered(a, torch, sd)
     m, d, V = a.m, a.d, a.vocab
     h = torch.randn(m, d, device="cuda").to(torch.bfloat16)
     copies = 1 if a.reps <= 1 else max(2, int(300e6 // (V * d * 2)) + 1)
@@ -138,15 +166,26 @@ def run_attn(a, torch, sd):
                        window=W, scale=1 / math.sqrt(D), dtype=sd.SD_BF16)
     kc, vc, tab, ctx = g(c["k_cache"]), g(c["v_cache"]), g(c["table"]), g(torch.from_numpy(L))
     q, kn, vn = g(s["q"]), g(s["k_new"]), g(s["v_new"])
-    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(max(256, sd.sd_verify_attn_workspace_size(desc)), dtype=torch.uint8,
-                     device="cuda")
-    us = _time(torch, lambda i: sd.sd_verify_attn(desc, q, kn, vn, kc, vc, tab, ctx, out, ws),
-               a.reps, a.warmup)
-    keys = (L + a.k + 1) if W == 0 else [min(int(x) + a.k + 1, W + a.k) for x in L]
+    if a.draft:  # the drafter's read-only cross-attention: one query per sequence at L - 1
+        desc.n_q = 1
+        q = q[:, :1].contiguous()
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(max(256, sd.sd_draft_xattn_workspace_size(desc)), dtype=torch.uint8,
+                         device="cuda")
+        qpos = (ctx - 1).to(torch.int32)
+        us = _time(torch, lambda i: sd.sd_draft_xattn(desc, q, kc, vc, tab, ctx, qpos, out, ws),
+                   a.reps, a.warmup)
+        keys = L if W == 0 else [min(int(x), W) for x in L]
+    else:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(max(256, sd.sd_verify_attn_workspace_size(desc)), dtype=torch.uint8,
+                         device="cuda")
+        us = _time(torch, lambda i: sd.sd_verify_attn(desc, q, kn, vn, kc, vc, tab, ctx, out,
+                                                      ws), a.reps, a.warmup)
+        keys = (L + a.k + 1) if W == 0 else [min(int(x) + a.k + 1, W + a.k) for x in L]
     gb = sum(int(x) for x in keys) * 4 * D * 2 * 2 / 1e9
-    print(f"attn B{a.batch} ctx{a.ctx} D{D} W{W} k{a.k}: {us:.1f} us, "
-          f"{gb / (us * 1e-6):.0f} GB/s of K/V")
+    print(f"{'xattn' if a.draft else 'attn'} B{a.batch} ctx{a.ctx} D{D} W{W} k{a.k}: "
+          f"{us:.1f} us, {gb / (us * 1e-6):.0f} GB/s of K/V")
 
 
 def main(argv=None):
@@ -167,6 +206,9 @@ def main(argv=None):
     ap.add_argument("--ctx", type=int, default=16384)
     ap.add_argument("--head-dim", type=int, default=512)
     ap.add_argument("--window", type=int, default=0)
+    ap.add_argument("--draft", action="store_true", help="attn: the drafter cross-attention")
+    ap.add_argument("--clusters", type=int, default=0, help="head: clustered head with C clusters")
+    ap.add_argument("--top-c", type=int, default=32)
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     a = ap.parse_args(argv)
