@@ -432,12 +432,12 @@ __global__ void __launch_bounds__(256) cluster_logits_kernel(
 // kClTok): the work is M * top_c * cs / kClTok units of kClTok tokens, each unit's weights one
 // contiguous block of the cluster-major matrix.  A persistent CTA per SM takes a contiguous
 // range of units; its producer warp streams them (weights and token ids, cp.async.bulk) through
-// a kClStages-deep mbarrier ring, and each of the kClWarps consumer warps takes two tokens of a
+// a kClStages-deep mbarrier ring, and each of the kClWarps consumer warps takes one token of a
 // unit: lane l multiplies elements l*8 + q*256 + [0, 8) of the staged row with the hidden
-// values it keeps in registers (reloaded when the row m changes).
+// values it keeps in registers (reloaded when the row m changes), in two accumulator chains.
 constexpr int kClTok = 16;
 constexpr int kClStages = 6;
-constexpr int kClWarps = kClTok / 2;
+constexpr int kClWarps = kClTok;  // one token per warp: 17 warps per SM hide the latency
 constexpr int kClUnitBytes = kClTok * 1024 * 2;  // largest unit (d = 1024)
 constexpr size_t kClSmem = 128 + (size_t)kClStages * kClUnitBytes + kClStages * kClTok * 4 +
                            kClStages * 16 + kClStages * 16 + 16;
@@ -530,32 +530,27 @@ __global__ void __launch_bounds__(32 * (kClWarps + 1), 1) cluster_logits_tma_ker
         }
         m_loaded = r.x;
       }
-      float acc[2];
+      const uint8_t *row = stages + (size_t)stg * kClUnitBytes + (size_t)warp * d * 2;
+      float acc2[2] = {0.f, 0.f};
 #pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        const uint8_t *row = stages + (size_t)stg * kClUnitBytes + (size_t)(warp * 2 + tt) * d * 2;
-        acc[tt] = 0.f;
+      for (int q = 0; q < 4; ++q) {
+        const int k0 = lane * 8 + q * 256;
+        if (q < nk && k0 < d) {
+          const uint4 raw = *reinterpret_cast<const uint4 *>(row + (size_t)k0 * 2);
+          const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int k0 = lane * 8 + q * 256;
-          if (q < nk && k0 < d) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(row + (size_t)k0 * 2);
-            const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&raw);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[tt] = fmaf(__bfloat162float(e[j]), hr[q][j], acc[tt]);
-          }
+          for (int j = 0; j < 8; ++j)
+            acc2[j & 1] = fmaf(__bfloat162float(e[j]), hr[q][j], acc2[j & 1]);
         }
       }
-#pragma unroll
-      for (int tt = 0; tt < 2; ++tt)
-        for (int o = 16; o > 0; o >>= 1) acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], o);
-      if (lane < 2) {
-        const int t = warp * 2 + lane;
-        const int id = tok[stg * kClTok + t];
+      float acc = acc2[0] + acc2[1];
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) {
+        const int id = tok[stg * kClTok + warp];
         if (id < 0 || id >= V)
           record_status(status, SD_ERR_DEVICE);
         else
-          logits[(size_t)r.x * ld + id] = lane == 0 ? acc[0] : acc[1];
+          logits[(size_t)r.x * ld + id] = acc;
       }
     }
     __syncwarp();
