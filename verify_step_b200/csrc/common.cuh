@@ -330,6 +330,15 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 
 // Every thread of every CTA of the cluster arrives (release) and waits (acquire): this CTA's
 // shared-memory writes before it are visible to the cluster's reads after it.
+// The two halves of a cluster barrier, for work between them (every thread of the cluster
+// arrives once and waits once per phase; warp-converged).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }

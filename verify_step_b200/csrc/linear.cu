@@ -20,9 +20,13 @@
 //     copies (no multicast; W evict-first, x' evict-last), warp 1 issues tcgen05.mma from one
 //     thread, warps 2-5 read the accumulator (thread = output row).  Persistent: one CTA per
 //     SM walks the work units (tile, K split); the K dimension is split so that the units
-//     spread evenly over the SMs.  A split writes its [128 x m] partial to the workspace; the
-//     last split of a tile to finish (atomic ticket, no waiting) adds the partials in split
-//     order, so the result does not depend on the timing, and applies the epilogue.
+//     spread evenly over the SMs.  When every unit gets its own SM and a tile has 2, 4 or 8
+//     splits, the splits are one thread-block cluster: each pushes its partial rows into the
+//     shared memory of the CTA owning them and, after one cluster barrier, the owners add the
+//     partials in split order and apply the epilogue.  Otherwise a split writes its [128 x m]
+//     partial to the workspace and the last split of a tile to finish (atomic ticket, no
+//     waiting) adds the partials in split order; either way the result does not depend on
+//     the timing.
 #include <algorithm>
 
 #include "common.cuh"
@@ -53,6 +57,7 @@ struct Params {
   __nv_bfloat16 *xp;  // x' [m][k64] bf16 (workspace)
   // product
   int tiles, kblocks, splits, kb_per_split, units;
+  int cluster;  // the splits of a tile are one thread-block cluster: partials summed via DSMEM
   int epi, out_f32;
   long long ld_out;
   void *out;
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(kStageThreads) linear_stage_kernel(const Param
   pdl_wait();
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (r == 0 && p.splits > 1)
+  if (r == 0 && p.splits > 1 && !p.cluster)
     for (int t = tid; t < p.tiles; t += blockDim.x) p.tickets[t] = 0u;
   if (tid == 0) {
     int t = -1;
@@ -158,17 +163,20 @@ struct UCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (192 * 1024 / STAGE_BYTES) < 8 ? (192 * 1024 / STAGE_BYTES) : 8;
   static constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : 128;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 8 * (2 * STAGES + 4) + 64;
+  static constexpr int RECV_BYTES = BM * N * 4;  // partial rows pushed by the cluster's CTAs
+  static constexpr size_t SMEM =
+      1024 + (size_t)STAGES * STAGE_BYTES + RECV_BYTES + 8 * (2 * STAGES + 4) + 64;
   static constexpr int THREADS = 192;
 };
 
 // The epilogue of one output row i (this thread's) for token r: y = the row's product.  The
 // gated form pairs row i (a gate row: i % 16 < 8) with row i + 8 of the same warp (lane + 8);
 // every lane of the warp calls it for the same r.
-__device__ __forceinline__ void apply_epilogue(const Params &p, int i, int r, float y, int lane) {
+__device__ __forceinline__ void apply_epilogue(const Params &p, int i, int r, float y, int lane,
+                                               bool active = true) {
   if (p.epi == SD_EPI_GEGLU) {
     const float yu = __shfl_down_sync(0xffffffffu, y, 8);
-    if ((lane & 8) == 0 && r < p.m) {
+    if (active && (lane & 8) == 0 && r < p.m) {
       const int f = (i >> 4) * 8 + (i & 7);
       if (f < p.n / 2)
         static_cast<__nv_bfloat16 *>(p.out)[r * p.ld_out + f] =
@@ -176,7 +184,7 @@ __device__ __forceinline__ void apply_epilogue(const Params &p, int i, int r, fl
     }
     return;
   }
-  if (r >= p.m || i >= p.n) return;
+  if (!active || r >= p.m || i >= p.n) return;
   const long long o = r * p.ld_out + i;
   if (p.epi == SD_EPI_ADD)
     static_cast<float *>(p.out)[o] += y;
@@ -195,7 +203,9 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)STAGES * C::STAGE_BYTES);
+  float *recv = reinterpret_cast<float *>(smem + (size_t)STAGES * C::STAGE_BYTES);  // [BM][N]
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)STAGES * C::STAGE_BYTES +
+                                                C::RECV_BYTES);
   uint64_t *empty = full + STAGES;
   uint64_t *tfull = empty + STAGES;   // [2] accumulator ready
   uint64_t *tempty = tfull + 2;       // [2] accumulator drained
@@ -223,6 +233,9 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // cluster mode: an arrival now, and a wait before the first distributed-shared-memory store,
+  // so that no CTA writes into a peer that has not started
+  if (p.cluster) cluster_arrive_relaxed();
   const uint32_t tmem_base = *tmem_slot;
   // x' and the tickets come from the staging kernel, which this kernel may overlap (it is
   // launched as its programmatic dependent): every role waits for it before touching global
@@ -330,8 +343,46 @@ __global__ void __launch_bounds__(192, 1)
     // warp skips the work (later waits return at once) but keeps the barriers.
     const int quad = warp & 3;  // tensor-memory lanes 32*quad .. 32*quad+31
     const int row_in_tile = quad * 32 + lane;
+    if (p.cluster) {
+      // one unit per CTA; the tile's splits are the cluster's CTAs.  Each row of this split's
+      // partial goes to the shared memory of the CTA owning the row (CTA r owns rows
+      // [r BM/S, (r+1) BM/S)); the owners add them after the cluster barrier below.
+      bool ok = *abort_flag == 0 && mbar_wait(&tfull[0], 0, abort_flag);
+      if (!ok && *abort_flag == 0) {
+        record_status(p.status, SD_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      tc_fence_after();
+      float y[N];
+      if (ok) {
+        const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+#pragma unroll
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          uint32_t rr[16];
+          tmem_ld16(taddr + c0, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) y[c0 + e] = __uint_as_float(rr[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < N; ++e) y[e] = 0.f;
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[0]);
+      cluster_wait();
+      const uint32_t rank = cluster_ctarank();
+      const int rows_per = BM / p.splits;
+      const int owner = row_in_tile / rows_per;
+      const uint32_t dst = dsmem_addr(
+          smem_u32(recv + ((size_t)rank * rows_per + (row_in_tile - owner * rows_per)) * N),
+          (uint32_t)owner);
+#pragma unroll
+      for (int r = 0; r < N; r += 4)
+        st_dsmem_f4(dst + r * 4, make_float4(y[r], y[r + 1], y[r + 2], y[r + 3]));
+    }
     uint32_t i = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++i) {
+    for (int u = blockIdx.x; u < p.units && !p.cluster; u += gridDim.x, ++i) {
       const int tile = u / p.splits;
       const uint32_t buf = i & 1, tph = (i >> 1) & 1;
       bool ok = *abort_flag == 0 && mbar_wait(&tfull[buf], tph, abort_flag);
@@ -411,6 +462,40 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   }
+  if (p.cluster) {
+    // every CTA of the cluster reaches this barrier once (no role returns early), so all partial
+    // rows have landed in their owners after it; each owner adds its rows' S partials in split
+    // order and applies the epilogue
+    if (warp < 2) cluster_wait();  // the first phase (the epilogue warps waited before storing)
+    cluster_sync();
+    if (warp >= 2) {
+      const int quad = warp & 3;
+      const int row_in_tile = quad * 32 + lane;
+      const int rank = (int)cluster_ctarank();
+      const int rows_per = BM / p.splits;
+      const bool mine = row_in_tile / rows_per == rank;
+      const int tile = blockIdx.x / p.splits;
+      float acc[N];
+#pragma unroll
+      for (int r = 0; r < N; ++r) acc[r] = 0.f;
+      if (mine) {
+        for (int sp = 0; sp < p.splits; ++sp) {
+          const float4 *src = reinterpret_cast<const float4 *>(
+              recv + ((size_t)sp * rows_per + (row_in_tile - rank * rows_per)) * N);
+#pragma unroll
+          for (int r = 0; r < N; r += 4) {
+            const float4 v = src[r / 4];
+            acc[r] += v.x;
+            acc[r + 1] += v.y;
+            acc[r + 2] += v.z;
+            acc[r + 3] += v.w;
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < N; ++r) apply_epilogue(p, tile * BM + row_in_tile, r, acc[r], lane, mine);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -429,6 +514,7 @@ __global__ void __launch_bounds__(192, 1)
 
 struct Shape {
   int N, tiles, kblocks, splits, kb_per_split, units, grid;
+  bool cluster;
 };
 
 static int n_of(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 48 ? 48 : 64; }
@@ -438,7 +524,11 @@ static int n_of(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 48 ? 48 : 64;
 // of weights and 4 KB of x' at a fair share of the HBM rate) plus, when split, about 2.5 us of
 // partial write, fence and ticket; and the reductions the SM finishes (ceil(tiles / SMs) tiles,
 // about 0.5 us per split read back).
-static Shape shape_of(int m, int n, int k) {
+// Clusters of S CTAs of the product kernel for N that fit on the device at once (0 where the
+// device cannot say, e.g. without a GPU).
+static int max_clusters(int N, int S);
+
+static Shape shape_of(int m, int n, int k, bool allow_cluster = false) {
   Shape s;
   s.N = n_of(m);
   s.tiles = (n + BM - 1) / BM;
@@ -459,10 +549,26 @@ static Shape shape_of(int m, int n, int k) {
       best_s = S;
     }
   }
+  // the splits of a tile as one cluster (2, 4 or 8 CTAs, whole 16-row blocks per owner) when
+  // every unit gets its own SM: partials summed through distributed shared memory, about
+  // 0.8 us, no workspace round trip or ticket
+  bool cluster = false;
+  for (int S = 2; S <= 8 && allow_cluster; S *= 2) {
+    if (S > s.kblocks || (long long)s.tiles * S > sms || s.tiles > max_clusters(s.N, S)) break;
+    const int kps = (s.kblocks + S - 1) / S;
+    if ((s.kblocks + kps - 1) / kps != S) continue;
+    const double cost = kps * 0.36 + 0.8;
+    if (cost < best) {
+      best = cost;
+      best_s = S;
+      cluster = true;
+    }
+  }
   s.splits = best_s;
+  s.cluster = cluster;
   s.kb_per_split = (s.kblocks + best_s - 1) / best_s;
   s.units = s.tiles * best_s;
-  s.grid = std::min(s.units, sms);
+  s.grid = cluster ? s.units : std::min(s.units, sms);
   return s;
 }
 
@@ -475,7 +581,7 @@ static Layout layout_of(const sd_linear_desc *d, const Shape &s) {
   const size_t k64 = (size_t)s.kblocks * BK;
   l.xp = 0;
   l.part = round_up((size_t)d->m * k64 * 2, 256);
-  const size_t part_bytes = s.splits > 1 ? (size_t)s.units * s.N * BM * 4 : 0;
+  const size_t part_bytes = s.splits > 1 && !s.cluster ? (size_t)s.units * s.N * BM * 4 : 0;
   l.tickets = l.part + round_up(part_bytes, 256);
   l.total = l.tickets + round_up((size_t)s.tiles * 4, 256);
   return l;
@@ -517,7 +623,7 @@ static sd_status validate(const sd_linear_desc *d, const void *x, const void *W,
 // are one call), so its launch, set-up and first weight copies overlap the staging.
 template <int N>
 static sd_status launch_product(const CUtensorMap &wm, const CUtensorMap &xm, const Params &p,
-                                int grid, cudaStream_t st) {
+                                int grid, int cluster, cudaStream_t st) {
   using C = UCfg<N>;
   static int configured[64];
   int dev = 0;
@@ -533,12 +639,63 @@ static sd_status launch_product(const CUtensorMap &wm, const CUtensorMap &xm, co
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster > 1 ? cluster : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, linear_umma_kernel<N>, wm, xm, p));
+}
+
+template <int N>
+static int max_clusters_n(int S) {
+  using C = UCfg<N>;
+  if (cudaFuncSetAttribute(linear_umma_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)C::SMEM) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeClusterDimension;
+  a[0].val.clusterDim.x = S;
+  a[0].val.clusterDim.y = 1;
+  a[0].val.clusterDim.z = 1;
+  cfg.attrs = a;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, linear_umma_kernel<N>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return n;
+}
+
+static int max_clusters(int N, int S) {
+  static int cache[64][4][4];  // [device][N / 16 - 1][log2 S - 1] = value + 1
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  const int ni = N / 16 - 1, si = S == 2 ? 0 : S == 4 ? 1 : 2;
+  if (dev < 64 && cache[dev][ni][si] > 0) return cache[dev][ni][si] - 1;
+  int v = 0;
+  switch (N) {
+    case 16: v = max_clusters_n<16>(S); break;
+    case 32: v = max_clusters_n<32>(S); break;
+    case 48: v = max_clusters_n<48>(S); break;
+    default: v = max_clusters_n<64>(S); break;
+  }
+  if (dev < 64) cache[dev][ni][si] = v + 1;
+  return v;
 }
 
 }  // namespace lin
@@ -558,8 +715,10 @@ extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const voi
   using namespace sdv::lin;
   sd_status s = validate(d, x, W, out, table, tokens);
   if (s != SD_OK || d->m == 0) return s;
-  const Shape sh = shape_of(d->m, d->n, d->k);
-  const Layout lay = layout_of(d, sh);
+  // the workspace is laid out for the plan without clusters (the larger one), so its size
+  // does not depend on what the device reports
+  const Shape sh = shape_of(d->m, d->n, d->k, true);
+  const Layout lay = layout_of(d, shape_of(d->m, d->n, d->k));
   if (!d->ws || d->ws_bytes < lay.total || !aligned16(d->ws)) return SD_ERR_WORKSPACE;
   uint8_t *ws = static_cast<uint8_t *>(d->ws);
 
@@ -588,6 +747,7 @@ extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const voi
   p.splits = sh.splits;
   p.kb_per_split = sh.kb_per_split;
   p.units = sh.units;
+  p.cluster = sh.cluster ? 1 : 0;
   p.epi = d->epilogue;
   p.out_f32 = d->out_dtype == SD_F32;
   p.ld_out = d->ld_out;
@@ -606,10 +766,11 @@ extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const voi
   cudaStream_t st = (cudaStream_t)stream;
   if (launch(linear_stage_kernel, dim3(d->m), dim3(kStageThreads), 0, st, p) != cudaSuccess)
     return SD_ERR_CUDA;
+  const int cl = sh.cluster ? sh.splits : 1;
   switch (sh.N) {
-    case 16: return launch_product<16>(wm, xm, p, sh.grid, st);
-    case 32: return launch_product<32>(wm, xm, p, sh.grid, st);
-    case 48: return launch_product<48>(wm, xm, p, sh.grid, st);
-    default: return launch_product<64>(wm, xm, p, sh.grid, st);
+    case 16: return launch_product<16>(wm, xm, p, sh.grid, cl, st);
+    case 32: return launch_product<32>(wm, xm, p, sh.grid, cl, st);
+    case 48: return launch_product<48>(wm, xm, p, sh.grid, cl, st);
+    default: return launch_product<64>(wm, xm, p, sh.grid, cl, st);
   }
 }
