@@ -8,7 +8,8 @@
 // rows a projection reads each weight once and does 2m FLOPs with it: the weights' single pass
 // through HBM bounds it, as it bounds the LM head.
 //
-// Two kernels per call:
+// Two kernels per call (the first is skipped when the input is already bf16 rows that need no
+// normalisation, gather or padding and no tickets are used: the product then reads x itself):
 //  1. linear_stage_kernel: one CTA per token row gathers the row (the input columns and, for
 //     the drafter's first projection, an embedding row chosen by token id), normalises it
 //     (RMSNorm with gain) and writes it once as bf16 into the workspace, zero-padded to a
@@ -758,13 +759,23 @@ extern "C" sd_status sd_linear(const sd_linear_desc *d, const void *x, const voi
 
   // weights: [128 rows x 64 columns] boxes, 128-byte swizzle (rows past n and columns past k
   // arrive as zeros); x': [N rows x 64 columns] boxes of the m staged rows (rows past m zero)
+  // A bf16 input that needs no normalisation, gather or padding (and no split tickets to
+  // clear) is read by the product directly: no staging kernel
+  const bool direct = d->x_dtype == SD_BF16 && !d->norm_gain && d->k_gather == 0 &&
+                      d->k % BK == 0 && d->ld_x % 8 == 0 && !d->norm_out &&
+                      (sh.cluster || sh.splits == 1);
   CUtensorMap wm, xm;
+  const bool xok =
+      direct ? encode_tmap_2d_bf16(&xm, x, (uint64_t)d->k, (uint64_t)d->m,
+                                   (uint64_t)d->ld_x * 2, BK, (uint32_t)sh.N)
+             : encode_tmap_2d_bf16(&xm, p.xp, (uint64_t)p.k64, (uint64_t)d->m,
+                                   (uint64_t)p.k64 * 2, BK, (uint32_t)sh.N);
   if (!encode_tmap_2d_bf16(&wm, W, (uint64_t)d->k, (uint64_t)d->n, (uint64_t)d->k * 2, BK, BM) ||
-      !encode_tmap_2d_bf16(&xm, p.xp, (uint64_t)p.k64, (uint64_t)d->m, (uint64_t)p.k64 * 2, BK,
-                           (uint32_t)sh.N))
+      !xok)
     return SD_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  if (launch(linear_stage_kernel, dim3(d->m), dim3(kStageThreads), 0, st, p) != cudaSuccess)
+  if (!direct &&
+      launch(linear_stage_kernel, dim3(d->m), dim3(kStageThreads), 0, st, p) != cudaSuccess)
     return SD_ERR_CUDA;
   const int cl = sh.cluster ? sh.splits : 1;
   switch (sh.N) {
