@@ -275,3 +275,78 @@ def test_margin_flags_on_constructed_near_ties():
     assert gflags.tolist() == [1, 0]
     assert out[1, 0] == ref["out_tokens"][1, 0] == live[1]
     assert status_ok()
+
+
+def test_two_level_draw_over_several_groups_follows_p():
+    """Plain draws over 1300 tokens (groups of 512, 512 and a ragged 276, the last carrying
+    most of the mass): 200 000 GPU draws follow p (chi-square), and the first 2000 equal the
+    oracle's outside the margin."""
+    V, n = 1300, 200_000
+    rng = np.random.default_rng(31)
+    logp = rng.standard_normal(V) * 0.5
+    logp[1024:] += 1.2
+    p = np.exp(logp) / np.exp(logp).sum()
+    z = torch.from_numpy(np.broadcast_to(logp.astype(np.float32), (n, 1, V)).copy())
+    n_acc, out, flags = gpu_accept(z, None, torch.zeros(n, 0, dtype=torch.int32), 1.0, seed=9,
+                                   step=2, purpose=2)
+    counts = np.bincount(out[:, 0], minlength=V)
+    assert stats.chisquare(counts, p * n).pvalue > 0.01
+    m = 2000
+    ref = OACC.accept(z[:m].double().numpy(), None, np.zeros((m, 0), np.int64), 1.0, seed=9,
+                      step=2, purpose=2)
+    ok = ~ref["margin"]
+    assert np.array_equal(out[:m][ok], ref["out_tokens"][ok])
+    differ = out[:m, 0] != ref["out_tokens"][:, 0]
+    assert np.all(flags[:m][differ] == 1)
+    assert status_ok()
+
+
+def test_residual_draw_over_several_groups_follows_the_residual():
+    """k = 1 over 1100 tokens (groups 512, 512, 76) with q heavier than p on the first 600
+    tokens: among the rejected sequences the GPU's emitted token follows norm(max(0, p - q))."""
+    V, n = 1100, 200_000
+    rng = np.random.default_rng(4)
+    zp = rng.standard_normal(V).astype(np.float32)
+    zq = zp.copy()
+    zq[:600] += 1.0
+    p = np.exp(zp.astype(np.float64)) / np.exp(zp.astype(np.float64)).sum()
+    q = np.exp(zq.astype(np.float64)) / np.exp(zq.astype(np.float64)).sum()
+    resid = np.maximum(0.0, p - q)
+    resid /= resid.sum()
+    z = torch.from_numpy(np.broadcast_to(np.stack([zp, zp]), (n, 2, V)).copy())
+    y = torch.from_numpy(np.broadcast_to(zq, (n, 1, V)).copy())
+    drafts = torch.from_numpy(rng.choice(V, size=(n, 1), p=q).astype(np.int32))
+    n_acc, out, _ = gpu_accept(z, y, drafts, 1.0, seed=23, step=5)
+    rej = n_acc == 0
+    assert rej.sum() > 30_000
+    counts = np.bincount(out[rej, 0], minlength=V)
+    exp = resid * rej.sum()
+    big = exp >= 5
+    obs = np.append(counts[big], counts[~big].sum())
+    ex = np.append(exp[big], exp[~big].sum())
+    assert stats.chisquare(obs, ex).pvalue > 0.01
+    assert status_ok()
+
+
+def test_group_level_near_tie_is_flagged_on_the_gpu():
+    """Two groups of equal-weight tokens whose level-1 keys differ by 1e-5 (both sides flag
+    it) or by 2 (neither does); the token comes from the winning group either way."""
+    from oracle.philox import group_uniform_rows
+    V, seed, step = 1024, 5, 9
+    ug = group_uniform_rows(seed, step, [0], OACC.PURPOSE_DRAFTER, 2)[0]
+    lnEg = np.log(-np.log1p(-ug))
+    for gap, want in ((1e-5, 1), (2.0, 0)):
+        lnW1 = lnEg[1] - lnEg[0] + gap
+        z = np.empty((1, 1, V), np.float32)
+        z[0, 0, :512] = -np.log(512)
+        z[0, 0, 512:] = lnW1 - np.log(512)
+        n_acc, out, flags = gpu_accept(torch.from_numpy(z), None,
+                                       torch.zeros(1, 0, dtype=torch.int32), 1.0, seed=seed,
+                                       step=step, purpose=2)
+        ref = OACC.accept(z.astype(np.float64), None, np.zeros((1, 0), np.int64), 1.0,
+                          seed=seed, step=step, purpose=2)
+        assert int(flags[0]) == want == int(ref["margin"][0])
+        if not want:
+            assert out[0, 0] == ref["out_tokens"][0, 0]
+        assert 0 <= out[0, 0] < V
+    assert status_ok()
