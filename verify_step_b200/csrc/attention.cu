@@ -525,12 +525,18 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES, SPLIT>::THREADS,
       const uint32_t vbase = kbase + C::TILE_BYTES;
       const int p0 = (s.tf + t_begin + t) * kTile;
 
-      // ---- partial S^T = K Q^T over this warp's D slice
-      float sc[NB][4];
+      // ---- partial S^T = K Q^T over this warp's D slice (with the registers of the warpgroup
+      // split, even and odd 16-column steps in separate accumulators: two dependency chains of
+      // half the length)
+      constexpr int NCH = C::WS ? 2 : 1;
+      float sc[NB][4], s2[NCH][NB][4];
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nb][e] = 0.f;
+        for (int e = 0; e < 4; ++e) {
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) s2[c][nb][e] = 0.f;
+        }
       {
         const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
         const int coff = (lane >> 4) * 8;
@@ -539,9 +545,18 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES, SPLIT>::THREADS,
           uint32_t ka[4];
           ldsm_x4(ka, kbase + swz(key, dg * DS + ks * 16 + coff));
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(sc[nb], ka, qb[ks][nb][0], qb[ks][nb][1]);
+          for (int nb = 0; nb < NB; ++nb)
+            mma_bf16_16816(s2[ks % NCH][nb], ka, qb[ks][nb][0], qb[ks][nb][1]);
         }
       }
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          sc[nb][e] = s2[0][nb][e];
+#pragma unroll
+          for (int c = 1; c < NCH; ++c) sc[nb][e] += s2[c][nb][e];
+        }
       if constexpr (NDG > 1) {
         float4 *myred = reinterpret_cast<float4 *>(red) + ((buf * NCW + dg) * 32 + lane) * NB;
 #pragma unroll
