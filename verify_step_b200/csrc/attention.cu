@@ -304,9 +304,8 @@ struct Cfg {
 };
 
 // Rows per CTA group for an item of M query rows: groups of at most 24 rows (three 8-row
-// blocks), R groups of NB blocks each.  At D 512 a single group of two or three blocks takes
-// the warpgroup register split; groups of a larger item do better without it (measured at
-// 28 rows, two groups of two blocks: 288 against 331 us).
+// blocks), R groups of NB blocks each.  At D 512 groups of two or three blocks take the
+// warpgroup register split (28 rows, two groups of two blocks: 271 against 290 us without).
 struct RowSplit {
   int R, NB;
   bool split;
@@ -316,7 +315,7 @@ __host__ __device__ inline RowSplit row_split(int M, int D) {
   s.R = (M + 23) / 24;
   const int per = (M + s.R - 1) / s.R;
   s.NB = (per + 7) / 8;
-  s.split = D == 512 && s.NB >= 2 && s.R == 1;
+  s.split = D == 512 && s.NB >= 2;
   return s;
 }
 
