@@ -75,6 +75,9 @@ CASES = [
     (8, [0, 3], 4, 4, 4, 256, 16, 0),
     (9, [200, 31], 3, 32, 2, 128, 16, 16),  # 48 rows: three 16-row tiles
     (10, [64, 70], 8, 32, 4, 256, 16, 0),    # 64 rows
+    (13, [300, 17, 1000], 7, 16, 4, 512, 16, 0),  # 28 rows at D 512
+    (14, [90, 260], 8, 16, 2, 512, 16, 0),        # 64 rows at D 512
+    (15, [500, 40], 8, 16, 4, 512, 32, 100),      # 32 rows at D 512, sliding window
 ]
 
 
