@@ -439,23 +439,30 @@ __global__ void __launch_bounds__(192, 1)
         __threadfence();
         const int own = u % p.splits;
         const int s0 = u - own;  // first unit of the tile
-        // partials added in split order; each split's N loads are issued together (this
+        // partials added in split order; the loads of RB splits are issued together (this
         // split's own partial is still in registers)
+        constexpr int RB = N <= 16 ? 8 : N <= 32 ? 4 : N <= 48 ? 2 : 1;
         float acc[N];
 #pragma unroll
         for (int r = 0; r < N; ++r) acc[r] = 0.f;
-        for (int sp = 0; sp < p.splits; ++sp) {
-          if (sp == own) {
+        for (int sp0 = 0; sp0 < p.splits; sp0 += RB) {
+          float v[RB][N];
 #pragma unroll
-            for (int r = 0; r < N; ++r) acc[r] += y[r];
-            continue;
+          for (int q = 0; q < RB; ++q) {
+            const int sp = sp0 + q;
+            const bool load = sp < p.splits && sp != own;
+            const float *src = p.part + (size_t)(s0 + sp) * N * BM + row_in_tile;
+#pragma unroll
+            for (int r = 0; r < N; ++r)
+              v[q][r] = load && r < p.m ? __ldcg(src + (size_t)r * BM) : 0.f;
           }
-          const float *src = p.part + (size_t)(s0 + sp) * N * BM + row_in_tile;
-          float v[N];
 #pragma unroll
-          for (int r = 0; r < N; ++r) v[r] = r < p.m ? __ldcg(src + (size_t)r * BM) : 0.f;
+          for (int q = 0; q < RB; ++q) {
+            const int sp = sp0 + q;
+            if (sp >= p.splits) break;
 #pragma unroll
-          for (int r = 0; r < N; ++r) acc[r] += v[r];
+            for (int r = 0; r < N; ++r) acc[r] += sp == own ? y[r] : v[q][r];
+          }
         }
 #pragma unroll
         for (int r = 0; r < N; ++r) apply_epilogue(p, row, r, acc[r], lane);
@@ -522,9 +529,10 @@ static int n_of(int m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 48 ? 48 : 64;
 
 // Work split of a call: S splits of the K blocks per 128-row tile, chosen to minimise a time
 // model of the busiest SM: ceil(tiles S / SMs) units, each its K blocks at about 0.36 us (16 KB
-// of weights and 4 KB of x' at a fair share of the HBM rate) plus, when split, about 2.5 us of
+// of weights and 4 KB of x' at a fair share of the HBM rate) plus, when split, about 2 us of
 // partial write, fence and ticket; and the reductions the SM finishes (ceil(tiles / SMs) tiles,
-// about 0.5 us per split read back).
+// about 0.5 us per split read back).  (At 24 rows, d 5376: the gated MLP's 336 tiles take 2
+// splits, 87.9 us against 94.7 unsplit.)
 // Clusters of S CTAs of the product kernel for N that fit on the device at once (0 where the
 // device cannot say, e.g. without a GPU).
 static int max_clusters(int N, int S);
@@ -542,7 +550,7 @@ static Shape shape_of(int m, int n, int k, bool allow_cluster = false) {
     const int S_eff = (s.kblocks + kps - 1) / kps;  // every split non-empty
     if (S_eff != S) continue;
     const long long units = (long long)s.tiles * S;
-    const double per_unit = kps * 0.36 + (S > 1 ? 2.5 : 0.0);
+    const double per_unit = kps * 0.36 + (S > 1 ? 2.0 : 0.0);
     double cost = (double)((units + sms - 1) / sms) * per_unit;
     if (S > 1) cost += (double)((s.tiles + sms - 1) / sms) * 0.5 * S;
     if (best < 0.0 || cost < best) {
