@@ -1241,15 +1241,20 @@ __global__ void __launch_bounds__(WCfg<D, MT>::THREADS, 1)
   }
 }
 
-// Merges the partials of items that several CTAs shared, in CTA order; writes zero rows for
-// drafter items with an empty key range.  One CTA per (item, query row).
-template <typename T>
-__global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
+// Merges the partials of items that several CTAs shared; writes zero rows for drafter items
+// with an empty key range.  One CTA per (item, query row) of G groups of 128 threads (4
+// columns a thread): the groups take runs of 8 partials in turn, and the group sums are added
+// in group order (a fixed order for a given partition of the tiles and G).  More groups
+// shorten the chain of dependent loads when an item has many partials; the host picks them
+// when the CTAs still fit one wave.
+template <typename T, int G>
+__global__ void __launch_bounds__(128 * G) attn_combine_kernel(const Params p) {
   constexpr int kChunk = 512;
   __shared__ long long s_F, s_Fl, s_T;
   __shared__ int s_n;
   __shared__ float s_w[kChunk];
-  __shared__ float s_red[4];
+  __shared__ float s_red[4 * G];
+  __shared__ float4 s_acc[G > 1 ? G - 1 : 1][128];
   pdl_trigger();
   pdl_wait();
   const int item = blockIdx.x, row = blockIdx.y;
@@ -1321,9 +1326,11 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
       }
   const float den = block_reduce(den_loc, false);
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  // weighted sum of the partial rows, slots in CTA order, kChunk slots at a time; the loads
-  // of 8 slots are issued before their multiply-adds (they are independent L2 reads)
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // D <= 512 with 128 threads
+  // weighted sum of the partial rows, kChunk slots at a time; group grp takes runs of 8
+  // slots u0 = 8 grp, 8 (grp + G), ..., the loads of a run issued before its multiply-adds
+  // (they are independent L2 reads)
+  const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // D <= 512: 4 columns per thread of a group
   for (int t0 = 0; t0 < S; t0 += kChunk) {
     const int n = min(kChunk, S - t0);
     __syncthreads();
@@ -1334,7 +1341,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
                    : 0.f;
     }
     __syncthreads();
-    for (int u0 = 0; u0 < n; u0 += 8) {
+    for (int u0 = 8 * grp; u0 < n; u0 += 8 * G) {
       float v[8][4];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -1342,7 +1349,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
         const float *o = p.ws_o + ((slot0 + c_first + t0 + u0 + u) * p.Mpad + row) * p.D;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int d = threadIdx.x + e * 128;
+          const int d = tid + e * 128;
           v[u][e] = (w != 0.f && d < p.D) ? __ldcg(o + d) : 0.f;
         }
       }
@@ -1354,9 +1361,22 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p) {
       }
     }
   }
+  if constexpr (G > 1) {
+    if (grp > 0) s_acc[grp - 1][tid] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    if (grp > 0) return;
+#pragma unroll
+    for (int g2 = 0; g2 < G - 1; ++g2) {
+      const float4 a = s_acc[g2][tid];
+      acc[0] += a.x;
+      acc[1] += a.y;
+      acc[2] += a.z;
+      acc[3] += a.w;
+    }
+  }
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const int d = threadIdx.x + e * 128;
+    const int d = tid + e * 128;
     if (d < p.D) dst[d] = T(acc[e] * inv);
   }
 }
@@ -1564,6 +1584,15 @@ static int persistent_ctas(int D, const RowSplit &rs) {
   const int sms = sm_count();
   if (occ <= 0 || sms <= 0) return 0;
   return occ * sms;
+}
+
+// Four combine groups when an item spreads over 32 or more CTAs (P CTA groups over `items`
+// items of similar length) and one CTA per SM covers the grid of `ctas`; else one (with a few
+// partials per item the extra groups only add scheduling: B 8, k 2, about 10 partials: 180 ->
+// 182 us with two groups).
+static bool combine_wide(int ctas, int P, int items) {
+  const int sms = std::max(sm_count(), 1);
+  return ctas <= sms && P >= 32 * items;
 }
 
 static sd_status launch_bf16(int D, const RowSplit &rs, const CUtensorMap &km,
@@ -1786,7 +1815,11 @@ static sd_status run(const sd_attn_desc *d, bool draft, const void *q, const voi
   s = launch_bf16(p.D, rs, km, vm, p, st);
   if (s != SD_OK) return s;
   return cuda_status(
-      launch(attn_combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hkv, p.M), dim3(128), 0, st, p));
+      combine_wide(p.B * p.Hkv * p.M, p.P, p.B * p.Hkv)
+          ? launch(attn_combine_kernel<__nv_bfloat16, 4>, dim3(p.B * p.Hkv, p.M), dim3(512), 0,
+                   st, p)
+          : launch(attn_combine_kernel<__nv_bfloat16, 1>, dim3(p.B * p.Hkv, p.M), dim3(128), 0,
+                   st, p));
 }
 
 }  // namespace attn
