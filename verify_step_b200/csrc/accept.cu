@@ -6,16 +6,18 @@
 // u_i < p_i(d_i) / q_i(d_i); at the first rejection emit x ~ norm(max(0, p_i - q_i)); if all
 // are accepted emit the bonus x ~ p_{k+1}.  T = 0: accept iff d_i == argmax, emit argmax.
 //
-// Three kernels (a plain draw, k = 0 at T > 0, runs a ticket clear and the last):
+// Two kernels at T > 0 (a plain draw, k = 0, runs a ticket clear and the second), two at T = 0
+// (the first and accept_decide):
 //  1. accept_stats: one CTA per (logit row, token chunk) over every row the sequences need (the
 //     k+1 target rows and, for T > 0, the k draft rows), sized to one wave of CTAs: online max /
 //     sum of exp(x / T) of the chunk (T > 0), or its top two values and the argmax (T = 0),
-//     with 16-byte loads kept in flight.
-//  2. accept_decide: one CTA per sequence merges the chunks of each row (a warp per row, fixed
-//     order), tests the k drafts lane-parallel and writes the sequence's decision record
-//     (accepted count, acceptance margin flag, the normalisers of the draw row); at T = 0 it
-//     writes the outputs itself.
-//  3. accept_mass: the categorical draw as a two-level exponential race.  CTAs per (sequence,
+//     with 16-byte loads kept in flight.  It also clears the draw's tickets.
+//  The decisions (decide_seq): a CTA merges the chunks of each row of its sequence (a warp per
+//     row, fixed order) and tests the k drafts lane-parallel: the accepted count, the
+//     acceptance margin flag and the normalisers of the draw row.  At T = 0 accept_decide (one
+//     CTA per sequence) takes them and writes the outputs; at T > 0 every CTA of accept_mass
+//     takes them first (all reach the same ones), which saves a launch between the passes.
+//  2. accept_mass: the categorical draw as a two-level exponential race.  CTAs per (sequence,
 //     run of 512-token groups), one wave of them, reduce each group of the draw row to its mass
 //     (max(0, p - q) after a rejection; p for the bonus draw and plain draws) with the sums the
 //     margin bounds need.  The last CTA of a sequence (atomic ticket; no waiting) races the
@@ -35,7 +37,7 @@ namespace acc {
 
 constexpr int kStatThreads = 256;
 constexpr int kChunk = 8192;        // tokens per statistics CTA at least
-constexpr int kDecideThreads = 256;
+constexpr int kDecideThreads = 256;  // the decisions also run inside the group-mass CTAs
 constexpr int kMaxRows = 31;        // rows per sequence: 2k + 1 with k <= 15
 constexpr int kMassSlots = 592;     // group-mass CTAs aimed at: one wave at 4 CTAs per SM
 constexpr int kMassThreads = 256;   // the last CTA races 2 groups / 2 tokens per thread
@@ -49,7 +51,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kMargin2 = kMargin * kLog2e;
 constexpr float kAbsKey2 = kAbsKey * kLog2e;
 
-// Decision record of one sequence (T > 0): written by the decision kernel, read by the draw.
+// Decision record of one sequence (T > 0), taken by each CTA of the draw.
 struct Record {
   int a;          // accepted drafts
   int flag;       // an acceptance test within the margin
@@ -210,6 +212,8 @@ __global__ void __launch_bounds__(kStatThreads) accept_stats_kernel(const Params
   pdl_wait();  // many waves: no early trigger, so the next kernel does not take their slots
   const int rr = blockIdx.x, c = blockIdx.y;
   const int b = rr / p.rps, ri = rr - b * p.rps;
+  // the tickets of the group-mass kernel that follows start from zero
+  if (p.T > 0.f && ri == 0 && c == 0 && threadIdx.x == 0) p.counters[b] = 0u;
   const float *row = seq_row(p, b, ri);
   const int v0 = c * p.stats_chunk;
   const int v1 = min(p.V, v0 + p.stats_chunk);
@@ -283,19 +287,16 @@ __global__ void __launch_bounds__(kStatThreads) accept_stats_kernel(const Params
   }
 }
 
-// ------------------------------------------------------------------ decision kernel
+// ------------------------------------------------------------------ decisions
 
-__global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Params p) {
-  __shared__ float4 s_row[kMaxRows];  // merged rows
-  __shared__ uint32_t s_step;
-  pdl_wait();
-  const int b = blockIdx.x;
+// The decisions of sequence b, taken by one CTA of kDecideThreads threads from the merged row
+// statistics: greedy (T = 0) writes the outputs; sampling leaves the record of the draw in
+// *rec_out (shared memory; valid after the CTA's next barrier, which every thread must reach).
+__device__ __forceinline__ void decide_seq(const Params &p, int b, float4 *s_row,
+                                           uint32_t *s_step, Record *rec_out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool sampling = p.T > 0.f;
-  if (threadIdx.x == 0) {
-    s_step = counter_step(p);
-    if (sampling) p.counters[b] = 0u;  // tickets of the group-mass kernel
-  }
+  if (threadIdx.x == 0) *s_step = counter_step(p);
   // the drafts and their logits, loaded before the merge so that their round trips overlap it
   // (warp 0, lane i - 1 for draft i)
   int d = -1;
@@ -333,7 +334,7 @@ __global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Par
   if (warp != 0) return;
 
   // ---- decisions (one warp): lane i-1 tests draft i; the first rejection stops the scan
-  const uint32_t step = s_step;
+  const uint32_t step = *s_step;
   const float inv_t = sampling ? 1.f / p.T : 1.f;
   bool acc = true;
   int flag = 0;
@@ -382,7 +383,18 @@ __global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Par
   r.isz = 1.f / sz.y;
   r.my = sy.x;
   r.isy = 1.f / sy.y;
-  p.rec[b] = r;
+  *rec_out = r;
+}
+
+static_assert(kDecideThreads == kMassThreads, "the group-mass CTAs take the decisions too");
+
+// Greedy acceptance (T = 0): one CTA per sequence takes the decisions and writes the outputs.
+__global__ void __launch_bounds__(kDecideThreads) accept_decide_kernel(const Params p) {
+  __shared__ float4 s_row[kMaxRows];  // merged rows
+  __shared__ uint32_t s_step;
+  __shared__ Record s_rec;
+  pdl_wait();
+  decide_seq(p, blockIdx.x, s_row, &s_step, &s_rec);
 }
 
 // ------------------------------------------------------------------ group masses and the race
@@ -441,13 +453,19 @@ __global__ void __launch_bounds__(kMassThreads) accept_mass_kernel(const Params 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   __shared__ Race s_red[kMassThreads / 32];
   __shared__ int s_last;
+  __shared__ float4 s_row[kMaxRows];
+  __shared__ uint32_t s_step;
+  __shared__ Record s_rec;
 
-  // every thread reads the record itself (one broadcast load): no barrier before the loads
+  // Every CTA of the sequence takes the decisions itself (the same ones: they read the same
+  // statistics), then reads the row they select.
   Record rec;
   if (p.k == 0) {  // plain draw: no decisions, unnormalised keys
     rec = Record{0, 0, 0u, 0, 0.f, 1.f, 0.f, 1.f};
   } else {
-    rec = p.rec[b];
+    decide_seq(p, b, s_row, &s_step, &s_rec);
+    __syncthreads();
+    rec = s_rec;
   }
   const int a = rec.a;
   const bool resid = a < p.k;
@@ -639,7 +657,7 @@ __global__ void __launch_bounds__(kMassThreads) accept_mass_kernel(const Params 
   p.counters[b] = 0u;
 }
 
-// Zeroes the per-sequence tickets of the draw (plain draws, which have no decision pass to
+// Zeroes the per-sequence tickets of the draw (plain draws, which have no statistics pass to
 // clear them).
 __global__ void clear_tickets_kernel(unsigned int *counters, int B) {
   pdl_wait();
@@ -778,9 +796,9 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
     if (launch(accept_stats_kernel, dim3(p.B * p.rps, p.nchunks), dim3(kStatThreads), 0, st,
                p) != cudaSuccess)
       return SD_ERR_CUDA;
-    if (launch(accept_decide_kernel, dim3(p.B), dim3(kDecideThreads), 0, st, p) != cudaSuccess)
-      return SD_ERR_CUDA;
-    if (!sampling) return SD_OK;  // greedy: the decision pass wrote the outputs
+    if (!sampling)  // greedy: the decision pass writes the outputs
+      return cuda_status(
+          launch(accept_decide_kernel, dim3(p.B), dim3(kDecideThreads), 0, st, p));
   }
   return cuda_status(
       launch(accept_mass_kernel, dim3(p.B, p.nmass), dim3(kMassThreads), 0, st, p));
@@ -822,7 +840,7 @@ extern "C" sd_status sd_accept_noalloc(const sd_accept_desc *desc, const float *
   void *scratch = sdv::acc::noalloc_scratch();
   if (scratch == nullptr) return SD_ERR_CUDA;
   // The per-sequence tickets in the scratch are cleared at the start of every call (by the
-  // decision kernel, or a one-block kernel for a plain draw), and every other byte the kernels
+  // statistics kernel, or a one-block kernel for a plain draw), and every other byte the kernels
   // read is written earlier in the same call, so the array's leftover contents from an earlier
   // call do not matter.
   return sd_accept(desc, target_logits, draft_logits, draft_tokens, n_accepted, out_tokens,
