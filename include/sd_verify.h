@@ -226,7 +226,7 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
  * SD_ACCEPT_NOALLOC_MAX_SCRATCH bytes compiled into the library, which every GPU that loads the
  * library holds until the process exits.  A request whose sd_accept_workspace_size exceeds that
  * limit is rejected with SD_ERR_WORKSPACE before anything is launched (at V = 262144 the limit
- * covers up to 281 sequences at k = 6, 388 at k = 2).  The first call on a device, and the
+ * covers up to 282 sequences at k = 6, 389 at k = 2).  The first call on a device, and the
  * first after the device's context changes (e.g. after a device reset), looks up the array's
  * device address (cudaGetSymbolAddress), so make that first call before any stream capture.
  * All calls share the one array: calls that may overlap on the GPU (other streams, other host

@@ -78,6 +78,8 @@ CASES = [
     (13, [300, 17, 1000], 7, 16, 4, 512, 16, 0),  # 28 rows at D 512
     (14, [90, 260], 8, 16, 2, 512, 16, 0),        # 64 rows at D 512
     (15, [500, 40], 8, 16, 4, 512, 32, 100),      # 32 rows at D 512, sliding window
+    (16, [20000], 1, 8, 1, 64, 16, 0),   # one item over every CTA: more than 512 partials
+    (17, [9000], 2, 8, 2, 128, 16, 0),   # a few items, hundreds of partials each
 ]
 
 

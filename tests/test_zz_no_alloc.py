@@ -76,11 +76,11 @@ def test_noalloc_other_shapes_in_a_row():
 
 def test_noalloc_refuses_requests_beyond_its_scratch():
     V, k = 262144, 6
-    desc = sd.AcceptDesc(batch=282, k=k, vocab=V, temperature=1.0, seed=0, step=0, purpose=1)
+    desc = sd.AcceptDesc(batch=283, k=k, vocab=V, temperature=1.0, seed=0, step=0, purpose=1)
     assert sd.sd_accept_workspace_size(desc) > (4 << 20)
-    desc.batch = 281
-    assert sd.sd_accept_workspace_size(desc) <= (4 << 20)
     desc.batch = 282
+    assert sd.sd_accept_workspace_size(desc) <= (4 << 20)
+    desc.batch = 283
     # nothing is dereferenced or launched: null data pointers are fine for the size check
     st = sd.lib().sd_accept_noalloc(ctypes.byref(desc), None, None, None, None, None, None,
                                     None)

@@ -78,7 +78,6 @@ struct Params {
   int32_t *out;
   int32_t *margin;
   float4 *stats;           // [B * rps][nchunks] chunk partials
-  Record *rec;             // [B]
   float4 *gm;              // [B][ngroups] group masses of the draw row
   unsigned int *counters;  // [B]
   int *status;
@@ -725,7 +724,6 @@ static size_t ws_size(const sd_accept_desc *d) {
   if (validate(d) != SD_OK) return 0;
   const size_t rows = (size_t)d->batch * (2 * d->k + 1);
   return round_up(rows * nchunks_of(d->vocab) * 16, 256) +
-         round_up((size_t)d->batch * sizeof(Record), 256) +
          round_up((size_t)d->batch * ngroups_of(d->vocab) * 16, 256) +
          round_up((size_t)d->batch * 4, 256);
 }
@@ -778,8 +776,6 @@ sd_status sd_accept(const sd_accept_desc *desc, const float *target_logits,
   uint8_t *w8 = reinterpret_cast<uint8_t *>(ws);
   p.stats = reinterpret_cast<float4 *>(w8);
   w8 += round_up((size_t)p.B * (2 * p.k + 1) * nchunks_of(p.V) * 16, 256);
-  p.rec = reinterpret_cast<Record *>(w8);
-  w8 += round_up((size_t)p.B * sizeof(Record), 256);
   p.gm = reinterpret_cast<float4 *>(w8);
   w8 += round_up((size_t)p.B * p.ngroups * 16, 256);
   p.counters = reinterpret_cast<unsigned int *>(w8);
