@@ -509,26 +509,12 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES, SPLIT>::THREADS,
         for (int e = 0; e < 4; ++e) o[mb][nb][e] = 0.f;
     }
 
-    for (int t = 0; t < seg_n; ++t) {
-      const int stage = it % STAGES;
-      const uint32_t ph = (it / STAGES) & 1;
-      // (the warp leaves together: its later shuffles and votes need every lane)
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], ph, abort_flag))) {
-        record_status(p.status, SD_ERR_TIMEOUT);
-        *abort_flag = 1;
-        ok = false;
-        break;
-      }
-      const int is_bad = bad[stage];
-      const uint32_t kbase = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
-      const uint32_t vbase = kbase + C::TILE_BYTES;
-      const int p0 = (s.tf + t_begin + t) * kTile;
-
-      // ---- partial S^T = K Q^T over this warp's D slice (with the registers of the warpgroup
-      // split, even and odd 16-column steps in separate accumulators: two dependency chains of
-      // half the length)
-      constexpr int NCH = C::WS ? 2 : 1;
-      float sc[NB][4], s2[NCH][NB][4];
+    // ---- partial S^T = K Q^T of one tile over this warp's D slice (with the registers of the
+    // warpgroup split, even and odd 16-column steps in separate accumulators: two dependency
+    // chains of half the length)
+    constexpr int NCH = C::WS ? 2 : 1;
+    auto qk_tile = [&](uint32_t kb, float (&part)[NB][4]) {
+      float s2[NCH][NB][4];
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -536,32 +522,94 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES, SPLIT>::THREADS,
 #pragma unroll
           for (int c = 0; c < NCH; ++c) s2[c][nb][e] = 0.f;
         }
-      {
-        const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int coff = (lane >> 4) * 8;
+      const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int coff = (lane >> 4) * 8;
 #pragma unroll
-        for (int ks = 0; ks < DS / 16; ++ks) {
-          uint32_t ka[4];
-          ldsm_x4(ka, kbase + swz(key, dg * DS + ks * 16 + coff));
+      for (int ks = 0; ks < DS / 16; ++ks) {
+        uint32_t ka[4];
+        ldsm_x4(ka, kb + swz(key, dg * DS + ks * 16 + coff));
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb)
-            mma_bf16_16816(s2[ks % NCH][nb], ka, qb[ks][nb][0], qb[ks][nb][1]);
-        }
+        for (int nb = 0; nb < NB; ++nb)
+          mma_bf16_16816(s2[ks % NCH][nb], ka, qb[ks][nb][0], qb[ks][nb][1]);
       }
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          sc[nb][e] = s2[0][nb][e];
+          part[nb][e] = s2[0][nb][e];
 #pragma unroll
-          for (int c = 1; c < NCH; ++c) sc[nb][e] += s2[c][nb][e];
+          for (int c = 1; c < NCH; ++c) part[nb][e] += s2[c][nb][e];
         }
-      if constexpr (NDG > 1) {
-        float4 *myred = reinterpret_cast<float4 *>(red) + ((buf * NCW + dg) * 32 + lane) * NB;
+    };
+    // (the warp leaves a wait together: its later shuffles and votes need every lane)
+    auto wait_full = [&](uint32_t itx) {
+      return __all_sync(0xffffffffu,
+                        mbar_wait(&full[itx % STAGES], (itx / STAGES) & 1, abort_flag));
+    };
+    auto stage_k = [&](uint32_t itx) {
+      return smem_u32(stages + (size_t)(itx % STAGES) * C::STAGE_BYTES);
+    };
+    // With several D slices and one row block (the drafter's call) the partials of tile t + 1
+    // are computed and published before the exchange of tile t is awaited: the wait for the
+    // other warps overlaps this warp's next products, nxt holding them in between (D 512,
+    // B 8: 168.6 -> 163.5 us).  With more row blocks the extra live registers cost more than
+    // the overlap gains (k 6: 270 -> 279 us), so those tiles keep the plain order.
+    constexpr bool PIPE = NDG > 1 && NB == 1;
+    static_assert(!PIPE || STAGES >= 2, "the next tile is awaited before this one is released");
+    auto publish = [&](int bf, const float (&part)[NB][4]) {
+      float4 *myred = reinterpret_cast<float4 *>(red) + ((bf * NCW + dg) * 32 + lane) * NB;
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-          myred[nb] = make_float4(sc[nb][0], sc[nb][1], sc[nb][2], sc[nb][3]);
-        mbar_arrive(&red_bar[buf]);
+      for (int nb = 0; nb < NB; ++nb)
+        myred[nb] = make_float4(part[nb][0], part[nb][1], part[nb][2], part[nb][3]);
+      mbar_arrive(&red_bar[bf]);
+    };
+    if constexpr (PIPE) {
+      if (seg_n > 0) {
+        if (!wait_full(it)) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+        } else {
+          float part[NB][4];
+          qk_tile(stage_k(it), part);
+          publish(buf, part);
+        }
+      }
+    }
+
+    for (int t = 0; t < seg_n && ok; ++t) {
+      const int stage = it % STAGES;
+      if constexpr (!PIPE) {
+        if (!wait_full(it)) {
+          record_status(p.status, SD_ERR_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+      }
+      const int is_bad = bad[stage];
+      const uint32_t kbase = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
+      const uint32_t vbase = kbase + C::TILE_BYTES;
+      const int p0 = (s.tf + t_begin + t) * kTile;
+
+      float sc[NB][4];
+      float nxt[PIPE ? NB : 1][4];
+      const bool have_next = PIPE && t + 1 < seg_n;
+      if constexpr (!PIPE) {
+        qk_tile(kbase, sc);
+        if constexpr (NDG > 1) publish(buf, sc);
+      } else {
+        if (have_next) {
+          if (!wait_full(it + 1)) {
+            record_status(p.status, SD_ERR_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          qk_tile(stage_k(it + 1), nxt);
+        }
+      }
+      if constexpr (NDG > 1) {
         if (!__all_sync(0xffffffffu, mbar_wait(&red_bar[buf], (it >> 1) & 1, abort_flag))) {
           record_status(p.status, SD_ERR_TIMEOUT);
           *abort_flag = 1;
@@ -700,6 +748,9 @@ __global__ void __launch_bounds__(Cfg<D, NB, STAGES, SPLIT>::THREADS,
         }
       }
       mbar_arrive(&empty[stage]);
+      if constexpr (PIPE) {
+        if (have_next) publish(buf, nxt);  // buf was toggled after this tile's exchange
+      }
       ++it;
     }
     if (!ok) break;
