@@ -201,6 +201,8 @@ DRAFT_CASES = [
     (21, [37, 100, 5], [40, 99, 0], 8, 2, 256, 16, 24),
     (22, [300, 17], [299, 500], 16, 4, 512, 16, 0),
     (23, [64, 0, 9], [63, 5, 2], 16, 4, 256, 16, 512),
+    (24, [20000], [19999], 8, 1, 64, 16, 0),   # one item over every CTA: over 512 partials
+    (25, [9000], [8999], 8, 2, 512, 16, 0),    # B 1 at D 512: hundreds of partials per item
 ]
 
 
